@@ -1,0 +1,241 @@
+"""Selector-driven block-sparse attention for B200 (sm_100a).
+
+Thin Python binding of ``libsparse_attn.so`` (C ABI in ``include/sparse_attn.h``):
+argument marshalling only -- every step runs in the library's CUDA kernels.
+PyTorch provides device memory and streams.  The functions ``sparse_attn_*``
+mirror the C entry points one to one (pointers as ints, the stream as an int
+handle); the lower-case helpers take torch tensors, allocate outputs and raise
+``SparseAttnError`` on a non-zero return code.
+
+The library must have been built (``python -m block_sparse_long_landmark_b200.build``);
+there is no fallback of any kind when it is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+from .inputs import F_CAUSAL, F_GATE, F_HIER, F_LOCAL, F_PER_QHEAD, F_SINK  # noqa: F401
+
+SA_SINK, SA_LOCAL, SA_GATE, SA_HIER, SA_CAUSAL, SA_SELECT_PER_QHEAD = 1, 2, 4, 8, 16, 32
+SA_BF16, SA_FP32 = 0, 1
+SA_OP_LANDMARKS, SA_OP_SELECT, SA_OP_SELECT_DECODE, SA_OP_PREFILL, SA_OP_DECODE = 0, 1, 2, 3, 4
+SA_OK, SA_ERR_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_LAUNCH, SA_ERR_DEVICE = 0, -1, -2, -3, -4, -5
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libsparse_attn.so")
+
+EXPORTS = (
+    "sparse_attn_workspace_size", "sparse_attn_landmarks", "sparse_attn_select", "sparse_attn_select_decode",
+    "sparse_attn_prefill", "sparse_attn_decode", "sparse_attn_check_status", "sparse_attn_status_string",
+    "sparse_attn_version",
+)
+
+
+class sa_params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int),
+                ("N", ctypes.c_int), ("block", ctypes.c_int), ("top_k", ctypes.c_int), ("flags", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("scale", ctypes.c_float)]
+
+    def __repr__(self):
+        return "sa_params(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {sparse_attn_status_string(code)} (code {code})")
+        self.code = code
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it was not built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m block_sparse_long_landmark_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P = ctypes.POINTER(sa_params)
+            vp, sz, i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+            L.sparse_attn_workspace_size.argtypes = [P, i]
+            L.sparse_attn_workspace_size.restype = sz
+            L.sparse_attn_landmarks.argtypes = [P, vp, vp, vp]
+            L.sparse_attn_select.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.sparse_attn_select_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.sparse_attn_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.sparse_attn_check_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int)]
+            L.sparse_attn_status_string.argtypes = [i]
+            L.sparse_attn_status_string.restype = ctypes.c_char_p
+            L.sparse_attn_version.argtypes = []
+            for n in EXPORTS[1:7]:
+                getattr(L, n).restype = i
+            L.sparse_attn_version.restype = i
+            _lib = L
+    return _lib
+
+
+# ----------------------------------------------------------------------------
+# The C entry points, one to one
+# ----------------------------------------------------------------------------
+
+def sparse_attn_workspace_size(p: sa_params, op: int) -> int:
+    return int(lib().sparse_attn_workspace_size(ctypes.byref(p), op))
+
+
+def sparse_attn_landmarks(p, K, L, stream) -> int:
+    return lib().sparse_attn_landmarks(ctypes.byref(p), K, L, stream)
+
+
+def sparse_attn_select(p, Q, L, idx, score, count, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_select(ctypes.byref(p), Q, L, idx, score, count, ws, ws_bytes, stream)
+
+
+def sparse_attn_select_decode(p, q, L, idx, score, count, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_select_decode(ctypes.byref(p), q, L, idx, score, count, ws, ws_bytes, stream)
+
+
+def sparse_attn_prefill(p, Q, K, V, idx, score, count, O, lse, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_prefill(ctypes.byref(p), Q, K, V, idx, score, count, O, lse, ws, ws_bytes, stream)
+
+
+def sparse_attn_decode(p, q, K, V, idx, score, count, o, lse, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_decode(ctypes.byref(p), q, K, V, idx, score, count, o, lse, ws, ws_bytes, stream)
+
+
+def sparse_attn_check_status(ws, stream):
+    detail = ctypes.c_int(0)
+    rc = lib().sparse_attn_check_status(ws, stream, ctypes.byref(detail))
+    return rc, detail.value
+
+
+def sparse_attn_status_string(code: int) -> str:
+    return lib().sparse_attn_status_string(code).decode()
+
+
+def sparse_attn_version() -> int:
+    return lib().sparse_attn_version()
+
+
+# ----------------------------------------------------------------------------
+# Tensor helpers
+# ----------------------------------------------------------------------------
+
+def make_params(B, Hq, Hkv, d, N, block, top_k, flags, dtype="bf16", scale=0.0) -> sa_params:
+    dt = {"bf16": SA_BF16, "fp32": SA_FP32}[dtype] if isinstance(dtype, str) else int(dtype)
+    return sa_params(B, Hq, Hkv, d, N, block, top_k, flags, dt, float(scale))
+
+
+def params_for(wl, **over) -> sa_params:
+    """Parameters of an ``inputs.Workload`` (fields overridable)."""
+    kw = dict(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, N=wl.N, block=wl.block, top_k=wl.top_k, flags=wl.flags,
+              dtype=wl.dtype)
+    kw.update(over)
+    return make_params(**kw)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check(rc: int, what: str):
+    if rc != SA_OK:
+        raise SparseAttnError(rc, what)
+
+
+def _tdtype(p):
+    torch = _torch()
+    return torch.bfloat16 if p.dtype == SA_BF16 else torch.float32
+
+
+def _hsel(p):
+    return p.Hq if p.flags & SA_SELECT_PER_QHEAD else p.Hkv
+
+
+def workspace(p: sa_params, device="cuda"):
+    """A zero-filled workspace large enough for every operation of `p`."""
+    torch = _torch()
+    n = max(sparse_attn_workspace_size(p, op) for op in range(5))
+    if n == 0:
+        raise SparseAttnError(SA_ERR_ARG, "workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def landmarks(p, K, out=None, stream=None):
+    torch = _torch()
+    nb = (p.N + p.block - 1) // p.block
+    L = out if out is not None else torch.empty(p.B, p.Hkv, nb, p.d, dtype=_tdtype(p), device=K.device)
+    _check(sparse_attn_landmarks(p, _ptr(K), _ptr(L), _stream(stream)), "sparse_attn_landmarks")
+    return L
+
+
+def _sel_out(p, decode, device):
+    torch = _torch()
+    cap = p.top_k + 2
+    lead = (p.B, _hsel(p)) if decode else (p.B, _hsel(p), (p.N + p.block - 1) // p.block)
+    return (torch.empty(*lead, cap, dtype=torch.int32, device=device),
+            torch.empty(*lead, cap, dtype=torch.float32, device=device),
+            torch.empty(*lead, dtype=torch.int32, device=device))
+
+
+def select(p, Q, L, ws, out=None, stream=None):
+    idx, sc, cnt = out if out is not None else _sel_out(p, False, Q.device)
+    _check(sparse_attn_select(p, _ptr(Q), _ptr(L), _ptr(idx), _ptr(sc), _ptr(cnt), _ptr(ws), ws.numel(),
+                              _stream(stream)), "sparse_attn_select")
+    return idx, sc, cnt
+
+
+def select_decode(p, q, L, ws, out=None, stream=None):
+    idx, sc, cnt = out if out is not None else _sel_out(p, True, q.device)
+    _check(sparse_attn_select_decode(p, _ptr(q), _ptr(L), _ptr(idx), _ptr(sc), _ptr(cnt), _ptr(ws), ws.numel(),
+                                     _stream(stream)), "sparse_attn_select_decode")
+    return idx, sc, cnt
+
+
+def prefill(p, Q, K, V, idx, sc, cnt, ws, out=None, stream=None):
+    torch = _torch()
+    if out is None:
+        O = torch.empty_like(Q)
+        lse = torch.empty(p.B, p.Hq, p.N, dtype=torch.float32, device=Q.device)
+    else:
+        O, lse = out
+    _check(sparse_attn_prefill(p, _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(sc), _ptr(cnt), _ptr(O), _ptr(lse),
+                               _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_prefill")
+    return O, lse
+
+
+def decode(p, q, K, V, idx, sc, cnt, ws, out=None, stream=None):
+    torch = _torch()
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(p.B, p.Hq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(sparse_attn_decode(p, _ptr(q), _ptr(K), _ptr(V), _ptr(idx), _ptr(sc), _ptr(cnt), _ptr(o), _ptr(lse),
+                              _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_decode")
+    return o, lse
+
+
+def check_status(ws, stream=None):
+    """Raises SparseAttnError when the status word reports a device problem."""
+    rc, detail = sparse_attn_check_status(_ptr(ws), _stream(stream))
+    if rc != SA_OK:
+        raise SparseAttnError(rc, f"device status bits {detail:#x}")
+    return detail

@@ -1,0 +1,151 @@
+// api.cu -- the C ABI of libsparse_attn.so: argument checks, workspace
+// sizing, dispatch to the kernels, status word.  See include/sparse_attn.h.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+
+using namespace sa;
+
+namespace {
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Resolves and checks a parameter block.  Returns SA_OK or an error code.
+int resolve(const sa_params *p, Shape &s) {
+    if (!p) return SA_ERR_ARG;
+    if (p->B <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->N <= 0 || p->block <= 0) return SA_ERR_ARG;
+    if (p->Hq % p->Hkv) return SA_ERR_ARG;
+    if (p->dtype != SA_BF16 && p->dtype != SA_FP32) return SA_ERR_ARG;
+    if (p->top_k < 0 || p->top_k > 256) return SA_ERR_ARG;
+    if (p->flags & ~(SA_SINK | SA_LOCAL | SA_GATE | SA_HIER | SA_CAUSAL | SA_SELECT_PER_QHEAD)) return SA_ERR_ARG;
+    if (!(p->scale >= 0.f) || isinf(p->scale)) return SA_ERR_ARG;
+    if (p->d != 64 && p->d != 128) return SA_ERR_UNSUPPORTED;
+    if (p->block < 16 || p->block > 128 || p->block % 16) return SA_ERR_UNSUPPORTED;
+    if ((p->flags & SA_GATE) && (p->flags & SA_HIER)) return SA_ERR_UNSUPPORTED;
+    if ((p->flags & SA_GATE) && !(p->flags & SA_LOCAL)) return SA_ERR_UNSUPPORTED;
+    s.B = p->B;
+    s.Hq = p->Hq;
+    s.Hkv = p->Hkv;
+    s.G = p->Hq / p->Hkv;
+    s.d = p->d;
+    s.N = p->N;
+    s.bs = p->block;
+    s.nb = (p->N + p->block - 1) / p->block;
+    s.top_k = p->top_k;
+    s.cap = p->top_k + 2;
+    s.flags = p->flags;
+    s.dtype = p->dtype;
+    const bool perq = p->flags & SA_SELECT_PER_QHEAD;
+    s.Hsel = perq ? p->Hq : p->Hkv;
+    s.heads_per = perq ? 1 : s.G;
+    s.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+    if ((long long)s.B * s.Hq * s.nb > (1ll << 31) - 1) return SA_ERR_UNSUPPORTED;
+    if (s.heads_per * s.d > 2048) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+int launch_result(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_LAUNCH; }
+
+}  // namespace
+
+extern "C" {
+
+size_t sparse_attn_workspace_size(const sa_params *p, int op) {
+    Shape s;
+    if (resolve(p, s) != SA_OK) return 0;
+    size_t extra = 0;
+    switch (op) {
+        case SA_OP_SELECT: extra = select_workspace(s, false); break;
+        case SA_OP_SELECT_DECODE: extra = select_workspace(s, true); break;
+        case SA_OP_DECODE: extra = decode_workspace(s); break;
+        default: break;
+    }
+    return kStatusBytes + ((extra + 255) & ~(size_t)255);
+}
+
+int sparse_attn_landmarks(const sa_params *p, const void *K, void *L, void *stream) {
+    Shape s;
+    int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    if (!K || !L || !aligned16(K) || !aligned16(L)) return SA_ERR_ARG;
+    return launch_result(launch_landmarks(s, K, L, (cudaStream_t)stream));
+}
+
+static int select_common(const sa_params *p, bool decode, const void *Q, const void *L, int32_t *idx, float *score,
+                         int32_t *count, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    if (!Q || !L || !idx || !score || !count || !ws) return SA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(L) || !aligned16(ws)) return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_workspace_size(p, decode ? SA_OP_SELECT_DECODE : SA_OP_SELECT)) return SA_ERR_WORKSPACE;
+    return launch_result(launch_select(s, decode, Q, L, idx, score, count, ws, ws_bytes, (cudaStream_t)stream));
+}
+
+int sparse_attn_select(const sa_params *p, const void *Q, const void *L, int32_t *idx, float *score,
+                       int32_t *count, void *ws, size_t ws_bytes, void *stream) {
+    return select_common(p, false, Q, L, idx, score, count, ws, ws_bytes, stream);
+}
+
+int sparse_attn_select_decode(const sa_params *p, const void *q, const void *L, int32_t *idx, float *score,
+                              int32_t *count, void *ws, size_t ws_bytes, void *stream) {
+    return select_common(p, true, q, L, idx, score, count, ws, ws_bytes, stream);
+}
+
+int sparse_attn_prefill(const sa_params *p, const void *Q, const void *K, const void *V, const int32_t *idx,
+                        const float *score, const int32_t *count, void *O, float *lse, void *ws,
+                        size_t ws_bytes, void *stream) {
+    Shape s;
+    int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    if (!Q || !K || !V || !idx || !score || !count || !O || !lse || !ws) return SA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(ws)) return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_PREFILL)) return SA_ERR_WORKSPACE;
+    return launch_result(
+        launch_prefill_simt(s, Q, K, V, idx, score, count, O, lse, (unsigned *)ws, (cudaStream_t)stream));
+}
+
+int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
+                       const float *score, const int32_t *count, void *o, float *lse, void *ws, size_t ws_bytes,
+                       void *stream) {
+    Shape s;
+    int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    if (!q || !K || !V || !idx || !score || !count || !o || !lse || !ws) return SA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(o) || !aligned16(ws)) return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_DECODE)) return SA_ERR_WORKSPACE;
+    return launch_result(launch_decode(s, q, K, V, idx, score, count, o, lse, ws, ws_bytes, (cudaStream_t)stream));
+}
+
+int sparse_attn_check_status(void *ws, void *stream, int *detail) {
+    if (!ws) return SA_ERR_ARG;
+    unsigned word = 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SA_ERR_LAUNCH;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_LAUNCH;
+    if (detail) *detail = (int)word;
+    if (word) {
+        if (cudaMemsetAsync(ws, 0, sizeof(word), st) != cudaSuccess) return SA_ERR_LAUNCH;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_LAUNCH;
+        return SA_ERR_DEVICE;
+    }
+    return SA_OK;
+}
+
+const char *sparse_attn_status_string(int code) {
+    switch (code) {
+        case SA_OK: return "ok";
+        case SA_ERR_ARG: return "invalid argument (null or misaligned pointer, bad shape or flag)";
+        case SA_ERR_UNSUPPORTED: return "unsupported combination of shape, dtype or flags";
+        case SA_ERR_WORKSPACE: return "workspace missing or too small";
+        case SA_ERR_LAUNCH: return "CUDA launch or copy failed";
+        case SA_ERR_DEVICE: return "device-side problem recorded in the status word";
+        default: return "unknown status code";
+    }
+}
+
+int sparse_attn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+// common.cuh -- shared device helpers and the internal launch interface of
+// libsparse_attn.so.  sm_100a only.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sparse_attn.h"
+
+namespace sa {
+
+// Status word at the start of every workspace: bit 1 = index list entry out
+// of range, bit 2 = NaN score, bit 4 = bounded wait expired.
+constexpr unsigned kStatusBadIndex = 1u;
+constexpr unsigned kStatusNaN = 2u;
+constexpr unsigned kStatusTimeout = 4u;
+constexpr size_t kStatusBytes = 256;   // keeps what follows 256-byte aligned
+
+// Shape of one call, resolved on the host.
+struct Shape {
+    int B, Hq, Hkv, G, d, N, bs, nb, top_k, cap, flags, dtype;
+    int Hsel;        // heads that own a selection list (Hkv, or Hq per q-head)
+    int heads_per;   // query heads that share one list (G, or 1 per q-head)
+    float scale;
+};
+
+__device__ __forceinline__ void set_status(unsigned *status, unsigned bit) {
+    if (status) atomicOr(status, bit);
+}
+
+// fp32 -> uint32 key whose unsigned order is the float order (NaN -> 0).
+__device__ __forceinline__ uint32_t ord_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+__device__ __forceinline__ float log_sigmoid(float x) {
+    return x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));
+}
+
+// 16-byte vector loads converted to fp32.
+__device__ __forceinline__ void load16(const __nv_bfloat16 *p, float *f) {
+    uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+__device__ __forceinline__ void load16(const float *p, float *f) {
+    float4 u = *reinterpret_cast<const float4 *>(p);
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+}
+__device__ __forceinline__ void store16(__nv_bfloat16 *p, const float *f) {
+    uint4 u;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = u;
+}
+__device__ __forceinline__ void store16(float *p, const float *f) {
+    *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
+}
+template <typename T> struct Vec { static constexpr int n = 16 / sizeof(T); };
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void from_f(float &y, float x) { y = x; }
+__device__ __forceinline__ void from_f(__nv_bfloat16 &y, float x) { y = __float2bfloat16_rn(x); }
+
+// Inclusive scan over a CTA of 256 threads (8 warps); `tmp` holds 8 ints.
+__device__ __forceinline__ int block_scan_incl(int v, int *tmp, int *total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    if (lane == 31) tmp[w] = v;
+    __syncthreads();
+    int add = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int x = tmp[i];
+        if (i < w) add += x;
+        tot += x;
+    }
+    __syncthreads();
+    if (total) *total = tot;
+    return v + add;
+}
+
+// ---------------------------------------------------------------------------
+// Internal launchers (return cudaError_t of the launch)
+// ---------------------------------------------------------------------------
+cudaError_t launch_landmarks(const Shape &s, const void *K, void *L, cudaStream_t st);
+cudaError_t launch_select(const Shape &s, bool decode, const void *Q, const void *L, int32_t *idx, float *score,
+                          int32_t *count, void *ws, size_t ws_bytes, cudaStream_t st);
+size_t select_workspace(const Shape &s, bool decode);
+cudaError_t launch_prefill_simt(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
+                                const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
+                                cudaStream_t st);
+cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
+                          const float *score, const int32_t *count, void *o, float *lse, void *ws,
+                          size_t ws_bytes, cudaStream_t st);
+size_t decode_workspace(const Shape &s);
+
+}  // namespace sa

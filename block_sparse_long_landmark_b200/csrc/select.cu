@@ -1,0 +1,430 @@
+// select.cu -- pooled-query scoring against block landmarks and hard top-K.
+//
+// [SAS] opening section / "Ключевые факты": a light selector scores context
+// units and a hard top-K keeps the best; the current block is always kept.
+// The Latent Sparse Attention post ("Индекс перестаёт перебирать весь
+// контекст"): the start of the context is always added as well.
+//
+// One unit = (batch, kv-head, query tile) in prefill or (batch, kv-head) in
+// decode (per q-head with SA_SELECT_PER_QHEAD).  A CTA pools the unit's query
+// (mean over its query heads and the tile's rows), scores one chunk of the
+// candidate blocks (s_b = scale * <qbar, L_b>, fp32), and radix-selects the
+// chunk's top-K on 32-bit order-preserving keys of the fp32 score; equal
+// scores go to the lower block index (the candidates sit in index order and
+// ties are ranked by position).  With one chunk per unit the CTA writes the
+// final list; otherwise each chunk leaves its top-K in the workspace and a
+// merge kernel picks the unit's top-K from them.  Either way the result is
+// the exact top-K of the whole candidate set, independent of the split.
+#include "common.cuh"
+
+namespace sa {
+
+constexpr int kSelThreads = 256;
+constexpr int kMaxChunk = 8192;
+
+struct SelArgs {
+    Shape s;
+    const void *Q;       // prefill Q [B,Hq,N,d] or decode q [B,Hq,d]
+    const void *L;       // [B,Hkv,nb,d]
+    int32_t *idx;
+    float *score;
+    int32_t *count;
+    unsigned *status;
+    uint32_t *part_key;  // [units][S][top_k]
+    int32_t *part_idx;   // [units][S][top_k]
+    float *special;      // [units][2]: s_0, s_local
+    int S;               // chunks per unit
+    int CH;              // candidates per chunk
+    int decode;
+    int ntiles;          // prefill: nb; decode: 1
+};
+
+struct SelSmem {
+    float qbar[256];
+    int hist[256];
+    int tmp[8];
+    int sel_digit, sel_above;
+    float s_special[2];
+};
+
+// Decodes a unit number into (batch, selection head, tile) and its local block.
+__device__ __forceinline__ void unit_coords(const SelArgs &a, int u, int &b, int &hs, int &j, int &local) {
+    j = u % a.ntiles;
+    int r = u / a.ntiles;
+    hs = r % a.s.Hsel;
+    b = r / a.s.Hsel;
+    local = a.decode ? (a.s.N - 1) / a.s.bs : j;
+}
+
+// Pooled query of the unit into sm.qbar (fp32).  Every thread participates.
+template <typename T, int VPR>
+__device__ void pool_query(const SelArgs &a, int b, int hs, int j, SelSmem &sm, float *red) {
+    constexpr int EPV = Vec<T>::n;
+    constexpr int NG = kSelThreads / VPR;
+    const Shape &s = a.s;
+    const int d = VPR * EPV;
+    const int h0 = (s.flags & SA_SELECT_PER_QHEAD) ? hs : hs * s.G;
+    const int nh = s.heads_per;
+    const int r0 = a.decode ? 0 : j * s.bs;
+    const int nrows = a.decode ? 1 : min(s.bs, s.N - r0);
+    const int R = nh * nrows;
+    const int cv = threadIdx.x % VPR, rg = threadIdx.x / VPR;
+    float acc[EPV];
+#pragma unroll
+    for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
+    const T *Q = (const T *)a.Q;
+    for (int r = rg; r < R; r += NG) {
+        const int hh = h0 + r / nrows, row = r0 + r % nrows;
+        const T *p = a.decode ? Q + ((size_t)b * s.Hq + hh) * d : Q + (((size_t)b * s.Hq + hh) * s.N + row) * d;
+        float f[EPV];
+        load16(p + cv * EPV, f);
+#pragma unroll
+        for (int i = 0; i < EPV; ++i) acc[i] += f[i];
+    }
+#pragma unroll
+    for (int i = 0; i < EPV; ++i) red[rg * d + cv * EPV + i] = acc[i];
+    __syncthreads();
+    if (threadIdx.x < d) {
+        float t = 0.f;
+        for (int g = 0; g < NG; ++g) t += red[g * d + threadIdx.x];
+        sm.qbar[threadIdx.x] = t / (float)R;
+    }
+    __syncthreads();
+}
+
+// Score of landmark row `blk` for the VPR-lane group this lane belongs to.
+template <typename T, int VPR>
+__device__ __forceinline__ float group_score(const T *Lrow, const float *qv, float scale) {
+    constexpr int EPV = Vec<T>::n;
+    const int cv = (threadIdx.x & 31) % VPR;
+    float f[EPV];
+    load16(Lrow + cv * EPV, f);
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPV; ++i) dot = fmaf(qv[i], f[i], dot);
+#pragma unroll
+    for (int o = VPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    return scale * dot;
+}
+
+// Exact top-`k` of keys[0..n) (n > k): returns threshold key T and the number
+// of keys equal to T that are taken (the lowest positions first).
+__device__ void radix_select(const uint32_t *keys, int n, int k, SelSmem &sm, uint32_t &T, int &take_eq) {
+    uint32_t prefix = 0, mask = 0;
+    int remaining = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        sm.hist[threadIdx.x] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += kSelThreads) {
+            const uint32_t x = keys[i];
+            if ((x & mask) == prefix) atomicAdd(&sm.hist[(x >> shift) & 255], 1);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            const int hi = 255 - 8 * lane;
+            int local = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) local += sm.hist[hi - q];
+            int incl = local;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const int excl = incl - local;
+            if (excl < remaining && remaining <= incl) {
+                int cum = excl;
+                for (int q = 0; q < 8; ++q) {
+                    const int c = sm.hist[hi - q];
+                    if (cum + c >= remaining) {
+                        sm.sel_digit = hi - q;
+                        sm.sel_above = cum;
+                        break;
+                    }
+                    cum += c;
+                }
+            }
+        }
+        __syncthreads();
+        remaining -= sm.sel_above;
+        prefix |= (uint32_t)sm.sel_digit << shift;
+        mask |= 255u << shift;
+        __syncthreads();
+    }
+    T = prefix;
+    take_eq = remaining;
+}
+
+// Marks the top-k of keys[0..n) and writes their positions, ascending, to
+// out_pos[0..min(n,k)).  Returns the number written.
+__device__ int topk_positions(const uint32_t *keys, int n, int k, SelSmem &sm, int *out_pos) {
+    if (k <= 0 || n <= 0) return 0;
+    if (n <= k) {
+        for (int i = threadIdx.x; i < n; i += kSelThreads) out_pos[i] = i;
+        __syncthreads();
+        return n;
+    }
+    uint32_t T;
+    int take_eq;
+    radix_select(keys, n, k, sm, T, take_eq);
+    const int seg = (n + kSelThreads - 1) / kSelThreads;
+    const int i0 = min(n, threadIdx.x * seg), i1 = min(n, i0 + seg);
+    int neq = 0;
+    for (int i = i0; i < i1; ++i) neq += keys[i] == T;
+    int eq_base = block_scan_incl(neq, sm.tmp, nullptr) - neq;
+    int nsel = 0;
+    {
+        int e = eq_base;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t x = keys[i];
+            const bool take = x > T || (x == T && e < take_eq);
+            e += x == T;
+            nsel += take;
+        }
+    }
+    int total;
+    int pos = block_scan_incl(nsel, sm.tmp, &total) - nsel;
+    {
+        int e = eq_base;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t x = keys[i];
+            const bool take = x > T || (x == T && e < take_eq);
+            e += x == T;
+            if (take) out_pos[pos++] = i;
+        }
+    }
+    __syncthreads();
+    return total;
+}
+
+// Writes the final kept list of a unit: [0 (sink)] + selected (ascending) +
+// [local].  sel_idx/sel_score hold `nsel` selected blocks in ascending order.
+__device__ void write_final(const SelArgs &a, int u, int local, const int *sel_idx, const float *sel_score,
+                            int nsel, float s0, float slocal) {
+    const Shape &s = a.s;
+    int32_t *idx = a.idx + (size_t)u * s.cap;
+    float *sc = a.score + (size_t)u * s.cap;
+    const bool sink = s.flags & SA_SINK;
+    const bool loc = (s.flags & SA_LOCAL) && !(sink && local == 0);
+    const int off = sink ? 1 : 0;
+    const int cnt = off + nsel + (loc ? 1 : 0);
+    for (int i = threadIdx.x; i < s.cap; i += kSelThreads) {
+        int bi = -1;
+        float sv = 0.f;
+        if (i < cnt) {
+            if (sink && i == 0) { bi = 0; sv = s0; }
+            else if (loc && i == cnt - 1) { bi = local; sv = slocal; }
+            else { bi = sel_idx[i - off]; sv = sel_score[i - off]; }
+        }
+        idx[i] = bi;
+        sc[i] = sv;
+    }
+    if (threadIdx.x == 0) a.count[u] = cnt;
+}
+
+template <typename T, int VPR>
+__global__ void __launch_bounds__(kSelThreads) select_chunk_kernel(SelArgs a) {
+    constexpr int EPV = Vec<T>::n;
+    constexpr int NG = kSelThreads / VPR;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + sizeof(SelSmem));
+    int *pos = reinterpret_cast<int *>(keys + a.CH);
+    float *red = reinterpret_cast<float *>(pos + a.CH);
+
+    const Shape &s = a.s;
+    const int d = VPR * EPV;
+    const int u = blockIdx.x / a.S, chunk = blockIdx.x % a.S;
+    int b, hs, j, local;
+    unit_coords(a, u, b, hs, j, local);
+    const int g = (s.flags & SA_SELECT_PER_QHEAD) ? hs / s.G : hs;
+    const int first = (s.flags & SA_SINK) ? 1 : 0;
+    const int c0 = first + chunk * a.CH;
+    const int c1 = min(local, c0 + a.CH);
+    const int n = max(0, c1 - c0);
+
+    pool_query<T, VPR>(a, b, hs, j, sm, red);
+    float qv[EPV];
+    {
+        const int cv = (threadIdx.x & 31) % VPR;
+#pragma unroll
+        for (int i = 0; i < EPV; ++i) qv[i] = sm.qbar[cv * EPV + i];
+    }
+    const T *Lg = (const T *)a.L + ((size_t)b * s.Hkv + g) * s.nb * d;
+    // rows are handed out per warp so that every lane of a warp takes the
+    // same trip count (the group reduction shuffles over the full warp)
+    constexpr int RPW = 32 / VPR;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / VPR, cv = lane % VPR;
+    bool nan_seen = false;
+    for (int base = warp * RPW; base < n; base += NG) {
+        const int r = base + sub;
+        const float sc = group_score<T, VPR>(Lg + (size_t)(c0 + min(r, n - 1)) * d, qv, s.scale);
+        if (cv == 0 && r < n) {
+            nan_seen |= isnan(sc);
+            keys[r] = ord_key(sc);
+        }
+    }
+    if (chunk == 0 && warp == 0) {
+        const int blk = sub == 0 ? 0 : local;   // groups 0 and 1: sink and local scores
+        const float sc = group_score<T, VPR>(Lg + (size_t)blk * d, qv, s.scale);
+        if (cv == 0 && sub < 2) {
+            sm.s_special[sub] = sc;
+            nan_seen |= isnan(sc);
+        }
+    }
+    if (nan_seen) set_status(a.status, kStatusNaN);
+    __syncthreads();
+
+    const int nsel = topk_positions(keys, n, s.top_k, sm, pos);
+    if (a.S == 1) {
+        // reuse the pooling buffer for the ascending selected list
+        int *sel_idx = reinterpret_cast<int *>(red);
+        float *sel_sc = reinterpret_cast<float *>(sel_idx + s.top_k);
+        for (int i = threadIdx.x; i < nsel; i += kSelThreads) {
+            sel_idx[i] = c0 + pos[i];
+            sel_sc[i] = key_to_float(keys[pos[i]]);
+        }
+        __syncthreads();
+        write_final(a, u, local, sel_idx, sel_sc, nsel, sm.s_special[0], sm.s_special[1]);
+    } else {
+        uint32_t *pk = a.part_key + ((size_t)u * a.S + chunk) * s.top_k;
+        int32_t *pi = a.part_idx + ((size_t)u * a.S + chunk) * s.top_k;
+        for (int i = threadIdx.x; i < s.top_k; i += kSelThreads) {
+            pk[i] = i < nsel ? keys[pos[i]] : 0u;
+            pi[i] = i < nsel ? c0 + pos[i] : -1;
+        }
+        if (chunk == 0 && threadIdx.x < 2) a.special[(size_t)u * 2 + threadIdx.x] = sm.s_special[threadIdx.x];
+    }
+}
+
+// Merges the per-chunk top-K lists of one unit (they sit in ascending block
+// order, chunk after chunk) into the unit's final list.
+__global__ void __launch_bounds__(kSelThreads) select_merge_kernel(SelArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
+    const Shape &s = a.s;
+    const int M = a.S * s.top_k;
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + sizeof(SelSmem));
+    int *cidx = reinterpret_cast<int *>(keys + M);
+    int *pos = cidx + M;
+    int *sel_idx = pos + M;
+    float *sel_sc = reinterpret_cast<float *>(sel_idx + s.top_k);
+    const int u = blockIdx.x;
+    int b, hs, j, local;
+    unit_coords(a, u, b, hs, j, local);
+    const int first = (s.flags & SA_SINK) ? 1 : 0;
+    // chunk c holds min(top_k, its candidates) valid entries
+    int ntot = 0;
+    for (int c = 0; c < a.S; ++c) {
+        const int c0 = first + c * a.CH, c1 = min(local, c0 + a.CH);
+        ntot += min(s.top_k, max(0, c1 - c0));
+    }
+    // each chunk's valid prefix, in chunk order
+    int base = 0;
+    for (int c = 0; c < a.S; ++c) {
+        const int c0 = first + c * a.CH, c1 = min(local, c0 + a.CH);
+        const int nv = min(s.top_k, max(0, c1 - c0));
+        const uint32_t *pk = a.part_key + ((size_t)u * a.S + c) * s.top_k;
+        const int32_t *pi = a.part_idx + ((size_t)u * a.S + c) * s.top_k;
+        for (int i = threadIdx.x; i < nv; i += kSelThreads) {
+            keys[base + i] = pk[i];
+            cidx[base + i] = pi[i];
+        }
+        base += nv;
+    }
+    __syncthreads();
+    const int nsel = topk_positions(keys, ntot, s.top_k, sm, pos);
+    for (int i = threadIdx.x; i < nsel; i += kSelThreads) {
+        sel_idx[i] = cidx[pos[i]];
+        sel_sc[i] = key_to_float(keys[pos[i]]);
+    }
+    __syncthreads();
+    write_final(a, u, local, sel_idx, sel_sc, nsel, a.special[(size_t)u * 2], a.special[(size_t)u * 2 + 1]);
+}
+
+static void geometry(const Shape &s, bool decode, int &nunits, int &S, int &CH) {
+    const int ntiles = decode ? 1 : s.nb;
+    nunits = s.B * s.Hsel * ntiles;
+    const int local_max = decode ? (s.N - 1) / s.bs : s.nb - 1;
+    const int first = (s.flags & SA_SINK) ? 1 : 0;
+    const int ncand = max(1, local_max - first);
+    S = 1;
+    if (decode) {
+        // enough CTAs to keep every SM streaming landmarks
+        const int want = (4 * 148 + nunits - 1) / nunits;
+        S = max(1, min(want, (ncand + 511) / 512));
+    }
+    S = max(S, (ncand + kMaxChunk - 1) / kMaxChunk);
+    CH = (ncand + S - 1) / S;
+    if (s.top_k == 0) {   // nothing to rank: only the sink and local scores
+        S = 1;
+        CH = 0;
+    }
+}
+
+size_t select_workspace(const Shape &s, bool decode) {
+    int nunits, S, CH;
+    geometry(s, decode, nunits, S, CH);
+    if (S == 1) return 0;
+    return (size_t)nunits * S * s.top_k * (sizeof(uint32_t) + sizeof(int32_t)) + (size_t)nunits * 2 * sizeof(float) +
+           256;
+}
+
+template <typename T>
+static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L, int32_t *idx, float *score,
+                       int32_t *count, void *ws, cudaStream_t st) {
+    SelArgs a{};
+    a.s = s;
+    a.Q = Q;
+    a.L = L;
+    a.idx = idx;
+    a.score = score;
+    a.count = count;
+    a.status = (unsigned *)ws;
+    a.decode = decode;
+    a.ntiles = decode ? 1 : s.nb;
+    int nunits;
+    geometry(s, decode, nunits, a.S, a.CH);
+    if (a.S > 1) {
+        char *p = (char *)ws + kStatusBytes;
+        a.part_key = (uint32_t *)p;
+        p += (size_t)nunits * a.S * s.top_k * sizeof(uint32_t);
+        a.part_idx = (int32_t *)p;
+        p += (size_t)nunits * a.S * s.top_k * sizeof(int32_t);
+        a.special = (float *)p;
+    }
+    const int vpr = s.d * (int)sizeof(T) / 16;
+    const int d = s.d;
+    size_t red_bytes = (size_t)(kSelThreads / vpr) * d * sizeof(float);
+    red_bytes = max(red_bytes, (size_t)s.top_k * 8);
+    const size_t smem = sizeof(SelSmem) + (size_t)a.CH * 8 + red_bytes;
+    void (*kern)(SelArgs) = nullptr;
+    switch (vpr) {
+        case 8: kern = select_chunk_kernel<T, 8>; break;
+        case 16: kern = select_chunk_kernel<T, 16>; break;
+        case 32: kern = select_chunk_kernel<T, 32>; break;
+        default: return cudaErrorInvalidValue;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)nunits * a.S, kSelThreads, smem, st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.S == 1) return e;
+    const int M = a.S * s.top_k;
+    const size_t msmem = sizeof(SelSmem) + (size_t)M * 12 + (size_t)s.top_k * 8;
+    e = cudaFuncSetAttribute(select_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    if (e != cudaSuccess) return e;
+    select_merge_kernel<<<(unsigned)nunits, kSelThreads, msmem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Shape &s, bool decode, const void *Q, const void *L, int32_t *idx, float *score,
+                          int32_t *count, void *ws, size_t ws_bytes, cudaStream_t st) {
+    (void)ws_bytes;
+    return s.dtype == SA_BF16 ? run<__nv_bfloat16>(s, decode, Q, L, idx, score, count, ws, st)
+                              : run<float>(s, decode, Q, L, idx, score, count, ws, st);
+}
+
+}  // namespace sa

@@ -1,0 +1,179 @@
+/*
+ * sparse_attn.h -- C ABI of the B200 (sm_100a) selector-driven block-sparse
+ * attention library (libsparse_attn.so).
+ *
+ * The method: every query tile (prefill) or decode query scores each earlier
+ * KV block through a landmark (the mean of the block's keys), keeps the top-K
+ * blocks plus the sink block 0 and its own (local) block, and attends only to
+ * the kept blocks.  Pages followed, cited by title and section:
+ *   [SAS]  "Учёные научили трансформеры отбирать контекст напрямую, а не через
+ *          имитацию полного внимания" -- opening section and "Ключевые
+ *          факты": a light selector scores context units (tokens or blocks),
+ *          hard top-K keeps the best; the current block is always kept; the
+ *          selector's continuous score enters the attention logits inside the
+ *          softmax in log form, normalised against the current block; the
+ *          kernel runs FlashAttention-style, blockwise, without the square
+ *          matrix.
+ *   [HiLS] "HiLS-Attention: иерархическое разреженное внимание для
+ *          сверхдлинного контекста в языковых моделях" -- opening section:
+ *          each query reads every selected chunk on its own and the per-chunk
+ *          results are combined with weights given by the retrieval scores.
+ *   [LSA]  Latent Sparse Attention post (rit.work), section "Индекс перестаёт
+ *          перебирать весь контекст": adjacent keys are pooled before
+ *          scoring; the start of the context and a recent window are always
+ *          added.
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned, dense
+ *     row-major with the layouts given below; the caller owns every buffer.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  Host-side argument errors return
+ *     before anything is launched.
+ *   - Return value: SA_OK (0) or a negative SA_ERR_* code.  No exception and
+ *     no allocation crosses the ABI; the library keeps no global state
+ *     besides CUDA's own per-device kernel images and tensor-map caches.
+ *   - Device-side problems (an index list entry out of range, a NaN score, a
+ *     bounded wait that expired) never trap: the kernel skips the bad item
+ *     and records a code in the workspace's status word, which
+ *     sparse_attn_check_status() returns and clears.
+ *   - Layouts.  Q, O: [B, Hq, N, d]; K, V: [B, Hkv, N, d]; landmarks L:
+ *     [B, Hkv, nb, d] with nb = ceil(N / block); decode query q and output o:
+ *     [B, Hq, d]; LSE: [B, Hq, N] (prefill) or [B, Hq] (decode), fp32.
+ *     Query tile j = rows [j*block, (j+1)*block) and aligns with KV block j.
+ *     q-head h reads kv-head h / (Hq / Hkv).
+ *   - Selection lists, one per unit.  A unit is (batch, kv-head, query tile)
+ *     for prefill and (batch, kv-head) for decode -- with
+ *     SA_SELECT_PER_QHEAD, (batch, q-head, ...) instead.  Per unit:
+ *       idx   int32 [top_k + 2]  kept blocks, ascending, padded with -1
+ *       score fp32  [top_k + 2]  retrieval score s_b of each kept block,
+ *                                s_b = scale * <pooled query, L_b>, padded 0
+ *       count int32              number of kept blocks
+ *     so idx/score are [B, Hsel, ntiles, top_k + 2] (prefill) or
+ *     [B, Hsel, top_k + 2] (decode), count [B, Hsel, ntiles] or [B, Hsel],
+ *     where Hsel = Hkv (Hq with SA_SELECT_PER_QHEAD) and ntiles = nb.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* flags */
+enum {
+    SA_SINK = 1,              /* block 0 always kept [LSA]                         */
+    SA_LOCAL = 2,             /* the unit's own block always kept [SAS]            */
+    SA_GATE = 4,              /* log_sigmoid(s_b - s_local) added to the logits of
+                                 every selected (not forced) block [SAS]; needs
+                                 SA_LOCAL, excludes SA_HIER                        */
+    SA_HIER = 8,              /* hierarchical mode [HiLS]: per-block softmax,
+                                 outputs combined by softmax_b(s_b); lse returned
+                                 = logsumexp_b(s_b)                                */
+    SA_CAUSAL = 16,           /* inside the local block key t is visible from
+                                 query i only when t <= i                          */
+    SA_SELECT_PER_QHEAD = 32  /* one list per q-head instead of per kv-head        */
+};
+
+/* dtypes of Q/K/V/L/O */
+enum { SA_BF16 = 0, SA_FP32 = 1 };
+
+/* operations, for sparse_attn_workspace_size */
+enum {
+    SA_OP_LANDMARKS = 0,
+    SA_OP_SELECT = 1,         /* prefill selection                                 */
+    SA_OP_SELECT_DECODE = 2,
+    SA_OP_PREFILL = 3,
+    SA_OP_DECODE = 4
+};
+
+/* return codes */
+enum {
+    SA_OK = 0,
+    SA_ERR_ARG = -1,          /* null pointer, bad shape, misaligned pointer       */
+    SA_ERR_UNSUPPORTED = -2,  /* valid but unsupported combination                 */
+    SA_ERR_WORKSPACE = -3,    /* workspace missing or smaller than required        */
+    SA_ERR_LAUNCH = -4,       /* a CUDA launch failed                              */
+    SA_ERR_DEVICE = -5        /* the status word reports a device-side problem     */
+};
+
+typedef struct {
+    int B;        /* batch (independent sequences)                                 */
+    int Hq;       /* query heads                                                   */
+    int Hkv;      /* key/value heads; Hq % Hkv == 0                                */
+    int d;        /* head dim: 64 or 128 (bf16 prefill fast path: 128)             */
+    int N;        /* prefill: sequence length; decode: context length including
+                     the query's own key (the query sits at position N - 1)        */
+    int block;    /* block size in keys = query tile size: 16..128, multiple of 16 */
+    int top_k;    /* budget of selected blocks, 0..256                             */
+    int flags;    /* SA_* flags above                                              */
+    int dtype;    /* SA_BF16 or SA_FP32                                            */
+    float scale;  /* logit scale; 0 selects 1/sqrt(d)                              */
+} sa_params;
+
+/* Bytes of workspace `op` needs (at least 256: the first 16 bytes hold the
+ * status word).  The workspace must be zero-filled once when allocated; the
+ * library leaves the status word zero unless a device-side problem occurs.  */
+size_t sparse_attn_workspace_size(const sa_params *p, int op);
+
+/* Landmarks (first step of the path; [HiLS] landmark, [LSA] keys pooled
+ * before scoring): L[b,g,k,:] = mean of K[b,g,t,:] over the keys t of block k that
+ * exist (t < N), summed in fp32, stored in the KV dtype rounded to nearest
+ * even.  K [B,Hkv,N,d] -> L [B,Hkv,nb,d]. */
+int sparse_attn_landmarks(const sa_params *p, const void *K, void *L, void *stream);
+
+/* Prefill selection ([SAS] hard top-K over block scores; [LSA] start of
+ * context always added; [SAS] current block always kept).  For tile j of a
+ * unit: pooled query = mean of Q over the unit's query heads and the tile's
+ * rows; s_b = scale * <pooled, L_b> for b <= j; candidates = blocks before j
+ * (block 0 excluded with SA_SINK); the top_k candidates by (s desc, index
+ * asc, decided on fp32 scores) are kept together with block 0 (SA_SINK) and
+ * block j (SA_LOCAL).  Q [B,Hq,N,d], L [B,Hkv,nb,d] -> idx, score, count.
+ * A NaN score is ranked lowest and flagged in the status word. */
+int sparse_attn_select(const sa_params *p, const void *Q, const void *L, int32_t *idx, float *score,
+                       int32_t *count, void *ws, size_t ws_bytes, void *stream);
+
+/* Decode selection: as sparse_attn_select for the one query per sequence at
+ * position N-1; its local block is (N-1)/block.  q [B,Hq,d] -> idx, score,
+ * count of shape [B,Hsel,top_k+2] / [B,Hsel]. */
+int sparse_attn_select_decode(const sa_params *p, const void *q, const void *L, int32_t *idx, float *score,
+                              int32_t *count, void *ws, size_t ws_bytes, void *stream);
+
+/* Block-sparse prefill over the kept lists ([SAS] FlashAttention-style,
+ * blockwise, online softmax).  Gated mode: z_t = scale * <q_i, k_t> + gate_b
+ * for keys t of kept blocks (t <= i inside the local block when causal),
+ * gate_b = log_sigmoid(s_b - s_local) on selected blocks (SA_GATE), 0 on the
+ * sink and local blocks; O_i = softmax(z) V, LSE_i = log sum exp z.
+ * Hierarchical mode (SA_HIER): per-block softmax outputs combined with
+ * weights softmax_b(s_b).  An empty list gives O = 0, LSE = -inf.
+ * Q,K,V + idx/score/count (as written by sparse_attn_select) -> O, LSE. */
+int sparse_attn_prefill(const sa_params *p, const void *Q, const void *K, const void *V, const int32_t *idx,
+                        const float *score, const int32_t *count, void *O, float *lse, void *ws,
+                        size_t ws_bytes, void *stream);
+
+/* Block-sparse decode: the same attention for one query per sequence at
+ * position N-1 over the cache K, V [B,Hkv,N,d] (it already holds the query's
+ * own key/value); split over the kept blocks, partials merged by
+ * log-sum-exp.  q [B,Hq,d] + decode lists -> o [B,Hq,d], lse [B,Hq]. */
+int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
+                       const float *score, const int32_t *count, void *o, float *lse, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, returns SA_OK or SA_ERR_DEVICE from the status
+ * word in `ws`, and clears it.  *detail (may be NULL) receives the raw bits:
+ * 1 index list entry out of range, 2 NaN score, 4 bounded wait expired. */
+int sparse_attn_check_status(void *ws, void *stream, int *detail);
+
+/* Static string for a return code. */
+const char *sparse_attn_status_string(int code);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int sparse_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

@@ -1,0 +1,93 @@
+"""The C-ABI library loads without a GPU, exports every symbol the public
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_long_landmark_b200 as sa
+from block_sparse_long_landmark_b200 import build as sabuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    sabuild.build()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(sparse_attn_\w+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert {"sparse_attn_select", "sparse_attn_prefill", "sparse_attn_decode", "sparse_attn_landmarks"} <= names
+    lib = ctypes.CDLL(sa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(sa.EXPORTS) >= names
+
+
+def test_version_and_strings():
+    assert sa.sparse_attn_version() >= 100
+    for code in (0, -1, -2, -3, -4, -5):
+        assert isinstance(sa.sparse_attn_status_string(code), str)
+
+
+def _p(**kw):
+    base = dict(B=1, Hq=8, Hkv=2, d=128, N=4096, block=64, top_k=16,
+                flags=sa.SA_SINK | sa.SA_LOCAL | sa.SA_GATE | sa.SA_CAUSAL, dtype="bf16")
+    base.update(kw)
+    return sa.make_params(**base)
+
+
+def test_workspace_size_host_only():
+    p = _p()
+    for op in range(5):
+        n = sa.sparse_attn_workspace_size(p, op)
+        assert n >= 256 and n % 256 == 0
+    pd = _p(B=8, N=1 << 20, top_k=64, flags=sa.SA_SINK | sa.SA_LOCAL | sa.SA_HIER | sa.SA_CAUSAL)
+    assert sa.sparse_attn_workspace_size(pd, sa.SA_OP_DECODE) > 256
+    assert sa.sparse_attn_workspace_size(pd, sa.SA_OP_SELECT_DECODE) > 256
+    assert sa.sparse_attn_workspace_size(_p(Hq=7), 0) == 0       # invalid: no size
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=7), sa.SA_ERR_ARG),
+    (dict(N=0), sa.SA_ERR_ARG),
+    (dict(top_k=-1), sa.SA_ERR_ARG),
+    (dict(top_k=1000), sa.SA_ERR_ARG),
+    (dict(flags=1 << 10), sa.SA_ERR_ARG),
+    (dict(dtype=7), sa.SA_ERR_ARG),
+    (dict(d=96), sa.SA_ERR_UNSUPPORTED),
+    (dict(block=48 + 1), sa.SA_ERR_UNSUPPORTED),
+    (dict(flags=sa.SA_GATE | sa.SA_HIER | sa.SA_LOCAL), sa.SA_ERR_UNSUPPORTED),
+    (dict(flags=sa.SA_GATE | sa.SA_SINK), sa.SA_ERR_UNSUPPORTED),
+])
+def test_bad_params_rejected_before_launch(kw, code):
+    p = _p(**kw)
+    fake = 256   # 16-byte aligned, never dereferenced: the checks fail first
+    assert sa.sparse_attn_landmarks(p, fake, fake, None) == code
+    assert sa.sparse_attn_select(p, fake, fake, fake, fake, fake, fake, 1 << 20, None) == code
+    assert sa.sparse_attn_prefill(p, fake, fake, fake, fake, fake, fake, fake, fake, fake, 1 << 20, None) == code
+    assert sa.sparse_attn_decode(p, fake, fake, fake, fake, fake, fake, fake, fake, fake, 1 << 20, None) == code
+
+
+def test_null_misaligned_and_small_workspace_rejected():
+    p = _p()
+    a = 256
+    assert sa.sparse_attn_landmarks(p, None, a, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_landmarks(p, a + 8, a, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_select(p, a, a, a, a, a, None, 1 << 20, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_select(p, a, a, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.sparse_attn_prefill(p, a, a, a, a, a, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.sparse_attn_decode(p, a, a, a, a, a, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.sparse_attn_check_status(None, None)[0] == sa.SA_ERR_ARG

@@ -1,0 +1,236 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against
+the CPU oracle on the same seeded inputs (small and ragged problems here;
+full-size sampled checks live in test_gpu_fullsize.py)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_landmark_b200 as sa
+import oracle
+from block_sparse_long_landmark_b200 import inputs
+from _util import (GAP, LSE_TOL, O_TOL, compare_lists, f64, oracle_sel_tensors, round_mode, run_decode,
+                   run_prefill)
+
+pytestmark = pytest.mark.gpu
+
+W = inputs.WORKLOADS
+
+PREFILL_CASES = {
+    "tiny_fp32": W["tiny_fp32_prefill"],
+    "tiny_fp32_ragged": W["tiny_fp32_prefill"].scaled(N=1000),
+    "gqa_bf16_4k": W["gated_prefill_32k"].scaled(N=4096),
+    "gqa_bf16_ragged": W["gated_prefill_32k"].scaled(N=2000, Hq=8, Hkv=2),
+    "gqa_bf16_block128": W["long_prefill_256k"].scaled(N=8192, Hq=8, Hkv=2),
+    "fp32_d128_gqa": W["gated_prefill_32k"].scaled(N=1536, Hq=4, Hkv=2, dtype="fp32", sigma=1.0),
+}
+
+
+def _prefill_inputs(wl):
+    Q, K, V = inputs.make_prefill(wl, device="cuda")
+    return Q, K, V
+
+
+def _oracle_prefill(wl, Q, K, V, flags=None, top_k=None, sel_override=None):
+    return oracle.prefill(f64(Q), f64(K), f64(V), wl.block, wl.top_k if top_k is None else top_k,
+                          wl.flags if flags is None else flags, round_mode=round_mode(wl.dtype),
+                          sel_override=sel_override)
+
+
+def _check_outputs(wl, ref, O, lse, row_mask=None):
+    Og, lg = f64(O), f64(lse)
+    Or, lr = ref["O"], ref["LSE"]
+    if row_mask is not None:
+        Og, lg, Or, lr = Og[row_mask], lg[row_mask], Or[row_mask], lr[row_mask]
+    err = np.abs(Og - Or).max() if Og.size else 0.0
+    assert err <= O_TOL[wl.dtype], f"max |O - O_ref| = {err}"
+    fin = np.isfinite(lr)
+    assert np.array_equal(fin, np.isfinite(lg))
+    lerr = np.abs(lg[fin] - lr[fin]).max() if fin.any() else 0.0
+    assert lerr <= LSE_TOL, f"max |lse - lse_ref| = {lerr}"
+    return err, lerr
+
+
+@pytest.mark.parametrize("case", sorted(PREFILL_CASES))
+def test_landmarks(case):
+    wl = PREFILL_CASES[case]
+    p = sa.params_for(wl)
+    _, K, _ = _prefill_inputs(wl)
+    L = f64(sa.landmarks(p, K))
+    Kh = f64(K)
+    for b in range(wl.B):
+        for g in range(wl.Hkv):
+            ref = oracle.landmarks(Kh[b, g], wl.block, round_mode(wl.dtype))
+            if wl.dtype == "fp32":
+                assert np.abs(L[b, g] - ref).max() <= 1e-6
+            else:
+                # fp32 sum vs exact mean: at most one bf16 step apart, and rarely
+                ulp = np.maximum(np.abs(ref), 1e-30) * 2.0 ** -7
+                diff = np.abs(L[b, g] - ref)
+                assert np.all(diff <= ulp)
+                assert np.mean(diff > 0) < 1e-3
+
+
+@pytest.mark.parametrize("case", sorted(PREFILL_CASES))
+def test_prefill_end_to_end(case):
+    wl = PREFILL_CASES[case]
+    p = sa.params_for(wl)
+    Q, K, V = _prefill_inputs(wl)
+    L, (idx, sc, cnt), O, lse = run_prefill(p, Q, K, V)
+    ref = _oracle_prefill(wl, Q, K, V)
+    n, exact, mask = compare_lists(ref, idx, sc, cnt)
+    assert exact >= 0.9 * n
+    # rows of units whose lists agree: element-wise comparison
+    G = wl.Hq // wl.Hkv
+    rows = np.zeros((wl.B, wl.Hq, wl.N), dtype=bool)
+    for b, g, j in zip(*np.nonzero(mask)):
+        rows[b, g * G:(g + 1) * G, j * wl.block:(j + 1) * wl.block] = True
+    _check_outputs(wl, ref, O, lse, rows)
+
+
+@pytest.mark.parametrize("case", sorted(PREFILL_CASES))
+def test_prefill_on_oracle_lists(case):
+    """The attention step alone: GPU prefill fed with the oracle's lists."""
+    wl = PREFILL_CASES[case]
+    p = sa.params_for(wl)
+    Q, K, V = _prefill_inputs(wl)
+    ref = _oracle_prefill(wl, Q, K, V)
+    _, _, O, lse = run_prefill(p, Q, K, V, sel=oracle_sel_tensors(ref))
+    _check_outputs(wl, ref, O, lse)
+
+
+FLAG_CASES = [
+    ("no_sink", inputs.F_LOCAL | inputs.F_GATE | inputs.F_CAUSAL, 4),
+    ("no_gate", inputs.F_SINK | inputs.F_LOCAL | inputs.F_CAUSAL, 4),
+    ("keep_all", inputs.F_SINK | inputs.F_LOCAL | inputs.F_CAUSAL, 64),
+    ("top0", inputs.F_SINK | inputs.F_LOCAL | inputs.F_GATE | inputs.F_CAUSAL, 0),
+    ("empty_tile0", inputs.F_CAUSAL, 3),
+    ("sink_only", inputs.F_SINK | inputs.F_CAUSAL, 2),
+    ("not_causal", inputs.F_SINK | inputs.F_LOCAL | inputs.F_GATE, 3),
+    ("hier", inputs.F_SINK | inputs.F_LOCAL | inputs.F_HIER | inputs.F_CAUSAL, 3),
+    ("per_qhead", inputs.F_SINK | inputs.F_LOCAL | inputs.F_GATE | inputs.F_CAUSAL | inputs.F_PER_QHEAD, 3),
+]
+
+
+@pytest.mark.parametrize("name,flags,top_k", FLAG_CASES)
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_prefill_flags(name, flags, top_k, dtype):
+    wl = W["gated_prefill_32k"].scaled(N=1000, Hq=4, Hkv=2, block=64, top_k=top_k, dtype=dtype, n_plants=2)
+    p = sa.params_for(wl, flags=flags)
+    Q, K, V = _prefill_inputs(wl)
+    L, (idx, sc, cnt), O, lse = run_prefill(p, Q, K, V)
+    ref = _oracle_prefill(wl, Q, K, V, flags=flags)
+    n, exact, mask = compare_lists(ref, idx, sc, cnt)
+    per_q = bool(flags & inputs.F_PER_QHEAD)
+    G = wl.Hq // wl.Hkv
+    rows = np.zeros((wl.B, wl.Hq, wl.N), dtype=bool)
+    for b, s_, j in zip(*np.nonzero(mask)):
+        hs = slice(s_, s_ + 1) if per_q else slice(s_ * G, (s_ + 1) * G)
+        rows[b, hs, j * wl.block:(j + 1) * wl.block] = True
+    _check_outputs(wl, ref, O, lse, rows)
+    if name == "empty_tile0":
+        assert np.all(f64(O)[:, :, :wl.block] == 0) and np.all(np.isneginf(f64(lse)[:, :, :wl.block]))
+
+
+DECODE_CASES = {
+    "gated_8k": W["gated_decode_128k"].scaled(B=4, N=8192),
+    "gated_ragged": W["gated_decode_128k"].scaled(B=3, N=5000, top_k=8, n_plants=4),
+    "hier_16k": W["hils_decode_1m"].scaled(B=2, N=16384, top_k=16, n_plants=16),
+    "hier_ragged": W["hils_decode_1m"].scaled(B=2, N=3001, top_k=5, n_plants=3),
+    "gated_fp32_d64": W["gated_decode_128k"].scaled(B=2, N=4096, d=64, dtype="fp32", Hq=8, Hkv=8, top_k=6,
+                                                    n_plants=3, sigma=1.0),
+    "gated_big_k": W["gated_decode_128k"].scaled(B=2, N=65536, top_k=200, n_plants=16),
+}
+
+
+def _oracle_decode(wl, q, K, V, flags=None, sel_override=None):
+    return oracle.decode(f64(q), f64(K), f64(V), wl.block, wl.top_k, wl.flags if flags is None else flags,
+                         round_mode=round_mode(wl.dtype), sel_override=sel_override)
+
+
+@pytest.mark.parametrize("case", sorted(DECODE_CASES))
+def test_decode_end_to_end(case):
+    wl = DECODE_CASES[case]
+    p = sa.params_for(wl)
+    q, K, V = inputs.make_decode(wl, device="cuda")
+    L, (idx, sc, cnt), o, lse = run_decode(p, q, K, V)
+    ref = _oracle_decode(wl, q, K, V)
+    n, exact, mask = compare_lists(ref, idx, sc, cnt)
+    G = wl.Hq // wl.Hkv
+    rows = np.repeat(mask, G, axis=1)
+    _check_outputs(wl, ref, o, lse, rows)
+    assert exact >= 0.5 * n
+
+
+@pytest.mark.parametrize("case", sorted(DECODE_CASES))
+def test_decode_on_oracle_lists(case):
+    wl = DECODE_CASES[case]
+    p = sa.params_for(wl)
+    q, K, V = inputs.make_decode(wl, device="cuda")
+    ref = _oracle_decode(wl, q, K, V)
+    _, _, o, lse = run_decode(p, q, K, V, sel=oracle_sel_tensors(ref))
+    _check_outputs(wl, ref, o, lse)
+
+
+@pytest.mark.parametrize("flags", [inputs.F_SINK | inputs.F_LOCAL | inputs.F_CAUSAL,
+                                   inputs.F_LOCAL | inputs.F_GATE | inputs.F_CAUSAL,
+                                   inputs.F_SINK | inputs.F_LOCAL | inputs.F_GATE | inputs.F_PER_QHEAD,
+                                   inputs.F_SINK | inputs.F_HIER | inputs.F_PER_QHEAD])
+def test_decode_flags(flags):
+    wl = W["gated_decode_128k"].scaled(B=2, N=3000, top_k=5, n_plants=3)
+    p = sa.params_for(wl, flags=flags)
+    q, K, V = inputs.make_decode(wl, device="cuda")
+    _, (idx, sc, cnt), o, lse = run_decode(p, q, K, V)
+    ref = _oracle_decode(wl, q, K, V, flags=flags)
+    n, exact, mask = compare_lists(ref, idx, sc, cnt)
+    G = 1 if flags & inputs.F_PER_QHEAD else wl.Hq // wl.Hkv
+    _check_outputs(wl, ref, o, lse, np.repeat(mask, G, axis=1))
+
+
+def test_selection_is_deterministic():
+    wl = W["gated_prefill_32k"].scaled(N=4096)
+    p = sa.params_for(wl)
+    Q, K, _ = _prefill_inputs(wl)
+    ws = sa.workspace(p)
+    L = sa.landmarks(p, K)
+    a = [t.clone() for t in sa.select(p, Q, L, ws)]
+    b = sa.select(p, Q, L, ws)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    wd = W["hils_decode_1m"].scaled(B=2, N=65536)
+    pd = sa.params_for(wd)
+    q, Kd, _ = inputs.make_decode(wd, device="cuda")
+    wsd = sa.workspace(pd)
+    Ld = sa.landmarks(pd, Kd)
+    a = [t.clone() for t in sa.select_decode(pd, q, Ld, wsd)]
+    b = sa.select_decode(pd, q, Ld, wsd)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_bad_list_entry_sets_status_and_is_skipped():
+    wl = W["gated_prefill_32k"].scaled(N=1024, Hq=4, Hkv=2)
+    p = sa.params_for(wl)
+    Q, K, V = _prefill_inputs(wl)
+    ws = sa.workspace(p)
+    L = sa.landmarks(p, K)
+    idx, sc, cnt = sa.select(p, Q, L, ws)
+    idx[0, 0, 5, 1] = 10_000          # beyond the tile's own block
+    sa.prefill(p, Q, K, V, idx, sc, cnt, ws)
+    with pytest.raises(sa.SparseAttnError) as ei:
+        sa.check_status(ws)
+    assert ei.value.code == sa.SA_ERR_DEVICE
+    assert sa.check_status(ws) == 0   # cleared
+
+
+def test_nan_score_sets_status():
+    wl = W["gated_prefill_32k"].scaled(N=1024, Hq=4, Hkv=2)
+    p = sa.params_for(wl)
+    Q, K, V = _prefill_inputs(wl)
+    Q[0, 0, 300, 5] = float("nan")
+    ws = sa.workspace(p)
+    L = sa.landmarks(p, K)
+    sa.select(p, Q, L, ws)
+    rc, detail = sa.sparse_attn_check_status(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == sa.SA_ERR_DEVICE and detail & 2
