@@ -266,11 +266,11 @@ __global__ void __launch_bounds__(kSelThreads) select_chunk_kernel(SelArgs a) {
             keys[r] = ord_key(sc);
         }
     }
-    if (chunk == 0 && warp == 0) {
-        const int blk = sub == 0 ? 0 : local;   // groups 0 and 1: sink and local scores
+    if (chunk == 0 && warp < 2) {
+        const int blk = warp == 0 ? 0 : local;   // warp 0: sink score, warp 1: local score
         const float sc = group_score<T, VPR>(Lg + (size_t)blk * d, qv, s.scale);
-        if (cv == 0 && sub < 2) {
-            sm.s_special[sub] = sc;
+        if (lane == 0) {
+            sm.s_special[warp] = sc;
             nan_seen |= isnan(sc);
         }
     }
