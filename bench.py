@@ -1,0 +1,546 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse landmark attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-secondary]
+
+One step of the headline workload (gated_prefill_32k: B1, Hq 32, Hkv 8, d 128,
+N 32768, block 64, top-16 + sink + local, bf16) is one pass of the prefill
+path through the C ABI: landmarks -> selection -> gated block-sparse prefill.
+``value`` = prefill tokens/s over all ranks (each rank runs its own seeded
+sequence: weak scaling, no collective on the data path).  The same JSON line
+carries the decode workloads (gated_decode_128k: 64 sequences at 128K context;
+hils_decode_1m: hierarchical, 8 sequences at 1M context) and the 256K prefill
+under ``secondary`` at N = 1, each with its own roofline.
+
+Timing: CUDA events on the launching stream around each step and each C call,
+W warm-up steps, K timed steps bracketed by barrier + synchronize, L2 flushed
+(a 256 MiB write) before every timed step, max over ranks.  ``--impl
+reference`` times the CPU oracle (a deliberately slow, plain C reference) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse prefill tokens/s and decode queries/s at 128K ctx; % of TC/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------
+# ranks
+# ----------------------------------------------------------------------------
+
+class Ranks:
+    def __init__(self, backend="nccl"):
+        import torch.distributed as dist
+        self.dist = dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        if self.world > 1 and not dist.is_initialized():
+            import datetime
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+    @classmethod
+    def single(cls):
+        r = cls.__new__(cls)
+        r.world, r.rank, r.local, r.backend, r.dist = 1, 0, 0, "none", None
+        return r
+
+    def barrier(self):
+        if self.world > 1:
+            if self.backend == "nccl":
+                self.dist.barrier(device_ids=[self.local])
+            else:
+                self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.world == 1:
+            return float(x)
+        dev = torch.device("cuda", self.local) if self.backend == "nccl" else torch.device("cpu")
+        t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float) -> float:
+        if self.world == 1:
+            return float(x)
+        dev = torch.device("cuda", self.local) if self.backend == "nccl" else torch.device("cpu")
+        t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1 and self.dist.is_initialized():
+            self.dist.destroy_process_group()
+
+
+def aggregate(ranks: Ranks, elapsed_ms: float, units: float) -> tuple[float, float]:
+    """Whole-job throughput: units of all ranks / the slowest rank's time.
+    Returns (value per second, max elapsed ms)."""
+    t = ranks.max(elapsed_ms)
+    u = ranks.sum(units)
+    return (u / (t / 1e3) if t > 0 else 0.0), t
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            sel = ["-i", ("GPU-" + self.uuid) if self.uuid and not self.uuid.startswith("GPU-") else self.uuid] \
+                if self.uuid else []
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8], parts[3]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v.lower() == "active"})
+        loaded = [r[0] for r in rows if r[3] not in ("0", "[N/A]")] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_for(kernel: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if its kernel
+    source is unchanged since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
+        return None
+    return d["dram_bytes_per_launch"]
+
+
+class Timer:
+    """Per-name CUDA-event timing of calls on the current stream."""
+
+    def __init__(self):
+        self.ev = {}
+
+    def __call__(self, name, fn):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        out = fn()
+        e.record()
+        self.ev.setdefault(name, []).append((s, e))
+        return out
+
+    def ms(self):
+        return {k: statistics.fmean(s.elapsed_time(e) for s, e in v) for k, v in self.ev.items()}
+
+
+def flush_l2(buf):
+    buf.fill_(1)
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+
+def prefill_case(wl, device, seed_offset=0):
+    import block_sparse_long_landmark_b200 as sa
+    from block_sparse_long_landmark_b200 import inputs
+    wl = wl.scaled(seed=wl.seed + 1000 * seed_offset) if seed_offset else wl
+    p = sa.params_for(wl)
+    Q, K, V = inputs.make_prefill(wl, device=device)
+    ws = sa.workspace(p, device=device)
+    nb = wl.nb
+    L = torch.empty(wl.B, wl.Hkv, nb, wl.d, dtype=Q.dtype, device=device)
+    sel = sa._sel_out(p, False, device)
+    O = torch.empty_like(Q)
+    lse = torch.empty(wl.B, wl.Hq, wl.N, dtype=torch.float32, device=device)
+    return wl, p, dict(Q=Q, K=K, V=V, ws=ws, L=L, sel=sel, O=O, lse=lse)
+
+
+def prefill_step(p, t, timer=None):
+    import block_sparse_long_landmark_b200 as sa
+    tm = timer or (lambda n, f: f())
+    tm("landmarks", lambda: sa.landmarks(p, t["K"], out=t["L"]))
+    tm("select", lambda: sa.select(p, t["Q"], t["L"], t["ws"], out=t["sel"]))
+    tm("prefill", lambda: sa.prefill(p, t["Q"], t["K"], t["V"], *t["sel"], t["ws"], out=(t["O"], t["lse"])))
+
+
+def prefill_flops(wl, cnt) -> float:
+    """Gathered FLOPs of one prefill launch: QK^T and PV over every kept
+    (tile, block) pair, the local block counted whole: 4 * rows * keys * d."""
+    G = wl.Hq // wl.Hkv
+    pairs = float(cnt.sum().item())
+    return pairs * 4.0 * (G * wl.block) * wl.block * wl.d
+
+
+def decode_case(wl, device):
+    import block_sparse_long_landmark_b200 as sa
+    from block_sparse_long_landmark_b200 import inputs
+    p = sa.params_for(wl)
+    q, K, V = inputs.make_decode(wl, device=device)
+    ws = sa.workspace(p, device=device)
+    L = sa.landmarks(p, K)
+    sel = sa._sel_out(p, True, device)
+    o = torch.empty_like(q)
+    lse = torch.empty(wl.B, wl.Hq, dtype=torch.float32, device=device)
+    return p, dict(q=q, K=K, V=V, ws=ws, L=L, sel=sel, o=o, lse=lse)
+
+
+def decode_step(p, t, timer=None):
+    import block_sparse_long_landmark_b200 as sa
+    tm = timer or (lambda n, f: f())
+    tm("select_decode", lambda: sa.select_decode(p, t["q"], t["L"], t["ws"], out=t["sel"]))
+    tm("decode", lambda: sa.decode(p, t["q"], t["K"], t["V"], *t["sel"], t["ws"], out=(t["o"], t["lse"])))
+
+
+def run_timed(step, steps, warmup, ranks, flush_buf):
+    for _ in range(warmup):
+        step(None)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    import block_sparse_long_landmark_b200 as sa
+    n0 = sa.sparse_attn_launch_count()
+    timer = Timer()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    starts, ends = [], []
+    for _ in range(steps):
+        flush_l2(flush_buf)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        step(timer)
+        e.record()
+        starts.append(s)
+        ends.append(e)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    launches = sa.sparse_attn_launch_count() - n0
+    elapsed = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    return elapsed, timer.ms(), launches, clocks
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and --impl reference)
+# ----------------------------------------------------------------------------
+
+def oracle_prefill_sample(wl, Q64, K64, V64, n_units, seed=0):
+    """Times the oracle on ``n_units`` (batch, kv-head, tile) units drawn from
+    the upper tiles (every one with a full top-K list).  Returns (seconds,
+    token-equivalents, threads)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    lo = min(wl.nb - 1, wl.top_k + 2)
+    units = [(0, int(rng.integers(0, wl.Hkv)), int(rng.integers(lo, wl.nb))) for _ in range(n_units)]
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.prefill(Q64, K64, V64, wl.block, wl.top_k, wl.flags, round_mode=oracle.ROUND_BF16, units=units,
+                   threads=threads)
+    dt = time.perf_counter() - t0
+    return dt, n_units * wl.block / wl.Hkv, threads
+
+
+def cpu_inputs(wl):
+    from block_sparse_long_landmark_b200 import inputs
+    Q, K, V = inputs.make_prefill(wl, device="cpu")
+    return (Q.float().numpy().astype(np.float64), K.float().numpy().astype(np.float64),
+            V.float().numpy().astype(np.float64))
+
+
+def calibrate_units(wl, Q64, K64, V64, target_s):
+    dt, _, _ = oracle_prefill_sample(wl, Q64, K64, V64, 16, seed=99)
+    per = dt / 16
+    return max(16, min(20000, int(target_s / max(per, 1e-6))))
+
+
+def cpu_baseline(wl, target_s):
+    Q64, K64, V64 = cpu_inputs(wl)
+    n = calibrate_units(wl, Q64, K64, V64, target_s)
+    dt, tok, threads = oracle_prefill_sample(wl, Q64, K64, V64, n, seed=1)
+    return {"value": tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} random (kv-head, tile) units of {wl.name} with full top-{wl.top_k} lists "
+                      f"(landmarks of the touched kv-heads, selection and gated attention), "
+                      f"{dt:.1f} s on {threads} host threads; tokens counted as block/Hkv per unit"}
+
+
+def run_reference(args, ranks):
+    from block_sparse_long_landmark_b200 import inputs
+    if ranks.rank != 0:
+        return 0
+    wl = inputs.WORKLOADS[args.workload]
+    Q64, K64, V64 = cpu_inputs(wl)
+    per_step_s = max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
+    n = calibrate_units(wl, Q64, K64, V64, per_step_s)
+    rates, times = [], []
+    threads = os.cpu_count() or 1
+    for i in range(args.warmup + args.steps):
+        dt, tok, threads = oracle_prefill_sample(wl, Q64, K64, V64, n, seed=10 + i)
+        if i >= args.warmup:
+            rates.append(tok / dt)
+            times.append(dt)
+    value = statistics.fmean(rates)
+    sample = (f"each step: {n} random (kv-head, tile) units of {wl.name} on {threads} host threads; "
+              f"tokens counted as block/Hkv per unit")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.fmean(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, extra=None):
+    c = {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "seq_len": wl.N,
+         "block": wl.block, "top_k": wl.top_k, "flags": wl.flags, "mode": "hier" if wl.hier else "gated",
+         "global_batch": wl.B, "parallelism": "replicas (independent sequences per rank)",
+         "l2": "flushed before every timed step (256 MiB write)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ----------------------------------------------------------------------------
+# main arms
+# ----------------------------------------------------------------------------
+
+def e2e_prefill(wl, p, t, steps):
+    """Same metric through the public API with host buffers: pinned H2D of
+    Q, K, V, the three calls, D2H of O and LSE, all inside the events."""
+    hQ = t["Q"].cpu().pin_memory()
+    hK = t["K"].cpu().pin_memory()
+    hV = t["V"].cpu().pin_memory()
+    hO = torch.empty(t["O"].shape, dtype=t["O"].dtype).pin_memory()
+    hL = torch.empty(t["lse"].shape, dtype=torch.float32).pin_memory()
+    times = []
+    for i in range(steps + 1):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        t["Q"].copy_(hQ, non_blocking=True)
+        t["K"].copy_(hK, non_blocking=True)
+        t["V"].copy_(hV, non_blocking=True)
+        prefill_step(p, t)
+        hO.copy_(t["O"], non_blocking=True)
+        hL.copy_(t["lse"], non_blocking=True)
+        e.record()
+        torch.cuda.synchronize()
+        if i:
+            times.append(s.elapsed_time(e))
+    ms = statistics.fmean(times)
+    h2d = sum(x.numel() * x.element_size() for x in (hQ, hK, hV))
+    d2h = hO.numel() * hO.element_size() + hL.numel() * 4
+    return ms, h2d, d2h
+
+
+def secondary_prefill(name, args, pk, psrc):
+    from block_sparse_long_landmark_b200 import inputs
+    wl, p, t = prefill_case(inputs.WORKLOADS[name], "cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ranks1 = Ranks.single()
+    steps = max(2, min(args.steps, 5))
+    el, kms, launches, clocks = run_timed(lambda tm: prefill_step(p, t, tm), steps, max(3, args.warmup),
+                                          ranks1, flush)
+    flops = prefill_flops(wl, t["sel"][2])
+    ach = flops / (kms["prefill"] / 1e3) / 1e12
+    out = {"metric": "prefill tokens/s", "value": wl.N * wl.B / (el / steps / 1e3), "unit": "tokens/s",
+           "ms_per_step": el / steps, "kernels_ms": kms, "config": workload_config(wl), "gpu_launches": launches,
+           "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": ach / pk["bf16_tflops"], "peak_source": psrc + " bf16 burst",
+                        "gathered_flops_per_launch": flops, "traffic": traffic_for("prefill_" + wl.name)},
+           "clocks": clocks}
+    del t
+    torch.cuda.empty_cache()
+    return out
+
+
+def secondary_decode(name, args, pk, psrc):
+    from block_sparse_long_landmark_b200 import inputs
+    wl = inputs.WORKLOADS[name]
+    p, t = decode_case(wl, "cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ranks1 = Ranks.single()
+    steps = max(3, args.steps)
+    el, kms, launches, clocks = run_timed(lambda tm: decode_step(p, t, tm), steps, max(3, args.warmup),
+                                          ranks1, flush)
+    esz = 2 if wl.dtype == "bf16" else 4
+    cnt = t["sel"][2].to(torch.int64)
+    local = (wl.N - 1) // wl.block
+    scan_bytes = wl.B * wl.Hkv * (local + 1) * wl.d * esz
+    gather_bytes = float(cnt.sum().item()) * wl.block * wl.d * esz * 2
+    ach_dec = gather_bytes / (kms["decode"] / 1e3) / 1e9
+    ach_sel = scan_bytes / (kms["select_decode"] / 1e3) / 1e9
+    step_ach = (scan_bytes + gather_bytes) / (el / steps / 1e3) / 1e9
+    hbm = pk["hbm_gbs"]
+    out = {"metric": "decode queries/s", "value": wl.B / (el / steps / 1e3), "unit": "queries/s",
+           "ms_per_step": el / steps, "kernels_ms": kms, "config": workload_config(wl), "gpu_launches": launches,
+           "roofline": {"bound": "hbm", "achieved": step_ach, "peak": hbm, "unit": "GB/s", "frac": step_ach / hbm,
+                        "peak_source": psrc, "bytes_per_step": scan_bytes + gather_bytes,
+                        "traffic": None},
+           "kernels_roofline": {
+               "decode": {"bound": "hbm", "achieved": ach_dec, "peak": hbm, "unit": "GB/s", "frac": ach_dec / hbm,
+                          "algorithmic_bytes": gather_bytes, "traffic": traffic_for("decode_" + name)},
+               "select_decode": {"bound": "hbm", "achieved": ach_sel, "peak": hbm, "unit": "GB/s",
+                                 "frac": ach_sel / hbm, "algorithmic_bytes": scan_bytes,
+                                 "traffic": traffic_for("select_decode_" + name)}},
+           "clocks": clocks}
+    del t
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, ranks):
+    import block_sparse_long_landmark_b200 as sa
+    from block_sparse_long_landmark_b200 import inputs
+    sa.lib()   # fails loudly without the built CUDA library
+    dev = torch.device("cuda", ranks.local)
+    torch.cuda.set_device(dev)
+    pk, psrc = peaks()
+    base = inputs.WORKLOADS[args.workload]
+    wl, p, t = prefill_case(base, "cuda", seed_offset=ranks.rank)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    el, kms, launches, clocks = run_timed(lambda tm: prefill_step(p, t, tm), args.steps, args.warmup, ranks, flush)
+    value, el_max = aggregate(ranks, el, wl.N * wl.B * args.steps)
+    flops = prefill_flops(wl, t["sel"][2])
+    ach = flops / (kms["prefill"] / 1e3) / 1e12
+    e2e_ms, h2d, d2h = e2e_prefill(wl, p, t, min(args.steps, 5))
+    e2e_value, _ = aggregate(ranks, e2e_ms, wl.N * wl.B)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ranks.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": el_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic: seeded Gaussian Q/K/V with planted relevant blocks",
+        "config": workload_config(wl),
+        "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": ach / pk["bf16_tflops"], "traffic": traffic_for("prefill_" + wl.name),
+                     "kernel": "prefill", "peak_source": psrc + " bf16 burst",
+                     "gathered_flops_per_launch": flops},
+        "kernels_ms": kms,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    del t
+    torch.cuda.empty_cache()
+    if ranks.world == 1 and ranks.rank == 0:
+        if not args.no_cpu:
+            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+        if not args.no_secondary:
+            sec = {}
+            for name in ("gated_decode_128k", "hils_decode_1m", "long_prefill_256k"):
+                try:
+                    sec[name] = (secondary_decode if inputs.WORKLOADS[name].kind == "decode" else
+                                 secondary_prefill)(name, args, pk, psrc)
+                except torch.cuda.OutOfMemoryError as e:   # pragma: no cover
+                    sec[name] = {"error": f"out of memory: {e}"}
+                torch.cuda.empty_cache()
+            line["secondary"] = sec
+    if ranks.rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gated_prefill_32k")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        # rank 0 alone times the oracle; other ranks exit without work
+        return run_reference(args, Ranks.single()) if int(os.environ.get("RANK", "0")) == 0 else 0
+    ranks = Ranks(backend="nccl")
+    try:
+        return run_ours(args, ranks)
+    finally:
+        ranks.close()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libs
 EXPORTS = (
     "sparse_attn_workspace_size", "sparse_attn_landmarks", "sparse_attn_select", "sparse_attn_select_decode",
     "sparse_attn_prefill", "sparse_attn_decode", "sparse_attn_check_status", "sparse_attn_status_string",
-    "sparse_attn_version",
+    "sparse_attn_version", "sparse_attn_launch_count",
 )
 
 
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             for n in EXPORTS[1:7]:
                 getattr(L, n).restype = i
             L.sparse_attn_version.restype = i
+            L.sparse_attn_launch_count.argtypes = []
+            L.sparse_attn_launch_count.restype = ctypes.c_ulonglong
             _lib = L
     return _lib
 
@@ -120,6 +122,10 @@ def sparse_attn_status_string(code: int) -> str:
 
 def sparse_attn_version() -> int:
     return lib().sparse_attn_version()
+
+
+def sparse_attn_launch_count() -> int:
+    return int(lib().sparse_attn_launch_count())
 
 
 # ----------------------------------------------------------------------------

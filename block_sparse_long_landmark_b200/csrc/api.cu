@@ -4,9 +4,14 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 using namespace sa;
+
+static std::atomic<unsigned long long> g_launches{0};
+void sa::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 namespace {
 
@@ -147,5 +152,7 @@ const char *sparse_attn_status_string(int code) {
 }
 
 int sparse_attn_version(void) { return 100; }
+
+unsigned long long sparse_attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

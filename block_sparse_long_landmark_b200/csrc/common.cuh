@@ -99,6 +99,9 @@ __device__ __forceinline__ int block_scan_incl(int v, int *tmp, int *total) {
     return v + add;
 }
 
+// Process-wide count of kernels this library has launched (for reporting).
+void note_launch();
+
 // ---------------------------------------------------------------------------
 // Internal launchers (return cudaError_t of the launch)
 // ---------------------------------------------------------------------------

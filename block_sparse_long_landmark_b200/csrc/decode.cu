@@ -281,9 +281,11 @@ static cudaError_t run(DecArgs a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const unsigned units = (unsigned)(s.B * s.Hsel);
     decode_split_kernel<T><<<units * a.S, kDecThreads, smem, st>>>(a);
+    note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess || a.S == 1) return e;
     decode_merge_kernel<T><<<units, kDecThreads, 0, st>>>(a);
+    note_launch();
     return cudaGetLastError();
 }
 

@@ -71,6 +71,7 @@ static cudaError_t run(const Shape &s, const void *K, void *L, cudaStream_t st) 
         case 32: landmarks_kernel<T, 32><<<grid, 256, 0, st>>>(k, l, s.N, s.bs, s.nb, nunits); break;
         default: return cudaErrorInvalidValue;
     }
+    note_launch();
     return cudaGetLastError();
 }
 

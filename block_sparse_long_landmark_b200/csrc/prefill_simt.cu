@@ -201,6 +201,7 @@ static cudaError_t run(const Shape &s, const PrefArgs &a0, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, threads, smem, st>>>(a);
+    note_launch();
     return cudaGetLastError();
 }
 

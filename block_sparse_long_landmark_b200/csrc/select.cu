@@ -410,6 +410,7 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)nunits * a.S, kSelThreads, smem, st>>>(a);
+    note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess || a.S == 1) return e;
     const int M = a.S * s.top_k;
@@ -417,6 +418,7 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
     e = cudaFuncSetAttribute(select_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     if (e != cudaSuccess) return e;
     select_merge_kernel<<<(unsigned)nunits, kSelThreads, msmem, st>>>(a);
+    note_launch();
     return cudaGetLastError();
 }
 

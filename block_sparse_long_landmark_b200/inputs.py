@@ -127,7 +127,7 @@ def _add_to_blocks(K, block_vec, wl: Workload):
     if nbf == 0:
         return
     Kv = K.view(wl.B * wl.Hkv, wl.N, wl.d)[:, :nbf * wl.block].view(wl.B * wl.Hkv, nbf, wl.block, wl.d)
-    step = max(1, (1 << 26) // (wl.block * wl.d))   # bound the fp32 temporary
+    step = max(1, (1 << 26) // (wl.B * wl.Hkv * wl.block * wl.d))   # bound the fp32 temporary
     bv = block_vec.view(wl.B * wl.Hkv, nbf, 1, wl.d)
     for s in range(0, nbf, step):
         e = min(nbf, s + step)

@@ -31,7 +31,7 @@
  *     before anything is launched.
  *   - Return value: SA_OK (0) or a negative SA_ERR_* code.  No exception and
  *     no allocation crosses the ABI; the library keeps no global state
- *     besides CUDA's own per-device kernel images and tensor-map caches.
+ *     besides CUDA's own per-device kernel images and a launch counter.
  *   - Device-side problems (an index list entry out of range, a NaN score, a
  *     bounded wait that expired) never trap: the kernel skips the bad item
  *     and records a code in the workspace's status word, which
@@ -171,6 +171,10 @@ const char *sparse_attn_status_string(int code);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int sparse_attn_version(void);
+
+/* Number of CUDA kernels this library has launched in this process so far
+ * (a reporting counter; the only process-wide state the library keeps). */
+unsigned long long sparse_attn_launch_count(void);
 
 #ifdef __cplusplus
 }
