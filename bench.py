@@ -412,9 +412,15 @@ def e2e_prefill(wl, p, t, steps):
     return ms, h2d, d2h
 
 
-def secondary_prefill(name, args, pk, psrc):
+def _wl(name, args):
     from block_sparse_long_landmark_b200 import inputs
-    wl, p, t = prefill_case(inputs.WORKLOADS[name], "cuda")
+    wl = inputs.WORKLOADS[name]
+    over = {k: v for k, v in (("N", args.N), ("B", args.B)) if v}
+    return wl.scaled(**over) if over else wl
+
+
+def secondary_prefill(name, args, pk, psrc):
+    wl, p, t = prefill_case(_wl(name, args), "cuda")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     ranks1 = Ranks.single()
     steps = max(2, min(args.steps, 5))
@@ -434,8 +440,7 @@ def secondary_prefill(name, args, pk, psrc):
 
 
 def secondary_decode(name, args, pk, psrc):
-    from block_sparse_long_landmark_b200 import inputs
-    wl = inputs.WORKLOADS[name]
+    wl = _wl(name, args)
     p, t = decode_case(wl, "cuda")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     ranks1 = Ranks.single()
@@ -475,6 +480,11 @@ def run_ours(args, ranks):
     dev = torch.device("cuda", ranks.local)
     torch.cuda.set_device(dev)
     pk, psrc = peaks()
+    if args.only:
+        # one workload alone (small profiling cases): a short report, no baselines
+        fn = secondary_decode if inputs.WORKLOADS[args.only].kind == "decode" else secondary_prefill
+        print(json.dumps({"only": args.only, **fn(args.only, args, pk, psrc)}), flush=True)
+        return 0
     base = inputs.WORKLOADS[args.workload]
     wl, p, t = prefill_case(base, "cuda", seed_offset=ranks.rank)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -529,6 +539,9 @@ def main(argv=None):
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--only", default=None, help="measure this one workload alone (profiling)")
+    ap.add_argument("--N", type=int, default=0, help="with --only: override the sequence/context length")
+    ap.add_argument("--B", type=int, default=0, help="with --only: override the batch")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
