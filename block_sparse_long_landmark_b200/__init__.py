@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libs
 EXPORTS = (
     "sparse_attn_workspace_size", "sparse_attn_landmarks", "sparse_attn_select", "sparse_attn_select_decode",
     "sparse_attn_prefill", "sparse_attn_decode", "sparse_attn_check_status", "sparse_attn_status_string",
-    "sparse_attn_version", "sparse_attn_launch_count",
+    "sparse_attn_version", "sparse_attn_launch_count", "sparse_attn_decode_static",
 )
 
 
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             for n in EXPORTS[1:7]:
                 getattr(L, n).restype = i
             L.sparse_attn_version.restype = i
+            L.sparse_attn_decode_static.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.sparse_attn_decode_static.restype = i
             L.sparse_attn_launch_count.argtypes = []
             L.sparse_attn_launch_count.restype = ctypes.c_ulonglong
             _lib = L
@@ -108,6 +110,10 @@ def sparse_attn_prefill(p, Q, K, V, idx, score, count, O, lse, ws, ws_bytes, str
 
 def sparse_attn_decode(p, q, K, V, idx, score, count, o, lse, ws, ws_bytes, stream) -> int:
     return lib().sparse_attn_decode(ctypes.byref(p), q, K, V, idx, score, count, o, lse, ws, ws_bytes, stream)
+
+
+def sparse_attn_decode_static(p, q, K, V, idx, score, count, o, lse, stream) -> int:
+    return lib().sparse_attn_decode_static(ctypes.byref(p), q, K, V, idx, score, count, o, lse, stream)
 
 
 def sparse_attn_check_status(ws, stream):
@@ -236,6 +242,20 @@ def decode(p, q, K, V, idx, sc, cnt, ws, out=None, stream=None):
         o, lse = out
     _check(sparse_attn_decode(p, _ptr(q), _ptr(K), _ptr(V), _ptr(idx), _ptr(sc), _ptr(cnt), _ptr(o), _ptr(lse),
                               _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_decode")
+    return o, lse
+
+
+def decode_static(p, q, K, V, idx, sc, cnt, out=None, stream=None):
+    """sparse_attn_decode without a workspace: for callers that cannot
+    allocate device memory (the library's own static scratch is used)."""
+    torch = _torch()
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(p.B, p.Hq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(sparse_attn_decode_static(p, _ptr(q), _ptr(K), _ptr(V), _ptr(idx), _ptr(sc), _ptr(cnt), _ptr(o),
+                                     _ptr(lse), _stream(stream)), "sparse_attn_decode_static")
     return o, lse
 
 

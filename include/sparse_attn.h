@@ -31,7 +31,8 @@
  *     before anything is launched.
  *   - Return value: SA_OK (0) or a negative SA_ERR_* code.  No exception and
  *     no allocation crosses the ABI; the library keeps no global state
- *     besides CUDA's own per-device kernel images and a launch counter.
+ *     besides CUDA's own per-device kernel images, a launch counter and the
+ *     static scratch array of sparse_attn_decode_static.
  *   - Device-side problems (an index list entry out of range, a NaN score, a
  *     bounded wait that expired) never trap: the kernel skips the bad item
  *     and records a code in the workspace's status word, which
@@ -160,6 +161,22 @@ int sparse_attn_prefill(const sa_params *p, const void *Q, const void *K, const 
 int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
                        const float *score, const int32_t *count, void *o, float *lse, void *ws,
                        size_t ws_bytes, void *stream);
+
+/* Decode without a caller workspace, for callers that cannot allocate device
+ * memory (custom-allocator callbacks, servers whose memory pool owns every
+ * device byte, plugins handed only the tensors of one call).  The pages
+ * describe no counterpart: this is a deployment convenience.  Same arguments
+ * and results as sparse_attn_decode minus `ws`/`ws_bytes`; the scratch is an
+ * 2 MiB array inside the library (held on every GPU that loads it until
+ * exit).  The first call on each device looks up that array's address -- make
+ * it before any stream capture.  All calls on a device share the array, so
+ * calls that overlap on the GPU race: keep them on one stream.  Problems
+ * whose split partials exceed the array return SA_ERR_WORKSPACE before any
+ * launch.  Never calls cudaMalloc or cudaFree.  Device-side list problems are
+ * skipped as in sparse_attn_decode but not reported. */
+int sparse_attn_decode_static(const sa_params *p, const void *q, const void *K, const void *V,
+                              const int32_t *idx, const float *score, const int32_t *count, void *o, float *lse,
+                              void *stream);
 
 /* Synchronises `stream`, returns SA_OK or SA_ERR_DEVICE from the status
  * word in `ws`, and clears it.  *detail (may be NULL) receives the raw bits:
