@@ -29,6 +29,7 @@ EXPORTS = (
     "sparse_attn_workspace_size", "sparse_attn_landmarks", "sparse_attn_select", "sparse_attn_select_decode",
     "sparse_attn_prefill", "sparse_attn_decode", "sparse_attn_check_status", "sparse_attn_status_string",
     "sparse_attn_version", "sparse_attn_launch_count", "sparse_attn_decode_static",
+    "sparse_attn_prefill_kernel",
 )
 
 
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
             for n in EXPORTS[1:7]:
                 getattr(L, n).restype = i
             L.sparse_attn_version.restype = i
+            L.sparse_attn_prefill_kernel.argtypes = [P]
+            L.sparse_attn_prefill_kernel.restype = i
             L.sparse_attn_decode_static.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             L.sparse_attn_decode_static.restype = i
             L.sparse_attn_launch_count.argtypes = []
@@ -110,6 +113,10 @@ def sparse_attn_prefill(p, Q, K, V, idx, score, count, O, lse, ws, ws_bytes, str
 
 def sparse_attn_decode(p, q, K, V, idx, score, count, o, lse, ws, ws_bytes, stream) -> int:
     return lib().sparse_attn_decode(ctypes.byref(p), q, K, V, idx, score, count, o, lse, ws, ws_bytes, stream)
+
+
+def sparse_attn_prefill_kernel(p) -> int:
+    return lib().sparse_attn_prefill_kernel(ctypes.byref(p))
 
 
 def sparse_attn_decode_static(p, q, K, V, idx, score, count, o, lse, stream) -> int:

@@ -112,6 +112,10 @@ size_t select_workspace(const Shape &s, bool decode);
 cudaError_t launch_prefill_simt(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
                                 const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
                                 cudaStream_t st);
+bool prefill_tc_supported(const Shape &s);
+cudaError_t launch_prefill_tc(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
+                              const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
+                              cudaStream_t st);
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, void *ws,
                           size_t ws_bytes, cudaStream_t st);

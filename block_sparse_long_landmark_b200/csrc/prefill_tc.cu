@@ -1,0 +1,592 @@
+// prefill_tc.cu -- tensor-core (tcgen05 + TMEM + TMA) gated block-sparse
+// prefill for bf16, d = 128, block 64 or 128.
+//
+// [SAS] "Ключевые факты" / "Как это применить": FlashAttention-style blockwise
+// attention over the kept blocks only, the square matrix never materialised;
+// the selector's gate log_sigmoid(s_b - s_local) is added to the logits of
+// selected blocks inside the softmax (forced sink / local blocks get 0).
+//
+// One CTA = 256 query rows of one (batch, kv-head, tile): two M=128 tiles
+// that share every K/V tile of the kept list (GQA: with block 64 a CTA holds
+// the 4 query heads x 64 rows of the tile; with block 128, 2 heads x 128 rows
+// and a second CTA takes the other 2 heads).  Key tiles are 128 keys: two
+// kept blocks of 64, or one of 128.
+//
+// Warp roles (12 warps = 3 warpgroups):
+//   warp 0      TMA producer: Q once, then K/V key tiles into a 2-stage ring
+//   warp 1      TMEM owner + single-thread tcgen05.mma issuer
+//   warps 2-3   idle
+//   warps 4-7   softmax for M-tile 0, warps 8-11 softmax for M-tile 1; thread
+//               = one query row = one TMEM lane
+// Registers: launched at 168 per thread (3 warps per SM sub-partition); the
+// first warpgroup gives back down to 72 and the two softmax warpgroups take
+// 216 each: 128 x 72 + 256 x 216 = 384 x 168, the launch's own total.
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16) is
+// written over the first 64 columns of its S tile and read by the PV MMA
+// straight from TMEM.  MMA order per key tile i:
+//   S0(i) = Q0 K_i^T ; O1 += P1(i-1) V_(i-1) ; S1(i) = Q1 K_i^T ; O0 += P0(i) V_i
+// so the tensor core works on one M-tile while the other's softmax runs.
+// The running max is rescaled lazily: O is corrected in TMEM only when a
+// row's max grows by more than 2^8.
+//
+// Every mbarrier wait is bounded (about two seconds of %globaltimer); on
+// expiry the CTA records kStatusTimeout, drains, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsSoftmax = 216;
+static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+constexpr uint32_t kChunkBytes = 128 * 128;     // 128 rows x 64 bf16 (one 128-byte swizzle column)
+constexpr uint32_t kTileBytes = 2 * kChunkBytes;  // 128 x 128 bf16
+constexpr uint32_t kQOff = 0;                   // 2 M tiles
+constexpr uint32_t kKOff = 2 * kTileBytes;      // 2 stages
+constexpr uint32_t kVOff = 4 * kTileBytes;      // 2 stages
+constexpr uint32_t kBarOff = 6 * kTileBytes;
+constexpr int kMaxList = 258;
+constexpr uint32_t kSmemBytes = kBarOff + 1024 + 8 * kMaxList + 2048;   // + alignment slack
+constexpr unsigned long long kWaitNs = 2000000000ull;
+
+// barrier slots (uint64 each)
+enum { B_Q = 0, B_KF = 1, B_VF = 3, B_FREE = 5, B_S = 7, B_P = 9, B_O = 11, B_END = 13, NBAR = 14 };
+
+struct TcArgs {
+    Shape s;
+    const int32_t *idx;
+    const float *score;
+    const int32_t *count;
+    __nv_bfloat16 *O;
+    float *lse;
+    unsigned *status;
+    int npair;   // CTAs per (batch, kv-head, tile)
+    int hc;      // query heads per CTA
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait: true when the phase completed, false on timeout or abort.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned *status) {
+    if (mbar_try(bar, parity)) return true;
+    const unsigned long long t0 = gtimer();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 63) == 63) {
+            if (*abort_flag) return false;
+            if (gtimer() - t0 > kWaitNs) {
+                *abort_flag = 1;
+                set_status(status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptors (sm_100 format, version 1), 128-byte swizzle.
+// K-major: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// MN-major: 64 contiguous elements per 128-byte row, next 64 elements `lbo`
+// bytes away, 8-row (K) groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+    return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, M = 128, N = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((128u >> 3) << 17) |
+           ((128u >> 4) << 24);
+}
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+          "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+          "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ---------------------------------------------------------------------------
+// kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, TcArgs a) {
+    constexpr float kLog2e = 1.4426950408889634f;
+    constexpr float kLn2 = 0.6931471805599453f;
+    const Shape &s = a.s;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                            ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kBarOff + 8 * NBAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 8 * NBAR + 4);
+    int *blk_s = reinterpret_cast<int *>(smem + kBarOff + 1024);
+    float *gate_s = reinterpret_cast<float *>(smem + kBarOff + 1024 + 4 * kMaxList);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // CTA -> (batch, kv-head, tile, head pair); larger tiles first
+    int u = blockIdx.x;
+    const int pair = u % a.npair;
+    u /= a.npair;
+    const int j = s.nb - 1 - (u % s.nb);
+    u /= s.nb;
+    const int g = u % s.Hkv;
+    const int b = u / s.Hkv;
+    const int h0 = g * s.G + pair * a.hc;          // first query head of this CTA
+    const size_t lu = ((size_t)b * s.Hkv + g) * s.nb + j;
+    const int cnt = max(0, min(a.count[lu], s.cap));
+    const int per_tile = s.bs == 64 ? 2 : 1;       // kept blocks per key tile
+    const int T = (cnt + per_tile - 1) / per_tile;
+
+    // ---- set-up -----------------------------------------------------------
+    if (tid == 0) {
+        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == B_P || i == B_P + 1) ? 128 : 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (tid < cnt) {
+        const int32_t *il = a.idx + lu * s.cap;
+        const float *sl = a.score + lu * s.cap;
+        const int blk = il[tid];
+        const bool ok = blk >= 0 && blk <= j && (tid == 0 || il[tid - 1] < blk);
+        if (!ok) set_status(a.status, kStatusBadIndex);
+        blk_s[tid] = ok ? blk : -1;
+        const bool forced = (blk == j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
+        gate_s[tid] = ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[tid] - sl[cnt - 1]) * kLog2e : 0.f;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const float qk_scale = s.scale * kLog2e;
+
+    if (warp == 0) {
+        // ---- TMA producer -------------------------------------------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+        if (lane == 0 && T > 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
+            mbar_expect_tx(bar(B_Q), 2 * kTileBytes);
+            for (int m = 0; m < 2; ++m) {
+                for (int c = 0; c < 2; ++c) {
+                    if (s.bs == 64) {
+                        for (int e = 0; e < 2; ++e) {
+                            const int h = h0 + 2 * m + e;
+                            const int y = ((b * s.Hq + h) * s.N) + j * 64;
+                            tma_load_2d(sbase + kQOff + m * kTileBytes + c * kChunkBytes + e * 8192, &tmQ, bar(B_Q),
+                                        64 * c, y);
+                        }
+                    } else {
+                        const int h = h0 + m;
+                        const int y = ((b * s.Hq + h) * s.N) + j * 128;
+                        tma_load_2d(sbase + kQOff + m * kTileBytes + c * kChunkBytes, &tmQ, bar(B_Q), 64 * c, y);
+                    }
+                }
+            }
+            const int kvbase = (b * s.Hkv + g) * s.N;
+            int issued = 0;
+            for (int i = 0; i < T; ++i) {
+                const int st = i & 1;
+                if (i >= 2 && !mbar_wait(bar(B_FREE + st), ((i >> 1) - 1) & 1, abort_flag, a.status)) break;
+                const uint32_t kdst = sbase + kKOff + st * kTileBytes, vdst = sbase + kVOff + st * kTileBytes;
+                mbar_expect_tx(bar(B_KF + st), kTileBytes);
+                mbar_expect_tx(bar(B_VF + st), kTileBytes);
+                for (int e = 0; e < 2; ++e) {
+                    // block feeding rows [64e, 64e+64) (block 64) or all 128 rows (block 128)
+                    if (s.bs == 128 && e == 1) break;
+                    int c = i * per_tile + e;
+                    if (c >= cnt) c = i * per_tile;          // odd tail: repeat, masked later
+                    const int blk = max(0, blk_s[c]);
+                    const int y = kvbase + blk * s.bs;
+                    for (int ch = 0; ch < 2; ++ch) {
+                        tma_load_2d(kdst + ch * kChunkBytes + e * 8192, &tmK, bar(B_KF + st), 64 * ch, y);
+                        tma_load_2d(vdst + ch * kChunkBytes + e * 8192, &tmV, bar(B_VF + st), 64 * ch, y);
+                    }
+                }
+                issued = i + 1;
+            }
+            if (*abort_flag) {
+                // let the copies in flight land before the CTA exits (bounded)
+                volatile int never = 0;
+                mbar_wait(bar(B_Q), 0, &never, a.status);
+                for (int i = max(0, issued - 2); i < issued; ++i) {
+                    mbar_wait(bar(B_KF + (i & 1)), (i >> 1) & 1, &never, a.status);
+                    mbar_wait(bar(B_VF + (i & 1)), (i >> 1) & 1, &never, a.status);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer ---------------------------------------------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+        if (lane == 0 && T > 0) {
+            constexpr uint32_t idq = idesc_bf16(false), idp = idesc_bf16(true);
+            const uint32_t tS[2] = {tmem + 0, tmem + 128};
+            const uint32_t tO[2] = {tmem + 256, tmem + 384};
+            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, a.status);
+            tc_fence_after();
+            auto qk = [&](int m, int st) {
+                const uint32_t qa = sbase + kQOff + m * kTileBytes, kb = sbase + kKOff + st * kTileBytes;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
+                    mma_ss(tS[m], desc_k_sw128(qa + off), desc_k_sw128(kb + off), idq, k > 0);
+                }
+                mma_commit(bar(B_S + m));
+            };
+            auto pv = [&](int m, int st, bool first) {
+                const uint32_t vb = sbase + kVOff + st * kTileBytes;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tO[m], tS[m] + 8 * k, desc_mn_sw128(vb + k * 2048, kChunkBytes), idp, (!first || k > 0));
+                mma_commit(bar(B_O + m));
+            };
+            for (int i = 0; ok && i < T; ++i) {
+                const int st = i & 1, ph = (i >> 1) & 1;
+                if (!(ok = mbar_wait(bar(B_KF + st), ph, abort_flag, a.status))) break;
+                tc_fence_after();
+                qk(0, st);
+                if (i > 0) {
+                    const int sp = (i - 1) & 1, php = ((i - 1) >> 1) & 1;
+                    if (!(ok = mbar_wait(bar(B_P + 1), (i - 1) & 1, abort_flag, a.status))) break;
+                    if (!(ok = mbar_wait(bar(B_VF + sp), php, abort_flag, a.status))) break;
+                    tc_fence_after();
+                    pv(1, sp, i - 1 == 0);
+                    mma_commit(bar(B_FREE + sp));
+                }
+                qk(1, st);
+                if (!(ok = mbar_wait(bar(B_P + 0), i & 1, abort_flag, a.status))) break;
+                if (!(ok = mbar_wait(bar(B_VF + st), ph, abort_flag, a.status))) break;
+                tc_fence_after();
+                pv(0, st, i == 0);
+            }
+            if (ok) {
+                const int i = T - 1, sp = i & 1, php = (i >> 1) & 1;
+                ok = mbar_wait(bar(B_P + 1), i & 1, abort_flag, a.status) &&
+                     mbar_wait(bar(B_VF + sp), php, abort_flag, a.status);
+                if (ok) {
+                    tc_fence_after();
+                    pv(1, sp, i == 0);
+                    mma_commit(bar(B_FREE + sp));
+                }
+            }
+            // drain: every MMA issued above has completed once this arrives
+            // (waited on even after an abort: TMEM is freed only after it)
+            mma_commit(bar(B_END));
+            volatile int never = 0;
+            mbar_wait(bar(B_END), 0, &never, a.status);
+        }
+    } else if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+    } else {
+        // ---- softmax warpgroups ---------------------------------------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        const int m = (warp - 4) >> 2;                  // M tile
+        const int q4 = warp & 3;                         // TMEM lane quarter of this warp
+        const int r = 32 * q4 + lane;                    // row within the M tile
+        const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+        const uint32_t tS = tmem + lane_off + m * 128, tO = tmem + lane_off + 256 + m * 128;
+        int head, ri;
+        if (s.bs == 64) { head = h0 + 2 * m + (r >> 6); ri = r & 63; }
+        else { head = h0 + m; ri = r; }
+        const int qi = j * s.bs + ri;                    // query position of this row
+        float m_run = -CUDART_INF_F, l = 0.f;
+        bool ok = true;
+        for (int i = 0; i < T; ++i) {
+            ok = mbar_wait(bar(B_S + m), i & 1, abort_flag, a.status);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            float x[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, x + 32 * c);
+            tmem_wait_ld();
+            // logits in log2 units: scale, gate per half, masks on the last tile
+            const int c0 = i * per_tile;
+            const float g0 = gate_s[c0];
+            const float g1 = (per_tile == 2 && c0 + 1 < cnt) ? gate_s[c0 + 1] : g0;
+            float mx = -CUDART_INF_F;
+            if (i + 1 < T) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    x[c] = fmaf(x[c], qk_scale, (per_tile == 2 && c >= 64) ? g1 : g0);
+                    mx = fmaxf(mx, x[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    const int e = (per_tile == 2) ? (c >> 6) : 0;
+                    const int ce = c0 + e;
+                    const int blk = ce < cnt ? blk_s[ce] : -1;
+                    const int t = blk * s.bs + ((per_tile == 2) ? (c & 63) : c);
+                    const bool vis = blk >= 0 && t < s.N && !((s.flags & SA_CAUSAL) && blk == j && t > qi);
+                    x[c] = vis ? fmaf(x[c], qk_scale, e ? g1 : g0) : -CUDART_INF_F;
+                    mx = fmaxf(mx, x[c]);
+                }
+            }
+            // masked entries earlier in the list (bad indices) on non-final tiles
+            if (i + 1 < T) {
+                const bool bad0 = blk_s[c0] < 0, bad1 = per_tile == 2 && blk_s[c0 + 1] < 0;
+                if (bad0 || bad1) {
+                    mx = -CUDART_INF_F;
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) {
+                        const bool bad = (per_tile == 2 && c >= 64) ? bad1 : bad0;
+                        if (bad) x[c] = -CUDART_INF_F;
+                        mx = fmaxf(mx, x[c]);
+                    }
+                }
+            }
+            const float m_new = fmaxf(m_run, mx);
+            if (i == 0) {
+                m_run = m_new;
+            } else {
+                const bool need = m_new > m_run + 8.f;
+                if (__any_sync(0xffffffffu, need)) {
+                    ok = mbar_wait(bar(B_O + m), (i - 1) & 1, abort_flag, a.status);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    tc_fence_after();
+                    const float corr = need ? ex2(m_run - m_new) : 1.f;
+                    if (need) {
+                        l *= corr;
+                        m_run = m_new;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float o[32];
+                        tmem_ld32(tO + 32 * c, o);
+                        tmem_wait_ld();
+                        uint32_t w[32];
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(o[k] * corr);
+                        tmem_st32(tO + 32 * c, w);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            const float ref = m_run == -CUDART_INF_F ? 0.f : m_run;
+            float ls = 0.f;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2(x[64 * hf + 2 * c] - ref), p1 = ex2(x[64 * hf + 2 * c + 1] - ref);
+                    ls += p0 + p1;
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    pk[c] = *reinterpret_cast<uint32_t *>(&h2);
+                }
+                tmem_st32(tS + 32 * hf, pk);
+            }
+            l += ls;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_P + m));
+        }
+        // ---- epilogue: O / l -> bf16, LSE ---------------------------------
+        const bool have = T > 0 && ok;
+        if (have) {
+            ok = mbar_wait(bar(B_O + m), (T - 1) & 1, abort_flag, a.status);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+        }
+        const bool row_ok = ri < s.bs && qi < s.N;
+        __nv_bfloat16 *orow = a.O + (((size_t)b * s.Hq + head) * s.N + (row_ok ? qi : 0)) * 128;
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float o[32];
+            if (have && ok) {
+                tmem_ld32(tO + 32 * c, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) o[k] = 0.f;
+            }
+            if (row_ok) {
+#pragma unroll
+                for (int v = 0; v < 32; v += 8) {
+                    float f[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) f[k] = o[v + k] * inv;
+                    store16(orow + 32 * c + v, f);
+                }
+            }
+        }
+        if (row_ok)
+            a.lse[((size_t)b * s.Hq + head) * s.N + qi] =
+                (l > 0.f && ok) ? (m_run + log2f(l)) * kLn2 : -CUDART_INF_F;
+    }
+
+    // ---- teardown -----------------------------------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encode() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+bool make_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows) {
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {128 * sizeof(__nv_bfloat16)};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_tc_supported(const Shape &s) {
+    if (s.dtype != SA_BF16 || s.d != 128) return false;
+    if (s.flags & (SA_HIER | SA_SELECT_PER_QHEAD)) return false;
+    if (s.bs != 64 && s.bs != 128) return false;
+    const int hc = 256 / s.bs;
+    if (s.G % hc) return false;
+    if (s.cap > kMaxList) return false;
+    const char *e = getenv("SPARSE_ATTN_PREFILL_PATH");
+    if (e && strcmp(e, "simt") == 0) return false;
+    return true;
+}
+
+cudaError_t launch_prefill_tc(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
+                              const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
+                              cudaStream_t st) {
+    if (!get_encode()) return cudaErrorNotSupported;
+    CUtensorMap mq, mk, mv;
+    const uint64_t qrows = (uint64_t)s.B * s.Hq * s.N, krows = (uint64_t)s.B * s.Hkv * s.N;
+    if (!make_map(&mq, Q, qrows, s.bs) || !make_map(&mk, K, krows, s.bs) || !make_map(&mv, V, krows, s.bs))
+        return cudaErrorInvalidValue;
+    TcArgs a{};
+    a.s = s;
+    a.idx = idx;
+    a.score = score;
+    a.count = count;
+    a.O = (__nv_bfloat16 *)O;
+    a.lse = lse;
+    a.status = status;
+    a.hc = 256 / s.bs;
+    a.npair = s.G / a.hc;
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((size_t)s.B * s.Hkv * s.nb * a.npair);
+    prefill_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace sa

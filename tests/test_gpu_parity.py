@@ -113,10 +113,18 @@ FLAG_CASES = [
 ]
 
 
+FLAG_SHAPES = {
+    "fp32_g2": dict(Hq=4, Hkv=2, block=64, dtype="fp32"),
+    "bf16_g2": dict(Hq=4, Hkv=2, block=64, dtype="bf16"),       # CUDA-core kernel
+    "bf16_g4": dict(Hq=8, Hkv=2, block=64, dtype="bf16"),       # tensor-core kernel (block 64)
+    "bf16_g2_b128": dict(Hq=4, Hkv=2, block=128, dtype="bf16"),  # tensor-core kernel (block 128)
+}
+
+
 @pytest.mark.parametrize("name,flags,top_k", FLAG_CASES)
-@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_prefill_flags(name, flags, top_k, dtype):
-    wl = W["gated_prefill_32k"].scaled(N=1000, Hq=4, Hkv=2, block=64, top_k=top_k, dtype=dtype, n_plants=2)
+@pytest.mark.parametrize("shape", sorted(FLAG_SHAPES))
+def test_prefill_flags(name, flags, top_k, shape):
+    wl = W["gated_prefill_32k"].scaled(N=1000, top_k=top_k, n_plants=2, **FLAG_SHAPES[shape])
     p = sa.params_for(wl, flags=flags)
     Q, K, V = _prefill_inputs(wl)
     L, (idx, sc, cnt), O, lse = run_prefill(p, Q, K, V)
@@ -186,6 +194,35 @@ def test_decode_flags(flags):
     n, exact, mask = compare_lists(ref, idx, sc, cnt)
     G = 1 if flags & inputs.F_PER_QHEAD else wl.Hq // wl.Hkv
     _check_outputs(wl, ref, o, lse, np.repeat(mask, G, axis=1))
+
+
+TC_CASES = {
+    "b64_g4": W["gated_prefill_32k"].scaled(N=4096),
+    "b64_g8": W["gated_prefill_32k"].scaled(N=3000, Hq=16, Hkv=2),
+    "b128_g4": W["long_prefill_256k"].scaled(N=8192, Hq=8, Hkv=2),
+    "b128_ragged": W["long_prefill_256k"].scaled(N=5000, Hq=4, Hkv=2, top_k=5),
+    "b64_big_k": W["gated_prefill_32k"].scaled(N=8192, Hq=8, Hkv=2, top_k=100),
+    "b64_odd_k": W["gated_prefill_32k"].scaled(N=4096, Hq=8, Hkv=2, top_k=7),
+}
+
+
+@pytest.mark.parametrize("case", sorted(TC_CASES))
+def test_tensor_core_prefill_matches_oracle_and_cuda_core(case, monkeypatch):
+    """The tensor-core kernel on the oracle's lists, against the oracle and
+    against the CUDA-core kernel on the same lists."""
+    wl = TC_CASES[case]
+    p = sa.params_for(wl)
+    assert sa.sparse_attn_prefill_kernel(p) == 1
+    Q, K, V = _prefill_inputs(wl)
+    ref = _oracle_prefill(wl, Q, K, V)
+    sel = oracle_sel_tensors(ref)
+    _, _, O, lse = run_prefill(p, Q, K, V, sel=sel)
+    _check_outputs(wl, ref, O, lse)
+    monkeypatch.setenv("SPARSE_ATTN_PREFILL_PATH", "simt")
+    assert sa.sparse_attn_prefill_kernel(p) == 0
+    _, _, O2, lse2 = run_prefill(p, Q, K, V, sel=sel)
+    assert (O.float() - O2.float()).abs().max().item() <= 2e-2
+    assert (lse - lse2).abs().max().item() <= 1e-3
 
 
 def test_selection_is_deterministic():
