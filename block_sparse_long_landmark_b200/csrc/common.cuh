@@ -116,6 +116,11 @@ bool prefill_tc_supported(const Shape &s);
 cudaError_t launch_prefill_tc(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
                               const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
                               cudaStream_t st);
+bool decode_mma_supported(const Shape &s);
+void decode_mma_geometry(const Shape &s, int &S, int &bps);
+cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
+                              const float *score, const int32_t *count, void *o, float *lse, void *ws,
+                              cudaStream_t st, int &S_out);
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, void *ws,
                           size_t ws_bytes, cudaStream_t st);

@@ -258,12 +258,30 @@ __global__ void __launch_bounds__(kSelThreads) select_chunk_kernel(SelArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / VPR, cv = lane % VPR;
     bool nan_seen = false;
-    for (int base = warp * RPW; base < n; base += NG) {
-        const int r = base + sub;
-        const float sc = group_score<T, VPR>(Lg + (size_t)(c0 + min(r, n - 1)) * d, qv, s.scale);
-        if (cv == 0 && r < n) {
-            nan_seen |= isnan(sc);
-            keys[r] = ord_key(sc);
+    // U rows per group in flight: the scan is a pure HBM stream of landmarks
+    constexpr int U = 8;
+    for (int base = warp * RPW * U; base < n; base += NG * U) {
+        uint4 raw[U];
+#pragma unroll
+        for (int uu = 0; uu < U; ++uu) {
+            const int r = min(base + sub + RPW * uu, n - 1);
+            raw[uu] = *reinterpret_cast<const uint4 *>(Lg + (size_t)(c0 + r) * d + cv * EPV);
+        }
+#pragma unroll
+        for (int uu = 0; uu < U; ++uu) {
+            float f[EPV];
+            load16(reinterpret_cast<const T *>(&raw[uu]), f);
+            float dot = 0.f;
+#pragma unroll
+            for (int i = 0; i < EPV; ++i) dot = fmaf(qv[i], f[i], dot);
+#pragma unroll
+            for (int o = VPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            const float sc = s.scale * dot;
+            const int r = base + sub + RPW * uu;
+            if (cv == 0 && r < n) {
+                nan_seen |= isnan(sc);
+                keys[r] = ord_key(sc);
+            }
         }
     }
     if (chunk == 0 && warp < 2) {

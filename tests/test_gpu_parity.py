@@ -181,6 +181,22 @@ def test_decode_on_oracle_lists(case):
     _check_outputs(wl, ref, o, lse)
 
 
+@pytest.mark.parametrize("case", ["gated_8k", "gated_ragged", "hier_16k", "hier_ragged", "gated_big_k"])
+def test_decode_mma_matches_cuda_core(case, monkeypatch):
+    """The tensor-core decode (TMA ring + mma.sync) against the CUDA-core decode
+    on the oracle's lists."""
+    wl = DECODE_CASES[case]
+    p = sa.params_for(wl)
+    q, K, V = inputs.make_decode(wl, device="cuda")
+    ref = _oracle_decode(wl, q, K, V)
+    sel = oracle_sel_tensors(ref)
+    _, _, o, lse = run_decode(p, q, K, V, sel=sel)
+    monkeypatch.setenv("SPARSE_ATTN_DECODE_PATH", "simt")
+    _, _, o2, lse2 = run_decode(p, q, K, V, sel=sel)
+    assert (o.float() - o2.float()).abs().max().item() <= 2e-2
+    assert (lse - lse2).abs().max().item() <= 1e-3
+
+
 @pytest.mark.parametrize("flags", [inputs.F_SINK | inputs.F_LOCAL | inputs.F_CAUSAL,
                                    inputs.F_LOCAL | inputs.F_GATE | inputs.F_CAUSAL,
                                    inputs.F_SINK | inputs.F_LOCAL | inputs.F_GATE | inputs.F_PER_QHEAD,
