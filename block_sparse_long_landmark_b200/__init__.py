@@ -29,7 +29,7 @@ EXPORTS = (
     "sparse_attn_workspace_size", "sparse_attn_landmarks", "sparse_attn_select", "sparse_attn_select_decode",
     "sparse_attn_prefill", "sparse_attn_decode", "sparse_attn_check_status", "sparse_attn_status_string",
     "sparse_attn_version", "sparse_attn_launch_count", "sparse_attn_decode_static",
-    "sparse_attn_prefill_kernel",
+    "sparse_attn_prefill_kernel", "sparse_attn_last_cuda_error", "sparse_attn_cuda_error_string",
 )
 
 
@@ -44,7 +44,11 @@ class sa_params(ctypes.Structure):
 
 class SparseAttnError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {sparse_attn_status_string(code)} (code {code})")
+        msg = f"{what}: {sparse_attn_status_string(code)} (code {code})"
+        if code == SA_ERR_LAUNCH:
+            err = lib().sparse_attn_last_cuda_error()
+            msg += f"; CUDA error {err}: {lib().sparse_attn_cuda_error_string(err).decode()}"
+        super().__init__(msg)
         self.code = code
 
 
@@ -77,6 +81,10 @@ def lib() -> ctypes.CDLL:
             for n in EXPORTS[1:7]:
                 getattr(L, n).restype = i
             L.sparse_attn_version.restype = i
+            L.sparse_attn_last_cuda_error.argtypes = []
+            L.sparse_attn_last_cuda_error.restype = i
+            L.sparse_attn_cuda_error_string.argtypes = [i]
+            L.sparse_attn_cuda_error_string.restype = ctypes.c_char_p
             L.sparse_attn_prefill_kernel.argtypes = [P]
             L.sparse_attn_prefill_kernel.restype = i
             L.sparse_attn_decode_static.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]

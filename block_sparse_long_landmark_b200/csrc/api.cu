@@ -51,7 +51,13 @@ int resolve(const sa_params *p, Shape &s) {
     return SA_OK;
 }
 
-int launch_result(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_LAUNCH; }
+thread_local int t_last_cuda_error = 0;
+
+int launch_result(cudaError_t e) {
+    if (e == cudaSuccess) return SA_OK;
+    t_last_cuda_error = (int)e;
+    return SA_ERR_LAUNCH;
+}
 
 }  // namespace
 
@@ -162,6 +168,10 @@ const char *sparse_attn_status_string(int code) {
 }
 
 int sparse_attn_version(void) { return 100; }
+
+int sparse_attn_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char *sparse_attn_cuda_error_string(int err) { return cudaGetErrorString((cudaError_t)err); }
 
 unsigned long long sparse_attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 

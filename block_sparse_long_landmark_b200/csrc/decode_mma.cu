@@ -10,8 +10,9 @@
 // The step is HBM-bound: every kept block is 16 KB of K and 16 KB of V read
 // once.  A CTA (unit, split) owns up to `bps` kept blocks of one (batch,
 // kv-head) list.  Warp 0 streams them with cp.async.bulk.tensor (128-byte
-// swizzle) into a 3-stage shared-memory ring; consumer warps take whole
-// blocks round-robin and compute, with mma.sync m16n8k16 bf16 tiles,
+// swizzle) into a shared-memory ring with one stage per consumer warp (three
+// CTAs fit an SM); consumer warps take whole blocks round-robin and compute,
+// with mma.sync m16n8k16 bf16 tiles,
 //   S[16 x 64] = q[16 x 128] K_b^T     (rows = the group's query heads, padded)
 //   O[16 x 128] += P[16 x 64] V_b      (P straight from S's registers)
 // keeping a per-warp online softmax.  The warps' states are merged in shared
@@ -32,7 +33,12 @@ namespace {
 
 constexpr int kNW = 2;                          // consumer warps
 constexpr int kThreadsD = 32 * (kNW + 1);
-constexpr int kNST = 3;                         // ring stages
+constexpr int kNST = 2;                         // ring stages
+// Block li goes to stage li % kNST and to consumer warp li % kNW.  With
+// kNST a multiple of kNW every stage has a single consumer warp, which waits
+// on its phases strictly in order; a shared stage would let one warp wait on a
+// parity two phases ahead of the barrier and pass before its data landed.
+static_assert(kNST % kNW == 0, "each ring stage must belong to one consumer warp");
 constexpr uint32_t kHalf = 64 * 128;            // one 64-row x 64-col bf16 box (8 KB)
 constexpr uint32_t kBlockBytes = 2 * kHalf;     // 64 x 128 bf16 (16 KB)
 constexpr uint32_t kStageBytes = 2 * kBlockBytes;  // K + V
@@ -407,7 +413,7 @@ bool decode_mma_supported(const Shape &s) {
 
 void decode_mma_geometry(const Shape &s, int &S, int &bps) {
     const int units = s.B * s.Hsel;
-    const int want = (4 * 296 + units - 1) / units;          // about four waves of CTAs
+    const int want = (3 * 3 * 148 + units - 1) / units;      // about three waves of 3 CTAs per SM
     S = max(1, min(want, (s.cap + 5) / 6));
     bps = (s.cap + S - 1) / S;
     if (bps > kMaxBps) bps = kMaxBps;

@@ -197,6 +197,11 @@ const char *sparse_attn_status_string(int code);
 /* Library version: major * 10000 + minor * 100 + patch. */
 int sparse_attn_version(void);
 
+/* The cudaError_t behind the last SA_ERR_LAUNCH returned on the calling host
+ * thread (0 if none), and CUDA's text for such a code. */
+int sparse_attn_last_cuda_error(void);
+const char *sparse_attn_cuda_error_string(int err);
+
 /* Number of CUDA kernels this library has launched in this process so far
  * (a reporting counter; the only process-wide state the library keeps). */
 unsigned long long sparse_attn_launch_count(void);

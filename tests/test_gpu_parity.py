@@ -149,6 +149,8 @@ DECODE_CASES = {
     "gated_fp32_d64": W["gated_decode_128k"].scaled(B=2, N=4096, d=64, dtype="fp32", Hq=8, Hkv=8, top_k=6,
                                                     n_plants=3, sigma=1.0),
     "gated_big_k": W["gated_decode_128k"].scaled(B=2, N=65536, top_k=200, n_plants=16),
+    # many units: 12 kept blocks per CTA, so every ring stage is reused several times
+    "gated_wide": W["gated_decode_128k"].scaled(B=64, N=4096),
 }
 
 
@@ -181,7 +183,8 @@ def test_decode_on_oracle_lists(case):
     _check_outputs(wl, ref, o, lse)
 
 
-@pytest.mark.parametrize("case", ["gated_8k", "gated_ragged", "hier_16k", "hier_ragged", "gated_big_k"])
+@pytest.mark.parametrize("case", ["gated_8k", "gated_ragged", "hier_16k", "hier_ragged", "gated_big_k",
+                                  "gated_wide"])
 def test_decode_mma_matches_cuda_core(case, monkeypatch):
     """The tensor-core decode (TMA ring + mma.sync) against the CUDA-core decode
     on the oracle's lists."""
