@@ -37,17 +37,12 @@ struct SelArgs {
     int CH;              // candidates per chunk
     int decode;
     int ntiles;          // prefill: nb; decode: 1
-    int mode;            // kFinal, kPartial or kScores
-    uint32_t *all_keys;  // kScores: [units][ncm] order-preserving score keys
-    int ncm;             // kScores: candidates per unit (row length of all_keys)
+    int mode;            // kFinal or kPartial
 };
 
 // What a chunk CTA leaves behind: the unit's final list (one chunk per
-// unit), its chunk's top-K for a merge, or only its chunk's scores for a
-// separate per-unit top-K pass (decode: the scan then runs at full HBM rate
-// and the selection work is taken off its critical path).
-enum { kFinal = 0, kPartial = 1, kScores = 2 };
-constexpr int kMaxSmemCand = 32768;
+// unit) or its chunk's top-K for the merge kernel.
+enum { kFinal = 0, kPartial = 1 };
 
 struct SelSmem {
     float qbar[256];
@@ -83,13 +78,26 @@ __device__ void pool_query(const SelArgs &a, int b, int hs, int j, SelSmem &sm, 
 #pragma unroll
     for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
     const T *Q = (const T *)a.Q;
-    for (int r = rg; r < R; r += NG) {
-        const int hh = h0 + r / nrows, row = r0 + r % nrows;
-        const T *p = a.decode ? Q + ((size_t)b * s.Hq + hh) * d : Q + (((size_t)b * s.Hq + hh) * s.N + row) * d;
-        float f[EPV];
-        load16(p + cv * EPV, f);
+    // U rows in flight per thread: pooling streams the tile's queries from HBM
+    constexpr int U = 8;
+    for (int r0u = rg; r0u < R; r0u += NG * U) {
+        uint4 raw[U];
 #pragma unroll
-        for (int i = 0; i < EPV; ++i) acc[i] += f[i];
+        for (int uu = 0; uu < U; ++uu) {
+            const int r = r0u + NG * uu;
+            const int rc = r < R ? r : r0u;
+            const int hh = h0 + rc / nrows, row = r0 + rc % nrows;
+            const T *p = a.decode ? Q + ((size_t)b * s.Hq + hh) * d : Q + (((size_t)b * s.Hq + hh) * s.N + row) * d;
+            raw[uu] = *reinterpret_cast<const uint4 *>(p + cv * EPV);
+        }
+#pragma unroll
+        for (int uu = 0; uu < U; ++uu) {
+            if (r0u + NG * uu >= R) break;
+            float f[EPV];
+            load16(reinterpret_cast<const T *>(&raw[uu]), f);
+#pragma unroll
+            for (int i = 0; i < EPV; ++i) acc[i] += f[i];
+        }
     }
 #pragma unroll
     for (int i = 0; i < EPV; ++i) red[rg * d + cv * EPV + i] = acc[i];
@@ -125,9 +133,18 @@ __device__ void radix_select(const uint32_t *keys, int n, int k, SelSmem &sm, ui
     for (int shift = 24; shift >= 0; shift -= 8) {
         sm.hist[threadIdx.x] = 0;
         __syncthreads();
-        for (int i = threadIdx.x; i < n; i += kSelThreads) {
-            const uint32_t x = keys[i];
-            if ((x & mask) == prefix) atomicAdd(&sm.hist[(x >> shift) & 255], 1);
+        // warp-aggregated histogram: scores cluster in few top digits, so
+        // lanes with the same digit add once per warp instead of once each
+        for (int i0 = threadIdx.x - (threadIdx.x & 31); i0 < n; i0 += kSelThreads) {
+            const int i = i0 + (threadIdx.x & 31);
+            const uint32_t x = i < n ? keys[i] : 0u;
+            const bool take = i < n && (x & mask) == prefix;
+            const unsigned act = __ballot_sync(0xffffffffu, take);
+            if (take) {
+                const int digit = (int)((x >> shift) & 255);
+                const unsigned same = __match_any_sync(act, digit);
+                if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sm.hist[digit], __popc(same));
+            }
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -239,10 +256,9 @@ __global__ void __launch_bounds__(kSelThreads) select_chunk_kernel(SelArgs a) {
     constexpr int NG = kSelThreads / VPR;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
-    const int chs = a.mode == kScores ? 0 : a.CH;   // kScores keeps no keys in shared memory
     uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + sizeof(SelSmem));
-    int *pos = reinterpret_cast<int *>(keys + chs);
-    float *red = reinterpret_cast<float *>(pos + chs);
+    int *pos = reinterpret_cast<int *>(keys + a.CH);
+    float *red = reinterpret_cast<float *>(pos + a.CH);
 
     const Shape &s = a.s;
     const int d = VPR * EPV;
@@ -291,8 +307,7 @@ __global__ void __launch_bounds__(kSelThreads) select_chunk_kernel(SelArgs a) {
             const int r = base + sub + RPW * uu;
             if (cv == 0 && r < n) {
                 nan_seen |= isnan(sc);
-                if (a.mode == kScores) a.all_keys[(size_t)u * a.ncm + (c0 - first) + r] = ord_key(sc);
-                else keys[r] = ord_key(sc);
+                keys[r] = ord_key(sc);
             }
         }
     }
@@ -306,10 +321,6 @@ __global__ void __launch_bounds__(kSelThreads) select_chunk_kernel(SelArgs a) {
     }
     if (nan_seen) set_status(a.status, kStatusNaN);
     __syncthreads();
-    if (a.mode == kScores) {
-        if (chunk == 0 && threadIdx.x < 2) a.special[(size_t)u * 2 + threadIdx.x] = sm.s_special[threadIdx.x];
-        return;
-    }
 
     const int nsel = topk_positions(keys, n, s.top_k, sm, pos);
     if (a.mode == kFinal) {
@@ -378,38 +389,6 @@ __global__ void __launch_bounds__(kSelThreads) select_merge_kernel(SelArgs a) {
     write_final(a, u, local, sel_idx, sel_sc, nsel, a.special[(size_t)u * 2], a.special[(size_t)u * 2 + 1]);
 }
 
-// Top-K of one unit over the scores a kScores pass stored.
-__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(SelArgs a) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
-    const Shape &s = a.s;
-    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + sizeof(SelSmem));
-    int *pos = reinterpret_cast<int *>(keys + a.ncm);
-    int *sel_idx = pos + s.top_k;
-    float *sel_sc = reinterpret_cast<float *>(sel_idx + s.top_k);
-    const int u = blockIdx.x;
-    int b, hs, j, local;
-    unit_coords(a, u, b, hs, j, local);
-    const int first = (s.flags & SA_SINK) ? 1 : 0;
-    const int n = max(0, local - first);
-    const uint32_t *src = a.all_keys + (size_t)u * a.ncm;
-    for (int i = threadIdx.x; i < n; i += kSelThreads) keys[i] = src[i];
-    __syncthreads();
-    const int nsel = topk_positions(keys, n, s.top_k, sm, pos);
-    for (int i = threadIdx.x; i < nsel; i += kSelThreads) {
-        sel_idx[i] = first + pos[i];
-        sel_sc[i] = key_to_float(keys[pos[i]]);
-    }
-    __syncthreads();
-    write_final(a, u, local, sel_idx, sel_sc, nsel, a.special[(size_t)u * 2], a.special[(size_t)u * 2 + 1]);
-}
-
-static int scores_mode_ok(const Shape &s, bool decode) {
-    const int first = (s.flags & SA_SINK) ? 1 : 0;
-    const int ncand = (s.N - 1) / s.bs - first;
-    return decode && s.top_k > 0 && ncand > s.top_k && ncand <= kMaxSmemCand;
-}
-
 static void geometry(const Shape &s, bool decode, int &nunits, int &S, int &CH) {
     const int ntiles = decode ? 1 : s.nb;
     nunits = s.B * s.Hsel * ntiles;
@@ -418,9 +397,9 @@ static void geometry(const Shape &s, bool decode, int &nunits, int &S, int &CH) 
     const int ncand = max(1, local_max - first);
     S = 1;
     if (decode) {
-        // enough CTAs to keep every SM streaming landmarks
-        const int want = (4 * 148 + nunits - 1) / nunits;
-        S = max(1, min(want, (ncand + 511) / 512));
+        // chunks of about 1024 candidates: thousands of CTAs keep every SM
+        // streaming landmarks while others run their chunk's top-K
+        S = max(1, (ncand + 1023) / 1024);
     }
     S = max(S, (ncand + kMaxChunk - 1) / kMaxChunk);
     CH = (ncand + S - 1) / S;
@@ -433,11 +412,6 @@ static void geometry(const Shape &s, bool decode, int &nunits, int &S, int &CH) 
 size_t select_workspace(const Shape &s, bool decode) {
     int nunits, S, CH;
     geometry(s, decode, nunits, S, CH);
-    if (scores_mode_ok(s, decode)) {
-        const int first = (s.flags & SA_SINK) ? 1 : 0;
-        const int ncand = (s.N - 1) / s.bs - first;
-        return (size_t)nunits * ncand * sizeof(uint32_t) + (size_t)nunits * 2 * sizeof(float) + 256;
-    }
     if (S == 1) return 0;
     return (size_t)nunits * S * s.top_k * (sizeof(uint32_t) + sizeof(int32_t)) + (size_t)nunits * 2 * sizeof(float) +
            256;
@@ -459,18 +433,7 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
     int nunits;
     geometry(s, decode, nunits, a.S, a.CH);
     a.mode = a.S == 1 ? kFinal : kPartial;
-    if (scores_mode_ok(s, decode)) {
-        // decode: stream all scores, then one top-K CTA per unit
-        const int first = (s.flags & SA_SINK) ? 1 : 0;
-        a.ncm = (s.N - 1) / s.bs - first;
-        a.CH = 1024;
-        a.S = (a.ncm + a.CH - 1) / a.CH;
-        a.mode = kScores;
-        char *p = (char *)ws + kStatusBytes;
-        a.all_keys = (uint32_t *)p;
-        p += (size_t)nunits * a.ncm * sizeof(uint32_t);
-        a.special = (float *)p;
-    } else if (a.S > 1) {
+    if (a.S > 1) {
         char *p = (char *)ws + kStatusBytes;
         a.part_key = (uint32_t *)p;
         p += (size_t)nunits * a.S * s.top_k * sizeof(uint32_t);
@@ -482,7 +445,7 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
     const int d = s.d;
     size_t red_bytes = (size_t)(kSelThreads / vpr) * d * sizeof(float);
     red_bytes = max(red_bytes, (size_t)s.top_k * 8);
-    const size_t smem = sizeof(SelSmem) + (a.mode == kScores ? 0 : (size_t)a.CH * 8) + red_bytes;
+    const size_t smem = sizeof(SelSmem) + (size_t)a.CH * 8 + red_bytes;
     void (*kern)(SelArgs) = nullptr;
     switch (vpr) {
         case 8: kern = select_chunk_kernel<T, 8>; break;
@@ -496,14 +459,6 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
     note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess || a.mode == kFinal) return e;
-    if (a.mode == kScores) {
-        const size_t tsmem = sizeof(SelSmem) + (size_t)a.ncm * 4 + (size_t)s.top_k * 12;
-        e = cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem);
-        if (e != cudaSuccess) return e;
-        select_topk_kernel<<<(unsigned)nunits, kSelThreads, tsmem, st>>>(a);
-        note_launch();
-        return cudaGetLastError();
-    }
     const int M = a.S * s.top_k;
     const size_t msmem = sizeof(SelSmem) + (size_t)M * 12 + (size_t)s.top_k * 8;
     e = cudaFuncSetAttribute(select_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
