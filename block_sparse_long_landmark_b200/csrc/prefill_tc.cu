@@ -9,11 +9,11 @@
 // One CTA = 256 query rows of one (batch, kv-head, tile): two M=128 tiles
 // that share every K/V tile of the kept list (GQA: with block 64 a CTA holds
 // the 4 query heads x 64 rows of the tile; with block 128, 2 heads x 128 rows
-// and a second CTA takes the other 2 heads).  Key tiles are 128 keys: two
-// kept blocks of 64, or one of 128.
+// and a second CTA takes the other 2 heads).  Key tiles are 64 keys: one kept
+// block of 64, or one half of a block of 128.
 //
 // Warp roles (12 warps = 3 warpgroups):
-//   warp 0      TMA producer: Q once, then K/V key tiles into a 2-stage ring
+//   warp 0      TMA producer: Q once, then K/V key tiles into a 4-stage ring
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
 //   warps 2-3   idle
 //   warps 4-7   softmax for M-tile 0, warps 8-11 softmax for M-tile 1; thread
@@ -21,11 +21,12 @@
 // Registers: launched at 168 per thread (3 warps per SM sub-partition); the
 // first warpgroup gives back down to 72 and the two softmax warpgroups take
 // 216 each: 128 x 72 + 256 x 216 = 384 x 168, the launch's own total.
-// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16) is
-// written over the first 64 columns of its S tile and read by the PV MMA
-// straight from TMEM.  MMA order per key tile i:
-//   S0(i) = Q0 K_i^T ; O1 += P1(i-1) V_(i-1) ; S1(i) = Q1 K_i^T ; O0 += P0(i) V_i
-// so the tensor core works on one M-tile while the other's softmax runs.
+// TMEM (512 columns), per M-tile m: S buffers A and B (64 fp32 columns each)
+// and O (128 columns) at m*256 + {0, 64, 128}.  P (bf16) is written over the
+// first 32 columns of its S buffer and read by the PV MMA straight from TMEM.
+// S is double-buffered: while a softmax warpgroup works on key tile i, the
+// tensor core already computes S for tile i+1.  MMA order, per key tile i:
+//   O0 += P0(i) V_i ; S0(i+2) = Q0 K_(i+2)^T ; O1 += P1(i) V_i ; S1(i+2) = Q1 K_(i+2)^T
 // The running max is rescaled lazily: O is corrected in TMEM only when a
 // row's max grows by more than 2^8.
 //
@@ -47,18 +48,31 @@ namespace {
 constexpr int kThreads = 384;
 constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsSoftmax = 216;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
-constexpr uint32_t kChunkBytes = 128 * 128;     // 128 rows x 64 bf16 (one 128-byte swizzle column)
-constexpr uint32_t kTileBytes = 2 * kChunkBytes;  // 128 x 128 bf16
+constexpr int kStages = 4;
+constexpr uint32_t kQChunk = 128 * 128;         // 128 rows x 64 bf16 (one 128-byte swizzle column)
+constexpr uint32_t kQTile = 2 * kQChunk;        // an M tile: 128 rows x 128 bf16
+constexpr uint32_t kKChunk = 64 * 128;          // 64 keys x 64 bf16
+constexpr uint32_t kKTile = 2 * kKChunk;        // a key tile: 64 keys x 128 bf16
 constexpr uint32_t kQOff = 0;                   // 2 M tiles
-constexpr uint32_t kKOff = 2 * kTileBytes;      // 2 stages
-constexpr uint32_t kVOff = 4 * kTileBytes;      // 2 stages
-constexpr uint32_t kBarOff = 6 * kTileBytes;
+constexpr uint32_t kKOff = 2 * kQTile;          // kStages K tiles
+constexpr uint32_t kVOff = kKOff + kStages * kKTile;
+constexpr uint32_t kBarOff = kVOff + kStages * kKTile;
 constexpr int kMaxList = 258;
 constexpr uint32_t kSmemBytes = kBarOff + 1024 + 8 * kMaxList + 2048;   // + alignment slack
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
 // barrier slots (uint64 each)
-enum { B_Q = 0, B_KF = 1, B_VF = 3, B_FREE = 5, B_S = 7, B_P = 9, B_O = 11, B_END = 13, NBAR = 14 };
+enum {
+    B_Q = 0,
+    B_KF = 1,                   // [kStages]
+    B_VF = B_KF + kStages,      // [kStages]
+    B_FREE = B_VF + kStages,    // [kStages]
+    B_S = B_FREE + kStages,     // [2 M tiles][2 buffers]
+    B_P = B_S + 4,              // [2][2], 128 arrivals each
+    B_O = B_P + 4,              // [2]
+    B_END = B_O + 2,
+    NBAR
+};
 
 struct TcArgs {
     Shape s;
@@ -141,9 +155,9 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) 
     return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
            ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
-// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, M = 128, N = 128.
-__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((128u >> 3) << 17) |
+// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major, uint32_t n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((n >> 3) << 17) |
            ((128u >> 4) << 24);
 }
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -225,12 +239,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const int h0 = g * s.G + pair * a.hc;          // first query head of this CTA
     const size_t lu = ((size_t)b * s.Hkv + g) * s.nb + j;
     const int cnt = max(0, min(a.count[lu], s.cap));
-    const int per_tile = s.bs == 64 ? 2 : 1;       // kept blocks per key tile
-    const int T = (cnt + per_tile - 1) / per_tile;
+    const int sub = s.bs / 64;                     // 64-key tiles per kept block
+    const int T = cnt * sub;                       // key tiles
 
     // ---- set-up -----------------------------------------------------------
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == B_P || i == B_P + 1) ? 128 : 1);
+        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i >= B_P && i < B_P + 4) ? 128 : 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -252,7 +266,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
     const float qk_scale = s.scale * kLog2e;
 
     if (warp == 0) {
@@ -262,52 +275,47 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
-            mbar_expect_tx(bar(B_Q), 2 * kTileBytes);
+            mbar_expect_tx(bar(B_Q), 2 * kQTile);
             for (int m = 0; m < 2; ++m) {
                 for (int c = 0; c < 2; ++c) {
                     if (s.bs == 64) {
                         for (int e = 0; e < 2; ++e) {
                             const int h = h0 + 2 * m + e;
                             const int y = ((b * s.Hq + h) * s.N) + j * 64;
-                            tma_load_2d(sbase + kQOff + m * kTileBytes + c * kChunkBytes + e * 8192, &tmQ, bar(B_Q),
-                                        64 * c, y);
+                            tma_load_2d(sbase + kQOff + m * kQTile + c * kQChunk + e * 8192, &tmQ, bar(B_Q), 64 * c,
+                                        y);
                         }
                     } else {
                         const int h = h0 + m;
                         const int y = ((b * s.Hq + h) * s.N) + j * 128;
-                        tma_load_2d(sbase + kQOff + m * kTileBytes + c * kChunkBytes, &tmQ, bar(B_Q), 64 * c, y);
+                        for (int e = 0; e < 2; ++e)
+                            tma_load_2d(sbase + kQOff + m * kQTile + c * kQChunk + e * 8192, &tmQ, bar(B_Q), 64 * c,
+                                        y + 64 * e);
                     }
                 }
             }
             const int kvbase = (b * s.Hkv + g) * s.N;
             int issued = 0;
-            for (int i = 0; i < T; ++i) {
-                const int st = i & 1;
-                if (i >= 2 && !mbar_wait(bar(B_FREE + st), ((i >> 1) - 1) & 1, abort_flag, a.status)) break;
-                const uint32_t kdst = sbase + kKOff + st * kTileBytes, vdst = sbase + kVOff + st * kTileBytes;
-                mbar_expect_tx(bar(B_KF + st), kTileBytes);
-                mbar_expect_tx(bar(B_VF + st), kTileBytes);
-                for (int e = 0; e < 2; ++e) {
-                    // block feeding rows [64e, 64e+64) (block 64) or all 128 rows (block 128)
-                    if (s.bs == 128 && e == 1) break;
-                    int c = i * per_tile + e;
-                    if (c >= cnt) c = i * per_tile;          // odd tail: repeat, masked later
-                    const int blk = max(0, blk_s[c]);
-                    const int y = kvbase + blk * s.bs;
-                    for (int ch = 0; ch < 2; ++ch) {
-                        tma_load_2d(kdst + ch * kChunkBytes + e * 8192, &tmK, bar(B_KF + st), 64 * ch, y);
-                        tma_load_2d(vdst + ch * kChunkBytes + e * 8192, &tmV, bar(B_VF + st), 64 * ch, y);
-                    }
-                }
-                issued = i + 1;
+            for (int t = 0; t < T; ++t) {
+                const int st = t % kStages;
+                if (t >= kStages && !mbar_wait(bar(B_FREE + st), ((t / kStages) - 1) & 1, abort_flag, a.status))
+                    break;
+                const int blk = max(0, blk_s[t / sub]);
+                const int y = kvbase + blk * s.bs + (t % sub) * 64;
+                const uint32_t kdst = sbase + kKOff + st * kKTile, vdst = sbase + kVOff + st * kKTile;
+                mbar_expect_tx(bar(B_KF + st), kKTile);
+                for (int ch = 0; ch < 2; ++ch) tma_load_2d(kdst + ch * kKChunk, &tmK, bar(B_KF + st), 64 * ch, y);
+                mbar_expect_tx(bar(B_VF + st), kKTile);
+                for (int ch = 0; ch < 2; ++ch) tma_load_2d(vdst + ch * kKChunk, &tmV, bar(B_VF + st), 64 * ch, y);
+                issued = t + 1;
             }
             if (*abort_flag) {
                 // let the copies in flight land before the CTA exits (bounded)
                 volatile int never = 0;
                 mbar_wait(bar(B_Q), 0, &never, a.status);
-                for (int i = max(0, issued - 2); i < issued; ++i) {
-                    mbar_wait(bar(B_KF + (i & 1)), (i >> 1) & 1, &never, a.status);
-                    mbar_wait(bar(B_VF + (i & 1)), (i >> 1) & 1, &never, a.status);
+                for (int t = max(0, issued - kStages); t < issued; ++t) {
+                    mbar_wait(bar(B_KF + t % kStages), (t / kStages) & 1, &never, a.status);
+                    mbar_wait(bar(B_VF + t % kStages), (t / kStages) & 1, &never, a.status);
                 }
             }
         }
@@ -315,54 +323,53 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         // ---- MMA issuer ---------------------------------------------------
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
         if (lane == 0 && T > 0) {
-            constexpr uint32_t idq = idesc_bf16(false), idp = idesc_bf16(true);
-            const uint32_t tS[2] = {tmem + 0, tmem + 128};
-            const uint32_t tO[2] = {tmem + 256, tmem + 384};
+            constexpr uint32_t idq = idesc_bf16(false, 64), idp = idesc_bf16(true, 128);
             bool ok = mbar_wait(bar(B_Q), 0, abort_flag, a.status);
             tc_fence_after();
-            auto qk = [&](int m, int st) {
-                const uint32_t qa = sbase + kQOff + m * kTileBytes, kb = sbase + kKOff + st * kTileBytes;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
-                    mma_ss(tS[m], desc_k_sw128(qa + off), desc_k_sw128(kb + off), idq, k > 0);
-                }
-                mma_commit(bar(B_S + m));
-            };
-            auto pv = [&](int m, int st, bool first) {
-                const uint32_t vb = sbase + kVOff + st * kTileBytes;
+            // S_m(t) = Q_m K_t^T into buffer t & 1 of M tile m
+            auto qk = [&](int m, int t) {
+                const int st = t % kStages;
+                const uint32_t qa = sbase + kQOff + m * kQTile, kb = sbase + kKOff + st * kKTile;
+                const uint32_t dS = tmem + m * 256 + (t & 1) * 64;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_ts(tO[m], tS[m] + 8 * k, desc_mn_sw128(vb + k * 2048, kChunkBytes), idp, (!first || k > 0));
+                    mma_ss(dS, desc_k_sw128(qa + (k >> 2) * kQChunk + (k & 3) * 32),
+                           desc_k_sw128(kb + (k >> 2) * kKChunk + (k & 3) * 32), idq, k > 0);
+                mma_commit(bar(B_S + 2 * m + (t & 1)));
+            };
+            // O_m += P_m(t) V_t, P read from the first 32 columns of S buffer t & 1
+            auto pv = [&](int m, int t) {
+                const int st = t % kStages;
+                const uint32_t vb = sbase + kVOff + st * kKTile;
+                const uint32_t aP = tmem + m * 256 + (t & 1) * 64, dO = tmem + m * 256 + 128;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ts(dO, aP + 8 * k, desc_mn_sw128(vb + k * 2048, kKChunk), idp, (t > 0 || k > 0));
                 mma_commit(bar(B_O + m));
             };
-            for (int i = 0; ok && i < T; ++i) {
-                const int st = i & 1, ph = (i >> 1) & 1;
-                if (!(ok = mbar_wait(bar(B_KF + st), ph, abort_flag, a.status))) break;
+            for (int t = 0; ok && t < min(2, T); ++t) {
+                if (!(ok = mbar_wait(bar(B_KF + t % kStages), (t / kStages) & 1, abort_flag, a.status))) break;
                 tc_fence_after();
-                qk(0, st);
-                if (i > 0) {
-                    const int sp = (i - 1) & 1, php = ((i - 1) >> 1) & 1;
-                    if (!(ok = mbar_wait(bar(B_P + 1), (i - 1) & 1, abort_flag, a.status))) break;
-                    if (!(ok = mbar_wait(bar(B_VF + sp), php, abort_flag, a.status))) break;
-                    tc_fence_after();
-                    pv(1, sp, i - 1 == 0);
-                    mma_commit(bar(B_FREE + sp));
-                }
-                qk(1, st);
-                if (!(ok = mbar_wait(bar(B_P + 0), i & 1, abort_flag, a.status))) break;
-                if (!(ok = mbar_wait(bar(B_VF + st), ph, abort_flag, a.status))) break;
-                tc_fence_after();
-                pv(0, st, i == 0);
+                qk(0, t);
+                qk(1, t);
             }
-            if (ok) {
-                const int i = T - 1, sp = i & 1, php = (i >> 1) & 1;
-                ok = mbar_wait(bar(B_P + 1), i & 1, abort_flag, a.status) &&
-                     mbar_wait(bar(B_VF + sp), php, abort_flag, a.status);
-                if (ok) {
+            for (int i = 0; ok && i < T; ++i) {
+                const int st = i % kStages, ph = (i / kStages) & 1;
+                const int t2 = i + 2;
+                const bool next = t2 < T;
+                if (!(ok = mbar_wait(bar(B_VF + st), ph, abort_flag, a.status))) break;
+                for (int m = 0; m < 2; ++m) {
+                    if (!(ok = mbar_wait(bar(B_P + 2 * m + (i & 1)), (i >> 1) & 1, abort_flag, a.status))) break;
                     tc_fence_after();
-                    pv(1, sp, i == 0);
-                    mma_commit(bar(B_FREE + sp));
+                    pv(m, i);
+                    if (m == 1) mma_commit(bar(B_FREE + st));
+                    if (next) {
+                        if (m == 0 &&
+                            !(ok = mbar_wait(bar(B_KF + t2 % kStages), (t2 / kStages) & 1, abort_flag, a.status)))
+                            break;
+                        tc_fence_after();
+                        qk(m, t2);
+                    }
                 }
             }
             // drain: every MMA issued above has completed once this arrives
@@ -380,56 +387,43 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int q4 = warp & 3;                         // TMEM lane quarter of this warp
         const int r = 32 * q4 + lane;                    // row within the M tile
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-        const uint32_t tS = tmem + lane_off + m * 128, tO = tmem + lane_off + 256 + m * 128;
+        const uint32_t tM = tmem + lane_off + m * 256, tO = tM + 128;
         int head, ri;
         if (s.bs == 64) { head = h0 + 2 * m + (r >> 6); ri = r & 63; }
         else { head = h0 + m; ri = r; }
         const int qi = j * s.bs + ri;                    // query position of this row
+        const bool causal = s.flags & SA_CAUSAL;
         float m_run = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int i = 0; i < T; ++i) {
-            ok = mbar_wait(bar(B_S + m), i & 1, abort_flag, a.status);
+            const uint32_t tS = tM + (i & 1) * 64;
+            ok = mbar_wait(bar(B_S + 2 * m + (i & 1)), (i >> 1) & 1, abort_flag, a.status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-            float x[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, x + 32 * c);
+            float x[64];
+            tmem_ld32(tS, x);
+            tmem_ld32(tS + 32, x + 32);
             tmem_wait_ld();
-            // logits in log2 units: scale, gate per half, masks on the last tile
-            const int c0 = i * per_tile;
-            const float g0 = gate_s[c0];
-            const float g1 = (per_tile == 2 && c0 + 1 < cnt) ? gate_s[c0 + 1] : g0;
+            const int c = i / sub;
+            const int blk = blk_s[c];
+            const float gl = gate_s[c];
+            const int t0 = blk * s.bs + (i % sub) * 64;  // first key of this tile
+            // masks: a bad list entry, the ragged end of the sequence, causality in the local block
+            const bool masked = blk < 0 || t0 + 64 > s.N || (causal && blk == j);
             float mx = -CUDART_INF_F;
-            if (i + 1 < T) {
+            if (!masked) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    x[c] = fmaf(x[c], qk_scale, (per_tile == 2 && c >= 64) ? g1 : g0);
-                    mx = fmaxf(mx, x[c]);
-                }
+                for (int k = 0; k < 64; ++k) mx = fmaxf(mx, x[k]);
+                mx = fmaf(mx, qk_scale, gl);
             } else {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const int e = (per_tile == 2) ? (c >> 6) : 0;
-                    const int ce = c0 + e;
-                    const int blk = ce < cnt ? blk_s[ce] : -1;
-                    const int t = blk * s.bs + ((per_tile == 2) ? (c & 63) : c);
-                    const bool vis = blk >= 0 && t < s.N && !((s.flags & SA_CAUSAL) && blk == j && t > qi);
-                    x[c] = vis ? fmaf(x[c], qk_scale, e ? g1 : g0) : -CUDART_INF_F;
-                    mx = fmaxf(mx, x[c]);
+                for (int k = 0; k < 64; ++k) {
+                    const int t = t0 + k;
+                    const bool vis = blk >= 0 && t < s.N && !(causal && blk == j && t > qi);
+                    x[k] = vis ? x[k] : -CUDART_INF_F;
+                    mx = fmaxf(mx, x[k]);
                 }
-            }
-            // masked entries earlier in the list (bad indices) on non-final tiles
-            if (i + 1 < T) {
-                const bool bad0 = blk_s[c0] < 0, bad1 = per_tile == 2 && blk_s[c0 + 1] < 0;
-                if (bad0 || bad1) {
-                    mx = -CUDART_INF_F;
-#pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        const bool bad = (per_tile == 2 && c >= 64) ? bad1 : bad0;
-                        if (bad) x[c] = -CUDART_INF_F;
-                        mx = fmaxf(mx, x[c]);
-                    }
-                }
+                mx = mx == -CUDART_INF_F ? mx : fmaf(mx, qk_scale, gl);
             }
             const float m_new = fmaxf(m_run, mx);
             if (i == 0) {
@@ -437,6 +431,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             } else {
                 const bool need = m_new > m_run + 8.f;
                 if (__any_sync(0xffffffffu, need)) {
+                    // PV(i-2) is done (S(i) was computed after it), so PV(i-1)
+                    // is either running or done: parity (i-1) is unambiguous
                     ok = mbar_wait(bar(B_O + m), (i - 1) & 1, abort_flag, a.status);
                     if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                     tc_fence_after();
@@ -446,52 +442,54 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         m_run = m_new;
                     }
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int cc = 0; cc < 4; ++cc) {
                         float o[32];
-                        tmem_ld32(tO + 32 * c, o);
+                        tmem_ld32(tO + 32 * cc, o);
                         tmem_wait_ld();
                         uint32_t w[32];
 #pragma unroll
                         for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(o[k] * corr);
-                        tmem_st32(tO + 32 * c, w);
+                        tmem_st32(tO + 32 * cc, w);
                     }
                     tmem_wait_st();
                 }
             }
-            const float ref = m_run == -CUDART_INF_F ? 0.f : m_run;
+            // p = 2^(x * scale + gate - ref): one FFMA and one ex2 per element
+            const float bias = gl - (m_run == -CUDART_INF_F ? 0.f : m_run);
+            uint32_t pk[32];
             float ls = 0.f;
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2(x[64 * hf + 2 * c] - ref), p1 = ex2(x[64 * hf + 2 * c + 1] - ref);
-                    ls += p0 + p1;
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    pk[c] = *reinterpret_cast<uint32_t *>(&h2);
-                }
-                tmem_st32(tS + 32 * hf, pk);
+            for (int k = 0; k < 32; ++k) {
+                const float p0 = ex2(fmaf(x[2 * k], qk_scale, bias)), p1 = ex2(fmaf(x[2 * k + 1], qk_scale, bias));
+                ls += p0 + p1;
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                pk[k] = *reinterpret_cast<uint32_t *>(&h2);
             }
             l += ls;
+            tmem_st32(tS, pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(B_P + m));
+            mbar_arrive(bar(B_P + 2 * m + (i & 1)));
         }
         // ---- epilogue: O / l -> bf16, LSE ---------------------------------
+        // O is final once the MMA thread's drain barrier (committed after its
+        // last MMA) completes: a single phase, so no parity can alias.  The
+        // per-PV barrier would not do here -- up to two of its phases may
+        // still be pending, and a parity wait cannot tell them apart.
         const bool have = T > 0 && ok;
         if (have) {
-            ok = mbar_wait(bar(B_O + m), (T - 1) & 1, abort_flag, a.status);
+            ok = mbar_wait(bar(B_END), 0, abort_flag, a.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
         }
-        const bool row_ok = ri < s.bs && qi < s.N;
+        const bool row_ok = qi < s.N;
         __nv_bfloat16 *orow = a.O + (((size_t)b * s.Hq + head) * s.N + (row_ok ? qi : 0)) * 128;
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
             float o[32];
             if (have && ok) {
-                tmem_ld32(tO + 32 * c, o);
+                tmem_ld32(tO + 32 * cc, o);
                 tmem_wait_ld();
             } else {
 #pragma unroll
@@ -503,7 +501,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     float f[8];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) f[k] = o[v + k] * inv;
-                    store16(orow + 32 * c + v, f);
+                    store16(orow + 32 * cc + v, f);
                 }
             }
         }
@@ -568,7 +566,7 @@ cudaError_t launch_prefill_tc(const Shape &s, const void *Q, const void *K, cons
     if (!get_encode()) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
     const uint64_t qrows = (uint64_t)s.B * s.Hq * s.N, krows = (uint64_t)s.B * s.Hkv * s.N;
-    if (!make_map(&mq, Q, qrows, s.bs) || !make_map(&mk, K, krows, s.bs) || !make_map(&mv, V, krows, s.bs))
+    if (!make_map(&mq, Q, qrows, 64) || !make_map(&mk, K, krows, 64) || !make_map(&mv, V, krows, 64))
         return cudaErrorInvalidValue;
     TcArgs a{};
     a.s = s;

@@ -38,10 +38,12 @@ struct SelArgs {
     int decode;
     int ntiles;          // prefill: nb; decode: 1
     int mode;            // kFinal or kPartial
+    unsigned *done;      // kPartial: [units] chunks finished; back to 0 after each call
 };
 
 // What a chunk CTA leaves behind: the unit's final list (one chunk per
-// unit) or its chunk's top-K for the merge kernel.
+// unit) or its chunk's top-K; in the second case the unit's last chunk CTA
+// to finish merges the chunks' lists into the final one.
 enum { kFinal = 0, kPartial = 1 };
 
 struct SelSmem {
@@ -50,6 +52,7 @@ struct SelSmem {
     int tmp[8];
     int sel_digit, sel_above;
     float s_special[2];
+    int last;
 };
 
 // Decodes a unit number into (batch, selection head, tile) and its local block.
@@ -250,8 +253,53 @@ __device__ void write_final(const SelArgs &a, int u, int local, const int *sel_i
     if (threadIdx.x == 0) a.count[u] = cnt;
 }
 
+// Merges the per-chunk top-K lists of unit u (they sit in ascending block
+// order, chunk after chunk) into the unit's final list.  Run by the unit's
+// last chunk CTA; the partial lists are read past L1 (written by other CTAs).
+__device__ void merge_unit(const SelArgs &a, int u, unsigned char *smem_raw) {
+    SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
+    const Shape &s = a.s;
+    const int M = a.S * s.top_k;
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + sizeof(SelSmem));
+    int *cidx = reinterpret_cast<int *>(keys + M);
+    int *pos = cidx + M;
+    int *sel_idx = pos + M;
+    float *sel_sc = reinterpret_cast<float *>(sel_idx + s.top_k);
+    int b, hs, j, local;
+    unit_coords(a, u, b, hs, j, local);
+    const int first = (s.flags & SA_SINK) ? 1 : 0;
+    // chunk c holds nv(c) = min(top_k, its candidates) valid entries, packed
+    // in chunk order; the chunk sizes are known, so every thread finds its
+    // entry's slot by arithmetic and all loads are in flight together
+    auto nv = [&](int c) {
+        const int c0 = first + c * a.CH, c1 = min(local, c0 + a.CH);
+        return min(s.top_k, max(0, c1 - c0));
+    };
+    int ntot = 0;
+    for (int c = 0; c < a.S; ++c) ntot += nv(c);
+    for (int e = threadIdx.x; e < M; e += kSelThreads) {
+        const int c = e / s.top_k, i = e - c * s.top_k;
+        if (i < nv(c)) {
+            int base = 0;
+            for (int q = 0; q < c; ++q) base += nv(q);
+            const size_t src = ((size_t)u * a.S + c) * s.top_k + i;
+            keys[base + i] = __ldcg(a.part_key + src);
+            cidx[base + i] = __ldcg(a.part_idx + src);
+        }
+    }
+    __syncthreads();
+    const int nsel = topk_positions(keys, ntot, s.top_k, sm, pos);
+    for (int i = threadIdx.x; i < nsel; i += kSelThreads) {
+        sel_idx[i] = cidx[pos[i]];
+        sel_sc[i] = key_to_float(keys[pos[i]]);
+    }
+    __syncthreads();
+    write_final(a, u, local, sel_idx, sel_sc, nsel, __ldcg(a.special + (size_t)u * 2),
+                __ldcg(a.special + (size_t)u * 2 + 1));
+}
+
 template <typename T, int VPR>
-__global__ void __launch_bounds__(kSelThreads) select_chunk_kernel(SelArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 5) select_chunk_kernel(SelArgs a) {
     constexpr int EPV = Vec<T>::n;
     constexpr int NG = kSelThreads / VPR;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -341,52 +389,17 @@ __global__ void __launch_bounds__(kSelThreads) select_chunk_kernel(SelArgs a) {
             pi[i] = i < nsel ? c0 + pos[i] : -1;
         }
         if (chunk == 0 && threadIdx.x < 2) a.special[(size_t)u * 2 + threadIdx.x] = sm.s_special[threadIdx.x];
-    }
-}
-
-// Merges the per-chunk top-K lists of one unit (they sit in ascending block
-// order, chunk after chunk) into the unit's final list.
-__global__ void __launch_bounds__(kSelThreads) select_merge_kernel(SelArgs a) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
-    const Shape &s = a.s;
-    const int M = a.S * s.top_k;
-    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + sizeof(SelSmem));
-    int *cidx = reinterpret_cast<int *>(keys + M);
-    int *pos = cidx + M;
-    int *sel_idx = pos + M;
-    float *sel_sc = reinterpret_cast<float *>(sel_idx + s.top_k);
-    const int u = blockIdx.x;
-    int b, hs, j, local;
-    unit_coords(a, u, b, hs, j, local);
-    const int first = (s.flags & SA_SINK) ? 1 : 0;
-    // chunk c holds min(top_k, its candidates) valid entries
-    int ntot = 0;
-    for (int c = 0; c < a.S; ++c) {
-        const int c0 = first + c * a.CH, c1 = min(local, c0 + a.CH);
-        ntot += min(s.top_k, max(0, c1 - c0));
-    }
-    // each chunk's valid prefix, in chunk order
-    int base = 0;
-    for (int c = 0; c < a.S; ++c) {
-        const int c0 = first + c * a.CH, c1 = min(local, c0 + a.CH);
-        const int nv = min(s.top_k, max(0, c1 - c0));
-        const uint32_t *pk = a.part_key + ((size_t)u * a.S + c) * s.top_k;
-        const int32_t *pi = a.part_idx + ((size_t)u * a.S + c) * s.top_k;
-        for (int i = threadIdx.x; i < nv; i += kSelThreads) {
-            keys[base + i] = pk[i];
-            cidx[base + i] = pi[i];
+        // the unit's last chunk to finish merges (writes fenced before the count)
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) sm.last = atomicAdd(a.done + u, 1u) == (unsigned)(a.S - 1);
+        __syncthreads();
+        if (sm.last) {
+            __threadfence();
+            merge_unit(a, u, smem_raw);
+            if (threadIdx.x == 0) a.done[u] = 0u;
         }
-        base += nv;
     }
-    __syncthreads();
-    const int nsel = topk_positions(keys, ntot, s.top_k, sm, pos);
-    for (int i = threadIdx.x; i < nsel; i += kSelThreads) {
-        sel_idx[i] = cidx[pos[i]];
-        sel_sc[i] = key_to_float(keys[pos[i]]);
-    }
-    __syncthreads();
-    write_final(a, u, local, sel_idx, sel_sc, nsel, a.special[(size_t)u * 2], a.special[(size_t)u * 2 + 1]);
 }
 
 static void geometry(const Shape &s, bool decode, int &nunits, int &S, int &CH) {
@@ -397,9 +410,9 @@ static void geometry(const Shape &s, bool decode, int &nunits, int &S, int &CH) 
     const int ncand = max(1, local_max - first);
     S = 1;
     if (decode) {
-        // chunks of about 1024 candidates: thousands of CTAs keep every SM
+        // chunks of about 512 candidates: thousands of CTAs keep every SM
         // streaming landmarks while others run their chunk's top-K
-        S = max(1, (ncand + 1023) / 1024);
+        S = max(1, (ncand + 511) / 512);
     }
     S = max(S, (ncand + kMaxChunk - 1) / kMaxChunk);
     CH = (ncand + S - 1) / S;
@@ -414,7 +427,7 @@ size_t select_workspace(const Shape &s, bool decode) {
     geometry(s, decode, nunits, S, CH);
     if (S == 1) return 0;
     return (size_t)nunits * S * s.top_k * (sizeof(uint32_t) + sizeof(int32_t)) + (size_t)nunits * 2 * sizeof(float) +
-           256;
+           (size_t)nunits * sizeof(unsigned) + 256;
 }
 
 template <typename T>
@@ -440,12 +453,16 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
         a.part_idx = (int32_t *)p;
         p += (size_t)nunits * a.S * s.top_k * sizeof(int32_t);
         a.special = (float *)p;
+        p += (size_t)nunits * 2 * sizeof(float);
+        a.done = (unsigned *)p;
     }
     const int vpr = s.d * (int)sizeof(T) / 16;
     const int d = s.d;
     size_t red_bytes = (size_t)(kSelThreads / vpr) * d * sizeof(float);
     red_bytes = max(red_bytes, (size_t)s.top_k * 8);
-    const size_t smem = sizeof(SelSmem) + (size_t)a.CH * 8 + red_bytes;
+    size_t smem = sizeof(SelSmem) + (size_t)a.CH * 8 + red_bytes;
+    if (a.mode == kPartial)   // the merging CTA reuses the same shared memory
+        smem = max(smem, sizeof(SelSmem) + (size_t)a.S * s.top_k * 12 + (size_t)s.top_k * 8);
     void (*kern)(SelArgs) = nullptr;
     switch (vpr) {
         case 8: kern = select_chunk_kernel<T, 8>; break;
@@ -458,14 +475,7 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
     kern<<<(unsigned)nunits * a.S, kSelThreads, smem, st>>>(a);
     note_launch();
     e = cudaGetLastError();
-    if (e != cudaSuccess || a.mode == kFinal) return e;
-    const int M = a.S * s.top_k;
-    const size_t msmem = sizeof(SelSmem) + (size_t)M * 12 + (size_t)s.top_k * 8;
-    e = cudaFuncSetAttribute(select_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
-    if (e != cudaSuccess) return e;
-    select_merge_kernel<<<(unsigned)nunits, kSelThreads, msmem, st>>>(a);
-    note_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_select(const Shape &s, bool decode, const void *Q, const void *L, int32_t *idx, float *score,

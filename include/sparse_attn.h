@@ -116,7 +116,9 @@ typedef struct {
 
 /* Bytes of workspace `op` needs (at least 256: the first 16 bytes hold the
  * status word).  The workspace must be zero-filled once when allocated; the
- * library leaves the status word zero unless a device-side problem occurs.  */
+ * library leaves the status word zero unless a device-side problem occurs,
+ * and returns every completion counter it keeps there to zero by the end of
+ * each call.  Calls that share a workspace must not overlap on the GPU.  */
 size_t sparse_attn_workspace_size(const sa_params *p, int op);
 
 /* Landmarks (first step of the path; [HiLS] landmark, [LSA] keys pooled

@@ -244,6 +244,21 @@ def test_tensor_core_prefill_matches_oracle_and_cuda_core(case, monkeypatch):
     assert (lse - lse2).abs().max().item() <= 1e-3
 
 
+def test_prefill_selection_in_chunks_with_merge():
+    """More than 8192 candidate blocks: prefill selection splits every tile's
+    candidates into chunks and merges the chunks' top-K lists."""
+    wl = W["tiny_fp32_prefill"].scaled(N=140000, Hq=1, Hkv=1, block=16, top_k=4, n_plants=2)
+    p = sa.params_for(wl)
+    assert sa.sparse_attn_workspace_size(p, sa.SA_OP_SELECT) > 256     # the chunked path
+    Q, K, V = _prefill_inputs(wl)
+    L, (idx, sc, cnt), O, lse = run_prefill(p, Q, K, V)
+    units = [(0, 0, j) for j in list(range(0, 40)) + list(range(8180, 8200)) + list(range(wl.nb - 40, wl.nb))]
+    ref = oracle.prefill(f64(Q), f64(K), f64(V), wl.block, wl.top_k, wl.flags, round_mode=oracle.ROUND_FP32,
+                         units=units)
+    n, exact, mask = compare_lists(ref, idx, sc, cnt, units=units)
+    assert exact >= 0.9 * n
+
+
 def test_selection_is_deterministic():
     wl = W["gated_prefill_32k"].scaled(N=4096)
     p = sa.params_for(wl)
