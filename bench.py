@@ -325,9 +325,14 @@ def cpu_inputs(wl):
 
 
 def calibrate_units(wl, Q64, K64, V64, target_s):
-    dt, _, _ = oracle_prefill_sample(wl, Q64, K64, V64, 16, seed=99)
-    per = dt / 16
-    return max(16, min(20000, int(target_s / max(per, 1e-6))))
+    """Units whose oracle time is about target_s: two probes fit t = a + b n
+    (a: the landmarks of the touched kv-heads, b: one unit's selection and
+    attention)."""
+    t1, _, _ = oracle_prefill_sample(wl, Q64, K64, V64, 16, seed=98)
+    t2, _, _ = oracle_prefill_sample(wl, Q64, K64, V64, 64, seed=99)
+    b = max((t2 - t1) / 48, 1e-6)
+    a = max(t1 - 16 * b, 0.0)
+    return max(16, min(50000, int((target_s - a) / b)))
 
 
 def cpu_baseline(wl, target_s):

@@ -6,27 +6,27 @@
 // the selector's gate log_sigmoid(s_b - s_local) is added to the logits of
 // selected blocks inside the softmax (forced sink / local blocks get 0).
 //
-// One CTA = 256 query rows of one (batch, kv-head, tile): two M=128 tiles
-// that share every K/V tile of the kept list (GQA: with block 64 a CTA holds
-// the 4 query heads x 64 rows of the tile; with block 128, 2 heads x 128 rows
-// and a second CTA takes the other 2 heads).  Key tiles are 64 keys: one kept
-// block of 64, or one half of a block of 128.
+// One CTA = one M=128 tile: 128 query rows of one (batch, kv-head, tile) that
+// share the tile's kept list (GQA: with block 64 the rows of 2 query heads,
+// with block 128 those of 1; the other heads of the group are neighbouring
+// CTAs, which find the same K/V tiles in L2).  Two CTAs run on every SM, each
+// with half the tensor memory, so one CTA's start and end overlap the other's
+// main loop.  Key tiles are 64 keys: one kept block of 64, or half of a block
+// of 128.
 //
-// Warp roles (12 warps = 3 warpgroups):
-//   warp 0      TMA producer: Q once, then K/V key tiles into a 4-stage ring
+// Warp roles (8 warps = 2 warpgroups):
+//   warp 0      TMA producer: Q once, then K and V key tiles into 2-stage rings
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
 //   warps 2-3   idle
-//   warps 4-7   softmax for M-tile 0, warps 8-11 softmax for M-tile 1; thread
-//               = one query row = one TMEM lane
-// Registers: launched at 168 per thread (3 warps per SM sub-partition); the
-// first warpgroup gives back down to 72 and the two softmax warpgroups take
-// 216 each: 128 x 72 + 256 x 216 = 384 x 168, the launch's own total.
-// TMEM (512 columns), per M-tile m: S buffers A and B (64 fp32 columns each)
-// and O (128 columns) at m*256 + {0, 64, 128}.  P (bf16) is written over the
-// first 32 columns of its S buffer and read by the PV MMA straight from TMEM.
-// S is double-buffered: while a softmax warpgroup works on key tile i, the
-// tensor core already computes S for tile i+1.  MMA order, per key tile i:
-//   O0 += P0(i) V_i ; S0(i+2) = Q0 K_(i+2)^T ; O1 += P1(i) V_i ; S1(i+2) = Q1 K_(i+2)^T
+//   warps 4-7   softmax; thread = one query row = one TMEM lane
+// Registers: launched at 128 per thread (two CTAs, 4 warps per SM
+// sub-partition); the first warpgroup gives back down to 56 and the softmax
+// warpgroup takes 200: 128 x 56 + 128 x 200 = 256 x 128, the launch's total.
+// TMEM (256 columns): S buffers A and B (64 fp32 columns each) and O (128).
+// P (bf16) is written over the first 32 columns of its S buffer and read by
+// the PV MMA straight from TMEM.  S is double-buffered: while the softmax
+// warpgroup works on key tile i, the tensor core already holds S(i+1) and,
+// once P(i) is in, runs  O += P(i) V_i ; S(i+2) = Q K_(i+2)^T.
 // The running max is rescaled lazily: O is corrected in TMEM only when a
 // row's max grows by more than 2^8.
 //
@@ -45,32 +45,34 @@
 namespace sa {
 namespace {
 
-constexpr int kThreads = 384;
-constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsSoftmax = 216;
-static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
-constexpr int kStages = 4;
+constexpr int kThreads = 256;
+constexpr int kRegsLaunch = 128, kRegsProducer = 56, kRegsSoftmax = 200;
+static_assert(128 * kRegsProducer + 128 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+constexpr int kStages = 2;                      // per ring (K and V)
 constexpr uint32_t kQChunk = 128 * 128;         // 128 rows x 64 bf16 (one 128-byte swizzle column)
-constexpr uint32_t kQTile = 2 * kQChunk;        // an M tile: 128 rows x 128 bf16
+constexpr uint32_t kQTile = 2 * kQChunk;        // the M tile: 128 rows x 128 bf16
 constexpr uint32_t kKChunk = 64 * 128;          // 64 keys x 64 bf16
 constexpr uint32_t kKTile = 2 * kKChunk;        // a key tile: 64 keys x 128 bf16
-constexpr uint32_t kQOff = 0;                   // 2 M tiles
-constexpr uint32_t kKOff = 2 * kQTile;          // kStages K tiles
+constexpr uint32_t kQOff = 0;
+constexpr uint32_t kKOff = kQTile;              // kStages K tiles
 constexpr uint32_t kVOff = kKOff + kStages * kKTile;
 constexpr uint32_t kBarOff = kVOff + kStages * kKTile;
 constexpr int kMaxList = 258;
 constexpr uint32_t kSmemBytes = kBarOff + 1024 + 8 * kMaxList + 2048;   // + alignment slack
 constexpr unsigned long long kWaitNs = 2000000000ull;
+constexpr uint32_t kTmemCols = 256;
 
 // barrier slots (uint64 each)
 enum {
     B_Q = 0,
-    B_KF = 1,                   // [kStages]
-    B_VF = B_KF + kStages,      // [kStages]
-    B_FREE = B_VF + kStages,    // [kStages]
-    B_S = B_FREE + kStages,     // [2 M tiles][2 buffers]
-    B_P = B_S + 4,              // [2][2], 128 arrivals each
-    B_O = B_P + 4,              // [2]
-    B_END = B_O + 2,
+    B_KF = 1,                   // [kStages] K tile landed
+    B_VF = B_KF + kStages,      // [kStages] V tile landed
+    B_KE = B_VF + kStages,      // [kStages] K tile consumed (QK done)
+    B_VE = B_KE + kStages,      // [kStages] V tile consumed (PV done)
+    B_S = B_VE + kStages,       // [2 buffers] S ready
+    B_P = B_S + 2,              // [2 buffers] P ready, 128 arrivals each
+    B_O = B_P + 2,              // one phase per PV
+    B_END = B_O + 1,
     NBAR
 };
 
@@ -210,7 +212,7 @@ __device__ __forceinline__ float ex2(float x) {
 // ---------------------------------------------------------------------------
 // kernel
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, TcArgs a) {
     constexpr float kLog2e = 1.4426950408889634f;
@@ -228,7 +230,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // CTA -> (batch, kv-head, tile, head pair); larger tiles first
+    // CTA -> (batch, kv-head, tile, head group); larger tiles first
     int u = blockIdx.x;
     const int pair = u % a.npair;
     u /= a.npair;
@@ -244,7 +246,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
     // ---- set-up -----------------------------------------------------------
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i >= B_P && i < B_P + 4) ? 128 : 1);
+        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == B_P || i == B_P + 1) ? 128 : 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -259,7 +261,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         gate_s[tid] = ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[tid] - sl[cnt - 1]) * kLog2e : 0.f;
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot)));
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "n"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -275,48 +278,39 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
-            mbar_expect_tx(bar(B_Q), 2 * kQTile);
-            for (int m = 0; m < 2; ++m) {
-                for (int c = 0; c < 2; ++c) {
-                    if (s.bs == 64) {
-                        for (int e = 0; e < 2; ++e) {
-                            const int h = h0 + 2 * m + e;
-                            const int y = ((b * s.Hq + h) * s.N) + j * 64;
-                            tma_load_2d(sbase + kQOff + m * kQTile + c * kQChunk + e * 8192, &tmQ, bar(B_Q), 64 * c,
-                                        y);
-                        }
-                    } else {
-                        const int h = h0 + m;
-                        const int y = ((b * s.Hq + h) * s.N) + j * 128;
-                        for (int e = 0; e < 2; ++e)
-                            tma_load_2d(sbase + kQOff + m * kQTile + c * kQChunk + e * 8192, &tmQ, bar(B_Q), 64 * c,
-                                        y + 64 * e);
-                    }
+            mbar_expect_tx(bar(B_Q), kQTile);
+            for (int c = 0; c < 2; ++c)
+                for (int e = 0; e < 2; ++e) {
+                    // block 64: rows of heads h0 and h0+1; block 128: rows 0-63 and 64-127 of head h0
+                    const int y = s.bs == 64 ? ((b * s.Hq + h0 + e) * s.N) + j * 64
+                                             : ((b * s.Hq + h0) * s.N) + j * 128 + 64 * e;
+                    tma_load_2d(sbase + kQOff + c * kQChunk + e * 8192, &tmQ, bar(B_Q), 64 * c, y);
                 }
-            }
             const int kvbase = (b * s.Hkv + g) * s.N;
-            int issued = 0;
+            int nk = 0, nv = 0;   // K and V tiles issued
             for (int t = 0; t < T; ++t) {
-                const int st = t % kStages;
-                if (t >= kStages && !mbar_wait(bar(B_FREE + st), ((t / kStages) - 1) & 1, abort_flag, a.status))
-                    break;
+                const int st = t % kStages, use = t / kStages;
                 const int blk = max(0, blk_s[t / sub]);
                 const int y = kvbase + blk * s.bs + (t % sub) * 64;
-                const uint32_t kdst = sbase + kKOff + st * kKTile, vdst = sbase + kVOff + st * kKTile;
+                if (t >= kStages && !mbar_wait(bar(B_KE + st), (use - 1) & 1, abort_flag, a.status)) break;
                 mbar_expect_tx(bar(B_KF + st), kKTile);
-                for (int ch = 0; ch < 2; ++ch) tma_load_2d(kdst + ch * kKChunk, &tmK, bar(B_KF + st), 64 * ch, y);
+                for (int ch = 0; ch < 2; ++ch)
+                    tma_load_2d(sbase + kKOff + st * kKTile + ch * kKChunk, &tmK, bar(B_KF + st), 64 * ch, y);
+                nk = t + 1;
+                if (t >= kStages && !mbar_wait(bar(B_VE + st), (use - 1) & 1, abort_flag, a.status)) break;
                 mbar_expect_tx(bar(B_VF + st), kKTile);
-                for (int ch = 0; ch < 2; ++ch) tma_load_2d(vdst + ch * kKChunk, &tmV, bar(B_VF + st), 64 * ch, y);
-                issued = t + 1;
+                for (int ch = 0; ch < 2; ++ch)
+                    tma_load_2d(sbase + kVOff + st * kKTile + ch * kKChunk, &tmV, bar(B_VF + st), 64 * ch, y);
+                nv = t + 1;
             }
             if (*abort_flag) {
                 // let the copies in flight land before the CTA exits (bounded)
                 volatile int never = 0;
                 mbar_wait(bar(B_Q), 0, &never, a.status);
-                for (int t = max(0, issued - kStages); t < issued; ++t) {
+                for (int t = max(0, nk - kStages); t < nk; ++t)
                     mbar_wait(bar(B_KF + t % kStages), (t / kStages) & 1, &never, a.status);
+                for (int t = max(0, nv - kStages); t < nv; ++t)
                     mbar_wait(bar(B_VF + t % kStages), (t / kStages) & 1, &never, a.status);
-                }
             }
         }
     } else if (warp == 1) {
@@ -326,50 +320,45 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             constexpr uint32_t idq = idesc_bf16(false, 64), idp = idesc_bf16(true, 128);
             bool ok = mbar_wait(bar(B_Q), 0, abort_flag, a.status);
             tc_fence_after();
-            // S_m(t) = Q_m K_t^T into buffer t & 1 of M tile m
-            auto qk = [&](int m, int t) {
+            const uint32_t qa = sbase + kQOff;
+            // S(t) = Q K_t^T into buffer t & 1; frees K stage when done
+            auto qk = [&](int t) {
                 const int st = t % kStages;
-                const uint32_t qa = sbase + kQOff + m * kQTile, kb = sbase + kKOff + st * kKTile;
-                const uint32_t dS = tmem + m * 256 + (t & 1) * 64;
+                const uint32_t kb = sbase + kKOff + st * kKTile;
+                const uint32_t dS = tmem + (t & 1) * 64;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     mma_ss(dS, desc_k_sw128(qa + (k >> 2) * kQChunk + (k & 3) * 32),
                            desc_k_sw128(kb + (k >> 2) * kKChunk + (k & 3) * 32), idq, k > 0);
-                mma_commit(bar(B_S + 2 * m + (t & 1)));
+                mma_commit(bar(B_S + (t & 1)));
+                mma_commit(bar(B_KE + st));
             };
-            // O_m += P_m(t) V_t, P read from the first 32 columns of S buffer t & 1
-            auto pv = [&](int m, int t) {
+            // O += P(t) V_t, P read from the first 32 columns of S buffer t & 1
+            auto pv = [&](int t) {
                 const int st = t % kStages;
                 const uint32_t vb = sbase + kVOff + st * kKTile;
-                const uint32_t aP = tmem + m * 256 + (t & 1) * 64, dO = tmem + m * 256 + 128;
+                const uint32_t aP = tmem + (t & 1) * 64, dO = tmem + 128;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_ts(dO, aP + 8 * k, desc_mn_sw128(vb + k * 2048, kKChunk), idp, (t > 0 || k > 0));
-                mma_commit(bar(B_O + m));
+                mma_commit(bar(B_O));
+                mma_commit(bar(B_VE + st));
             };
             for (int t = 0; ok && t < min(2, T); ++t) {
                 if (!(ok = mbar_wait(bar(B_KF + t % kStages), (t / kStages) & 1, abort_flag, a.status))) break;
                 tc_fence_after();
-                qk(0, t);
-                qk(1, t);
+                qk(t);
             }
             for (int i = 0; ok && i < T; ++i) {
-                const int st = i % kStages, ph = (i / kStages) & 1;
+                if (!(ok = mbar_wait(bar(B_P + (i & 1)), (i >> 1) & 1, abort_flag, a.status))) break;
+                if (!(ok = mbar_wait(bar(B_VF + i % kStages), (i / kStages) & 1, abort_flag, a.status))) break;
+                tc_fence_after();
+                pv(i);
                 const int t2 = i + 2;
-                const bool next = t2 < T;
-                if (!(ok = mbar_wait(bar(B_VF + st), ph, abort_flag, a.status))) break;
-                for (int m = 0; m < 2; ++m) {
-                    if (!(ok = mbar_wait(bar(B_P + 2 * m + (i & 1)), (i >> 1) & 1, abort_flag, a.status))) break;
+                if (t2 < T) {
+                    if (!(ok = mbar_wait(bar(B_KF + t2 % kStages), (t2 / kStages) & 1, abort_flag, a.status))) break;
                     tc_fence_after();
-                    pv(m, i);
-                    if (m == 1) mma_commit(bar(B_FREE + st));
-                    if (next) {
-                        if (m == 0 &&
-                            !(ok = mbar_wait(bar(B_KF + t2 % kStages), (t2 / kStages) & 1, abort_flag, a.status)))
-                            break;
-                        tc_fence_after();
-                        qk(m, t2);
-                    }
+                    qk(t2);
                 }
             }
             // drain: every MMA issued above has completed once this arrives
@@ -381,23 +370,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     } else if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
     } else {
-        // ---- softmax warpgroups ---------------------------------------------
+        // ---- softmax warpgroup ----------------------------------------------
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-        const int m = (warp - 4) >> 2;                  // M tile
         const int q4 = warp & 3;                         // TMEM lane quarter of this warp
         const int r = 32 * q4 + lane;                    // row within the M tile
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-        const uint32_t tM = tmem + lane_off + m * 256, tO = tM + 128;
+        const uint32_t tM = tmem + lane_off, tO = tM + 128;
         int head, ri;
-        if (s.bs == 64) { head = h0 + 2 * m + (r >> 6); ri = r & 63; }
-        else { head = h0 + m; ri = r; }
+        if (s.bs == 64) { head = h0 + (r >> 6); ri = r & 63; }
+        else { head = h0; ri = r; }
         const int qi = j * s.bs + ri;                    // query position of this row
         const bool causal = s.flags & SA_CAUSAL;
         float m_run = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int i = 0; i < T; ++i) {
             const uint32_t tS = tM + (i & 1) * 64;
-            ok = mbar_wait(bar(B_S + 2 * m + (i & 1)), (i >> 1) & 1, abort_flag, a.status);
+            ok = mbar_wait(bar(B_S + (i & 1)), (i >> 1) & 1, abort_flag, a.status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
             float x[64];
@@ -433,7 +421,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 if (__any_sync(0xffffffffu, need)) {
                     // PV(i-2) is done (S(i) was computed after it), so PV(i-1)
                     // is either running or done: parity (i-1) is unambiguous
-                    ok = mbar_wait(bar(B_O + m), (i - 1) & 1, abort_flag, a.status);
+                    ok = mbar_wait(bar(B_O), (i - 1) & 1, abort_flag, a.status);
                     if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                     tc_fence_after();
                     const float corr = need ? ex2(m_run - m_new) : 1.f;
@@ -469,7 +457,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             tmem_st32(tS, pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(B_P + 2 * m + (i & 1)));
+            mbar_arrive(bar(B_P + (i & 1)));
         }
         // ---- epilogue: O / l -> bf16, LSE ---------------------------------
         // O is final once the MMA thread's drain barrier (committed after its
@@ -515,7 +503,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kTmemCols));
     }
 }
 
@@ -552,7 +540,7 @@ bool prefill_tc_supported(const Shape &s) {
     if (s.dtype != SA_BF16 || s.d != 128) return false;
     if (s.flags & (SA_HIER | SA_SELECT_PER_QHEAD)) return false;
     if (s.bs != 64 && s.bs != 128) return false;
-    const int hc = 256 / s.bs;
+    const int hc = 128 / s.bs;   // query heads per CTA
     if (s.G % hc) return false;
     if (s.cap > kMaxList) return false;
     const char *e = getenv("SPARSE_ATTN_PREFILL_PATH");
@@ -576,7 +564,7 @@ cudaError_t launch_prefill_tc(const Shape &s, const void *Q, const void *K, cons
     a.O = (__nv_bfloat16 *)O;
     a.lse = lse;
     a.status = status;
-    a.hc = 256 / s.bs;
+    a.hc = 128 / s.bs;
     a.npair = s.G / a.hc;
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);

@@ -115,7 +115,7 @@ FLAG_CASES = [
 
 FLAG_SHAPES = {
     "fp32_g2": dict(Hq=4, Hkv=2, block=64, dtype="fp32"),
-    "bf16_g2": dict(Hq=4, Hkv=2, block=64, dtype="bf16"),       # CUDA-core kernel
+    "bf16_g1": dict(Hq=2, Hkv=2, block=64, dtype="bf16"),       # CUDA-core kernel (odd group)
     "bf16_g4": dict(Hq=8, Hkv=2, block=64, dtype="bf16"),       # tensor-core kernel (block 64)
     "bf16_g2_b128": dict(Hq=4, Hkv=2, block=128, dtype="bf16"),  # tensor-core kernel (block 128)
 }
@@ -220,6 +220,8 @@ TC_CASES = {
     "b64_g8": W["gated_prefill_32k"].scaled(N=3000, Hq=16, Hkv=2),
     "b128_g4": W["long_prefill_256k"].scaled(N=8192, Hq=8, Hkv=2),
     "b128_ragged": W["long_prefill_256k"].scaled(N=5000, Hq=4, Hkv=2, top_k=5),
+    "b64_g2": W["gated_prefill_32k"].scaled(N=3000, Hq=4, Hkv=2),
+    "b128_g1": W["long_prefill_256k"].scaled(N=4096, Hq=2, Hkv=2),
     "b64_big_k": W["gated_prefill_32k"].scaled(N=8192, Hq=8, Hkv=2, top_k=100),
     "b64_odd_k": W["gated_prefill_32k"].scaled(N=4096, Hq=8, Hkv=2, top_k=7),
 }
