@@ -521,7 +521,7 @@ def run_ours(args, ranks):
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
         if not args.no_secondary:
             sec = {}
-            for name in ("gated_decode_128k", "hils_decode_1m", "long_prefill_256k"):
+            for name in ("gated_decode_128k", "hils_decode_1m", "long_prefill_256k", "hils_prefill_32k"):
                 try:
                     sec[name] = (secondary_decode if inputs.WORKLOADS[name].kind == "decode" else
                                  secondary_prefill)(name, args, pk, psrc)

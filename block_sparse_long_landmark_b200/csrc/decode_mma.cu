@@ -116,7 +116,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // byte offset of (row, 16-byte unit u) in a 64-row box with 128-byte swizzle
 __device__ __forceinline__ uint32_t swz(int row, int u) { return row * 128 + ((u ^ (row & 7)) << 4); }
 
-__global__ void __launch_bounds__(kThreadsD)
+__global__ void __launch_bounds__(kThreadsD, 3)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DmArgs a) {
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr float kLn2 = 0.6931471805599453f;

@@ -258,7 +258,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         if (!ok) set_status(a.status, kStatusBadIndex);
         blk_s[tid] = ok ? blk : -1;
         const bool forced = (blk == j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
-        gate_s[tid] = ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[tid] - sl[cnt - 1]) * kLog2e : 0.f;
+        // gated: the log2-unit gate of the block; hierarchical: its log2-unit retrieval score
+        gate_s[tid] = (s.flags & SA_HIER) ? sl[tid] * kLog2e
+                      : ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[tid] - sl[cnt - 1]) * kLog2e : 0.f;
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -383,6 +385,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const bool causal = s.flags & SA_CAUSAL;
         float m_run = -CUDART_INF_F, l = 0.f;
         bool ok = true;
+        // hierarchical mode ([HiLS]): every block gets its own softmax, and the
+        // block outputs are weighted by softmax_b(s_b).  With M the largest
+        // retrieval score of the list (known before the first tile), block b
+        // enters O as P_b V_b * 2^(s_b - M) / l_b and W sums 2^(s_b - M), so
+        // O never needs rescaling and the result is O / W.
+        const bool hier = s.flags & SA_HIER;
+        float mh = -CUDART_INF_F;
+        if (hier) {
+            for (int c = 0; c < cnt; ++c)
+                if (blk_s[c] >= 0) mh = fmaxf(mh, gate_s[c]);
+            m_run = mh;
+        }
         for (int i = 0; i < T; ++i) {
             const uint32_t tS = tM + (i & 1) * 64;
             ok = mbar_wait(bar(B_S + (i & 1)), (i >> 1) & 1, abort_flag, a.status);
@@ -412,6 +426,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     mx = fmaxf(mx, x[k]);
                 }
                 mx = mx == -CUDART_INF_F ? mx : fmaf(mx, qk_scale, gl);
+            }
+            if (hier) {
+                // this block's own softmax (scores without gate), weighted by its retrieval score
+                const float mb = mx == -CUDART_INF_F ? 0.f : mx - gl;   // mx carried the score: drop it
+                float lb = 0.f;
+#pragma unroll
+                for (int k = 0; k < 64; ++k) {
+                    x[k] = ex2(fmaf(x[k], qk_scale, -mb));
+                    lb += x[k];
+                }
+                const float wb = lb > 0.f ? ex2(gl - mh) : 0.f;
+                const float f = lb > 0.f ? wb / lb : 0.f;
+                l += wb;
+                uint32_t pk[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * k] * f, x[2 * k + 1] * f);
+                    pk[k] = *reinterpret_cast<uint32_t *>(&h2);
+                }
+                tmem_st32(tS, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B_P + (i & 1)));
+                continue;
             }
             const float m_new = fmaxf(m_run, mx);
             if (i == 0) {
@@ -538,7 +576,8 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows) {
 
 bool prefill_tc_supported(const Shape &s) {
     if (s.dtype != SA_BF16 || s.d != 128) return false;
-    if (s.flags & (SA_HIER | SA_SELECT_PER_QHEAD)) return false;
+    if (s.flags & SA_SELECT_PER_QHEAD) return false;
+    if ((s.flags & SA_HIER) && s.bs != 64) return false;   // hierarchical: one block per key tile
     if (s.bs != 64 && s.bs != 128) return false;
     const int hc = 128 / s.bs;   // query heads per CTA
     if (s.G % hc) return false;

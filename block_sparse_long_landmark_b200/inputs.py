@@ -77,6 +77,9 @@ WORKLOADS = {
     # B1 N262144 block 128 top-16, bf16.
     "long_prefill_256k": Workload("long_prefill_256k", "prefill", 1, 32, 8, 128, 262144, 128, 16, "bf16", False,
                                   0.5, 3, "every_4096", 4),
+    # the 32K prefill in hierarchical mode (per-block softmax, retrieval-score weights).
+    "hils_prefill_32k": Workload("hils_prefill_32k", "prefill", 1, 32, 8, 128, 32768, 64, 16, "bf16", True,
+                                 0.5, 5, "per_tile", 8),
     # 8 sequences x one query at context 1048576, block 64 top-64, hierarchical.
     "hils_decode_1m": Workload("hils_decode_1m", "decode", 8, 32, 8, 128, 1048576, 64, 64, "bf16", True,
                                0.5, 4, "per_seq", 64),

@@ -221,6 +221,8 @@ TC_CASES = {
     "b128_g4": W["long_prefill_256k"].scaled(N=8192, Hq=8, Hkv=2),
     "b128_ragged": W["long_prefill_256k"].scaled(N=5000, Hq=4, Hkv=2, top_k=5),
     "b64_g2": W["gated_prefill_32k"].scaled(N=3000, Hq=4, Hkv=2),
+    "b64_hier": W["gated_prefill_32k"].scaled(N=4096, Hq=8, Hkv=2, hier=True),
+    "b64_hier_ragged": W["gated_prefill_32k"].scaled(N=3001, Hq=4, Hkv=2, hier=True, top_k=7),
     "b128_g1": W["long_prefill_256k"].scaled(N=4096, Hq=2, Hkv=2),
     "b64_big_k": W["gated_prefill_32k"].scaled(N=8192, Hq=8, Hkv=2, top_k=100),
     "b64_odd_k": W["gated_prefill_32k"].scaled(N=4096, Hq=8, Hkv=2, top_k=7),
