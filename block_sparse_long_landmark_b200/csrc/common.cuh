@@ -109,6 +109,9 @@ cudaError_t launch_landmarks(const Shape &s, const void *K, void *L, cudaStream_
 cudaError_t launch_select(const Shape &s, bool decode, const void *Q, const void *L, int32_t *idx, float *score,
                           int32_t *count, void *ws, size_t ws_bytes, cudaStream_t st);
 size_t select_workspace(const Shape &s, bool decode);
+bool select_tiles_supported(const Shape &s);
+cudaError_t launch_select_tiles(const Shape &s, const void *Q, const void *L, int32_t *idx, float *score,
+                                int32_t *count, unsigned *status, cudaStream_t st);
 cudaError_t launch_prefill_simt(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
                                 const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
                                 cudaStream_t st);

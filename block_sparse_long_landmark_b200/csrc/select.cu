@@ -481,6 +481,9 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
 cudaError_t launch_select(const Shape &s, bool decode, const void *Q, const void *L, int32_t *idx, float *score,
                           int32_t *count, void *ws, size_t ws_bytes, cudaStream_t st) {
     (void)ws_bytes;
+    // prefill: eight tiles per CTA share one landmark scan (select_tiles.cu)
+    if (!decode && select_tiles_supported(s))
+        return launch_select_tiles(s, Q, L, idx, score, count, (unsigned *)ws, st);
     return s.dtype == SA_BF16 ? run<__nv_bfloat16>(s, decode, Q, L, idx, score, count, ws, st)
                               : run<float>(s, decode, Q, L, idx, score, count, ws, st);
 }
