@@ -319,12 +319,27 @@ __global__ void __launch_bounds__(kSelThreads, 5) select_chunk_kernel(SelArgs a)
     const int c1 = min(local, c0 + a.CH);
     const int n = max(0, c1 - c0);
 
-    pool_query<T, VPR>(a, b, hs, j, sm, red);
     float qv[EPV];
-    {
-        const int cv = (threadIdx.x & 31) % VPR;
+    if (a.decode) {
+        // one query per head: every lane averages its own slice over the
+        // group's heads (no shared memory, no barrier before the scan)
+        const int cvq = (threadIdx.x & 31) % VPR;
+        const int hq0 = (s.flags & SA_SELECT_PER_QHEAD) ? hs : hs * s.G;
 #pragma unroll
-        for (int i = 0; i < EPV; ++i) qv[i] = sm.qbar[cv * EPV + i];
+        for (int i = 0; i < EPV; ++i) qv[i] = 0.f;
+        for (int hh = 0; hh < s.heads_per; ++hh) {
+            float f[EPV];
+            load16((const T *)a.Q + ((size_t)b * s.Hq + hq0 + hh) * d + cvq * EPV, f);
+#pragma unroll
+            for (int i = 0; i < EPV; ++i) qv[i] += f[i];
+        }
+#pragma unroll
+        for (int i = 0; i < EPV; ++i) qv[i] /= (float)s.heads_per;
+    } else {
+        pool_query<T, VPR>(a, b, hs, j, sm, red);
+        const int cvq = (threadIdx.x & 31) % VPR;
+#pragma unroll
+        for (int i = 0; i < EPV; ++i) qv[i] = sm.qbar[cvq * EPV + i];
     }
     const T *Lg = (const T *)a.L + ((size_t)b * s.Hkv + g) * s.nb * d;
     // rows are handed out per warp so that every lane of a warp takes the

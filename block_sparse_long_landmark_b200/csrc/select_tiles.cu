@@ -19,6 +19,7 @@
 //   3. warp w radix-selects its tile's top-K with a per-warp histogram
 //      (warp-aggregated atomics, __syncwarp only) and writes the list.
 #include "common.cuh"
+#include "warp_select.cuh"
 
 namespace sa {
 namespace {
@@ -36,77 +37,6 @@ struct TilesArgs {
     unsigned *status;
     int ngroups;                 // ceil(nb / kTpc)
 };
-
-// Exact top-k (n > k) of keys[0..n) for one warp; T = threshold key,
-// take_eq = how many keys equal to T are taken (lowest positions first).
-__device__ void warp_radix_select(const uint32_t *keys, int n, int k, int *hist, uint32_t &T, int &take_eq) {
-    const int lane = threadIdx.x & 31;
-    uint32_t prefix = 0, mask = 0;
-    int remaining = k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int b = lane; b < 256; b += 32) hist[b] = 0;
-        __syncwarp();
-        for (int i0 = 0; i0 < n; i0 += 32) {
-            const int i = i0 + lane;
-            const uint32_t x = i < n ? keys[i] : 0u;
-            const bool take = i < n && (x & mask) == prefix;
-            const unsigned act = __ballot_sync(0xffffffffu, take);
-            if (take) {
-                const int digit = (int)((x >> shift) & 255);
-                const unsigned same = __match_any_sync(act, digit);
-                if (lane == __ffs(same) - 1) atomicAdd(&hist[digit], __popc(same));
-            }
-        }
-        __syncwarp();
-        const int hi = 255 - 8 * lane;
-        int loc = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) loc += hist[hi - q];
-        int incl = loc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const int excl = incl - loc;
-        int digit = 0, above = 0;
-        if (excl < remaining && remaining <= incl) {
-            int cum = excl;
-            for (int q = 0; q < 8; ++q) {
-                const int c = hist[hi - q];
-                if (cum + c >= remaining) {
-                    digit = hi - q;
-                    above = cum;
-                    break;
-                }
-                cum += c;
-            }
-        }
-        const unsigned who = __ballot_sync(0xffffffffu, excl < remaining && remaining <= incl);
-        const int src = __ffs(who) - 1;
-        digit = __shfl_sync(0xffffffffu, digit, src);
-        above = __shfl_sync(0xffffffffu, above, src);
-        remaining -= above;
-        prefix |= (uint32_t)digit << shift;
-        mask |= 255u << shift;
-        __syncwarp();
-    }
-    T = prefix;
-    take_eq = remaining;
-}
-
-// Warp exclusive prefix sum.
-__device__ __forceinline__ int warp_excl(int v, int &total) {
-    const int lane = threadIdx.x & 31;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    total = __shfl_sync(0xffffffffu, incl, 31);
-    return incl - v;
-}
 
 template <typename T, int VPR>
 __global__ void __launch_bounds__(kThreadsT) select_tiles_kernel(TilesArgs a) {
@@ -242,41 +172,7 @@ __global__ void __launch_bounds__(kThreadsT) select_tiles_kernel(TilesArgs a) {
     const int n = max(0, j - first);
     const uint32_t *cand = kw + first;
     int *op = outp + warp * max(s.top_k, 1);
-    int nsel = 0;
-    if (s.top_k > 0 && n > 0) {
-        if (n <= s.top_k) {
-            for (int i = lane; i < n; i += 32) op[i] = i;
-            nsel = n;
-        } else {
-            uint32_t Tk;
-            int take_eq;
-            warp_radix_select(cand, n, s.top_k, hist + warp * 256, Tk, take_eq);
-            const int seg = (n + 31) / 32;
-            const int i0 = min(n, lane * seg), i1 = min(n, i0 + seg);
-            int neq = 0;
-            for (int i = i0; i < i1; ++i) neq += cand[i] == Tk;
-            int tot;
-            const int eq_base = warp_excl(neq, tot);
-            int cntsel = 0;
-            {
-                int e = eq_base;
-                for (int i = i0; i < i1; ++i) {
-                    const uint32_t x = cand[i];
-                    cntsel += x > Tk || (x == Tk && e < take_eq);
-                    e += x == Tk;
-                }
-            }
-            int pos = warp_excl(cntsel, nsel);
-            {
-                int e = eq_base;
-                for (int i = i0; i < i1; ++i) {
-                    const uint32_t x = cand[i];
-                    if (x > Tk || (x == Tk && e < take_eq)) op[pos++] = i;
-                    e += x == Tk;
-                }
-            }
-        }
-    }
+    const int nsel = warp_topk_positions(cand, n, s.top_k, hist + warp * 256, op);
     __syncwarp();
     const size_t u = ((size_t)b * s.Hsel + hs) * s.nb + j;
     int32_t *idx = a.idx + u * s.cap;
