@@ -247,22 +247,35 @@ def prefill_flops(wl, cnt) -> float:
     return pairs * 4.0 * (G * wl.block) * wl.block * wl.d
 
 
-def decode_case(wl, device):
+def decode_case(wl, device, lens=None):
+    """Decode inputs; with `lens` a ragged batch (sequence b holds lens[b]
+    keys of the cache) that runs through the varlen entry points."""
     import block_sparse_long_landmark_b200 as sa
     from block_sparse_long_landmark_b200 import inputs
     p = sa.params_for(wl)
     q, K, V = inputs.make_decode(wl, device=device)
     ws = sa.workspace(p, device=device)
-    L = sa.landmarks(p, K)
-    sel = sa._sel_out(p, True, device)
-    o = torch.empty_like(q)
-    lse = torch.empty(wl.B, wl.Hq, dtype=torch.float32, device=device)
-    return p, dict(q=q, K=K, V=V, ws=ws, L=L, sel=sel, o=o, lse=lse)
+    t = dict(q=q, K=K, V=V, ws=ws)
+    if lens is None:
+        t["L"] = sa.landmarks(p, K)
+    else:
+        t["sl"] = torch.tensor(lens, dtype=torch.int32, device=device)
+        t["L"] = torch.zeros(wl.B, wl.Hkv, wl.nb, wl.d, dtype=K.dtype, device=device)
+        sa.landmarks_update(p, K, t["L"], seq_len=t["sl"])
+    t["sel"] = sa._sel_out(p, True, device)
+    t["o"] = torch.empty_like(q)
+    t["lse"] = torch.empty(wl.B, wl.Hq, dtype=torch.float32, device=device)
+    return p, t
 
 
 def decode_step(p, t, timer=None):
     import block_sparse_long_landmark_b200 as sa
     tm = timer or (lambda n, f: f())
+    if "sl" in t:
+        tm("select_decode", lambda: sa.select_decode_varlen(p, t["q"], t["L"], t["sl"], t["ws"], out=t["sel"]))
+        tm("decode", lambda: sa.decode_varlen(p, t["q"], t["K"], t["V"], t["sl"], *t["sel"], t["ws"],
+                                              out=(t["o"], t["lse"])))
+        return
     tm("select_decode", lambda: sa.select_decode(p, t["q"], t["L"], t["ws"], out=t["sel"]))
     tm("decode", lambda: sa.decode(p, t["q"], t["K"], t["V"], *t["sel"], t["ws"], out=(t["o"], t["lse"])))
 
@@ -445,8 +458,13 @@ def secondary_prefill(name, args, pk, psrc):
 
 
 def secondary_decode(name, args, pk, psrc):
-    wl = _wl(name, args)
-    p, t = decode_case(wl, "cuda")
+    varlen = name.endswith("_varlen")
+    wl = _wl(name[:-len("_varlen")] if varlen else name, args)
+    lens = None
+    if varlen:
+        # ragged batch: lengths uniform in [N/2, N], seeded
+        lens = np.random.default_rng(11).integers(wl.N // 2, wl.N + 1, size=wl.B)
+    p, t = decode_case(wl, "cuda", lens)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     ranks1 = Ranks.single()
     steps = max(3, args.steps)
@@ -454,15 +472,19 @@ def secondary_decode(name, args, pk, psrc):
                                           ranks1, flush)
     esz = 2 if wl.dtype == "bf16" else 4
     cnt = t["sel"][2].to(torch.int64)
-    local = (wl.N - 1) // wl.block
-    scan_bytes = wl.B * wl.Hkv * (local + 1) * wl.d * esz
+    if lens is None:
+        scan_bytes = wl.B * wl.Hkv * ((wl.N - 1) // wl.block + 1) * wl.d * esz
+    else:
+        scan_bytes = sum(wl.Hkv * ((int(n) - 1) // wl.block + 1) * wl.d * esz for n in lens)
     gather_bytes = float(cnt.sum().item()) * wl.block * wl.d * esz * 2
     ach_dec = gather_bytes / (kms["decode"] / 1e3) / 1e9
     ach_sel = scan_bytes / (kms["select_decode"] / 1e3) / 1e9
     step_ach = (scan_bytes + gather_bytes) / (el / steps / 1e3) / 1e9
     hbm = pk["hbm_gbs"]
+    cfg = workload_config(wl, {"seq_len_min": int(min(lens)), "seq_len_mean": float(np.mean(lens)),
+                               "varlen": True} if varlen else None)
     out = {"metric": "decode queries/s", "value": wl.B / (el / steps / 1e3), "unit": "queries/s",
-           "ms_per_step": el / steps, "kernels_ms": kms, "config": workload_config(wl), "gpu_launches": launches,
+           "ms_per_step": el / steps, "kernels_ms": kms, "config": cfg, "gpu_launches": launches,
            "roofline": {"bound": "hbm", "achieved": step_ach, "peak": hbm, "unit": "GB/s", "frac": step_ach / hbm,
                         "peak_source": psrc, "bytes_per_step": scan_bytes + gather_bytes,
                         "traffic": None},
@@ -487,7 +509,8 @@ def run_ours(args, ranks):
     pk, psrc = peaks()
     if args.only:
         # one workload alone (small profiling cases): a short report, no baselines
-        fn = secondary_decode if inputs.WORKLOADS[args.only].kind == "decode" else secondary_prefill
+        kind = inputs.WORKLOADS[args.only.replace("_varlen", "")].kind
+        fn = secondary_decode if kind == "decode" else secondary_prefill
         print(json.dumps({"only": args.only, **fn(args.only, args, pk, psrc)}), flush=True)
         return 0
     base = inputs.WORKLOADS[args.workload]
@@ -521,10 +544,11 @@ def run_ours(args, ranks):
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
         if not args.no_secondary:
             sec = {}
-            for name in ("gated_decode_128k", "hils_decode_1m", "long_prefill_256k", "hils_prefill_32k"):
+            for name in ("gated_decode_128k", "hils_decode_1m", "long_prefill_256k", "hils_prefill_32k",
+                         "gated_decode_128k_varlen"):
                 try:
-                    sec[name] = (secondary_decode if inputs.WORKLOADS[name].kind == "decode" else
-                                 secondary_prefill)(name, args, pk, psrc)
+                    kind = inputs.WORKLOADS[name.replace("_varlen", "")].kind
+                    sec[name] = (secondary_decode if kind == "decode" else secondary_prefill)(name, args, pk, psrc)
                 except torch.cuda.OutOfMemoryError as e:   # pragma: no cover
                     sec[name] = {"error": f"out of memory: {e}"}
                 torch.cuda.empty_cache()

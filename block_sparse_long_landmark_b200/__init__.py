@@ -30,6 +30,7 @@ EXPORTS = (
     "sparse_attn_prefill", "sparse_attn_decode", "sparse_attn_check_status", "sparse_attn_status_string",
     "sparse_attn_version", "sparse_attn_launch_count", "sparse_attn_decode_static",
     "sparse_attn_prefill_kernel", "sparse_attn_last_cuda_error", "sparse_attn_cuda_error_string",
+    "sparse_attn_landmarks_update", "sparse_attn_select_decode_varlen", "sparse_attn_decode_varlen",
 )
 
 
@@ -81,6 +82,12 @@ def lib() -> ctypes.CDLL:
             for n in EXPORTS[1:7]:
                 getattr(L, n).restype = i
             L.sparse_attn_version.restype = i
+            L.sparse_attn_landmarks_update.argtypes = [P, vp, vp, vp, vp, vp]
+            L.sparse_attn_landmarks_update.restype = i
+            L.sparse_attn_select_decode_varlen.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.sparse_attn_select_decode_varlen.restype = i
+            L.sparse_attn_decode_varlen.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.sparse_attn_decode_varlen.restype = i
             L.sparse_attn_last_cuda_error.argtypes = []
             L.sparse_attn_last_cuda_error.restype = i
             L.sparse_attn_cuda_error_string.argtypes = [i]
@@ -129,6 +136,20 @@ def sparse_attn_prefill_kernel(p) -> int:
 
 def sparse_attn_decode_static(p, q, K, V, idx, score, count, o, lse, stream) -> int:
     return lib().sparse_attn_decode_static(ctypes.byref(p), q, K, V, idx, score, count, o, lse, stream)
+
+
+def sparse_attn_landmarks_update(p, K, L, seq_len, first_block, stream) -> int:
+    return lib().sparse_attn_landmarks_update(ctypes.byref(p), K, L, seq_len, first_block, stream)
+
+
+def sparse_attn_select_decode_varlen(p, q, L, seq_len, idx, score, count, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_select_decode_varlen(ctypes.byref(p), q, L, seq_len, idx, score, count, ws, ws_bytes,
+                                                  stream)
+
+
+def sparse_attn_decode_varlen(p, q, K, V, seq_len, idx, score, count, o, lse, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_decode_varlen(ctypes.byref(p), q, K, V, seq_len, idx, score, count, o, lse, ws,
+                                           ws_bytes, stream)
 
 
 def sparse_attn_check_status(ws, stream):
@@ -271,6 +292,34 @@ def decode_static(p, q, K, V, idx, sc, cnt, out=None, stream=None):
         o, lse = out
     _check(sparse_attn_decode_static(p, _ptr(q), _ptr(K), _ptr(V), _ptr(idx), _ptr(sc), _ptr(cnt), _ptr(o),
                                      _ptr(lse), _stream(stream)), "sparse_attn_decode_static")
+    return o, lse
+
+
+def landmarks_update(p, K, L, seq_len=None, first_block=None, stream=None):
+    """Refresh the landmarks of blocks first_block[b] .. (for appends) over
+    each sequence's own length; int32 device tensors or None."""
+    _check(sparse_attn_landmarks_update(p, _ptr(K), _ptr(L), _ptr(seq_len), _ptr(first_block), _stream(stream)),
+           "sparse_attn_landmarks_update")
+    return L
+
+
+def select_decode_varlen(p, q, L, seq_len, ws, out=None, stream=None):
+    idx, sc, cnt = out if out is not None else _sel_out(p, True, q.device)
+    _check(sparse_attn_select_decode_varlen(p, _ptr(q), _ptr(L), _ptr(seq_len), _ptr(idx), _ptr(sc), _ptr(cnt),
+                                            _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_select_decode_varlen")
+    return idx, sc, cnt
+
+
+def decode_varlen(p, q, K, V, seq_len, idx, sc, cnt, ws, out=None, stream=None):
+    torch = _torch()
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(p.B, p.Hq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(sparse_attn_decode_varlen(p, _ptr(q), _ptr(K), _ptr(V), _ptr(seq_len), _ptr(idx), _ptr(sc), _ptr(cnt),
+                                     _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "sparse_attn_decode_varlen")
     return o, lse
 
 

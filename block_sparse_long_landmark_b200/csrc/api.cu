@@ -46,6 +46,8 @@ int resolve(const sa_params *p, Shape &s) {
     s.Hsel = perq ? p->Hq : p->Hkv;
     s.heads_per = perq ? 1 : s.G;
     s.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+    s.seq_len = nullptr;
+    s.first_block = nullptr;
     if ((long long)s.B * s.Hq * s.nb > (1ll << 31) - 1) return SA_ERR_UNSUPPORTED;
     if (s.heads_per * s.d > 2048) return SA_ERR_UNSUPPORTED;
     return SA_OK;
@@ -84,11 +86,23 @@ int sparse_attn_landmarks(const sa_params *p, const void *K, void *L, void *stre
     return launch_result(launch_landmarks(s, K, L, (cudaStream_t)stream));
 }
 
-static int select_common(const sa_params *p, bool decode, const void *Q, const void *L, int32_t *idx, float *score,
-                         int32_t *count, void *ws, size_t ws_bytes, void *stream) {
+int sparse_attn_landmarks_update(const sa_params *p, const void *K, void *L, const int32_t *seq_len,
+                                 const int32_t *first_block, void *stream) {
     Shape s;
     int r = resolve(p, s);
     if (r != SA_OK) return r;
+    if (!K || !L || !aligned16(K) || !aligned16(L)) return SA_ERR_ARG;
+    s.seq_len = seq_len;
+    s.first_block = first_block;
+    return launch_result(launch_landmarks(s, K, L, (cudaStream_t)stream));
+}
+
+static int select_common(const sa_params *p, bool decode, const void *Q, const void *L, int32_t *idx, float *score,
+                         int32_t *count, void *ws, size_t ws_bytes, void *stream, const int32_t *seq_len = nullptr) {
+    Shape s;
+    int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    s.seq_len = seq_len;
     if (!Q || !L || !idx || !score || !count || !ws) return SA_ERR_ARG;
     if (!aligned16(Q) || !aligned16(L) || !aligned16(ws)) return SA_ERR_ARG;
     if (ws_bytes < sparse_attn_workspace_size(p, decode ? SA_OP_SELECT_DECODE : SA_OP_SELECT)) return SA_ERR_WORKSPACE;
@@ -103,6 +117,13 @@ int sparse_attn_select(const sa_params *p, const void *Q, const void *L, int32_t
 int sparse_attn_select_decode(const sa_params *p, const void *q, const void *L, int32_t *idx, float *score,
                               int32_t *count, void *ws, size_t ws_bytes, void *stream) {
     return select_common(p, true, q, L, idx, score, count, ws, ws_bytes, stream);
+}
+
+int sparse_attn_select_decode_varlen(const sa_params *p, const void *q, const void *L, const int32_t *seq_len,
+                                     int32_t *idx, float *score, int32_t *count, void *ws, size_t ws_bytes,
+                                     void *stream) {
+    if (!seq_len) return SA_ERR_ARG;
+    return select_common(p, true, q, L, idx, score, count, ws, ws_bytes, stream, seq_len);
 }
 
 int sparse_attn_prefill(const sa_params *p, const void *Q, const void *K, const void *V, const int32_t *idx,
@@ -128,16 +149,30 @@ int sparse_attn_prefill_kernel(const sa_params *p) {
     return prefill_tc_supported(s) ? 1 : 0;
 }
 
-int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
-                       const float *score, const int32_t *count, void *o, float *lse, void *ws, size_t ws_bytes,
-                       void *stream) {
+static int decode_common(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *seq_len,
+                         const int32_t *idx, const float *score, const int32_t *count, void *o, float *lse,
+                         void *ws, size_t ws_bytes, void *stream) {
     Shape s;
     int r = resolve(p, s);
     if (r != SA_OK) return r;
+    s.seq_len = seq_len;
     if (!q || !K || !V || !idx || !score || !count || !o || !lse || !ws) return SA_ERR_ARG;
     if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(o) || !aligned16(ws)) return SA_ERR_ARG;
     if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_DECODE)) return SA_ERR_WORKSPACE;
     return launch_result(launch_decode(s, q, K, V, idx, score, count, o, lse, ws, ws_bytes, (cudaStream_t)stream));
+}
+
+int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
+                       const float *score, const int32_t *count, void *o, float *lse, void *ws, size_t ws_bytes,
+                       void *stream) {
+    return decode_common(p, q, K, V, nullptr, idx, score, count, o, lse, ws, ws_bytes, stream);
+}
+
+int sparse_attn_decode_varlen(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *seq_len,
+                              const int32_t *idx, const float *score, const int32_t *count, void *o, float *lse,
+                              void *ws, size_t ws_bytes, void *stream) {
+    if (!seq_len) return SA_ERR_ARG;
+    return decode_common(p, q, K, V, seq_len, idx, score, count, o, lse, ws, ws_bytes, stream);
 }
 
 int sparse_attn_check_status(void *ws, void *stream, int *detail) {

@@ -23,7 +23,16 @@ struct Shape {
     int Hsel;        // heads that own a selection list (Hkv, or Hq per q-head)
     int heads_per;   // query heads that share one list (G, or 1 per q-head)
     float scale;
+    const int32_t *seq_len;      // decode / landmarks: per-sequence lengths [B] (device) or null = N
+    const int32_t *first_block;  // landmarks: per-sequence first block to recompute [B] or null = 0
 };
+
+// Context length of sequence b: seq_len[b] clamped to [1, N], or N.
+__device__ __forceinline__ int seq_n(const Shape &s, int b) {
+    if (!s.seq_len) return s.N;
+    const int n = s.seq_len[b];
+    return n < 1 ? 1 : (n > s.N ? s.N : n);
+}
 
 __device__ __forceinline__ void set_status(unsigned *status, unsigned bit) {
     if (status) atomicOr(status, bit);

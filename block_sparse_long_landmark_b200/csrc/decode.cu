@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecArgs a) {
     const int32_t *idx = a.idx + (size_t)u * s.cap;
     const float *sc = a.score + (size_t)u * s.cap;
     const int cnt = min(a.count[u], s.cap);
-    const int local = (s.N - 1) / bs;
+    const int nseq = seq_n(s, b);                       // this sequence's context length
+    const int local = (nseq - 1) / bs;
     const bool hier = s.flags & SA_HIER, gate_on = s.flags & SA_GATE;
     const float s_local = cnt > 0 ? sc[cnt - 1] : 0.f;
 
@@ -84,7 +85,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecArgs a) {
         }
         const bool forced = (blk == local && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
         const float gate = (gate_on && !forced) ? log_sigmoid(sc[c] - s_local) * kLog2e : 0.f;
-        const int t0 = blk * bs, nk = min(bs, s.N - t0);
+        const int t0 = blk * bs, nk = min(bs, nseq - t0);
         __syncthreads();
         {
             constexpr int EPV = Vec<T>::n;

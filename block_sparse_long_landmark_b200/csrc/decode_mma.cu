@@ -140,7 +140,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     const int32_t *il = a.idx + (size_t)u * s.cap;
     const float *sl = a.score + (size_t)u * s.cap;
     const int cnt = max(0, min(a.count[u], s.cap));
-    const int local = (s.N - 1) / 64;
+    const int nseq = seq_n(s, b);                       // this sequence's context length
+    const int local = (nseq - 1) / 64;
     const int c0 = split * a.bps, c1 = min(cnt, c0 + a.bps);
     const int nloc = max(0, c1 - c0);
     const bool hier = s.flags & SA_HIER;
@@ -236,7 +237,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             const uint32_t kb = sb + st * kStageBytes, vb = kb + kBlockBytes;
             const int blk = blk_s[li];
-            const int nk = blk < 0 ? 0 : min(64, s.N - blk * 64);
+            const int nk = blk < 0 ? 0 : min(64, nseq - blk * 64);
             // S = q K^T over 8 key n-tiles
             float sacc[8][4];
 #pragma unroll

@@ -14,7 +14,7 @@ namespace sa {
 
 template <typename T, int VPR>
 __global__ void __launch_bounds__(256) landmarks_kernel(const T *__restrict__ K, T *__restrict__ L, int N, int bs,
-                                                        int nb, long long nunits) {
+                                                        int nb, long long nunits, Shape s) {
     constexpr int EPV = Vec<T>::n;           // elements per 16-byte vector
     constexpr int RSTEP = 32 / VPR;          // rows a warp covers per step
     const int lane = threadIdx.x & 31;
@@ -24,7 +24,12 @@ __global__ void __launch_bounds__(256) landmarks_kernel(const T *__restrict__ K,
     const int blk = (int)(unit - bg * nb);
     const int d = VPR * EPV;
     const int t0 = blk * bs;
-    const int cnt = min(bs, N - t0);
+    // per-sequence length and first block to refresh (appends), when given
+    const int bb = (int)(bg / s.Hkv);
+    const int n = seq_n(s, bb);
+    const int fb = s.first_block ? max(0, s.first_block[bb]) : 0;
+    if (blk < fb || t0 >= n) return;   // the whole warp leaves together
+    const int cnt = min(bs, n - t0);
     const int cv = lane % VPR, rs = lane / VPR;
     const T *base = K + ((size_t)bg * N + t0) * d + cv * EPV;
     float acc[EPV];
@@ -66,9 +71,9 @@ static cudaError_t run(const Shape &s, const void *K, void *L, cudaStream_t st) 
     auto k = (const T *)K;
     auto l = (T *)L;
     switch (vpr) {
-        case 8: landmarks_kernel<T, 8><<<grid, 256, 0, st>>>(k, l, s.N, s.bs, s.nb, nunits); break;
-        case 16: landmarks_kernel<T, 16><<<grid, 256, 0, st>>>(k, l, s.N, s.bs, s.nb, nunits); break;
-        case 32: landmarks_kernel<T, 32><<<grid, 256, 0, st>>>(k, l, s.N, s.bs, s.nb, nunits); break;
+        case 8: landmarks_kernel<T, 8><<<grid, 256, 0, st>>>(k, l, s.N, s.bs, s.nb, nunits, s); break;
+        case 16: landmarks_kernel<T, 16><<<grid, 256, 0, st>>>(k, l, s.N, s.bs, s.nb, nunits, s); break;
+        case 32: landmarks_kernel<T, 32><<<grid, 256, 0, st>>>(k, l, s.N, s.bs, s.nb, nunits, s); break;
         default: return cudaErrorInvalidValue;
     }
     note_launch();

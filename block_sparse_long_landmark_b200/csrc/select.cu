@@ -61,7 +61,7 @@ __device__ __forceinline__ void unit_coords(const SelArgs &a, int u, int &b, int
     int r = u / a.ntiles;
     hs = r % a.s.Hsel;
     b = r / a.s.Hsel;
-    local = a.decode ? (a.s.N - 1) / a.s.bs : j;
+    local = a.decode ? (seq_n(a.s, b) - 1) / a.s.bs : j;
 }
 
 // Pooled query of the unit into sm.qbar (fp32).  Every thread participates.

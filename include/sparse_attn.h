@@ -127,6 +127,19 @@ size_t sparse_attn_workspace_size(const sa_params *p, int op);
  * even.  K [B,Hkv,N,d] -> L [B,Hkv,nb,d]. */
 int sparse_attn_landmarks(const sa_params *p, const void *K, void *L, void *stream);
 
+/* Landmarks of the blocks that changed: for every kv-head of sequence b,
+ * recompute blocks first_block[b] .. ceil(seq_len[b] / block) - 1 and leave
+ * the others untouched.  After an append that grew sequence b from n0 to n1
+ * keys, first_block[b] = n0 / block refreshes exactly the partial block and
+ * the new ones (the Latent Sparse Attention post, "Индекс перестаёт
+ * перебирать весь контекст": a block's composition is fixed once complete).
+ * seq_len (device, [B], may be NULL = N for all) gives each sequence's
+ * length; a length outside [1, N] is clamped to it.  first_block (device,
+ * [B], may be NULL = 0) gives the first block to refresh.  K and L as in
+ * sparse_attn_landmarks (N = the cache capacity). */
+int sparse_attn_landmarks_update(const sa_params *p, const void *K, void *L, const int32_t *seq_len,
+                                 const int32_t *first_block, void *stream);
+
 /* Prefill selection ([SAS] hard top-K over block scores; [LSA] start of
  * context always added; [SAS] current block always kept).  For tile j of a
  * unit: pooled query = mean of Q over the unit's query heads and the tile's
@@ -143,6 +156,16 @@ int sparse_attn_select(const sa_params *p, const void *Q, const void *L, int32_t
  * count of shape [B,Hsel,top_k+2] / [B,Hsel]. */
 int sparse_attn_select_decode(const sa_params *p, const void *q, const void *L, int32_t *idx, float *score,
                               int32_t *count, void *ws, size_t ws_bytes, void *stream);
+
+/* Decode selection for a ragged batch: sequence b holds seq_len[b] keys
+ * (device, [B], clamped to [1, N]; N = the cache capacity of K/V/L) and its
+ * query sits at position seq_len[b] - 1, so its local block is
+ * (seq_len[b] - 1) / block.  L must hold each sequence's landmarks over its
+ * own length (sparse_attn_landmarks_update with the same seq_len).
+ * Otherwise as sparse_attn_select_decode; seq_len NULL returns SA_ERR_ARG. */
+int sparse_attn_select_decode_varlen(const sa_params *p, const void *q, const void *L, const int32_t *seq_len,
+                                     int32_t *idx, float *score, int32_t *count, void *ws, size_t ws_bytes,
+                                     void *stream);
 
 /* Block-sparse prefill over the kept lists ([SAS] FlashAttention-style,
  * blockwise, online softmax).  Gated mode: z_t = scale * <q_i, k_t> + gate_b
@@ -187,6 +210,15 @@ int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const v
 int sparse_attn_decode_static(const sa_params *p, const void *q, const void *K, const void *V,
                               const int32_t *idx, const float *score, const int32_t *count, void *o, float *lse,
                               void *stream);
+
+/* Block-sparse decode for a ragged batch: as sparse_attn_decode with
+ * sequence b reading only its first seq_len[b] cached keys (clamped to
+ * [1, N]), its query at position seq_len[b] - 1; lists from
+ * sparse_attn_select_decode_varlen.  Uses the workspace size of
+ * SA_OP_DECODE; seq_len NULL returns SA_ERR_ARG. */
+int sparse_attn_decode_varlen(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *seq_len,
+                              const int32_t *idx, const float *score, const int32_t *count, void *o, float *lse,
+                              void *ws, size_t ws_bytes, void *stream);
 
 /* Synchronises `stream`, returns SA_OK or SA_ERR_DEVICE from the status
  * word in `ws`, and clears it.  *detail (may be NULL) receives the raw bits:

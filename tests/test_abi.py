@@ -91,3 +91,12 @@ def test_null_misaligned_and_small_workspace_rejected():
     assert sa.sparse_attn_prefill(p, a, a, a, a, a, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
     assert sa.sparse_attn_decode(p, a, a, a, a, a, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
     assert sa.sparse_attn_check_status(None, None)[0] == sa.SA_ERR_ARG
+
+
+def test_varlen_entry_points_need_lengths():
+    p = _p()
+    a = 256
+    assert sa.sparse_attn_select_decode_varlen(p, a, a, None, a, a, a, a, 1 << 20, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_decode_varlen(p, a, a, a, None, a, a, a, a, a, a, 1 << 20, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_landmarks_update(p, None, a, None, None, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_landmarks_update(_p(Hq=7), a, a, None, None, None) == sa.SA_ERR_ARG
