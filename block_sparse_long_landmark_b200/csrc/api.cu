@@ -135,6 +135,9 @@ int sparse_attn_prefill(const sa_params *p, const void *Q, const void *K, const 
     if (!Q || !K || !V || !idx || !score || !count || !O || !lse || !ws) return SA_ERR_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(ws)) return SA_ERR_ARG;
     if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_PREFILL)) return SA_ERR_WORKSPACE;
+    if (prefill_tc2_supported(s))
+        return launch_result(
+            launch_prefill_tc2(s, Q, K, V, idx, score, count, O, lse, (unsigned *)ws, (cudaStream_t)stream));
     if (prefill_tc_supported(s))
         return launch_result(
             launch_prefill_tc(s, Q, K, V, idx, score, count, O, lse, (unsigned *)ws, (cudaStream_t)stream));
@@ -146,7 +149,7 @@ int sparse_attn_prefill_kernel(const sa_params *p) {
     Shape s;
     int r = resolve(p, s);
     if (r != SA_OK) return r;
-    return prefill_tc_supported(s) ? 1 : 0;
+    return prefill_tc2_supported(s) ? 2 : prefill_tc_supported(s) ? 1 : 0;
 }
 
 static int decode_common(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *seq_len,

@@ -128,6 +128,10 @@ bool prefill_tc_supported(const Shape &s);
 cudaError_t launch_prefill_tc(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
                               const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
                               cudaStream_t st);
+bool prefill_tc2_supported(const Shape &s);
+cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
+                               const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
+                               cudaStream_t st);
 bool decode_mma_supported(const Shape &s);
 void decode_mma_geometry(const Shape &s, int &S, int &bps);
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,

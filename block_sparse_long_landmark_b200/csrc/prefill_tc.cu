@@ -32,15 +32,13 @@
 //
 // Every mbarrier wait is bounded (about two seconds of %globaltimer); on
 // expiry the CTA records kStatusTimeout, drains, frees TMEM and exits.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <math_constants.h>
 
 #include <cstdlib>
 #include <cstring>
-#include <mutex>
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace sa {
 namespace {
@@ -59,7 +57,6 @@ constexpr uint32_t kVOff = kKOff + kStages * kKTile;
 constexpr uint32_t kBarOff = kVOff + kStages * kKTile;
 constexpr int kMaxList = 258;
 constexpr uint32_t kSmemBytes = kBarOff + 1024 + 8 * kMaxList + 2048;   // + alignment slack
-constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr uint32_t kTmemCols = 256;
 
 // barrier slots (uint64 each)
@@ -88,126 +85,7 @@ struct TcArgs {
     int hc;      // query heads per CTA
 };
 
-// ---------------------------------------------------------------------------
-// PTX wrappers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ unsigned long long gtimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-// Bounded wait: true when the phase completed, false on timeout or abort.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          unsigned *status) {
-    if (mbar_try(bar, parity)) return true;
-    const unsigned long long t0 = gtimer();
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try(bar, parity)) return true;
-        if ((it & 63) == 63) {
-            if (*abort_flag) return false;
-            if (gtimer() - t0 > kWaitNs) {
-                *abort_flag = 1;
-                set_status(status, kStatusTimeout);
-                return false;
-            }
-        }
-    }
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-        : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptors (sm_100 format, version 1), 128-byte swizzle.
-// K-major: rows of 128 bytes, 8-row groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// MN-major: 64 contiguous elements per 128-byte row, next 64 elements `lbo`
-// bytes away, 8-row (K) groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
-    return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, M = 128, N = n.
-__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major, uint32_t n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((n >> 3) << 17) |
-           ((128u >> 4) << 24);
-}
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-          "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-          "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
+using namespace tc;
 
 // ---------------------------------------------------------------------------
 // kernel
@@ -406,27 +284,35 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             tmem_ld32(tS, x);
             tmem_ld32(tS + 32, x + 32);
             tmem_wait_ld();
+            reg_fence<64>(x);
             const int c = i / sub;
             const int blk = blk_s[c];
             const float gl = gate_s[c];
             const int t0 = blk * s.bs + (i % sub) * 64;  // first key of this tile
             // masks: a bad list entry, the ragged end of the sequence, causality in the local block
             const bool masked = blk < 0 || t0 + 64 > s.N || (causal && blk == j);
-            float mx = -CUDART_INF_F;
-            if (!masked) {
-#pragma unroll
-                for (int k = 0; k < 64; ++k) mx = fmaxf(mx, x[k]);
-                mx = fmaf(mx, qk_scale, gl);
-            } else {
+            if (masked) {
 #pragma unroll
                 for (int k = 0; k < 64; ++k) {
                     const int t = t0 + k;
                     const bool vis = blk >= 0 && t < s.N && !(causal && blk == j && t > qi);
                     x[k] = vis ? x[k] : -CUDART_INF_F;
-                    mx = fmaxf(mx, x[k]);
                 }
-                mx = mx == -CUDART_INF_F ? mx : fmaf(mx, qk_scale, gl);
             }
+            // row max: eight independent chains, then a three-level tree
+            float mq[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mq[e] = x[e];
+#pragma unroll
+            for (int k = 8; k < 64; k += 8)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mq[e] = fmaxf(mq[e], x[k + e]);
+#pragma unroll
+            for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                for (int e = 0; e < w; ++e) mq[e] = fmaxf(mq[e], mq[e + w]);
+            float mx = mq[0];
+            mx = mx == -CUDART_INF_F ? mx : fmaf(mx, qk_scale, gl);
             if (hier) {
                 // this block's own softmax (scores without gate), weighted by its retrieval score
                 const float mb = mx == -CUDART_INF_F ? 0.f : mx - gl;   // mx carried the score: drop it
@@ -472,6 +358,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         float o[32];
                         tmem_ld32(tO + 32 * cc, o);
                         tmem_wait_ld();
+                        reg_fence<32>(o);
                         uint32_t w[32];
 #pragma unroll
                         for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(o[k] * corr);
@@ -517,6 +404,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             if (have && ok) {
                 tmem_ld32(tO + 32 * cc, o);
                 tmem_wait_ld();
+                reg_fence<32>(o);
             } else {
 #pragma unroll
                 for (int k = 0; k < 32; ++k) o[k] = 0.f;
@@ -548,30 +436,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-bool get_encode() {
-    std::call_once(g_encode_once, [] {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    });
-    return g_encode != nullptr;
-}
-
-bool make_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows) {
-    cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {128 * sizeof(__nv_bfloat16)};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool prefill_tc_supported(const Shape &s) {
@@ -590,10 +454,16 @@ bool prefill_tc_supported(const Shape &s) {
 cudaError_t launch_prefill_tc(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
                               const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
                               cudaStream_t st) {
-    if (!get_encode()) return cudaErrorNotSupported;
+    // The register split assumes a launch at exactly kRegsLaunch registers
+    // per thread; anything else could stall the register exchange.
+    cudaFuncAttributes fa;
+    cudaError_t fe = cudaFuncGetAttributes(&fa, prefill_tc_kernel);
+    if (fe != cudaSuccess) return fe;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidDeviceFunction;
     CUtensorMap mq, mk, mv;
     const uint64_t qrows = (uint64_t)s.B * s.Hq * s.N, krows = (uint64_t)s.B * s.Hkv * s.N;
-    if (!make_map(&mq, Q, qrows, 64) || !make_map(&mk, K, krows, 64) || !make_map(&mv, V, krows, 64))
+    if (!make_map_d128(&mq, Q, qrows, 64) || !make_map_d128(&mk, K, krows, 64) ||
+        !make_map_d128(&mv, V, krows, 64))
         return cudaErrorInvalidValue;
     TcArgs a{};
     a.s = s;

@@ -1,0 +1,569 @@
+// prefill_tc2.cu -- persistent tensor-core gated block-sparse prefill for
+// bf16, d = 128, block 64 or 128, query groups of at least 256 rows.
+//
+// Computes what prefill_tc.cu computes ([SAS] "Ключевые факты" / "Как это
+// применить": blockwise softmax attention over the kept blocks only, the
+// selector's gate log_sigmoid(s_b - s_local) added to the logits of selected
+// blocks, forced sink / local blocks gated by 0), with a layout built for
+// one CTA per SM:
+//
+//   * a work unit is 256 query rows of one (batch, kv-head, block): the four
+//     query heads of a block-64 tile or two heads of a block-128 tile, all of
+//     which share one kept list, so each K/V key tile is loaded once for
+//     256 rows;
+//   * the unit is two M=128 Q tiles, each with its own softmax warpgroup,
+//     S buffer and O accumulator in tensor memory (4 x 128 columns = all
+//     512).  While one warpgroup turns S into P, the tensor core runs the
+//     other tile's PV and QK, so the two warpgroups take turns on it;
+//   * key tiles are 128 keys (two kept blocks of 64, or one of 128), which
+//     halves the per-tile hand-off cost against 64-key tiles;
+//   * the grid is one CTA per SM, each looping over units: the next unit's
+//     list and Q tiles load while the current one runs, and a warpgroup's
+//     epilogue overlaps the other's last tile.
+//
+// Warp roles (12 warps):
+//   warp 0      loads each unit's list into shared memory (all lanes), then
+//               issues the TMA loads: Q tiles, K and V key tiles (2-stage rings)
+//   warp 1      TMEM owner; one thread issues every tcgen05.mma
+//   warps 2-3   idle
+//   warps 4-7   softmax for Q tile 0, warps 8-11 for Q tile 1; thread = row
+// Registers: launched at 168; the first warpgroup drops to 56 and the two
+// softmax warpgroups rise to 224: 128 x 56 + 256 x 224 = 384 x 168.
+//
+// Per Q tile q and key tile g the MMA thread issues, in this order,
+//   O_q += P_q(g-1) V_(g-1)   then   S_q = Q_q K_g^T
+// (P_q is written over the first 64 columns of S_q and read from TMEM), so
+// when S_q(g) is ready, the PV before it has completed too: the lazy O
+// rescale (when a row max grows by more than 2^8) never waits on the tensor
+// core.
+//
+// Every mbarrier wait is bounded; on expiry the CTA records kStatusTimeout,
+// stops, lets its copies land, frees TMEM and exits.
+#include <math_constants.h>
+
+#include <cstdlib>
+#include <cstring>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace sa {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads2 = 384;
+constexpr int kRegsLaunch2 = 168, kRegsLow2 = 56, kRegsHigh2 = 224;
+static_assert(128 * kRegsLow2 + 256 * kRegsHigh2 <= kThreads2 * kRegsLaunch2, "register split");
+constexpr int kRows = 256;                          // query rows per unit
+constexpr uint32_t kChunk2 = 128 * 128;             // 128 rows x 64 bf16 (one swizzle atom wide)
+constexpr uint32_t kTile2 = 2 * kChunk2;            // 128 rows x 128 bf16
+constexpr int kStages2 = 2;
+constexpr uint32_t kQOff2 = 0;                      // Q tiles 0 and 1
+constexpr uint32_t kKOff2 = 2 * kTile2;             // K ring
+constexpr uint32_t kVOff2 = kKOff2 + kStages2 * kTile2;
+constexpr uint32_t kBarOff2 = kVOff2 + kStages2 * kTile2;
+constexpr int kMaxList2 = 258;
+constexpr uint32_t kListOff2 = kBarOff2 + 512;      // [2 slots] blk[kMaxList2], gate[kMaxList2]
+constexpr uint32_t kListBytes = 8 * kMaxList2;
+constexpr uint32_t kSmem2 = kListOff2 + 2 * kListBytes + 64 + 1024;   // + counts + alignment slack
+
+enum {
+    C_Q = 0,                    // Q tiles landed (one phase per unit with work)
+    C_QFREE = 1,                // every QK of the unit done: Q may be overwritten
+    C_KF = 2,                   // [2] K tile landed
+    C_VF = C_KF + kStages2,     // [2] V tile landed
+    C_KE = C_VF + kStages2,     // [2] K stage free (both QKs done)
+    C_VE = C_KE + kStages2,     // [2] V stage free (both PVs done)
+    C_S = C_VE + kStages2,      // [2 Q tiles] S ready
+    C_P = C_S + 2,              // [2 Q tiles] P written, 128 arrivals
+    C_OD = C_P + 2,             // [2 Q tiles] last PV of the unit done
+    C_L = C_OD + 2,             // [2 slots] list loaded
+    C_LF = C_L + 2,             // [2 slots] list released, 8 arrivals (one per softmax warp)
+    C_END = C_LF + 2,
+    NBAR2
+};
+static_assert(8 * NBAR2 + 8 <= 512, "barrier area");
+
+struct Tc2Args {
+    Shape s;
+    const int32_t *idx;
+    const float *score;
+    const int32_t *count;
+    __nv_bfloat16 *O;
+    float *lse;
+    unsigned *status;
+    int npair;   // units per (batch, kv-head, block)
+    int hc;      // query heads per unit
+    int units;
+};
+
+struct Unit {
+    int b, g, j, h0;
+    size_t lu;   // (b, g, j) list row
+};
+
+// Units run heaviest first: the block index j is the slowest-varying
+// coordinate, descending, so the round-robin over CTAs ends on short lists.
+__device__ __forceinline__ Unit unit_at(const Tc2Args &a, int u) {
+    const Shape &s = a.s;
+    const int per_j = s.B * s.Hkv * a.npair;
+    Unit w;
+    w.j = s.nb - 1 - u / per_j;
+    int r = u % per_j;
+    const int pair = r % a.npair;
+    r /= a.npair;
+    w.g = r % s.Hkv;
+    w.b = r / s.Hkv;
+    w.h0 = w.g * s.G + pair * a.hc;
+    w.lu = ((size_t)w.b * s.Hkv + w.g) * s.nb + w.j;
+    return w;
+}
+
+// 128-key tiles of a list of cnt blocks
+__device__ __forceinline__ int key_tiles(const Shape &s, int cnt) { return s.bs == 64 ? (cnt + 1) >> 1 : cnt; }
+
+
+__global__ void __launch_bounds__(kThreads2, 1)
+prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, Tc2Args a) {
+    constexpr float kLog2e = 1.4426950408889634f;
+    constexpr float kLn2 = 0.6931471805599453f;
+    const Shape &s = a.s;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                            ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kBarOff2 + 8 * NBAR2);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff2 + 8 * NBAR2 + 4);
+    int *cnt_s = reinterpret_cast<int *>(smem + kListOff2 + 2 * kListBytes);   // [2 slots]
+    auto blk_of = [&](int slot) { return reinterpret_cast<int *>(smem + kListOff2 + slot * kListBytes); };
+    auto gate_of = [&](int slot) {
+        return reinterpret_cast<float *>(smem + kListOff2 + slot * kListBytes + 4 * kMaxList2);
+    };
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- set-up -----------------------------------------------------------
+    if (tid == 0) {
+        for (int i = 0; i < NBAR2; ++i)
+            mbar_init(bar(i), (i == C_P || i == C_P + 1) ? 128 : (i == C_LF || i == C_LF + 1) ? 8 : 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "n"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- lists and TMA loads ------------------------------------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow2));
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
+        }
+        bool ok = true;
+        int gt = 0, nq = 0, ul = 0;   // key tiles, Q loads and units so far
+        int nk = 0, nv = 0;           // K and V tiles issued
+        for (int u = blockIdx.x; u < a.units; u += gridDim.x, ++ul) {
+            const Unit w = unit_at(a, u);
+            const int slot = ul & 1;
+            if (ul >= 2) ok = mbar_wait(bar(C_LF + slot), ((ul >> 1) - 1) & 1, abort_flag, a.status);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            // the unit's list: block ids (bad entries -> -1) and log2-unit gates
+            const int cnt = max(0, min(a.count[w.lu], s.cap));
+            int *blk_s = blk_of(slot);
+            float *gate_s = gate_of(slot);
+            const int32_t *il = a.idx + w.lu * s.cap;
+            const float *sl = a.score + w.lu * s.cap;
+            const float s_loc = cnt > 0 ? sl[cnt - 1] : 0.f;
+            for (int e = lane; e < cnt; e += 32) {
+                const int blk = il[e];
+                const bool good = blk >= 0 && blk <= w.j && (e == 0 || il[e - 1] < blk);
+                if (!good) set_status(a.status, kStatusBadIndex);
+                blk_s[e] = good ? blk : -1;
+                const bool forced = (blk == w.j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
+                gate_s[e] = ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[e] - s_loc) * kLog2e : 0.f;
+            }
+            if (lane == 0) cnt_s[slot] = cnt;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C_L + slot));
+            const int T = key_tiles(s, cnt);
+            if (lane == 0 && T > 0) {
+                // Q tiles: rows of heads h0 .. h0+3 (block 64) or h0, h0+1 (block 128)
+                if (nq >= 1) ok = mbar_wait(bar(C_QFREE), (nq - 1) & 1, abort_flag, a.status);
+                if (ok) {
+                    mbar_expect_tx(bar(C_Q), 2 * kTile2);
+                    for (int q = 0; q < 2; ++q)
+                        for (int c = 0; c < 2; ++c)
+                            for (int e = 0; e < 2; ++e) {
+                                const int y = s.bs == 64 ? (w.b * s.Hq + w.h0 + 2 * q + e) * s.N + w.j * 64
+                                                         : (w.b * s.Hq + w.h0 + q) * s.N + w.j * 128 + 64 * e;
+                                tma_load_2d(sbase + kQOff2 + q * kTile2 + c * kChunk2 + e * 8192, &tmQ, bar(C_Q),
+                                            64 * c, y);
+                            }
+                }
+                // key tiles: two 64-row halves each (two blocks of 64, or one block of 128)
+                const int kvbase = (w.b * s.Hkv + w.g) * s.N;
+                for (int t = 0; ok && t < T; ++t) {
+                    const int gg = gt + t, st = gg % kStages2, use = gg / kStages2;
+                    int y0, y1;
+                    if (s.bs == 64) {
+                        // an odd list's last tile repeats its block in the second half (masked later)
+                        y0 = kvbase + max(0, blk_s[2 * t]) * 64;
+                        y1 = kvbase + max(0, blk_s[min(2 * t + 1, cnt - 1)]) * 64;
+                    } else {
+                        y0 = kvbase + max(0, blk_s[t]) * 128;
+                        y1 = y0 + 64;
+                    }
+                    if (gg >= kStages2 && !(ok = mbar_wait(bar(C_KE + st), (use - 1) & 1, abort_flag, a.status)))
+                        break;
+                    mbar_expect_tx(bar(C_KF + st), kTile2);
+                    for (int c = 0; c < 2; ++c) {
+                        const uint32_t d = sbase + kKOff2 + st * kTile2 + c * kChunk2;
+                        tma_load_2d(d, &tmK, bar(C_KF + st), 64 * c, y0);
+                        tma_load_2d(d + 8192, &tmK, bar(C_KF + st), 64 * c, y1);
+                    }
+                    nk = gg + 1;
+                    if (gg >= kStages2 && !(ok = mbar_wait(bar(C_VE + st), (use - 1) & 1, abort_flag, a.status)))
+                        break;
+                    mbar_expect_tx(bar(C_VF + st), kTile2);
+                    for (int c = 0; c < 2; ++c) {
+                        const uint32_t d = sbase + kVOff2 + st * kTile2 + c * kChunk2;
+                        tma_load_2d(d, &tmV, bar(C_VF + st), 64 * c, y0);
+                        tma_load_2d(d + 8192, &tmV, bar(C_VF + st), 64 * c, y1);
+                    }
+                    nv = gg + 1;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            gt += T;
+            if (T > 0) ++nq;
+        }
+        if (lane == 0 && *abort_flag) {
+            // let the copies in flight land before the CTA exits (bounded)
+            volatile int never = 0;
+            if (nq > 0) mbar_wait(bar(C_Q), (nq - 1) & 1, &never, a.status);
+            for (int t = max(0, nk - kStages2); t < nk; ++t)
+                mbar_wait(bar(C_KF + t % kStages2), (t / kStages2) & 1, &never, a.status);
+            for (int t = max(0, nv - kStages2); t < nv; ++t)
+                mbar_wait(bar(C_VF + t % kStages2), (t / kStages2) & 1, &never, a.status);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer -----------------------------------------------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow2));
+        if (lane == 0) {
+            constexpr uint32_t idq = idesc_bf16(false, 128), idp = idesc_bf16(true, 128);
+            // S_q = Q_q K^T for key tile gg (8 MMAs of K = 16 over d = 128)
+            // (descriptor start addresses advance in 16-byte units: offset >> 4;
+            // the bases are rebuilt per call -- hoisting every (tile, stage)
+            // variant out of the loop would not fit this warp's registers)
+            auto qk = [&](int q, int gg) {
+                uint64_t da = desc_k_sw128(sbase + kQOff2 + q * kTile2);
+                uint64_t db = desc_k_sw128(sbase + kKOff2 + (gg % kStages2) * kTile2);
+                asm volatile("" : "+l"(da), "+l"(db));
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = ((k >> 2) * kChunk2 + (k & 3) * 32) >> 4;
+                    mma_ss(tmem + q * 128, da + off, db + off, idq, k > 0);
+                }
+                mma_commit(bar(C_S + q));
+            };
+            // O_q += P_q V for key tile gg; P_q (bf16) is the first 64 columns of S_q
+            auto pv = [&](int q, int gg, bool acc) {
+                uint64_t db = desc_mn_sw128(sbase + kVOff2 + (gg % kStages2) * kTile2, kChunk2);
+                asm volatile("" : "+l"(db));
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tmem + 256 + q * 128, tmem + q * 128 + 8 * k, db + ((k * 2048) >> 4), idp, acc || k > 0);
+            };
+            bool ok = true;
+            int gt = 0, nq = 0, ul = 0;
+            for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x, ++ul) {
+                const int slot = ul & 1;
+                if (!(ok = mbar_wait(bar(C_L + slot), (ul >> 1) & 1, abort_flag, a.status))) break;
+                const int T = key_tiles(s, cnt_s[slot]);
+                if (T == 0) continue;
+                if (!(ok = mbar_wait(bar(C_Q), nq & 1, abort_flag, a.status))) break;
+                if (!(ok = mbar_wait(bar(C_KF + gt % kStages2), (gt / kStages2) & 1, abort_flag, a.status))) break;
+                tc_fence_after();
+                qk(0, gt);
+                qk(1, gt);
+                mma_commit(bar(C_KE + gt % kStages2));
+                if (T == 1) mma_commit(bar(C_QFREE));
+                for (int t = 0; ok && t < T; ++t) {
+                    const int gg = gt + t;
+                    if (!(ok = mbar_wait(bar(C_P), gg & 1, abort_flag, a.status))) break;
+                    if (!(ok = mbar_wait(bar(C_VF + gg % kStages2), (gg / kStages2) & 1, abort_flag, a.status)))
+                        break;
+                    tc_fence_after();
+                    pv(0, gg, t > 0);
+                    if (t == T - 1) mma_commit(bar(C_OD));
+                    if (t + 1 < T) {
+                        const int g1 = gg + 1;
+                        if (!(ok = mbar_wait(bar(C_KF + g1 % kStages2), (g1 / kStages2) & 1, abort_flag, a.status)))
+                            break;
+                        tc_fence_after();
+                        qk(0, g1);
+                    }
+                    if (!(ok = mbar_wait(bar(C_P + 1), gg & 1, abort_flag, a.status))) break;
+                    tc_fence_after();
+                    pv(1, gg, t > 0);
+                    mma_commit(bar(C_VE + gg % kStages2));
+                    if (t == T - 1) mma_commit(bar(C_OD + 1));
+                    if (t + 1 < T) {
+                        qk(1, gg + 1);
+                        mma_commit(bar(C_KE + (gg + 1) % kStages2));
+                        if (t + 2 == T) mma_commit(bar(C_QFREE));
+                    }
+                }
+                gt += T;
+                ++nq;
+            }
+            // drain: every MMA issued above has completed once this arrives
+            // (waited on even after an abort: TMEM is freed only after it)
+            mma_commit(bar(C_END));
+            volatile int never = 0;
+            mbar_wait(bar(C_END), 0, &never, a.status);
+        }
+    } else if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow2));
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh2));
+        // ---- softmax warpgroups --------------------------------------------
+        const int q = (warp - 4) >> 2;                   // Q tile of this warpgroup
+        const int qq = warp & 3;                         // TMEM lane quarter of this warp
+        const int r = 32 * qq + lane;                    // row within the Q tile
+        const uint32_t lane_off = (uint32_t)(32 * qq) << 16;
+        const uint32_t tS = tmem + lane_off + q * 128, tO = tmem + lane_off + 256 + q * 128;
+        const bool causal = s.flags & SA_CAUSAL;
+        const float qk_scale = s.scale * kLog2e;
+        bool ok = true;
+        int gt = 0, nq = 0, ul = 0;
+        for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x, ++ul) {
+            const Unit w = unit_at(a, u);
+            const int slot = ul & 1;
+            ok = mbar_wait(bar(C_L + slot), (ul >> 1) & 1, abort_flag, a.status);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            const int cnt = cnt_s[slot];
+            const int *blk_s = blk_of(slot);
+            const float *gate_s = gate_of(slot);
+            const int T = key_tiles(s, cnt);
+            int head, ri;
+            if (s.bs == 64) { head = w.h0 + 2 * q + (r >> 6); ri = r & 63; }
+            else { head = w.h0 + q; ri = r; }
+            const int qi = w.j * s.bs + ri;              // query position of this row
+            float m_run = -CUDART_INF_F, l = 0.f;
+            for (int t = 0; t < T; ++t) {
+                ok = mbar_wait(bar(C_S + q), (gt + t) & 1, abort_flag, a.status);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                float x[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, x + 32 * c);
+                tmem_wait_ld();
+                reg_fence<128>(x);
+                // per 64-key half: its block, gate and masks (a bad entry, an
+                // odd list's empty half, the ragged end, causality in the local block)
+                float gh[2], mh[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    int blk, t0;
+                    float gl;
+                    if (s.bs == 64) {
+                        const int e = 2 * t + h;
+                        blk = e < cnt ? blk_s[e] : -1;
+                        gl = e < cnt ? gate_s[e] : 0.f;
+                        t0 = blk * 64;
+                    } else {
+                        blk = blk_s[t];
+                        gl = gate_s[t];
+                        t0 = blk * 128 + 64 * h;
+                    }
+                    float *xh = x + 64 * h;
+                    if (blk < 0 || t0 + 64 > s.N || (causal && blk == w.j)) {
+#pragma unroll
+                        for (int k = 0; k < 64; ++k) {
+                            const int key = t0 + k;
+                            const bool vis = blk >= 0 && key < s.N && !(causal && blk == w.j && key > qi);
+                            xh[k] = vis ? xh[k] : -CUDART_INF_F;
+                        }
+                    }
+                    float mq[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mq[e] = xh[e];
+#pragma unroll
+                    for (int k = 8; k < 64; k += 8)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mq[e] = fmaxf(mq[e], xh[k + e]);
+#pragma unroll
+                    for (int v = 4; v > 0; v >>= 1)
+#pragma unroll
+                        for (int e = 0; e < v; ++e) mq[e] = fmaxf(mq[e], mq[e + v]);
+                    mh[h] = mq[0] == -CUDART_INF_F ? -CUDART_INF_F : fmaf(mq[0], qk_scale, gl);
+                    gh[h] = gl;
+                }
+                const float mx = fmaxf(mh[0], mh[1]);
+                if (t == 0) {
+                    m_run = mx;
+                } else {
+                    const bool need = mx > m_run + 8.f;
+                    if (__any_sync(0xffffffffu, need)) {
+                        // the PV before this S has completed: O_q is stable
+                        const float corr = need ? ex2(m_run - mx) : 1.f;
+                        if (need) {
+                            l *= corr;
+                            m_run = mx;
+                        }
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            float o[32];
+                            tmem_ld32(tO + 32 * cc, o);
+                            tmem_wait_ld();
+                            reg_fence<32>(o);
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) o[k] *= corr;
+                            tmem_st32(tO + 32 * cc, reinterpret_cast<const uint32_t *>(o));
+                        }
+                        tmem_wait_st();
+                    }
+                }
+                // p = 2^(x * scale + gate - ref), written as bf16 pairs over S columns 0..63
+                const float ref = m_run == -CUDART_INF_F ? 0.f : m_run;
+                float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float bias = gh[c >> 1] - ref;
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float p0 = ex2(fmaf(x[32 * c + 2 * k], qk_scale, bias));
+                        const float p1 = ex2(fmaf(x[32 * c + 2 * k + 1], qk_scale, bias));
+                        ls0 += p0;
+                        ls1 += p1;
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                        pk[k] = *reinterpret_cast<uint32_t *>(&h2);
+                    }
+                    tmem_st16(tS + 16 * c, pk);
+                }
+                l += ls0 + ls1;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C_P + q));
+            }
+            if (!ok) break;
+            // ---- epilogue: O_q / l -> bf16, LSE ----------------------------
+            if (T > 0) {
+                ok = mbar_wait(bar(C_OD + q), nq & 1, abort_flag, a.status);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+            }
+            const bool row_ok = qi < s.N;
+            __nv_bfloat16 *orow = a.O + (((size_t)w.b * s.Hq + head) * s.N + (row_ok ? qi : 0)) * 128;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float o[32];
+                if (T > 0) {
+                    tmem_ld32(tO + 32 * cc, o);
+                    tmem_wait_ld();
+                    reg_fence<32>(o);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o[k] = 0.f;
+                }
+                if (row_ok) {
+#pragma unroll
+                    for (int v = 0; v < 32; v += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) f[k] = o[v + k] * inv;
+                        store16(orow + 32 * cc + v, f);
+                    }
+                }
+            }
+            if (row_ok)
+                a.lse[((size_t)w.b * s.Hq + head) * s.N + qi] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -CUDART_INF_F;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C_LF + slot));
+            gt += T;
+            if (T > 0) ++nq;
+        }
+    }
+
+    // ---- teardown -----------------------------------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(512));
+    }
+}
+
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+}  // namespace
+
+bool prefill_tc2_supported(const Shape &s) {
+    if (s.dtype != SA_BF16 || s.d != 128) return false;
+    if (s.flags & (SA_SELECT_PER_QHEAD | SA_HIER)) return false;
+    if (s.bs != 64 && s.bs != 128) return false;
+    if ((s.G * s.bs) % kRows) return false;
+    if (s.cap > kMaxList2) return false;
+    const char *e = getenv("SPARSE_ATTN_PREFILL_PATH");
+    if (e && (strcmp(e, "simt") == 0 || strcmp(e, "tc1") == 0)) return false;
+    return true;
+}
+
+cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
+                               const float *score, const int32_t *count, void *O, float *lse, unsigned *status,
+                               cudaStream_t st) {
+    // The register split above assumes the kernel is launched at exactly
+    // kRegsLaunch2 registers per thread; anything else could stall the
+    // warpgroups' register exchange, so refuse to launch.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_tc2_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch2) return cudaErrorInvalidDeviceFunction;
+    CUtensorMap mq, mk, mv;
+    const uint64_t qrows = (uint64_t)s.B * s.Hq * s.N, krows = (uint64_t)s.B * s.Hkv * s.N;
+    if (!make_map_d128(&mq, Q, qrows, 64) || !make_map_d128(&mk, K, krows, 64) ||
+        !make_map_d128(&mv, V, krows, 64))
+        return cudaErrorInvalidValue;
+    Tc2Args a{};
+    a.s = s;
+    a.idx = idx;
+    a.score = score;
+    a.count = count;
+    a.O = (__nv_bfloat16 *)O;
+    a.lse = lse;
+    a.status = status;
+    a.hc = kRows / s.bs;
+    a.npair = s.G / a.hc;
+    a.units = s.B * s.Hkv * s.nb * a.npair;
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorNoDevice;
+    e = cudaFuncSetAttribute(prefill_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem2);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)min(a.units, sms);
+    prefill_tc2_kernel<<<grid, kThreads2, kSmem2, st>>>(mq, mk, mv, a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace sa

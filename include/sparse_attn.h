@@ -179,12 +179,17 @@ int sparse_attn_prefill(const sa_params *p, const void *Q, const void *K, const 
                         const float *score, const int32_t *count, void *O, float *lse, void *ws,
                         size_t ws_bytes, void *stream);
 
-/* Which kernel sparse_attn_prefill runs for these parameters: 1 = the
- * tensor-core kernel (tcgen05/TMEM/TMA; bf16, d = 128, block 64 or 128,
- * query heads per kv-head a multiple of 256/block, gated or plain), 0 = the
- * CUDA-core kernel (every other supported shape, fp32, hierarchical mode,
- * per-q-head lists), negative = invalid parameters.  Setting the environment
- * variable SPARSE_ATTN_PREFILL_PATH=simt forces 0. */
+/* Which kernel sparse_attn_prefill runs for these parameters:
+ *   2 = the persistent tensor-core kernel (tcgen05/TMEM/TMA, one CTA per SM,
+ *       256 query rows per work unit; bf16, d = 128, block 64 or 128, query
+ *       heads per kv-head a multiple of 256/block, gated or plain),
+ *   1 = the two-CTA-per-SM tensor-core kernel (same types, query heads per
+ *       kv-head a multiple of 128/block; also hierarchical mode at block 64),
+ *   0 = the CUDA-core kernel (every other supported shape, fp32, per-q-head
+ *       lists),
+ *   negative = invalid parameters.
+ * The environment variable SPARSE_ATTN_PREFILL_PATH=tc1 rules out 2, and
+ * SPARSE_ATTN_PREFILL_PATH=simt forces 0. */
 int sparse_attn_prefill_kernel(const sa_params *p);
 
 /* Block-sparse decode: the same attention for one query per sequence at
