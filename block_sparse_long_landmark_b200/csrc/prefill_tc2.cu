@@ -24,15 +24,18 @@
 // Warp roles (12 warps):
 //   warp 0      loads each unit's list into shared memory (all lanes), then
 //               issues the TMA loads: Q tiles, K and V key tiles (2-stage rings)
-//   warp 1      TMEM owner; one thread issues every tcgen05.mma
+//   warp 1      TMEM owner and MMA issuer: the warp runs the schedule in
+//               lockstep, one elected lane issues each tcgen05.mma
 //   warps 2-3   idle
 //   warps 4-7   softmax for Q tile 0, warps 8-11 for Q tile 1; thread = row
 // Registers: launched at 168; the first warpgroup drops to 56 and the two
 // softmax warpgroups rise to 224: 128 x 56 + 256 x 224 = 384 x 168.
 //
-// Per Q tile q and key tile g the MMA thread issues, in this order,
+// Per Q tile q and key tile g the MMA warp issues, in this order,
 //   O_q += P_q(g-1) V_(g-1)   then   S_q = Q_q K_g^T
-// (P_q is written over the first 64 columns of S_q and read from TMEM), so
+// (P_q is written over the first 64 columns of S_q and read from TMEM; it is
+// handed over in two 64-key halves, so the first half's PV runs while the
+// softmax exponentiates the second), so
 // when S_q(g) is ready, the PV before it has completed too: the lazy O
 // rescale (when a row max grows by more than 2^8) never waits on the tensor
 // core.
@@ -76,8 +79,9 @@ enum {
     C_KE = C_VF + kStages2,     // [2] K stage free (both QKs done)
     C_VE = C_KE + kStages2,     // [2] V stage free (both PVs done)
     C_S = C_VE + kStages2,      // [2 Q tiles] S ready
-    C_P = C_S + 2,              // [2 Q tiles] P written, 128 arrivals
-    C_OD = C_P + 2,             // [2 Q tiles] last PV of the unit done
+    C_P = C_S + 2,              // [2 Q tiles] P of keys 0..63 written, 128 arrivals
+    C_P2 = C_P + 2,             // [2 Q tiles] P of keys 64..127 written, 128 arrivals
+    C_OD = C_P2 + 2,            // [2 Q tiles] last PV of the unit done
     C_L = C_OD + 2,             // [2 slots] list loaded
     C_LF = C_L + 2,             // [2 slots] list released, 8 arrivals (one per softmax warp)
     C_END = C_LF + 2,
@@ -148,7 +152,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // ---- set-up -----------------------------------------------------------
     if (tid == 0) {
         for (int i = 0; i < NBAR2; ++i)
-            mbar_init(bar(i), (i == C_P || i == C_P + 1) ? 128 : (i == C_LF || i == C_LF + 1) ? 8 : 1);
+            mbar_init(bar(i), (i >= C_P && i < C_P2 + 2) ? 128 : (i == C_LF || i == C_LF + 1) ? 8 : 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -260,81 +264,85 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
     } else if (warp == 1) {
         // ---- MMA issuer -----------------------------------------------------
+        // The whole warp runs this loop (waits, descriptor arithmetic) in
+        // lockstep; one elected lane issues each MMA and commit.
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow2));
-        if (lane == 0) {
-            constexpr uint32_t idq = idesc_bf16(false, 128), idp = idesc_bf16(true, 128);
-            // S_q = Q_q K^T for key tile gg (8 MMAs of K = 16 over d = 128)
-            // (descriptor start addresses advance in 16-byte units: offset >> 4;
-            // the bases are rebuilt per call -- hoisting every (tile, stage)
-            // variant out of the loop would not fit this warp's registers)
-            auto qk = [&](int q, int gg) {
-                uint64_t da = desc_k_sw128(sbase + kQOff2 + q * kTile2);
-                uint64_t db = desc_k_sw128(sbase + kKOff2 + (gg % kStages2) * kTile2);
-                asm volatile("" : "+l"(da), "+l"(db));
+        constexpr uint32_t idq = idesc_bf16(false, 128), idp = idesc_bf16(true, 128);
+        // S_q = Q_q K^T for key tile gg (8 MMAs of K = 16 over d = 128);
+        // descriptor start addresses advance in 16-byte units (offset >> 4)
+        auto qk = [&](int q, int gg) {
+            const uint64_t da = desc_k_sw128(sbase + kQOff2 + q * kTile2);
+            const uint64_t db = desc_k_sw128(sbase + kKOff2 + (gg % kStages2) * kTile2);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t off = ((k >> 2) * kChunk2 + (k & 3) * 32) >> 4;
-                    mma_ss(tmem + q * 128, da + off, db + off, idq, k > 0);
-                }
-                mma_commit(bar(C_S + q));
-            };
-            // O_q += P_q V for key tile gg; P_q (bf16) is the first 64 columns of S_q
-            auto pv = [&](int q, int gg, bool acc) {
-                uint64_t db = desc_mn_sw128(sbase + kVOff2 + (gg % kStages2) * kTile2, kChunk2);
-                asm volatile("" : "+l"(db));
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ts(tmem + 256 + q * 128, tmem + q * 128 + 8 * k, db + ((k * 2048) >> 4), idp, acc || k > 0);
-            };
-            bool ok = true;
-            int gt = 0, nq = 0, ul = 0;
-            for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x, ++ul) {
-                const int slot = ul & 1;
-                if (!(ok = mbar_wait(bar(C_L + slot), (ul >> 1) & 1, abort_flag, a.status))) break;
-                const int T = key_tiles(s, cnt_s[slot]);
-                if (T == 0) continue;
-                if (!(ok = mbar_wait(bar(C_Q), nq & 1, abort_flag, a.status))) break;
-                if (!(ok = mbar_wait(bar(C_KF + gt % kStages2), (gt / kStages2) & 1, abort_flag, a.status))) break;
-                tc_fence_after();
-                qk(0, gt);
-                qk(1, gt);
-                mma_commit(bar(C_KE + gt % kStages2));
-                if (T == 1) mma_commit(bar(C_QFREE));
-                for (int t = 0; ok && t < T; ++t) {
-                    const int gg = gt + t;
-                    if (!(ok = mbar_wait(bar(C_P), gg & 1, abort_flag, a.status))) break;
-                    if (!(ok = mbar_wait(bar(C_VF + gg % kStages2), (gg / kStages2) & 1, abort_flag, a.status)))
-                        break;
-                    tc_fence_after();
-                    pv(0, gg, t > 0);
-                    if (t == T - 1) mma_commit(bar(C_OD));
-                    if (t + 1 < T) {
-                        const int g1 = gg + 1;
-                        if (!(ok = mbar_wait(bar(C_KF + g1 % kStages2), (g1 / kStages2) & 1, abort_flag, a.status)))
-                            break;
-                        tc_fence_after();
-                        qk(0, g1);
-                    }
-                    if (!(ok = mbar_wait(bar(C_P + 1), gg & 1, abort_flag, a.status))) break;
-                    tc_fence_after();
-                    pv(1, gg, t > 0);
-                    mma_commit(bar(C_VE + gg % kStages2));
-                    if (t == T - 1) mma_commit(bar(C_OD + 1));
-                    if (t + 1 < T) {
-                        qk(1, gg + 1);
-                        mma_commit(bar(C_KE + (gg + 1) % kStages2));
-                        if (t + 2 == T) mma_commit(bar(C_QFREE));
-                    }
-                }
-                gt += T;
-                ++nq;
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t off = ((k >> 2) * kChunk2 + (k & 3) * 32) >> 4;
+                mma_ss_w(tmem + q * 128, da + off, db + off, idq, k > 0);
             }
-            // drain: every MMA issued above has completed once this arrives
-            // (waited on even after an abort: TMEM is freed only after it)
-            mma_commit(bar(C_END));
-            volatile int never = 0;
-            mbar_wait(bar(C_END), 0, &never, a.status);
+            mma_commit_w(bar(C_S + q));
+        };
+        // O_q += P_q V for keys 64h .. 64h+63 of key tile gg; P_q (bf16) is the
+        // first 64 columns of S_q, handed over in two halves
+        auto pv = [&](int q, int gg, int h, bool acc) {
+            const uint64_t db = desc_mn_sw128(sbase + kVOff2 + (gg % kStages2) * kTile2, kChunk2);
+#pragma unroll
+            for (int k = 4 * h; k < 4 * h + 4; ++k)
+                mma_ts_w(tmem + 256 + q * 128, tmem + q * 128 + 8 * k, db + ((k * 2048) >> 4), idp, acc || k > 0);
+        };
+        auto wait = [&](int i, int parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar(i), parity, abort_flag, a.status));
+        };
+        bool ok = true;
+        int gt = 0, nq = 0, ul = 0;
+        for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x, ++ul) {
+            const int slot = ul & 1;
+            if (!(ok = wait(C_L + slot, (ul >> 1) & 1))) break;
+            const int T = key_tiles(s, cnt_s[slot]);
+            if (T == 0) continue;
+            if (!(ok = wait(C_Q, nq & 1))) break;
+            if (!(ok = wait(C_KF + gt % kStages2, (gt / kStages2) & 1))) break;
+            tc_fence_after();
+            qk(0, gt);
+            qk(1, gt);
+            mma_commit_w(bar(C_KE + gt % kStages2));
+            if (T == 1) mma_commit_w(bar(C_QFREE));
+            for (int t = 0; ok && t < T; ++t) {
+                const int gg = gt + t;
+                if (!(ok = wait(C_P, gg & 1))) break;
+                if (!(ok = wait(C_VF + gg % kStages2, (gg / kStages2) & 1))) break;
+                tc_fence_after();
+                pv(0, gg, 0, t > 0);
+                if (!(ok = wait(C_P2, gg & 1))) break;
+                tc_fence_after();
+                pv(0, gg, 1, true);
+                if (t == T - 1) mma_commit_w(bar(C_OD));
+                if (t + 1 < T) {
+                    const int g1 = gg + 1;
+                    if (!(ok = wait(C_KF + g1 % kStages2, (g1 / kStages2) & 1))) break;
+                    tc_fence_after();
+                    qk(0, g1);
+                }
+                if (!(ok = wait(C_P + 1, gg & 1))) break;
+                tc_fence_after();
+                pv(1, gg, 0, t > 0);
+                if (!(ok = wait(C_P2 + 1, gg & 1))) break;
+                tc_fence_after();
+                pv(1, gg, 1, true);
+                mma_commit_w(bar(C_VE + gg % kStages2));
+                if (t == T - 1) mma_commit_w(bar(C_OD + 1));
+                if (t + 1 < T) {
+                    qk(1, gg + 1);
+                    mma_commit_w(bar(C_KE + (gg + 1) % kStages2));
+                    if (t + 2 == T) mma_commit_w(bar(C_QFREE));
+                }
+            }
+            gt += T;
+            ++nq;
         }
+        // drain: every MMA issued above has completed once this arrives
+        // (waited on even after an abort: TMEM is freed only after it)
+        mma_commit_w(bar(C_END));
+        volatile int never = 0;
+        mbar_wait(bar(C_END), 0, &never, a.status);
     } else if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow2));
     } else {
@@ -398,18 +406,16 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                             xh[k] = vis ? xh[k] : -CUDART_INF_F;
                         }
                     }
-                    float mq[8];
+                    // four independent chains of 3-input maxima
+                    float mq[4];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) mq[e] = xh[e];
+                    for (int e = 0; e < 4; ++e) mq[e] = fmaxf(xh[2 * e], xh[2 * e + 1]);
 #pragma unroll
                     for (int k = 8; k < 64; k += 8)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) mq[e] = fmaxf(mq[e], xh[k + e]);
-#pragma unroll
-                    for (int v = 4; v > 0; v >>= 1)
-#pragma unroll
-                        for (int e = 0; e < v; ++e) mq[e] = fmaxf(mq[e], mq[e + v]);
-                    mh[h] = mq[0] == -CUDART_INF_F ? -CUDART_INF_F : fmaf(mq[0], qk_scale, gl);
+                        for (int e = 0; e < 4; ++e) mq[e] = fmax3(mq[e], xh[k + 2 * e], xh[k + 2 * e + 1]);
+                    const float mm = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
+                    mh[h] = mm == -CUDART_INF_F ? -CUDART_INF_F : fmaf(mm, qk_scale, gl);
                     gh[h] = gl;
                 }
                 const float mx = fmaxf(mh[0], mh[1]);
@@ -438,6 +444,8 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     }
                 }
                 // p = 2^(x * scale + gate - ref), written as bf16 pairs over S columns 0..63
+                // each 64-key half is handed to the MMA warp as soon as it is written,
+                // so the first half's PV runs while the second half is exponentiated
                 const float ref = m_run == -CUDART_INF_F ? 0.f : m_run;
                 float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
@@ -454,11 +462,13 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         pk[k] = *reinterpret_cast<uint32_t *>(&h2);
                     }
                     tmem_st16(tS + 16 * c, pk);
+                    if (c & 1) {
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(bar((c == 1 ? C_P : C_P2) + q));
+                    }
                 }
                 l += ls0 + ls1;
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(C_P + q));
             }
             if (!ok) break;
             // ---- epilogue: O_q / l -> bf16, LSE ----------------------------
