@@ -183,8 +183,16 @@ def traffic_for(kernel: str):
         d = json.load(f).get(kernel)
     if not d:
         return None
-    src = os.path.join(ROOT, d["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
+    # the counters stand only while every source file of the kernel is unchanged
+    if "sources" not in d or "sources_sha256" not in d:
+        return None
+    h = hashlib.sha256()
+    for rel in d["sources"]:
+        src = os.path.join(ROOT, rel)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    if h.hexdigest() != d["sources_sha256"]:
         return None
     return d["dram_bytes_per_launch"]
 

@@ -34,8 +34,8 @@
 // Per Q tile q and key tile g the MMA warp issues, in this order,
 //   O_q += P_q(g-1) V_(g-1)   then   S_q = Q_q K_g^T
 // (P_q is written over the first 64 columns of S_q and read from TMEM; it is
-// handed over in two 64-key halves, so the first half's PV runs while the
-// softmax exponentiates the second), so
+// handed over in four 32-key quarters, so the PV of one quarter runs while the
+// softmax exponentiates the next), so
 // when S_q(g) is ready, the PV before it has completed too: the lazy O
 // rescale (when a row max grows by more than 2^8) never waits on the tensor
 // core.
@@ -79,9 +79,8 @@ enum {
     C_KE = C_VF + kStages2,     // [2] K stage free (both QKs done)
     C_VE = C_KE + kStages2,     // [2] V stage free (both PVs done)
     C_S = C_VE + kStages2,      // [2 Q tiles] S ready
-    C_P = C_S + 2,              // [2 Q tiles] P of keys 0..63 written, 128 arrivals
-    C_P2 = C_P + 2,             // [2 Q tiles] P of keys 64..127 written, 128 arrivals
-    C_OD = C_P2 + 2,            // [2 Q tiles] last PV of the unit done
+    C_P = C_S + 2,              // [2 Q tiles][4 quarters] P of 32 keys written, 128 arrivals
+    C_OD = C_P + 8,             // [2 Q tiles] last PV of the unit done
     C_L = C_OD + 2,             // [2 slots] list loaded
     C_LF = C_L + 2,             // [2 slots] list released, 8 arrivals (one per softmax warp)
     C_END = C_LF + 2,
@@ -107,18 +106,20 @@ struct Unit {
     size_t lu;   // (b, g, j) list row
 };
 
-// Units run heaviest first: the block index j is the slowest-varying
-// coordinate, descending, so the round-robin over CTAs ends on short lists.
+// Unit order: the units of one (batch, kv-head) are contiguous, so the CTAs
+// running at any moment read the K/V of one or two heads and their tiles are
+// re-read from L2 (all heads' K/V together would not fit); within a head the
+// block index runs from the end, so its longest lists go first.
 __device__ __forceinline__ Unit unit_at(const Tc2Args &a, int u) {
     const Shape &s = a.s;
-    const int per_j = s.B * s.Hkv * a.npair;
+    const int per_g = s.nb * a.npair;
     Unit w;
-    w.j = s.nb - 1 - u / per_j;
-    int r = u % per_j;
+    const int bg = u / per_g;
+    int r = u % per_g;
+    w.j = s.nb - 1 - r / a.npair;
     const int pair = r % a.npair;
-    r /= a.npair;
-    w.g = r % s.Hkv;
-    w.b = r / s.Hkv;
+    w.g = bg % s.Hkv;
+    w.b = bg / s.Hkv;
     w.h0 = w.g * s.G + pair * a.hc;
     w.lu = ((size_t)w.b * s.Hkv + w.g) * s.nb + w.j;
     return w;
@@ -152,7 +153,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // ---- set-up -----------------------------------------------------------
     if (tid == 0) {
         for (int i = 0; i < NBAR2; ++i)
-            mbar_init(bar(i), (i >= C_P && i < C_P2 + 2) ? 128 : (i == C_LF || i == C_LF + 1) ? 8 : 1);
+            mbar_init(bar(i), (i >= C_P && i < C_P + 8) ? 128 : (i == C_LF || i == C_LF + 1) ? 8 : 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -280,12 +281,12 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             }
             mma_commit_w(bar(C_S + q));
         };
-        // O_q += P_q V for keys 64h .. 64h+63 of key tile gg; P_q (bf16) is the
-        // first 64 columns of S_q, handed over in two halves
+        // O_q += P_q V for keys 32h .. 32h+31 of key tile gg; P_q (bf16) is the
+        // first 64 columns of S_q, handed over in quarters
         auto pv = [&](int q, int gg, int h, bool acc) {
             const uint64_t db = desc_mn_sw128(sbase + kVOff2 + (gg % kStages2) * kTile2, kChunk2);
 #pragma unroll
-            for (int k = 4 * h; k < 4 * h + 4; ++k)
+            for (int k = 2 * h; k < 2 * h + 2; ++k)
                 mma_ts_w(tmem + 256 + q * 128, tmem + q * 128 + 8 * k, db + ((k * 2048) >> 4), idp, acc || k > 0);
         };
         auto wait = [&](int i, int parity) {
@@ -311,9 +312,12 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (!(ok = wait(C_VF + gg % kStages2, (gg / kStages2) & 1))) break;
                 tc_fence_after();
                 pv(0, gg, 0, t > 0);
-                if (!(ok = wait(C_P2, gg & 1))) break;
-                tc_fence_after();
-                pv(0, gg, 1, true);
+                for (int h = 1; ok && h < 4; ++h) {
+                    if (!(ok = wait(C_P + h, gg & 1))) break;
+                    tc_fence_after();
+                    pv(0, gg, h, true);
+                }
+                if (!ok) break;
                 if (t == T - 1) mma_commit_w(bar(C_OD));
                 if (t + 1 < T) {
                     const int g1 = gg + 1;
@@ -321,12 +325,12 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tc_fence_after();
                     qk(0, g1);
                 }
-                if (!(ok = wait(C_P + 1, gg & 1))) break;
-                tc_fence_after();
-                pv(1, gg, 0, t > 0);
-                if (!(ok = wait(C_P2 + 1, gg & 1))) break;
-                tc_fence_after();
-                pv(1, gg, 1, true);
+                for (int h = 0; ok && h < 4; ++h) {
+                    if (!(ok = wait(C_P + 4 + h, gg & 1))) break;
+                    tc_fence_after();
+                    pv(1, gg, h, t > 0 || h > 0);
+                }
+                if (!ok) break;
                 mma_commit_w(bar(C_VE + gg % kStages2));
                 if (t == T - 1) mma_commit_w(bar(C_OD + 1));
                 if (t + 1 < T) {
@@ -444,31 +448,33 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     }
                 }
                 // p = 2^(x * scale + gate - ref), written as bf16 pairs over S columns 0..63
-                // each 64-key half is handed to the MMA warp as soon as it is written,
-                // so the first half's PV runs while the second half is exponentiated
+                // each 32-key quarter is handed to the MMA warp as soon as it is
+                // written, so its PV runs while the next quarter is exponentiated
+                // (pairs of elements go through the packed fp32 pipe: one FMA and
+                // one add per two keys)
                 const float ref = m_run == -CUDART_INF_F ? 0.f : m_run;
-                float ls0 = 0.f, ls1 = 0.f;
+                const float2 sc2 = make_float2(qk_scale, qk_scale);
+                float2 ls2a = make_float2(0.f, 0.f), ls2b = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const float bias = gh[c >> 1] - ref;
+                    const float2 b2 = make_float2(bias, bias);
                     uint32_t pk[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
-                        const float p0 = ex2(fmaf(x[32 * c + 2 * k], qk_scale, bias));
-                        const float p1 = ex2(fmaf(x[32 * c + 2 * k + 1], qk_scale, bias));
-                        ls0 += p0;
-                        ls1 += p1;
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                        const float2 z = ffma2(make_float2(x[32 * c + 2 * k], x[32 * c + 2 * k + 1]), sc2, b2);
+                        const float2 pp = make_float2(ex2(z.x), ex2(z.y));
+                        if (k & 1) ls2b = fadd2(ls2b, pp);
+                        else ls2a = fadd2(ls2a, pp);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
                         pk[k] = *reinterpret_cast<uint32_t *>(&h2);
                     }
                     tmem_st16(tS + 16 * c, pk);
-                    if (c & 1) {
-                        tmem_wait_st();
-                        tc_fence_before();
-                        mbar_arrive(bar((c == 1 ? C_P : C_P2) + q));
-                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(C_P + 4 * q + c));
                 }
-                l += ls0 + ls1;
+                l += (ls2a.x + ls2a.y) + (ls2b.x + ls2b.y);
             }
             if (!ok) break;
             // ---- epilogue: O_q / l -> bf16, LSE ----------------------------
@@ -480,24 +486,25 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const bool row_ok = qi < s.N;
             __nv_bfloat16 *orow = a.O + (((size_t)w.b * s.Hq + head) * s.N + (row_ok ? qi : 0)) * 128;
             const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float o[32];
+            {
+                // all 128 columns in one TMEM round trip
+                float o[128];
                 if (T > 0) {
-                    tmem_ld32(tO + 32 * cc, o);
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) tmem_ld32(tO + 32 * cc, o + 32 * cc);
                     tmem_wait_ld();
-                    reg_fence<32>(o);
+                    reg_fence<128>(o);
                 } else {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = 0.f;
+                    for (int k = 0; k < 128; ++k) o[k] = 0.f;
                 }
                 if (row_ok) {
 #pragma unroll
-                    for (int v = 0; v < 32; v += 8) {
+                    for (int v = 0; v < 128; v += 8) {
                         float f[8];
 #pragma unroll
                         for (int k = 0; k < 8; ++k) f[k] = o[v + k] * inv;
-                        store16(orow + 32 * cc + v, f);
+                        store16(orow + v, f);
                     }
                 }
             }
