@@ -1,5 +1,6 @@
-// prefill_tc2.cu -- persistent tensor-core gated block-sparse prefill for
-// bf16, d = 128, block 64 or 128, query groups of at least 256 rows.
+// prefill_tc2.cu -- persistent tensor-core block-sparse prefill (gated, plain
+// or hierarchical) for bf16, d = 128, block 64 or 128, query groups of at
+// least 256 rows.
 //
 // Computes what prefill_tc.cu computes ([SAS] "Ключевые факты" / "Как это
 // применить": blockwise softmax attention over the kept blocks only, the
@@ -39,6 +40,13 @@
 // when S_q(g) is ready, the PV before it has completed too: the lazy O
 // rescale (when a row max grows by more than 2^8) never waits on the tensor
 // core.
+//
+// Hierarchical mode ([HiLS]: each kept block gets its own softmax and the
+// blocks are mixed by softmax_b(s_b) of their retrieval scores) uses the same
+// pipeline: per block, P = 2^(x - max_b) * 2^(s_b - M) / l_b with M the list's
+// largest retrieval score, so O needs no rescaling; all of a tile's
+// exponentials are taken before its first quarter is handed over, since the
+// weights need each block's sum.
 //
 // Every mbarrier wait is bounded; on expiry the CTA records kStatusTimeout,
 // stops, lets its copies land, frees TMEM and exits.
@@ -129,6 +137,7 @@ __device__ __forceinline__ Unit unit_at(const Tc2Args &a, int u) {
 __device__ __forceinline__ int key_tiles(const Shape &s, int cnt) { return s.bs == 64 ? (cnt + 1) >> 1 : cnt; }
 
 
+template <bool kHier>
 __global__ void __launch_bounds__(kThreads2, 1)
 prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, Tc2Args a) {
@@ -196,7 +205,8 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (!good) set_status(a.status, kStatusBadIndex);
                 blk_s[e] = good ? blk : -1;
                 const bool forced = (blk == w.j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
-                gate_s[e] = ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[e] - s_loc) * kLog2e : 0.f;
+                gate_s[e] = kHier ? sl[e] * kLog2e
+                            : ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[e] - s_loc) * kLog2e : 0.f;
             }
             if (lane == 0) cnt_s[slot] = cnt;
             __syncwarp();
@@ -358,6 +368,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const uint32_t lane_off = (uint32_t)(32 * qq) << 16;
         const uint32_t tS = tmem + lane_off + q * 128, tO = tmem + lane_off + 256 + q * 128;
         const bool causal = s.flags & SA_CAUSAL;
+        constexpr bool hier = kHier;
         const float qk_scale = s.scale * kLog2e;
         bool ok = true;
         int gt = 0, nq = 0, ul = 0;
@@ -375,6 +386,15 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             else { head = w.h0 + q; ri = r; }
             const int qi = w.j * s.bs + ri;              // query position of this row
             float m_run = -CUDART_INF_F, l = 0.f;
+            // hierarchical mode ([HiLS]): every block gets its own softmax and
+            // the block outputs are weighted by softmax_b(s_b).  With M the
+            // largest retrieval score of the list, block b enters O as
+            // P_b V_b * 2^(s_b - M) / l_b and l sums 2^(s_b - M), so O is never
+            // rescaled and the result is O / l, with LSE = M + log2 l.
+            if constexpr (hier) {
+                for (int e = 0; e < cnt; ++e)
+                    if (blk_s[e] >= 0) m_run = fmaxf(m_run, gate_s[e]);
+            }
             for (int t = 0; t < T; ++t) {
                 ok = mbar_wait(bar(C_S + q), (gt + t) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -386,7 +406,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 reg_fence<128>(x);
                 // per 64-key half: its block, gate and masks (a bad entry, an
                 // odd list's empty half, the ragged end, causality in the local block)
-                float gh[2], mh[2];
+                float gh[2], mh[2], raw[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     int blk, t0;
@@ -419,8 +439,59 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
                         for (int e = 0; e < 4; ++e) mq[e] = fmax3(mq[e], xh[k + 2 * e], xh[k + 2 * e + 1]);
                     const float mm = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
+                    raw[h] = mm;
                     mh[h] = mm == -CUDART_INF_F ? -CUDART_INF_F : fmaf(mm, qk_scale, gl);
                     gh[h] = gl;
+                }
+                if constexpr (hier) {
+                    // per-block softmax: one block per 64-key half (block 64), each
+                    // half handed over as soon as its weight is known; or one block
+                    // per tile (block 128), handed over after both halves
+                    const float2 sc2 = make_float2(qk_scale, qk_scale);
+                    const bool one = s.bs == 128;
+                    const float mt = fmaxf(raw[0], raw[1]);
+                    float lsum0 = 0.f;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float mb = one ? mt : raw[h];
+                        const float nb2 = mb == -CUDART_INF_F ? 0.f : -mb * qk_scale;
+                        const float2 b2 = make_float2(nb2, nb2);
+                        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) {
+                            const float2 z = ffma2(make_float2(x[64 * h + 2 * k], x[64 * h + 2 * k + 1]), sc2, b2);
+                            const float2 pp = make_float2(ex2(z.x), ex2(z.y));
+                            x[64 * h + 2 * k] = pp.x;
+                            x[64 * h + 2 * k + 1] = pp.y;
+                            acc = fadd2(acc, pp);
+                        }
+                        const float lh = acc.x + acc.y;
+                        if (one && h == 0) {
+                            lsum0 = lh;
+                            continue;
+                        }
+                        const float lb = one ? lsum0 + lh : lh;
+                        const float wb = lb > 0.f ? ex2(gh[h] - m_run) : 0.f;
+                        const float fq = lb > 0.f ? wb / lb : 0.f;
+                        l += wb;
+                        // quarters of this half (both halves when the tile is one block)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            if (!one && (c >> 1) != h) continue;
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) {
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(x[32 * c + 2 * k] * fq,
+                                                                          x[32 * c + 2 * k + 1] * fq);
+                                pk[k] = *reinterpret_cast<uint32_t *>(&h2);
+                            }
+                            tmem_st16(tS + 16 * c, pk);
+                            tmem_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(bar(C_P + 4 * q + c));
+                        }
+                    }
+                    continue;
                 }
                 const float mx = fmaxf(mh[0], mh[1]);
                 if (t == 0) {
@@ -538,7 +609,7 @@ int sm_count() {
 
 bool prefill_tc2_supported(const Shape &s) {
     if (s.dtype != SA_BF16 || s.d != 128) return false;
-    if (s.flags & (SA_SELECT_PER_QHEAD | SA_HIER)) return false;
+    if (s.flags & SA_SELECT_PER_QHEAD) return false;
     if (s.bs != 64 && s.bs != 128) return false;
     if ((s.G * s.bs) % kRows) return false;
     if (s.cap > kMaxList2) return false;
@@ -553,8 +624,10 @@ cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, con
     // The register split above assumes the kernel is launched at exactly
     // kRegsLaunch2 registers per thread; anything else could stall the
     // warpgroups' register exchange, so refuse to launch.
+    void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, Tc2Args) =
+        (s.flags & SA_HIER) ? prefill_tc2_kernel<true> : prefill_tc2_kernel<false>;
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_tc2_kernel);
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kRegsLaunch2) return cudaErrorInvalidDeviceFunction;
     CUtensorMap mq, mk, mv;
@@ -575,10 +648,10 @@ cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, con
     a.units = s.B * s.Hkv * s.nb * a.npair;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorNoDevice;
-    e = cudaFuncSetAttribute(prefill_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem2);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem2);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)min(a.units, sms);
-    prefill_tc2_kernel<<<grid, kThreads2, kSmem2, st>>>(mq, mk, mv, a);
+    kern<<<grid, kThreads2, kSmem2, st>>>(mq, mk, mv, a);
     note_launch();
     return cudaGetLastError();
 }

@@ -11,13 +11,13 @@
 // (score desc, index asc) on order-preserving 32-bit keys.
 //
 // CTA = (batch, selection head, tiles j0 .. j0+7); warp w owns tile j0 + w.
-//   1. warp w pools its tile's queries (16-byte loads, 8 per lane in flight);
+//   1. warp w pools its tile's queries (16-byte loads, 16 per lane in flight);
 //   2. the CTA scans landmark rows 0 .. j0+7 once: a group of VPR lanes holds
 //      one row and all eight pooled queries' matching slices, forms the eight
 //      dot products and reduce-scatters them (3 halving exchanges + the rest
 //      of the butterfly), so every row costs eight shuffles, not 32;
-//   3. warp w radix-selects its tile's top-K with a per-warp histogram
-//      (warp-aggregated atomics, __syncwarp only) and writes the list.
+//   3. warp w finds its tile's top-K (bitwise search for the k-th key, then
+//      an index-ordered compaction; warp_select.cuh) and writes the list.
 #include "common.cuh"
 #include "warp_select.cuh"
 
@@ -48,8 +48,7 @@ __global__ void __launch_bounds__(kThreadsT) select_tiles_kernel(TilesArgs a) {
     const Shape &s = a.s;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *qbar = reinterpret_cast<float *>(smem_raw);                     // [kTpc][D]
-    int *hist = reinterpret_cast<int *>(qbar + kTpc * D);                  // [kTpc][256]
-    int *outp = hist + kTpc * 256;                                         // [kTpc][top_k]
+    int *outp = reinterpret_cast<int *>(qbar + kTpc * D);                  // [kTpc][top_k]
     uint32_t *keys = reinterpret_cast<uint32_t *>(outp + kTpc * max(s.top_k, 1));   // [kTpc][kcap]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -75,7 +74,7 @@ __global__ void __launch_bounds__(kThreadsT) select_tiles_kernel(TilesArgs a) {
             const int r0 = j * s.bs, nrows = min(s.bs, s.N - r0);
             R = s.heads_per * nrows;
             const T *Qb = (const T *)a.Q;
-            constexpr int UP = 8;
+            constexpr int UP = 16;
             for (int base = 0; base < R; base += RPW * UP) {
                 uint4 raw[UP];
 #pragma unroll
@@ -128,13 +127,15 @@ __global__ void __launch_bounds__(kThreadsT) select_tiles_kernel(TilesArgs a) {
         for (int uu = 0; uu < U; ++uu) {
             float f[EPV];
             load16(reinterpret_cast<const T *>(&raw[uu]), f);
+            // eight partial dot products, two elements per packed FMA
             float v[kTpc];
 #pragma unroll
             for (int t = 0; t < kTpc; ++t) {
-                float dot = 0.f;
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int i = 0; i < EPV; ++i) dot = fmaf(qv[t][i], f[i], dot);
-                v[t] = dot;
+                for (int i = 0; i < EPV; i += 2)
+                    acc = ffma2(make_float2(qv[t][i], qv[t][i + 1]), make_float2(f[i], f[i + 1]), acc);
+                v[t] = acc.x + acc.y;
             }
             // reduce-scatter 8 values over the VPR lanes of the group
 #pragma unroll
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kThreadsT) select_tiles_kernel(TilesArgs a) {
     const int n = max(0, j - first);
     const uint32_t *cand = kw + first;
     int *op = outp + warp * max(s.top_k, 1);
-    const int nsel = warp_topk_positions(cand, n, s.top_k, hist + warp * 256, op);
+    const int nsel = warp_topk_positions(cand, n, s.top_k, op);
     __syncwarp();
     const size_t u = ((size_t)b * s.Hsel + hs) * s.nb + j;
     int32_t *idx = a.idx + u * s.cap;
@@ -210,8 +211,7 @@ cudaError_t run_tiles(const Shape &s, const void *Q, const void *L, int32_t *idx
     a.ngroups = (s.nb + kTpc - 1) / kTpc;
     const int vpr = s.d * (int)sizeof(T) / 16;
     const int kcap_max = min(s.nb, a.ngroups * kTpc);
-    const size_t smem = (size_t)kTpc * s.d * 4 + (size_t)kTpc * 256 * 4 + (size_t)kTpc * max(s.top_k, 1) * 4 +
-                        (size_t)kTpc * kcap_max * 4;
+    const size_t smem = (size_t)kTpc * s.d * 4 + (size_t)kTpc * max(s.top_k, 1) * 4 + (size_t)kTpc * kcap_max * 4;
     void (*kern)(TilesArgs) = nullptr;
     switch (vpr) {
         case 8: kern = select_tiles_kernel<T, 8>; break;

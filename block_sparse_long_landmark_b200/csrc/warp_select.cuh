@@ -1,90 +1,43 @@
 // warp_select.cuh -- exact top-k of up to a few thousand order-preserving
-// score keys by one warp, with no block-wide barrier: a 4-pass MSB radix
-// select over a per-warp shared-memory histogram (lanes that share a digit add
-// once, via __match_any_sync), then an index-ordered compaction in which keys
-// equal to the threshold are taken lowest position first -- so equal scores
-// go to the lower block index, as the selection rule requires.
+// score keys by one warp, with no block-wide barrier and no shared-memory
+// atomics.
+//
+//   1. The k-th largest key T is found bit by bit, most significant first:
+//      T keeps a candidate bit when at least k keys are >= T with that bit
+//      set.  Bits above the highest bit in which the warp's largest and
+//      smallest keys differ are common to all keys and are taken as they are.
+//      Each step is one compare per key and one warp reduction.
+//   2. A compaction in position order takes every key > T and the first
+//      (k - #keys > T) keys equal to T, so equal scores go to the lower block
+//      index, as the selection rule requires; positions come out ascending.
+// Lists of up to 512 keys are held in registers (16 per lane), longer ones
+// are read from shared memory at every step.
 #pragma once
 
 #include "common.cuh"
 
 namespace sa {
 
-// Exact top-k (n > k) of keys[0..n) for one warp; T = threshold key,
-// take_eq = how many keys equal to T are taken (lowest positions first).
-__device__ __forceinline__ void warp_radix_select(const uint32_t *keys, int n, int k, int *hist, uint32_t &T, int &take_eq) {
-    const int lane = threadIdx.x & 31;
-    uint32_t prefix = 0, mask = 0;
-    int remaining = k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int b = lane; b < 256; b += 32) hist[b] = 0;
-        __syncwarp();
-        for (int i0 = 0; i0 < n; i0 += 32) {
-            const int i = i0 + lane;
-            const uint32_t x = i < n ? keys[i] : 0u;
-            const bool take = i < n && (x & mask) == prefix;
-            const unsigned act = __ballot_sync(0xffffffffu, take);
-            if (take) {
-                const int digit = (int)((x >> shift) & 255);
-                const unsigned same = __match_any_sync(act, digit);
-                if (lane == __ffs(same) - 1) atomicAdd(&hist[digit], __popc(same));
-            }
-        }
-        __syncwarp();
-        const int hi = 255 - 8 * lane;
-        int loc = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) loc += hist[hi - q];
-        int incl = loc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const int excl = incl - loc;
-        int digit = 0, above = 0;
-        if (excl < remaining && remaining <= incl) {
-            int cum = excl;
-            for (int q = 0; q < 8; ++q) {
-                const int c = hist[hi - q];
-                if (cum + c >= remaining) {
-                    digit = hi - q;
-                    above = cum;
-                    break;
-                }
-                cum += c;
-            }
-        }
-        const unsigned who = __ballot_sync(0xffffffffu, excl < remaining && remaining <= incl);
-        const int src = __ffs(who) - 1;
-        digit = __shfl_sync(0xffffffffu, digit, src);
-        above = __shfl_sync(0xffffffffu, above, src);
-        remaining -= above;
-        prefix |= (uint32_t)digit << shift;
-        mask |= 255u << shift;
-        __syncwarp();
-    }
-    T = prefix;
-    take_eq = remaining;
-}
+constexpr int kWarpSelRegSlots = 16;   // keys per lane kept in registers
 
-// Warp exclusive prefix sum.
-__device__ __forceinline__ int warp_excl(int v, int &total) {
-    const int lane = threadIdx.x & 31;
-    int incl = v;
+// Count of keys >= c over the warp.
+template <int SLOTS>
+__device__ __forceinline__ int warp_count_ge_reg(const uint32_t (&r)[SLOTS], uint32_t c) {
+    int n = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    total = __shfl_sync(0xffffffffu, incl, 31);
-    return incl - v;
+    for (int j = 0; j < SLOTS; ++j) n += r[j] >= c;
+    return __reduce_add_sync(0xffffffffu, n);
+}
+__device__ __forceinline__ int warp_count_ge_smem(const uint32_t *keys, int n, uint32_t c) {
+    const int lane = threadIdx.x & 31;
+    int m = 0;
+    for (int i = lane; i < n; i += 32) m += keys[i] >= c;
+    return __reduce_add_sync(0xffffffffu, m);
 }
 
 // Positions (ascending) of the top-k keys of keys[0..n) into out[0..):
-// every position when n <= k.  Returns how many (warp-uniform).  `hist`
-// holds 256 ints of this warp's own.
-__device__ __forceinline__ int warp_topk_positions(const uint32_t *keys, int n, int k, int *hist, int *out) {
+// every position when n <= k.  Returns how many (warp-uniform).
+__device__ __forceinline__ int warp_topk_positions(const uint32_t *keys, int n, int k, int *out) {
     const int lane = threadIdx.x & 31;
     if (k <= 0 || n <= 0) return 0;
     if (n <= k) {
@@ -92,36 +45,63 @@ __device__ __forceinline__ int warp_topk_positions(const uint32_t *keys, int n, 
         __syncwarp();
         return n;
     }
-    uint32_t Tk;
-    int take_eq;
-    warp_radix_select(keys, n, k, hist, Tk, take_eq);
-    const int seg = (n + 31) / 32;
-    const int i0 = min(n, lane * seg), i1 = min(n, i0 + seg);
-    int neq = 0;
-    for (int i = i0; i < i1; ++i) neq += keys[i] == Tk;
-    int tot;
-    const int eq_base = warp_excl(neq, tot);
-    int cntsel = 0;
-    {
-        int e = eq_base;
-        for (int i = i0; i < i1; ++i) {
+    // ---- 1. threshold T = the k-th largest key ----------------------------
+    const bool in_regs = n <= 32 * kWarpSelRegSlots;
+    uint32_t r[kWarpSelRegSlots];
+    uint32_t kmax = 0u, kmin = 0xffffffffu;
+    if (in_regs) {
+#pragma unroll
+        for (int j = 0; j < kWarpSelRegSlots; ++j) {
+            const int i = j * 32 + lane;
+            r[j] = i < n ? keys[i] : 0u;   // padding 0: below every candidate, never counted
+            if (i < n) {
+                kmax = max(kmax, r[j]);
+                kmin = min(kmin, r[j]);
+            }
+        }
+    } else {
+        for (int i = lane; i < n; i += 32) {
             const uint32_t x = keys[i];
-            cntsel += x > Tk || (x == Tk && e < take_eq);
-            e += x == Tk;
+            kmax = max(kmax, x);
+            kmin = min(kmin, x);
         }
     }
-    int nsel;
-    int pos = warp_excl(cntsel, nsel);
-    {
-        int e = eq_base;
-        for (int i = i0; i < i1; ++i) {
-            const uint32_t x = keys[i];
-            if (x > Tk || (x == Tk && e < take_eq)) out[pos++] = i;
-            e += x == Tk;
-        }
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    const uint32_t diff = kmax ^ kmin;
+    const int top = diff ? 31 - __clz(diff) : -1;           // highest differing bit
+    const uint32_t low = top >= 0 ? (0xffffffffu >> (31 - top)) : 0u;
+    uint32_t T = kmax & ~low;                                // common prefix: every key is >= T
+    for (int b = top; b >= 0; --b) {
+        const uint32_t c = T | (1u << b);
+        const int ge = in_regs ? warp_count_ge_reg(r, c) : warp_count_ge_smem(keys, n, c);
+        if (ge >= k) T = c;
+    }
+    int gt = 0;
+    if (in_regs) {
+#pragma unroll
+        for (int j = 0; j < kWarpSelRegSlots; ++j) gt += r[j] > T;
+    } else {
+        for (int i = lane; i < n; i += 32) gt += keys[i] > T;
+    }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    const int take_eq = k - gt;
+    // ---- 2. compaction in position order -----------------------------------
+    const unsigned below = (1u << lane) - 1u;
+    int base = 0, eq_before = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t x = i < n ? keys[i] : 0u;
+        const bool eq = i < n && x == T;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const bool sel = i < n && (x > T || (eq && eq_before + __popc(eqm & below) < take_eq));
+        const unsigned selm = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[base + __popc(selm & below)] = i;
+        base += __popc(selm);
+        eq_before += __popc(eqm);
     }
     __syncwarp();
-    return nsel;
+    return base;
 }
 
 }  // namespace sa

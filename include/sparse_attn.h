@@ -182,7 +182,8 @@ int sparse_attn_prefill(const sa_params *p, const void *Q, const void *K, const 
 /* Which kernel sparse_attn_prefill runs for these parameters:
  *   2 = the persistent tensor-core kernel (tcgen05/TMEM/TMA, one CTA per SM,
  *       256 query rows per work unit; bf16, d = 128, block 64 or 128, query
- *       heads per kv-head a multiple of 256/block, gated or plain),
+ *       heads per kv-head a multiple of 256/block; gated, plain or
+ *       hierarchical),
  *   1 = the two-CTA-per-SM tensor-core kernel (same types, query heads per
  *       kv-head a multiple of 128/block; also hierarchical mode at block 64),
  *   0 = the CUDA-core kernel (every other supported shape, fp32, per-q-head

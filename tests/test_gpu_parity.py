@@ -229,13 +229,22 @@ TC_CASES = {
     "b64_g4_ragged": W["gated_prefill_32k"].scaled(N=3001, Hq=8, Hkv=2, top_k=6),
     "b64_g4_batch2": W["gated_prefill_32k"].scaled(B=2, N=2048, Hq=8, Hkv=2, top_k=9),
     "b128_g2_batch3": W["long_prefill_256k"].scaled(B=3, N=3000, Hq=4, Hkv=2, top_k=4),
+    "b128_hier": W["long_prefill_256k"].scaled(N=4000, Hq=4, Hkv=2, top_k=5, hier=True),
+    "b64_hier_batch2": W["gated_prefill_32k"].scaled(B=2, N=2500, Hq=8, Hkv=2, top_k=6, hier=True),
 }
 
 
-def _expected_kernel(wl):
-    """2 = persistent kernel (256-row units), 1 = two-CTA kernel (128-row tiles)."""
+def _tc1_kernel(wl):
+    """1 when the two-CTA kernel takes the shape (128-row tiles; hierarchical
+    only at block 64), else 0 (CUDA cores)."""
     G = wl.Hq // wl.Hkv
-    return 2 if (G * wl.block) % 256 == 0 and not wl.hier else 1
+    return 1 if (G * wl.block) % 128 == 0 and (not wl.hier or wl.block == 64) else 0
+
+
+def _expected_kernel(wl):
+    """2 = persistent kernel (256-row units), else what the two-CTA kernel takes."""
+    G = wl.Hq // wl.Hkv
+    return 2 if (G * wl.block) % 256 == 0 else _tc1_kernel(wl)
 
 
 @pytest.mark.parametrize("case", sorted(TC_CASES))
@@ -252,9 +261,9 @@ def test_tensor_core_prefill_matches_oracle_and_cuda_core(case, monkeypatch):
     _, _, O, lse = run_prefill(p, Q, K, V, sel=sel)
     _check_outputs(wl, ref, O, lse)
     if kern == 2:
-        # the two tensor-core kernels agree on the same lists
+        # the persistent kernel agrees with the next path on the same lists
         monkeypatch.setenv("SPARSE_ATTN_PREFILL_PATH", "tc1")
-        assert sa.sparse_attn_prefill_kernel(p) == 1
+        assert sa.sparse_attn_prefill_kernel(p) == _tc1_kernel(wl)
         _, _, O1, lse1 = run_prefill(p, Q, K, V, sel=sel)
         _check_outputs(wl, ref, O1, lse1)
         assert (O.float() - O1.float()).abs().max().item() <= 2e-2
