@@ -10,15 +10,14 @@
 //   2. A compaction in position order takes every key > T and the first
 //      (k - #keys > T) keys equal to T, so equal scores go to the lower block
 //      index, as the selection rule requires; positions come out ascending.
-// Lists of up to 512 keys are held in registers (16 per lane), longer ones
-// are read from shared memory at every step.
+// Lists of up to 32 * REG_SLOTS keys are held in registers (REG_SLOTS per
+// lane), longer ones are read from shared memory at every step; REG_SLOTS = 0
+// keeps every list in shared memory (for kernels short of registers).
 #pragma once
 
 #include "common.cuh"
 
 namespace sa {
-
-constexpr int kWarpSelRegSlots = 16;   // keys per lane kept in registers
 
 // Count of keys >= c over the warp.
 template <int SLOTS>
@@ -37,7 +36,9 @@ __device__ __forceinline__ int warp_count_ge_smem(const uint32_t *keys, int n, u
 
 // Positions (ascending) of the top-k keys of keys[0..n) into out[0..):
 // every position when n <= k.  Returns how many (warp-uniform).
+template <int REG_SLOTS = 16>
 __device__ __forceinline__ int warp_topk_positions(const uint32_t *keys, int n, int k, int *out) {
+    constexpr int kSlots = REG_SLOTS > 0 ? REG_SLOTS : 1;
     const int lane = threadIdx.x & 31;
     if (k <= 0 || n <= 0) return 0;
     if (n <= k) {
@@ -46,12 +47,12 @@ __device__ __forceinline__ int warp_topk_positions(const uint32_t *keys, int n, 
         return n;
     }
     // ---- 1. threshold T = the k-th largest key ----------------------------
-    const bool in_regs = n <= 32 * kWarpSelRegSlots;
-    uint32_t r[kWarpSelRegSlots];
+    const bool in_regs = REG_SLOTS > 0 && n <= 32 * REG_SLOTS;
+    uint32_t r[kSlots];
     uint32_t kmax = 0u, kmin = 0xffffffffu;
     if (in_regs) {
 #pragma unroll
-        for (int j = 0; j < kWarpSelRegSlots; ++j) {
+        for (int j = 0; j < kSlots; ++j) {
             const int i = j * 32 + lane;
             r[j] = i < n ? keys[i] : 0u;   // padding 0: below every candidate, never counted
             if (i < n) {
@@ -80,7 +81,7 @@ __device__ __forceinline__ int warp_topk_positions(const uint32_t *keys, int n, 
     int gt = 0;
     if (in_regs) {
 #pragma unroll
-        for (int j = 0; j < kWarpSelRegSlots; ++j) gt += r[j] > T;
+        for (int j = 0; j < kSlots; ++j) gt += r[j] > T;
     } else {
         for (int i = lane; i < n; i += 32) gt += keys[i] > T;
     }
