@@ -465,6 +465,49 @@ def secondary_prefill(name, args, pk, psrc):
     return out
 
 
+# fp32 FMA peak of the CUDA cores, derived from unit counts and the clock:
+# 148 SMs x 128 FP32 lanes x 2 FLOP x 1.965 GHz (no measured figure exists).
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def secondary_backward(name, args, pk, psrc):
+    """One backward step (attention backward + selector backward) of the gated
+    prefill, the forward's outputs and an upstream gradient resident in HBM."""
+    import block_sparse_long_landmark_b200 as sa
+    base = name.replace("_backward", "")
+    wl, p, t = prefill_case(_wl(base, args), "cuda")
+    prefill_step(p, t)
+    g = torch.Generator(device="cuda").manual_seed(11)
+    dO = torch.randn(t["Q"].shape, generator=g, device="cuda", dtype=torch.float32).to(t["Q"].dtype)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    grads = (torch.empty(t["Q"].shape, **f32), torch.empty(t["K"].shape, **f32), torch.empty(t["V"].shape, **f32),
+             torch.empty(t["sel"][1].shape, **f32))
+
+    def step(tm):
+        tmr = tm or (lambda n, f: f())
+        tmr("prefill_backward", lambda: sa.prefill_backward(p, t["Q"], t["K"], t["V"], t["O"], t["lse"], dO,
+                                                            *t["sel"], t["ws"], out=grads))
+        tmr("select_backward", lambda: sa.select_backward(p, t["Q"], t["L"], t["sel"][0], grads[3], t["sel"][2],
+                                                          grads[0], grads[1], t["ws"]))
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    steps = 2
+    el, kms, launches, clocks = run_timed(step, steps, 3, Ranks.single(), flush)
+    # 10 d FLOP per kept (row, key) pair: z, dO.V, dQ, dK, dV; the forward's count is 4 d per pair
+    flops = prefill_flops(wl, t["sel"][2]) * 10 / 4
+    ach = flops / (kms["prefill_backward"] / 1e3) / 1e12
+    out = {"metric": "prefill backward tokens/s", "value": wl.N * wl.B / (el / steps / 1e3), "unit": "tokens/s",
+           "ms_per_step": el / steps, "kernels_ms": kms, "config": workload_config(wl), "gpu_launches": launches,
+           "roofline": {"bound": "alu", "achieved": ach, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                        "frac": ach / FP32_ALU_TFLOPS, "kernel": "prefill_backward",
+                        "peak_source": "derived: 148 SMs x 128 fp32 FMA x 2 x 1.965 GHz",
+                        "algorithmic_flops_per_launch": flops, "traffic": None},
+           "clocks": clocks}
+    del t, grads, dO
+    torch.cuda.empty_cache()
+    return out
+
+
 def secondary_decode(name, args, pk, psrc):
     varlen = name.endswith("_varlen")
     wl = _wl(name[:-len("_varlen")] if varlen else name, args)
@@ -517,8 +560,9 @@ def run_ours(args, ranks):
     pk, psrc = peaks()
     if args.only:
         # one workload alone (small profiling cases): a short report, no baselines
-        kind = inputs.WORKLOADS[args.only.replace("_varlen", "")].kind
-        fn = secondary_decode if kind == "decode" else secondary_prefill
+        kind = inputs.WORKLOADS[args.only.replace("_varlen", "").replace("_backward", "")].kind
+        fn = (secondary_backward if args.only.endswith("_backward") else
+              secondary_decode if kind == "decode" else secondary_prefill)
         print(json.dumps({"only": args.only, **fn(args.only, args, pk, psrc)}), flush=True)
         return 0
     base = inputs.WORKLOADS[args.workload]
@@ -553,8 +597,12 @@ def run_ours(args, ranks):
         if not args.no_secondary:
             sec = {}
             for name in ("gated_decode_128k", "hils_decode_1m", "long_prefill_256k", "hils_prefill_32k",
-                         "gated_decode_128k_varlen"):
+                         "gated_decode_128k_varlen", "gated_prefill_32k_backward"):
                 try:
+                    if name.endswith("_backward"):
+                        sec[name] = secondary_backward(name, args, pk, psrc)
+                        torch.cuda.empty_cache()
+                        continue
                     kind = inputs.WORKLOADS[name.replace("_varlen", "")].kind
                     sec[name] = (secondary_decode if kind == "decode" else secondary_prefill)(name, args, pk, psrc)
                 except torch.cuda.OutOfMemoryError as e:   # pragma: no cover

@@ -21,6 +21,7 @@ from .inputs import F_CAUSAL, F_GATE, F_HIER, F_LOCAL, F_PER_QHEAD, F_SINK  # no
 SA_SINK, SA_LOCAL, SA_GATE, SA_HIER, SA_CAUSAL, SA_SELECT_PER_QHEAD = 1, 2, 4, 8, 16, 32
 SA_BF16, SA_FP32 = 0, 1
 SA_OP_LANDMARKS, SA_OP_SELECT, SA_OP_SELECT_DECODE, SA_OP_PREFILL, SA_OP_DECODE = 0, 1, 2, 3, 4
+SA_OP_PREFILL_BACKWARD, SA_OP_SELECT_BACKWARD = 5, 6
 SA_OK, SA_ERR_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_LAUNCH, SA_ERR_DEVICE = 0, -1, -2, -3, -4, -5
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libsparse_attn.so")
@@ -31,6 +32,7 @@ EXPORTS = (
     "sparse_attn_version", "sparse_attn_launch_count", "sparse_attn_decode_static",
     "sparse_attn_prefill_kernel", "sparse_attn_last_cuda_error", "sparse_attn_cuda_error_string",
     "sparse_attn_landmarks_update", "sparse_attn_select_decode_varlen", "sparse_attn_decode_varlen",
+    "sparse_attn_prefill_backward", "sparse_attn_select_backward",
 )
 
 
@@ -96,6 +98,10 @@ def lib() -> ctypes.CDLL:
             L.sparse_attn_prefill_kernel.restype = i
             L.sparse_attn_decode_static.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             L.sparse_attn_decode_static.restype = i
+            L.sparse_attn_prefill_backward.argtypes = [P] + [vp] * 14 + [sz, vp]
+            L.sparse_attn_prefill_backward.restype = i
+            L.sparse_attn_select_backward.argtypes = [P] + [vp] * 8 + [sz, vp]
+            L.sparse_attn_select_backward.restype = i
             L.sparse_attn_launch_count.argtypes = []
             L.sparse_attn_launch_count.restype = ctypes.c_ulonglong
             _lib = L
@@ -128,6 +134,17 @@ def sparse_attn_prefill(p, Q, K, V, idx, score, count, O, lse, ws, ws_bytes, str
 
 def sparse_attn_decode(p, q, K, V, idx, score, count, o, lse, ws, ws_bytes, stream) -> int:
     return lib().sparse_attn_decode(ctypes.byref(p), q, K, V, idx, score, count, o, lse, ws, ws_bytes, stream)
+
+
+def sparse_attn_prefill_backward(p, Q, K, V, O, lse, dO, idx, score, count, dQ, dK, dV, dscore, ws, ws_bytes,
+                                 stream) -> int:
+    return lib().sparse_attn_prefill_backward(ctypes.byref(p), Q, K, V, O, lse, dO, idx, score, count, dQ, dK, dV,
+                                              dscore, ws, ws_bytes, stream)
+
+
+def sparse_attn_select_backward(p, Q, L, idx, dscore, count, dQ, dK, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_select_backward(ctypes.byref(p), Q, L, idx, dscore, count, dQ, dK, ws, ws_bytes,
+                                             stream)
 
 
 def sparse_attn_prefill_kernel(p) -> int:
@@ -220,7 +237,7 @@ def _hsel(p):
 def workspace(p: sa_params, device="cuda"):
     """A zero-filled workspace large enough for every operation of `p`."""
     torch = _torch()
-    n = max(sparse_attn_workspace_size(p, op) for op in range(5))
+    n = max(sparse_attn_workspace_size(p, op) for op in range(7))
     if n == 0:
         raise SparseAttnError(SA_ERR_ARG, "workspace_size")
     return torch.zeros(n, dtype=torch.uint8, device=device)
@@ -279,6 +296,30 @@ def decode(p, q, K, V, idx, sc, cnt, ws, out=None, stream=None):
     _check(sparse_attn_decode(p, _ptr(q), _ptr(K), _ptr(V), _ptr(idx), _ptr(sc), _ptr(cnt), _ptr(o), _ptr(lse),
                               _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_decode")
     return o, lse
+
+
+def prefill_backward(p, Q, K, V, O, lse, dO, idx, sc, cnt, ws, out=None, stream=None):
+    """Gradients of the gated prefill: (dQ, dK, dV, dscore), all fp32."""
+    torch = _torch()
+    if out is None:
+        f32 = dict(dtype=torch.float32, device=Q.device)
+        dQ = torch.empty(Q.shape, **f32)
+        dK = torch.empty(K.shape, **f32)
+        dV = torch.empty(V.shape, **f32)
+        dscore = torch.empty(sc.shape, **f32)
+    else:
+        dQ, dK, dV, dscore = out
+    _check(sparse_attn_prefill_backward(p, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _ptr(dO), _ptr(idx),
+                                        _ptr(sc), _ptr(cnt), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dscore), _ptr(ws),
+                                        ws.numel(), _stream(stream)), "sparse_attn_prefill_backward")
+    return dQ, dK, dV, dscore
+
+
+def select_backward(p, Q, L, idx, dscore, cnt, dQ, dK, ws, stream=None):
+    """Adds the selector's gradient (through pooled query and landmarks) into dQ, dK."""
+    _check(sparse_attn_select_backward(p, _ptr(Q), _ptr(L), _ptr(idx), _ptr(dscore), _ptr(cnt), _ptr(dQ), _ptr(dK),
+                                       _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_select_backward")
+    return dQ, dK
 
 
 def decode_static(p, q, K, V, idx, sc, cnt, out=None, stream=None):

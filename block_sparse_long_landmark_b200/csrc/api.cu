@@ -73,6 +73,8 @@ size_t sparse_attn_workspace_size(const sa_params *p, int op) {
         case SA_OP_SELECT: extra = select_workspace(s, false); break;
         case SA_OP_SELECT_DECODE: extra = select_workspace(s, true); break;
         case SA_OP_DECODE: extra = decode_workspace(s); break;
+        case SA_OP_PREFILL_BACKWARD: extra = prefill_backward_workspace(s); break;
+        case SA_OP_SELECT_BACKWARD: extra = select_backward_workspace(s); break;
         default: break;
     }
     return kStatusBytes + ((extra + 255) & ~(size_t)255);
@@ -176,6 +178,37 @@ int sparse_attn_decode_varlen(const sa_params *p, const void *q, const void *K, 
                               void *ws, size_t ws_bytes, void *stream) {
     if (!seq_len) return SA_ERR_ARG;
     return decode_common(p, q, K, V, seq_len, idx, score, count, o, lse, ws, ws_bytes, stream);
+}
+
+int sparse_attn_prefill_backward(const sa_params *p, const void *Q, const void *K, const void *V, const void *O,
+                                 const float *lse, const void *dO, const int32_t *idx, const float *score,
+                                 const int32_t *count, float *dQ, float *dK, float *dV, float *dscore, void *ws,
+                                 size_t ws_bytes, void *stream) {
+    Shape s;
+    int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    if (!backward_supported(s)) return SA_ERR_UNSUPPORTED;
+    if (!Q || !K || !V || !O || !lse || !dO || !idx || !score || !count || !dQ || !dK || !dV || !dscore || !ws)
+        return SA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(dQ) ||
+        !aligned16(dK) || !aligned16(dV) || !aligned16(ws))
+        return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_PREFILL_BACKWARD)) return SA_ERR_WORKSPACE;
+    return launch_result(launch_prefill_backward(s, Q, K, V, O, lse, dO, idx, score, count, dQ, dK, dV, dscore, ws,
+                                                 (cudaStream_t)stream));
+}
+
+int sparse_attn_select_backward(const sa_params *p, const void *Q, const void *L, const int32_t *idx,
+                                const float *dscore, const int32_t *count, float *dQ, float *dK, void *ws,
+                                size_t ws_bytes, void *stream) {
+    Shape s;
+    int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    if (!backward_supported(s)) return SA_ERR_UNSUPPORTED;
+    if (!Q || !L || !idx || !dscore || !count || !dQ || !dK || !ws) return SA_ERR_ARG;
+    if (!aligned16(Q) || !aligned16(L) || !aligned16(dQ) || !aligned16(dK) || !aligned16(ws)) return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_SELECT_BACKWARD)) return SA_ERR_WORKSPACE;
+    return launch_result(launch_select_backward(s, Q, L, idx, dscore, count, dQ, dK, ws, (cudaStream_t)stream));
 }
 
 int sparse_attn_check_status(void *ws, void *stream, int *detail) {

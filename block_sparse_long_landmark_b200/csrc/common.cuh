@@ -160,5 +160,15 @@ cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const vo
                           const float *score, const int32_t *count, void *o, float *lse, void *ws,
                           size_t ws_bytes, cudaStream_t st);
 size_t decode_workspace(const Shape &s);
+bool backward_supported(const Shape &s);
+size_t prefill_backward_workspace(const Shape &s);
+size_t select_backward_workspace(const Shape &s);
+cudaError_t launch_prefill_backward(const Shape &s, const void *Q, const void *K, const void *V, const void *O,
+                                    const float *lse, const void *dO, const int32_t *idx, const float *score,
+                                    const int32_t *count, float *dQ, float *dK, float *dV, float *dscore,
+                                    void *ws, cudaStream_t st);
+cudaError_t launch_select_backward(const Shape &s, const void *Q, const void *L, const int32_t *idx,
+                                   const float *dscore, const int32_t *count, float *dQ, float *dK, void *ws,
+                                   cudaStream_t st);
 
 }  // namespace sa

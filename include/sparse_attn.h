@@ -87,7 +87,9 @@ enum {
     SA_OP_SELECT = 1,         /* prefill selection                                 */
     SA_OP_SELECT_DECODE = 2,
     SA_OP_PREFILL = 3,
-    SA_OP_DECODE = 4
+    SA_OP_DECODE = 4,
+    SA_OP_PREFILL_BACKWARD = 5,
+    SA_OP_SELECT_BACKWARD = 6
 };
 
 /* return codes */
@@ -225,6 +227,44 @@ int sparse_attn_decode_static(const sa_params *p, const void *q, const void *K, 
 int sparse_attn_decode_varlen(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *seq_len,
                               const int32_t *idx, const float *score, const int32_t *count, void *o, float *lse,
                               void *ws, size_t ws_bytes, void *stream);
+
+/* Backward of the gated (or plain) block-sparse prefill -- [SAS] "Как это
+ * применить": the selector's score enters the softmax as the gate
+ * g_c = log_sigmoid(s_c - s_local), which is how the loss reaches the
+ * selector; the top-K choice itself is hard ("Ключевые факты") and the kept
+ * lists of the forward pass are reused as they are.
+ * Inputs: Q [B,Hq,N,d], K, V [B,Hkv,N,d] (dtype of p), the forward's O
+ * [B,Hq,N,d] and LSE [B,Hq,N] (fp32, natural log), the upstream gradient dO
+ * [B,Hq,N,d] (dtype of p) and the lists idx/score/count of
+ * sparse_attn_select.  Outputs, all fp32 and overwritten:
+ *   dQ [B,Hq,N,d]  = scale dZ K over the kept keys of each row,
+ *   dK, dV [B,Hkv,N,d] = scale dZ^T Q and P^T dO summed over every row that
+ *                  keeps the key (accumulated with atomics, so the last bits
+ *                  may vary between runs),
+ *   dscore [B,Hkv,nb,cap]: gradient with respect to each list entry's score:
+ *                  dg_c sigmoid(-(s_c - s_local)) for gated entries, minus
+ *                  their sum for the local block's entry, 0 otherwise,
+ * with P = exp(z - LSE), dZ = P (dO V^T - rowsum(dO O)) and dg_c the sum of
+ * dZ over entry c's keys.  Workspace: SA_OP_PREFILL_BACKWARD.  Gated or plain
+ * mode with per-kv-head lists, d = 64 or 128; SA_HIER or
+ * SA_SELECT_PER_QHEAD give SA_ERR_UNSUPPORTED.  CUDA cores, fp32. */
+int sparse_attn_prefill_backward(const sa_params *p, const void *Q, const void *K, const void *V, const void *O,
+                                 const float *lse, const void *dO, const int32_t *idx, const float *score,
+                                 const int32_t *count, float *dQ, float *dK, float *dV, float *dscore, void *ws,
+                                 size_t ws_bytes, void *stream);
+
+/* The selector's part of the backward: the scores s_c = scale <qbar, L_c>
+ * ([SAS] "Ключевые факты": a light selector scores the blocks) carry dscore
+ * back to the pooled query qbar (mean of the unit's G heads x block rows of
+ * Q) and to the landmarks L (means of the blocks' keys, landmark rounding
+ * taken as the identity):  dQ[rows of the unit] += scale sum_c dscore_c L_c / R
+ * and dK[keys of block b] += scale sum over entries c with block b of
+ * dscore_c qbar / n_b.  Adds into the dQ and dK of
+ * sparse_attn_prefill_backward (fp32).  Q, L as given to sparse_attn_select.
+ * Workspace: SA_OP_SELECT_BACKWARD.  Same support as above. */
+int sparse_attn_select_backward(const sa_params *p, const void *Q, const void *L, const int32_t *idx,
+                                const float *dscore, const int32_t *count, float *dQ, float *dK, void *ws,
+                                size_t ws_bytes, void *stream);
 
 /* Synchronises `stream`, returns SA_OK or SA_ERR_DEVICE from the status
  * word in `ws`, and clears it.  *detail (may be NULL) receives the raw bits:

@@ -100,3 +100,21 @@ def test_varlen_entry_points_need_lengths():
     assert sa.sparse_attn_decode_varlen(p, a, a, a, None, a, a, a, a, a, a, 1 << 20, None) == sa.SA_ERR_ARG
     assert sa.sparse_attn_landmarks_update(p, None, a, None, None, None) == sa.SA_ERR_ARG
     assert sa.sparse_attn_landmarks_update(_p(Hq=7), a, a, None, None, None) == sa.SA_ERR_ARG
+
+
+def test_backward_entry_points_check_arguments():
+    """Every call below fails its host-side checks before any launch."""
+    p = _p()
+    a = 256
+    ptrs = [a] * 14                                   # Q K V O lse dO idx score count dQ dK dV dscore ws
+    hier = _p(flags=sa.SA_SINK | sa.SA_LOCAL | sa.SA_HIER | sa.SA_CAUSAL)
+    assert sa.sparse_attn_prefill_backward(hier, *ptrs, 1 << 20, None) == sa.SA_ERR_UNSUPPORTED
+    assert sa.sparse_attn_select_backward(hier, a, a, a, a, a, a, a, a, 1 << 20, None) == sa.SA_ERR_UNSUPPORTED
+    nulls = list(ptrs)
+    nulls[5] = None                                   # dO
+    assert sa.sparse_attn_prefill_backward(p, *nulls, 1 << 20, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_prefill_backward(p, *ptrs, 16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.sparse_attn_select_backward(p, a, a, a, a, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.sparse_attn_select_backward(p, None, a, a, a, a, a, a, a, 1 << 20, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_workspace_size(p, sa.SA_OP_PREFILL_BACKWARD) > 256
+    assert sa.sparse_attn_workspace_size(p, sa.SA_OP_SELECT_BACKWARD) > 256
