@@ -47,6 +47,23 @@ struct BwArgs {
 template <typename T>
 __device__ __forceinline__ float ld1(const T *p) { return to_f(*p); }
 
+// N = 2 or 4 consecutive floats (8- or 16-byte aligned)
+template <int N>
+__device__ __forceinline__ void vload(const float *p, float *v) {
+    if constexpr (N == 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(p);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    } else {
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        v[0] = x.x; v[1] = x.y;
+    }
+}
+template <int N>
+__device__ __forceinline__ void vatomic_add(float *p, const float *v) {
+    if constexpr (N == 4) atomicAdd(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
+    else atomicAdd(reinterpret_cast<float2 *>(p), make_float2(v[0], v[1]));
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kBwThreads) bwd_attn_kernel(BwArgs a) {
     const Shape &s = a.s;
@@ -136,12 +153,20 @@ __global__ void __launch_bounds__(kBwThreads) bwd_attn_kernel(BwArgs a) {
                 float z[8], dp[8];
 #pragma unroll
                 for (int m = 0; m < 8; ++m) z[m] = dp[m] = 0.f;
-                for (int e = 0; e < D; ++e) {
-                    const float kv = sk[t * DP + e], vv = sv[t * DP + e];
+                // row operands as 16-byte broadcast loads, key operands per lane
+                for (int e = 0; e < D; e += 4) {
+                    float kv[4], vv[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        kv[x] = sk[t * DP + e + x];
+                        vv[x] = sv[t * DP + e + x];
+                    }
 #pragma unroll
                     for (int m = 0; m < 8; ++m) {
-                        z[m] = fmaf(sq[(warp + 8 * m) * D + e], kv, z[m]);
-                        dp[m] = fmaf(sdo[(warp + 8 * m) * D + e], vv, dp[m]);
+                        const float4 q4 = *reinterpret_cast<const float4 *>(sq + (warp + 8 * m) * D + e);
+                        const float4 d4 = *reinterpret_cast<const float4 *>(sdo + (warp + 8 * m) * D + e);
+                        z[m] = fmaf(q4.x, kv[0], fmaf(q4.y, kv[1], fmaf(q4.z, kv[2], fmaf(q4.w, kv[3], z[m]))));
+                        dp[m] = fmaf(d4.x, vv[0], fmaf(d4.y, vv[1], fmaf(d4.z, vv[2], fmaf(d4.w, vv[3], dp[m]))));
                     }
                 }
 #pragma unroll
@@ -167,7 +192,8 @@ __global__ void __launch_bounds__(kBwThreads) bwd_attn_kernel(BwArgs a) {
                     for (int cc = 0; cc < EPT; ++cc) dq[m][cc] = fmaf(w, sk[t * DP + lane + 32 * cc], dq[m][cc]);
                 }
             }
-            // dK, dV (keys warp + 8m', columns lane + 32c)
+            // dK, dV (keys warp + 8m', columns lane*EPT .. lane*EPT+EPT-1: vector
+            // loads of the row operands and one vector atomic per key and lane)
 #pragma unroll
             for (int m = 0; m < kKC / 8; ++m) {
                 const int t = warp + 8 * m, key = kc + t;
@@ -176,18 +202,20 @@ __global__ void __launch_bounds__(kBwThreads) bwd_attn_kernel(BwArgs a) {
                 for (int cc = 0; cc < EPT; ++cc) ak[cc] = av[cc] = 0.f;
                 for (int i = 0; i < kRC; ++i) {
                     const float wz = sZ[i * (kKC + 1) + t], wp = sP[i * (kKC + 1) + t];
+                    float qv[EPT], dv[EPT];
+                    vload<EPT>(sq + i * D + lane * EPT, qv);
+                    vload<EPT>(sdo + i * D + lane * EPT, dv);
 #pragma unroll
                     for (int cc = 0; cc < EPT; ++cc) {
-                        ak[cc] = fmaf(wz, sq[i * D + lane + 32 * cc], ak[cc]);
-                        av[cc] = fmaf(wp, sdo[i * D + lane + 32 * cc], av[cc]);
+                        ak[cc] = fmaf(wz, qv[cc], ak[cc]);
+                        av[cc] = fmaf(wp, dv[cc], av[cc]);
                     }
                 }
                 if (key < t1) {
 #pragma unroll
-                    for (int cc = 0; cc < EPT; ++cc) {
-                        atomicAdd(a.dK + (kvhead + key) * D + lane + 32 * cc, s.scale * ak[cc]);
-                        atomicAdd(a.dV + (kvhead + key) * D + lane + 32 * cc, av[cc]);
-                    }
+                    for (int cc = 0; cc < EPT; ++cc) ak[cc] *= s.scale;
+                    vatomic_add<EPT>(a.dK + (kvhead + key) * D + lane * EPT, ak);
+                    vatomic_add<EPT>(a.dV + (kvhead + key) * D + lane * EPT, av);
                 }
             }
         }
