@@ -192,30 +192,39 @@ __global__ void __launch_bounds__(kBwThreads) bwd_attn_kernel(BwArgs a) {
                     for (int cc = 0; cc < EPT; ++cc) dq[m][cc] = fmaf(w, sk[t * DP + lane + 32 * cc], dq[m][cc]);
                 }
             }
-            // dK, dV (keys warp + 8m', columns lane*EPT .. lane*EPT+EPT-1: vector
-            // loads of the row operands and one vector atomic per key and lane)
+            // dK, dV (keys warp + 8m', columns lane*EPT .. lane*EPT+EPT-1): each
+            // row's q and dO slices are loaded once (vector loads) for the
+            // thread's four keys; one vector atomic per key and lane at the end
+            {
+                constexpr int KT = kKC / 8;
+                float ak[KT][EPT], av[KT][EPT];
 #pragma unroll
-            for (int m = 0; m < kKC / 8; ++m) {
-                const int t = warp + 8 * m, key = kc + t;
-                float ak[EPT], av[EPT];
+                for (int m = 0; m < KT; ++m)
 #pragma unroll
-                for (int cc = 0; cc < EPT; ++cc) ak[cc] = av[cc] = 0.f;
+                    for (int cc = 0; cc < EPT; ++cc) ak[m][cc] = av[m][cc] = 0.f;
                 for (int i = 0; i < kRC; ++i) {
-                    const float wz = sZ[i * (kKC + 1) + t], wp = sP[i * (kKC + 1) + t];
                     float qv[EPT], dv[EPT];
                     vload<EPT>(sq + i * D + lane * EPT, qv);
                     vload<EPT>(sdo + i * D + lane * EPT, dv);
 #pragma unroll
-                    for (int cc = 0; cc < EPT; ++cc) {
-                        ak[cc] = fmaf(wz, qv[cc], ak[cc]);
-                        av[cc] = fmaf(wp, dv[cc], av[cc]);
+                    for (int m = 0; m < KT; ++m) {
+                        const float wz = sZ[i * (kKC + 1) + warp + 8 * m], wp = sP[i * (kKC + 1) + warp + 8 * m];
+#pragma unroll
+                        for (int cc = 0; cc < EPT; ++cc) {
+                            ak[m][cc] = fmaf(wz, qv[cc], ak[m][cc]);
+                            av[m][cc] = fmaf(wp, dv[cc], av[m][cc]);
+                        }
                     }
                 }
-                if (key < t1) {
 #pragma unroll
-                    for (int cc = 0; cc < EPT; ++cc) ak[cc] *= s.scale;
-                    vatomic_add<EPT>(a.dK + (kvhead + key) * D + lane * EPT, ak);
-                    vatomic_add<EPT>(a.dV + (kvhead + key) * D + lane * EPT, av);
+                for (int m = 0; m < KT; ++m) {
+                    const int key = kc + warp + 8 * m;
+                    if (key < t1) {
+#pragma unroll
+                        for (int cc = 0; cc < EPT; ++cc) ak[m][cc] *= s.scale;
+                        vatomic_add<EPT>(a.dK + (kvhead + key) * D + lane * EPT, ak[m]);
+                        vatomic_add<EPT>(a.dV + (kvhead + key) * D + lane * EPT, av[m]);
+                    }
                 }
             }
         }
