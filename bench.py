@@ -349,9 +349,14 @@ def calibrate_units(wl, Q64, K64, V64, target_s):
     """Units whose oracle time is about target_s: two probes fit t = a + b n
     (a: the landmarks of the touched kv-heads, b: one unit's selection and
     attention)."""
+    # a first call pays one-time costs (the oracle's build and load, first
+    # touch of the inputs) that must not enter the fit
+    oracle_prefill_sample(wl, Q64, K64, V64, 4, seed=97)
     t1, _, _ = oracle_prefill_sample(wl, Q64, K64, V64, 16, seed=98)
     t2, _, _ = oracle_prefill_sample(wl, Q64, K64, V64, 64, seed=99)
-    b = max((t2 - t1) / 48, 1e-6)
+    # per-unit cost: the slope, but never below half the larger probe's mean
+    # (timing noise can flatten the slope and inflate the sample)
+    b = max((t2 - t1) / 48, 0.5 * t2 / 64, 1e-6)
     a = max(t1 - 16 * b, 0.0)
     return max(16, min(50000, int((target_s - a) / b)))
 
