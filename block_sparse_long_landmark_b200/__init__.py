@@ -33,6 +33,7 @@ EXPORTS = (
     "sparse_attn_prefill_kernel", "sparse_attn_last_cuda_error", "sparse_attn_cuda_error_string",
     "sparse_attn_landmarks_update", "sparse_attn_select_decode_varlen", "sparse_attn_decode_varlen",
     "sparse_attn_prefill_backward", "sparse_attn_select_backward",
+    "sparse_attn_lsa_clusters", "sparse_attn_lsa_workspace_size", "sparse_attn_lsa_build", "sparse_attn_lsa_decode",
 )
 
 
@@ -43,6 +44,13 @@ class sa_params(ctypes.Structure):
 
     def __repr__(self):
         return "sa_params(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class sa_lsa_params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int),
+                ("N", ctypes.c_int), ("pool", ctypes.c_int), ("seg", ctypes.c_int), ("clusters", ctypes.c_int),
+                ("top_clusters", ctypes.c_int), ("sink", ctypes.c_int), ("window", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("scale", ctypes.c_float)]
 
 
 class SparseAttnError(RuntimeError):
@@ -102,6 +110,15 @@ def lib() -> ctypes.CDLL:
             L.sparse_attn_prefill_backward.restype = i
             L.sparse_attn_select_backward.argtypes = [P] + [vp] * 8 + [sz, vp]
             L.sparse_attn_select_backward.restype = i
+            LP = ctypes.POINTER(sa_lsa_params)
+            L.sparse_attn_lsa_clusters.argtypes = [LP]
+            L.sparse_attn_lsa_clusters.restype = i
+            L.sparse_attn_lsa_workspace_size.argtypes = [LP]
+            L.sparse_attn_lsa_workspace_size.restype = sz
+            L.sparse_attn_lsa_build.argtypes = [LP, vp, vp, vp, vp, vp]
+            L.sparse_attn_lsa_build.restype = i
+            L.sparse_attn_lsa_decode.argtypes = [LP] + [vp] * 9 + [sz, vp]
+            L.sparse_attn_lsa_decode.restype = i
             L.sparse_attn_launch_count.argtypes = []
             L.sparse_attn_launch_count.restype = ctypes.c_ulonglong
             _lib = L
@@ -140,6 +157,23 @@ def sparse_attn_prefill_backward(p, Q, K, V, O, lse, dO, idx, score, count, dQ, 
                                  stream) -> int:
     return lib().sparse_attn_prefill_backward(ctypes.byref(p), Q, K, V, O, lse, dO, idx, score, count, dQ, dK, dV,
                                               dscore, ws, ws_bytes, stream)
+
+
+def sparse_attn_lsa_clusters(p: sa_lsa_params) -> int:
+    return int(lib().sparse_attn_lsa_clusters(ctypes.byref(p)))
+
+
+def sparse_attn_lsa_workspace_size(p: sa_lsa_params) -> int:
+    return int(lib().sparse_attn_lsa_workspace_size(ctypes.byref(p)))
+
+
+def sparse_attn_lsa_build(p, K, centres, members, sizes, stream) -> int:
+    return lib().sparse_attn_lsa_build(ctypes.byref(p), K, centres, members, sizes, stream)
+
+
+def sparse_attn_lsa_decode(p, q, K, V, centres, members, sizes, o, lse, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_lsa_decode(ctypes.byref(p), q, K, V, centres, members, sizes, o, lse, ws, ws_bytes,
+                                        stream)
 
 
 def sparse_attn_select_backward(p, Q, L, idx, dscore, count, dQ, dK, ws, ws_bytes, stream) -> int:
@@ -320,6 +354,49 @@ def select_backward(p, Q, L, idx, dscore, cnt, dQ, dK, ws, stream=None):
     _check(sparse_attn_select_backward(p, _ptr(Q), _ptr(L), _ptr(idx), _ptr(dscore), _ptr(cnt), _ptr(dQ), _ptr(dK),
                                        _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_select_backward")
     return dQ, dK
+
+
+def make_lsa_params(B, Hq, Hkv, d, N, pool, seg, clusters, top_clusters, sink, window, dtype="bf16",
+                    scale=0.0) -> sa_lsa_params:
+    dt = {"bf16": SA_BF16, "fp32": SA_FP32}.get(dtype, dtype)
+    return sa_lsa_params(B, Hq, Hkv, d, N, pool, seg, clusters, top_clusters, sink, window, dt, float(scale))
+
+
+def lsa_build(p: sa_lsa_params, K, stream=None):
+    """Flat clustered index of K: (centres fp64, members int32, sizes int32)."""
+    torch = _torch()
+    C = sparse_attn_lsa_clusters(p)
+    if C < 0:
+        raise SparseAttnError(C, "sparse_attn_lsa_clusters")
+    n = max(C, 1)
+    centres = torch.empty(p.B, p.Hkv, n, p.d, dtype=torch.float64, device=K.device)
+    members = torch.empty(p.B, p.Hkv, n, p.seg, dtype=torch.int32, device=K.device)
+    sizes = torch.empty(p.B, p.Hkv, n, dtype=torch.int32, device=K.device)
+    _check(sparse_attn_lsa_build(p, _ptr(K), _ptr(centres), _ptr(members), _ptr(sizes), _stream(stream)),
+           "sparse_attn_lsa_build")
+    return centres, members, sizes
+
+
+def lsa_workspace(p: sa_lsa_params, device="cuda"):
+    torch = _torch()
+    n = sparse_attn_lsa_workspace_size(p)
+    if n == 0:
+        raise SparseAttnError(SA_ERR_ARG, "sparse_attn_lsa_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def lsa_decode(p: sa_lsa_params, q, K, V, index, ws, out=None, stream=None):
+    """Decode through the flat index: (o, lse)."""
+    torch = _torch()
+    centres, members, sizes = index
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(p.B, p.Hq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(sparse_attn_lsa_decode(p, _ptr(q), _ptr(K), _ptr(V), _ptr(centres), _ptr(members), _ptr(sizes), _ptr(o),
+                                  _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_lsa_decode")
+    return o, lse
 
 
 def decode_static(p, q, K, V, idx, sc, cnt, out=None, stream=None):

@@ -7,6 +7,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "lsa.cuh"
 
 using namespace sa;
 
@@ -50,6 +51,38 @@ int resolve(const sa_params *p, Shape &s) {
     s.first_block = nullptr;
     if ((long long)s.B * s.Hq * s.nb > (1ll << 31) - 1) return SA_ERR_UNSUPPORTED;
     if (s.heads_per * s.d > 2048) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+// Resolves and checks a flat-index parameter block.
+int resolve_lsa(const sa_lsa_params *p, LsaShape &s) {
+    if (!p) return SA_ERR_ARG;
+    if (p->B <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->N <= 0 || p->pool <= 0) return SA_ERR_ARG;
+    if (p->Hq % p->Hkv) return SA_ERR_ARG;
+    if (p->dtype != SA_BF16 && p->dtype != SA_FP32) return SA_ERR_ARG;
+    if (p->seg < 2 || p->clusters < 1 || p->clusters > p->seg) return SA_ERR_ARG;
+    if (p->top_clusters < 0 || p->sink < 0 || p->window < 0) return SA_ERR_ARG;
+    if (!(p->scale >= 0.f) || isinf(p->scale)) return SA_ERR_ARG;
+    if (p->d != 64 && p->d != 128) return SA_ERR_UNSUPPORTED;
+    if (p->seg > 64 || p->N > (1 << 20) || p->top_clusters > 4096) return SA_ERR_UNSUPPORTED;
+    if ((long long)p->pool * p->seg > (1ll << 30)) return SA_ERR_UNSUPPORTED;
+    s.B = p->B;
+    s.Hq = p->Hq;
+    s.Hkv = p->Hkv;
+    s.G = p->Hq / p->Hkv;
+    s.d = p->d;
+    s.N = p->N;
+    s.pool = p->pool;
+    s.seg = p->seg;
+    s.clusters = p->clusters;
+    s.top_clusters = p->top_clusters;
+    s.sink = p->sink;
+    s.window = p->window;
+    s.dtype = p->dtype;
+    s.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+    s.nseg = p->N / (p->pool * p->seg);
+    s.ctotal = s.nseg * p->clusters;
+    if ((long long)s.B * s.Hkv * s.nseg > (1ll << 31) - 1) return SA_ERR_UNSUPPORTED;
     return SA_OK;
 }
 
@@ -209,6 +242,44 @@ int sparse_attn_select_backward(const sa_params *p, const void *Q, const void *L
     if (!aligned16(Q) || !aligned16(L) || !aligned16(dQ) || !aligned16(dK) || !aligned16(ws)) return SA_ERR_ARG;
     if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_SELECT_BACKWARD)) return SA_ERR_WORKSPACE;
     return launch_result(launch_select_backward(s, Q, L, idx, dscore, count, dQ, dK, ws, (cudaStream_t)stream));
+}
+
+int sparse_attn_lsa_clusters(const sa_lsa_params *p) {
+    LsaShape s;
+    const int r = resolve_lsa(p, s);
+    return r != SA_OK ? r : s.ctotal;
+}
+
+size_t sparse_attn_lsa_workspace_size(const sa_lsa_params *p) {
+    LsaShape s;
+    if (resolve_lsa(p, s) != SA_OK) return 0;
+    const size_t scores = (size_t)s.B * s.Hkv * (size_t)s.ctotal * sizeof(double);
+    return kStatusBytes + ((scores + 255) & ~(size_t)255);
+}
+
+int sparse_attn_lsa_build(const sa_lsa_params *p, const void *K, double *centres, int32_t *members, int32_t *sizes,
+                          void *stream) {
+    LsaShape s;
+    const int r = resolve_lsa(p, s);
+    if (r != SA_OK) return r;
+    if (!K || !aligned16(K)) return SA_ERR_ARG;
+    if (s.ctotal > 0 && (!centres || !members || !sizes)) return SA_ERR_ARG;
+    return launch_result(launch_lsa_build(s, K, centres, members, sizes, (cudaStream_t)stream));
+}
+
+int sparse_attn_lsa_decode(const sa_lsa_params *p, const void *q, const void *K, const void *V,
+                           const double *centres, const int32_t *members, const int32_t *sizes, void *o, float *lse,
+                           void *ws, size_t ws_bytes, void *stream) {
+    LsaShape s;
+    const int r = resolve_lsa(p, s);
+    if (r != SA_OK) return r;
+    if (!q || !K || !V || !o || !lse || !ws) return SA_ERR_ARG;
+    if (s.ctotal > 0 && (!centres || !members || !sizes)) return SA_ERR_ARG;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(ws)) return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_lsa_workspace_size(p)) return SA_ERR_WORKSPACE;
+    double *scores = reinterpret_cast<double *>(static_cast<unsigned char *>(ws) + kStatusBytes);
+    return launch_result(launch_lsa_decode(s, q, K, V, centres, members, sizes, scores, static_cast<unsigned *>(ws),
+                                           o, lse, (cudaStream_t)stream));
 }
 
 int sparse_attn_check_status(void *ws, void *stream, int *detail) {

@@ -266,6 +266,55 @@ int sparse_attn_select_backward(const sa_params *p, const void *Q, const void *L
                                 const float *dscore, const int32_t *count, float *dQ, float *dK, void *ws,
                                 size_t ws_bytes, void *stream);
 
+/* ---- Flat clustered index (the Latent Sparse Attention post, section
+ * "Индекс перестаёт перебирать весь контекст") -----------------------------
+ * Keys are pooled into items (means of `pool` adjacent keys); every complete
+ * segment of `seg` items (all seg * pool keys present) is clustered by Ward's
+ * method into `clusters` clusters, frozen from then on; the index keeps each
+ * cluster's centre and its items.  A decode query (the mean of its kv-group's
+ * query heads) is scored against every centre, scale * <q, centre>; the best
+ * `top_clusters`, by (score desc, cluster id asc), are expanded back to their
+ * key positions; the first `sink` and the last `window` positions are always
+ * added; each query head attends (plain softmax) to that set.  The clustering
+ * runs in the raw key space: the post's learned projections are not modelled.
+ * Clusters of a segment are numbered by their first item; cluster c of
+ * segment g has global id g * clusters + c. */
+typedef struct {
+    int B, Hq, Hkv;     /* batch, query heads, key/value heads (Hq % Hkv == 0)       */
+    int d;              /* head dim: 64 or 128                                         */
+    int N;              /* context length (the query sits at N - 1), 1 .. 2^20         */
+    int pool;           /* keys per item, >= 1                                         */
+    int seg;            /* items per segment, 2 .. 64                                  */
+    int clusters;       /* clusters per segment, 1 .. seg                              */
+    int top_clusters;   /* clusters a query expands, 0 .. 4096                         */
+    int sink, window;   /* always-kept first / last positions, >= 0                    */
+    int dtype;          /* SA_BF16 or SA_FP32 for q, K, V and o                        */
+    float scale;        /* score and logit scale; 0 -> 1/sqrt(d)                       */
+} sa_lsa_params;
+
+/* Clusters per (batch, kv-head): (N / (pool * seg)) * clusters, or a negative
+ * SA_ERR_* code for invalid / unsupported parameters. */
+int sparse_attn_lsa_clusters(const sa_lsa_params *p);
+
+/* Workspace bytes for sparse_attn_lsa_decode (status word + scores), 0 when
+ * the parameters are invalid. */
+size_t sparse_attn_lsa_workspace_size(const sa_lsa_params *p);
+
+/* Builds the index of every (batch, kv-head) from K [B,Hkv,N,d]:
+ * centres [B,Hkv,C,d] (fp64: the clustering's own precision), members
+ * [B,Hkv,C,seg] (item ids of each cluster, ascending, -1 padded), sizes
+ * [B,Hkv,C]; C = sparse_attn_lsa_clusters(p).  Caller-owned buffers. */
+int sparse_attn_lsa_build(const sa_lsa_params *p, const void *K, double *centres, int32_t *members, int32_t *sizes,
+                          void *stream);
+
+/* Decode through the index: q [B,Hq,d], K, V [B,Hkv,N,d] and the index of
+ * sparse_attn_lsa_build -> o [B,Hq,d] (dtype of p), lse [B,Hq] (fp32, natural
+ * log; -inf when nothing is kept).  A member entry outside the context sets
+ * status bit 1 and is skipped. */
+int sparse_attn_lsa_decode(const sa_lsa_params *p, const void *q, const void *K, const void *V,
+                           const double *centres, const int32_t *members, const int32_t *sizes, void *o, float *lse,
+                           void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronises `stream`, returns SA_OK or SA_ERR_DEVICE from the status
  * word in `ws`, and clears it.  *detail (may be NULL) receives the raw bits:
  * 1 index list entry out of range, 2 NaN score, 4 bounded wait expired. */

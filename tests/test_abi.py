@@ -118,3 +118,26 @@ def test_backward_entry_points_check_arguments():
     assert sa.sparse_attn_select_backward(p, None, a, a, a, a, a, a, a, 1 << 20, None) == sa.SA_ERR_ARG
     assert sa.sparse_attn_workspace_size(p, sa.SA_OP_PREFILL_BACKWARD) > 256
     assert sa.sparse_attn_workspace_size(p, sa.SA_OP_SELECT_BACKWARD) > 256
+
+
+def test_lsa_entry_points_check_arguments():
+    """Host-side checks of the flat-index entry points; nothing is launched."""
+    ok = sa.make_lsa_params(1, 4, 2, 128, 4096, 4, 32, 8, 6, 16, 64)
+    assert sa.sparse_attn_lsa_clusters(ok) == (4096 // 128) * 8
+    assert sa.sparse_attn_lsa_workspace_size(ok) > 256
+    for bad, code in [
+        (dict(Hq=5), sa.SA_ERR_ARG), (dict(pool=0), sa.SA_ERR_ARG), (dict(seg=1), sa.SA_ERR_ARG),
+        (dict(clusters=40), sa.SA_ERR_ARG), (dict(top_clusters=-1), sa.SA_ERR_ARG), (dict(d=96), sa.SA_ERR_UNSUPPORTED),
+        (dict(seg=65, clusters=4), sa.SA_ERR_UNSUPPORTED), (dict(N=(1 << 20) + 1), sa.SA_ERR_UNSUPPORTED),
+    ]:
+        kw = dict(B=1, Hq=4, Hkv=2, d=128, N=4096, pool=4, seg=32, clusters=8, top_clusters=6, sink=16, window=64)
+        kw.update(bad)
+        p = sa.make_lsa_params(**kw)
+        assert sa.sparse_attn_lsa_clusters(p) == code, bad
+        assert sa.sparse_attn_lsa_workspace_size(p) == 0
+        assert sa.sparse_attn_lsa_build(p, 256, 256, 256, 256, None) == code
+    a = 256
+    assert sa.sparse_attn_lsa_build(ok, None, a, a, a, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_lsa_build(ok, a, None, a, a, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_lsa_decode(ok, a, a, a, a, a, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.sparse_attn_lsa_decode(ok, None, a, a, a, a, a, a, a, a, 1 << 20, None) == sa.SA_ERR_ARG
