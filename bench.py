@@ -513,6 +513,53 @@ def secondary_backward(name, args, pk, psrc):
     return out
 
 
+# flat clustered index (Latent Sparse Attention style): 8 kv-heads of one
+# 32K sequence, 4-key items, 64-item segments of 16 clusters, 64 clusters
+# expanded per query, 64 sink and 1024 window positions
+LSA_DECODE_32K = dict(B=1, Hq=32, Hkv=8, d=128, N=32768, pool=4, seg=64, clusters=16, top_clusters=64, sink=64,
+                      window=1024)
+
+
+def secondary_lsa(name, args, pk, psrc):
+    """Decode through the flat clustered index; the index is built once,
+    outside the timed region (its build time is reported beside)."""
+    import block_sparse_long_landmark_b200 as sa
+    c = LSA_DECODE_32K
+    p = sa.make_lsa_params(**c)
+    g = torch.Generator(device="cuda").manual_seed(21)
+    q = torch.randn(c["B"], c["Hq"], c["d"], generator=g, device="cuda").to(torch.bfloat16)
+    K = torch.randn(c["B"], c["Hkv"], c["N"], c["d"], generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn(c["B"], c["Hkv"], c["N"], c["d"], generator=g, device="cuda").to(torch.bfloat16)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    index = sa.lsa_build(p, K)
+    s1.record()
+    torch.cuda.synchronize()
+    build_ms = s0.elapsed_time(s1)
+    ws = sa.lsa_workspace(p)
+    out = (torch.empty_like(q), torch.empty(c["B"], c["Hq"], dtype=torch.float32, device="cuda"))
+
+    def step(tm):
+        (tm or (lambda n, f: f()))("lsa_decode", lambda: sa.lsa_decode(p, q, K, V, index, ws, out=out))
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    steps = 5
+    el, kms, launches, clocks = run_timed(step, steps, 3, Ranks.single(), flush)
+    C = sa.sparse_attn_lsa_clusters(p)
+    per_cluster = c["seg"] * c["pool"]              # upper bound: a cluster holds at most a whole segment
+    kept = min(c["N"], c["sink"] + c["window"] + c["top_clusters"] * per_cluster)
+    nbytes = c["B"] * c["Hkv"] * (C * c["d"] * 8 + kept * c["d"] * 2 * 2)
+    hbm = pk["hbm_gbs"]
+    ach = nbytes / (kms["lsa_decode"] / 1e3) / 1e9
+    return {"metric": "lsa decode queries/s", "value": c["B"] / (el / steps / 1e3), "unit": "queries/s",
+            "ms_per_step": el / steps, "kernels_ms": kms, "index_build_ms": build_ms, "config": dict(c),
+            "gpu_launches": launches,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                         "algorithmic_bytes_upper_bound": nbytes, "traffic": None,
+                         "peak_source": psrc + " HBM copy"},
+            "clocks": clocks}
+
+
 def secondary_decode(name, args, pk, psrc):
     varlen = name.endswith("_varlen")
     wl = _wl(name[:-len("_varlen")] if varlen else name, args)
@@ -565,9 +612,12 @@ def run_ours(args, ranks):
     pk, psrc = peaks()
     if args.only:
         # one workload alone (small profiling cases): a short report, no baselines
-        kind = inputs.WORKLOADS[args.only.replace("_varlen", "").replace("_backward", "")].kind
-        fn = (secondary_backward if args.only.endswith("_backward") else
-              secondary_decode if kind == "decode" else secondary_prefill)
+        if args.only == "lsa_decode_32k":
+            fn = secondary_lsa
+        else:
+            kind = inputs.WORKLOADS[args.only.replace("_varlen", "").replace("_backward", "")].kind
+            fn = (secondary_backward if args.only.endswith("_backward") else
+                  secondary_decode if kind == "decode" else secondary_prefill)
         print(json.dumps({"only": args.only, **fn(args.only, args, pk, psrc)}), flush=True)
         return 0
     base = inputs.WORKLOADS[args.workload]
@@ -602,8 +652,15 @@ def run_ours(args, ranks):
         if not args.no_secondary:
             sec = {}
             for name in ("gated_decode_128k", "hils_decode_1m", "long_prefill_256k", "hils_prefill_32k",
-                         "gated_decode_128k_varlen", "gated_prefill_32k_backward"):
+                         "gated_decode_128k_varlen", "gated_prefill_32k_backward", "lsa_decode_32k"):
                 try:
+                    if name == "lsa_decode_32k":
+                        try:
+                            sec[name] = secondary_lsa(name, args, pk, psrc)
+                        except Exception as e:   # pragma: no cover -- recorded, the headline line still prints
+                            sec[name] = {"error": f"{type(e).__name__}: {e}"}
+                        torch.cuda.empty_cache()
+                        continue
                     if name.endswith("_backward"):
                         sec[name] = secondary_backward(name, args, pk, psrc)
                         torch.cuda.empty_cache()
