@@ -1,0 +1,75 @@
+"""Host-side logic of bench.py (no GPU): the traffic counters are used only
+while the kernel's sources are unchanged, the oracle sample is calibrated
+without one-time costs, and the single-rank aggregation and config fields."""
+from __future__ import annotations
+
+import hashlib
+import json
+import os
+import shutil
+
+import pytest
+
+import bench
+from block_sparse_long_landmark_b200 import inputs
+
+
+def test_traffic_is_used_only_for_the_measured_sources(tmp_path, monkeypatch):
+    entry = json.load(open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")))["prefill_gated_prefill_32k"]
+    # the committed counters match the committed sources
+    assert bench.traffic_for("prefill_gated_prefill_32k") == entry["dram_bytes_per_launch"]
+    # a copy of the tree with one source byte changed: the counters no longer apply
+    root = tmp_path / "repo"
+    for rel in entry["sources"] + ["profiles/ncu_traffic.json"]:
+        dst = root / rel
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy(os.path.join(bench.ROOT, rel), dst)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.traffic_for("prefill_gated_prefill_32k") == entry["dram_bytes_per_launch"]
+    src = root / entry["sources"][0]
+    src.write_bytes(src.read_bytes() + b"\n")
+    assert bench.traffic_for("prefill_gated_prefill_32k") is None
+    assert bench.traffic_for("no_such_kernel") is None
+
+
+def test_traffic_hash_covers_every_source():
+    entry = json.load(open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")))["prefill_gated_prefill_32k"]
+    h = hashlib.sha256()
+    for rel in entry["sources"]:
+        h.update(open(os.path.join(bench.ROOT, rel), "rb").read())
+    assert h.hexdigest() == entry["sources_sha256"]
+    assert any(r.endswith("prefill_tc2.cu") for r in entry["sources"])
+
+
+def test_calibration_ignores_one_time_costs(monkeypatch):
+    """The first oracle call pays the build and first-touch costs; the sample
+    size must come from the steady per-unit cost, not from that outlier."""
+    calls = []
+
+    def fake(wl, Q, K, V, n, seed=0):
+        first = not calls
+        calls.append(n)
+        return (30.0 if first else 0.0) + 0.01 * n, n * wl.block / wl.Hkv, 8
+
+    monkeypatch.setattr(bench, "oracle_prefill_sample", fake)
+    wl = inputs.WORKLOADS["gated_prefill_32k"]
+    n = bench.calibrate_units(wl, None, None, None, 15.0)
+    assert 1000 <= n <= 1600            # 15 s at 10 ms per unit, within the fit's slack
+    assert calls[0] < 16                # the warm-up call is a small one
+
+
+def test_calibration_with_a_flat_slope_stays_bounded(monkeypatch):
+    times = {4: 1.0, 16: 1.0, 64: 1.0}  # noise: no visible slope between the probes
+    monkeypatch.setattr(bench, "oracle_prefill_sample", lambda wl, Q, K, V, n, seed=0: (times[n], 1.0, 8))
+    n = bench.calibrate_units(inputs.WORKLOADS["gated_prefill_32k"], None, None, None, 15.0)
+    assert n <= 2 * 15.0 / (1.0 / 64)   # never more than twice what the larger probe's mean implies
+
+
+def test_single_rank_aggregation_and_config():
+    r = bench.Ranks.single()
+    value, t = bench.aggregate(r, 500.0, 1000.0)
+    assert t == 500.0 and value == pytest.approx(2000.0)
+    c = bench.workload_config(inputs.WORKLOADS["gated_prefill_32k"])
+    for k in ("workload", "global_batch", "seq_len", "parallelism", "l2"):
+        assert k in c
+    assert bench.FP32_ALU_TFLOPS == pytest.approx(148 * 128 * 2 * 1.965e9 / 1e12)
