@@ -21,7 +21,15 @@
  *   [LSA]  Latent Sparse Attention post (rit.work), section "Индекс перестаёт
  *          перебирать весь контекст": adjacent keys are pooled before
  *          scoring; the start of the context and a recent window are always
- *          added.
+ *          added; the flat clustered index (sparse_attn_lsa_*) follows its
+ *          cluster-centre scan.
+ *
+ * Groups of entry points: the path (landmarks, selection, prefill, decode),
+ * ragged decode batches and landmark refresh, the backward of the gated
+ * prefill (sparse_attn_prefill_backward, sparse_attn_select_backward), the
+ * flat clustered index (sparse_attn_lsa_*), a decode that allocates nothing
+ * (sparse_attn_decode_static), and helpers (workspace sizes, status word,
+ * error strings, counters).
  *
  * Conventions for every call
  *   - All tensor pointers are DEVICE pointers, 16-byte aligned, dense

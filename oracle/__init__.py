@@ -2,9 +2,11 @@
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  It shares no code with the CUDA library
-and never imports it.  The arithmetic lives in ``oracle.c`` (plain C, every
-step in double); this module compiles it with gcc, loads it with ctypes and
-walks the units of a problem in the order the method takes its steps:
+and never imports it.  The forward path's arithmetic lives in ``oracle.c``
+(plain C, every step in double); this module compiles it with gcc, loads it
+with ctypes and walks the units of a problem in the order the method takes its
+steps (the backward pass, ``backward.py``, and the flat clustered index,
+``lsa.py``, are plain numpy in float64):
 
   1. landmarks  -- mean of each block's keys ([HiLS] opening section: chunk
                    summaries named landmarks; [LSA] "Индекс перестаёт
