@@ -34,34 +34,39 @@ import numpy as np
 from . import default_scale
 
 
-def ward_merges(X: np.ndarray, n_clusters: int) -> np.ndarray:
+def ward_merges(X: np.ndarray, n_clusters: int, weights=None) -> np.ndarray:
     """Ward's agglomerative clustering of the rows of X down to n_clusters.
 
     Returns labels [len(X)] in 0..n_clusters-1, numbered in order of each
     cluster's first item.  Every step merges the two clusters A, B with the
     smallest increase of the within-cluster sum of squares,
         |A| |B| / (|A| + |B|) * ||c_A - c_B||^2,
-    ties to the pair with the lowest (first id, second id)."""
+    ties to the pair with the lowest (first id, second id).  ``weights``: the
+    mass of each row (default 1), so that rows standing for groups of points
+    merge as those groups would; |A| is then the summed mass."""
     X = np.asarray(X, np.float64)
     n = X.shape[0]
     n_clusters = max(1, min(n_clusters, n))
+    w = np.ones(n) if weights is None else np.asarray(weights, np.float64)
     members = {i: [i] for i in range(n)}
     cent = {i: X[i].copy() for i in range(n)}
+    mass = {i: float(w[i]) for i in range(n)}
     while len(members) > n_clusters:
         ids = sorted(members)
         best = None
         for ai, a in enumerate(ids):
             for b in ids[ai + 1:]:
-                na, nb = len(members[a]), len(members[b])
+                na, nb = mass[a], mass[b]
                 diff = cent[a] - cent[b]
                 cost = na * nb / (na + nb) * float(diff @ diff)
                 if best is None or cost < best[0]:
                     best = (cost, a, b)
         _, a, b = best
-        na, nb = len(members[a]), len(members[b])
+        na, nb = mass[a], mass[b]
         cent[a] = (na * cent[a] + nb * cent[b]) / (na + nb)
+        mass[a] = na + nb
         members[a] = sorted(members[a] + members[b])
-        del members[b], cent[b]
+        del members[b], cent[b], mass[b]
     labels = np.empty(n, dtype=np.int64)
     for new, cid in enumerate(sorted(members, key=lambda c: members[c][0])):
         labels[members[cid]] = new
@@ -151,3 +156,52 @@ def decode(q, K, V, pool: int, seg: int, clusters_per_seg: int, top_clusters: in
             for h in range(g * G, (g + 1) * G):
                 O[b, h], LSE[b, h] = attend(q[b, h], K[b, g], V[b, g], pos, scale)
     return {"O": O, "LSE": LSE, "kept": kept}
+
+
+# ---------------------------------------------------------------------------
+# Tree variant (same section of the post: the clusters are combined into a
+# hierarchy that a beam search walks, keeping a few good branches per level,
+# so a query needs a number of comparisons that grows logarithmically).
+# Reading: the flat index's clusters are the leaves; every level above is a
+# Ward clustering of the level below, weighted by the items each node holds,
+# into ceil(n / fanout) nodes; a node's centre is the mean of all its items.
+# ---------------------------------------------------------------------------
+
+def build_tree(index: dict, fanout: int) -> list:
+    """Levels from the leaves up: level 0 = the flat clusters.  Each level is
+    dict(centres, mass, children) with children = lists of ids one level down."""
+    cent = np.asarray(index["centres"], np.float64)
+    mass = np.asarray([len(p) for p in index["positions"]], np.float64)
+    levels = [{"centres": cent, "mass": mass, "children": [[c] for c in range(len(cent))]}]
+    while len(levels[-1]["centres"]) > fanout:
+        below = levels[-1]
+        n = len(below["centres"])
+        lab = ward_merges(below["centres"], (n + fanout - 1) // fanout, weights=below["mass"])
+        kids = [list(np.nonzero(lab == c)[0]) for c in range(lab.max() + 1)]
+        m = np.asarray([below["mass"][k].sum() for k in kids])
+        c = np.stack([(below["mass"][k][:, None] * below["centres"][k]).sum(axis=0) / below["mass"][k].sum()
+                      for k in kids])
+        levels.append({"centres": c, "mass": m, "children": kids})
+    return levels
+
+
+def tree_select(levels: list, q: np.ndarray, beam: int, top_clusters: int, scale: float):
+    """Beam search from the top level down; returns (leaf ids ascending, number
+    of centre comparisons).  At each level the `beam` best nodes by (score
+    desc, id asc) are kept and expanded; at the leaves the `top_clusters`
+    best of the reached ones are returned."""
+    q = np.asarray(q, np.float64)
+    if len(levels) == 0 or len(levels[0]["centres"]) == 0 or top_clusters <= 0:
+        return np.zeros(0, dtype=np.int64), 0
+    top = len(levels) - 1
+    frontier = list(range(len(levels[top]["centres"])))
+    compared = 0
+    for lv in range(top, -1, -1):
+        s = scale * (levels[lv]["centres"][frontier] @ q)
+        compared += len(frontier)
+        order = sorted(range(len(frontier)), key=lambda i: (-s[i], frontier[i]))
+        keep = [frontier[i] for i in order[:(top_clusters if lv == 0 else beam)]]
+        if lv == 0:
+            return np.asarray(sorted(keep), dtype=np.int64), compared
+        frontier = sorted(c for node in keep for c in levels[lv]["children"][node])
+    return np.zeros(0, dtype=np.int64), compared

@@ -84,3 +84,57 @@ def test_kept_positions_add_sink_and_window_and_stay_causal():
     assert {0, 1, 2, 36, 37, 38, 39, 40} <= set(pos.tolist())
     assert pos.max() <= 40 and np.all(np.diff(pos) > 0)
     assert set(idx["positions"][0].tolist()) & set(range(41)) <= set(pos.tolist())
+
+
+def test_weighted_ward_equals_ward_on_the_repeated_points():
+    """Rows of mass m merge as m copies of the row would (checked on the
+    first merge, where the copies themselves merge at zero cost first)."""
+    rng = np.random.default_rng(9)
+    X = rng.normal(size=(7, 3))
+    w = np.array([1, 3, 1, 2, 1, 1, 4])
+    lab_w = lsa.ward_merges(X, 3, weights=w)
+    rep = np.repeat(X, w, axis=0)
+    lab_r = lsa.ward_merges(rep, 3)
+    owner = np.repeat(np.arange(len(X)), w)
+    # every group of copies ends in one cluster, and the partitions agree
+    for i in range(len(X)):
+        assert len(set(lab_r[owner == i])) == 1
+    assert np.array_equal(_canon(lab_w), _canon(np.array([lab_r[owner == i][0] for i in range(len(X))])))
+
+
+def test_tree_with_a_full_beam_is_the_flat_scan():
+    rng = np.random.default_rng(10)
+    n, d, pool, seg, k = 512, 8, 2, 16, 4
+    K = rng.normal(size=(n, d))
+    idx = lsa.build_index(K, pool, seg, k)
+    levels = lsa.build_tree(idx, fanout=4)
+    assert len(levels) >= 3
+    scale = oracle.default_scale(d)
+    for t in range(5):
+        q = rng.normal(size=d)
+        flat = lsa.select_clusters(idx, q, 6, scale)
+        tree, comps = lsa.tree_select(levels, q, beam=10 ** 6, top_clusters=6, scale=scale)
+        assert np.array_equal(tree, flat)
+
+
+def test_tree_nodes_are_item_means_and_the_beam_bounds_the_work():
+    rng = np.random.default_rng(11)
+    n, d, pool, seg, k, fan, beam = 1024, 8, 2, 16, 4, 4, 3
+    idx = lsa.build_index(rng.normal(size=(n, d)), pool, seg, k)
+    levels = lsa.build_tree(idx, fanout=fan)
+    # every parent's centre is the mean of the items below it
+    def items_under(lv, node):
+        if lv == 0:
+            return sorted({int(t) // pool for t in idx["positions"][node]})
+        return sorted(x for c in levels[lv]["children"][node] for x in items_under(lv - 1, c))
+    for lv in range(1, len(levels)):
+        for node in range(len(levels[lv]["centres"])):
+            it = items_under(lv, node)
+            np.testing.assert_allclose(levels[lv]["centres"][node], idx["items"][it].mean(axis=0), rtol=1e-10,
+                                       atol=1e-12)
+    leaves = len(levels[0]["centres"])
+    _, comps = lsa.tree_select(levels, rng.normal(size=d), beam=beam, top_clusters=beam,
+                               scale=oracle.default_scale(d))
+    widest = max(len(ch) for lv in levels[1:] for ch in lv["children"])
+    assert comps <= len(levels[-1]["centres"]) + (len(levels) - 1) * beam * widest
+    assert comps < leaves
