@@ -377,7 +377,8 @@ def run_reference(args, ranks):
         return 0
     wl = inputs.WORKLOADS[args.workload]
     Q64, K64, V64 = cpu_inputs(wl)
-    per_step_s = max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
+    # a few minutes in all, each step's sample capped by --cpu-seconds
+    per_step_s = min(args.cpu_seconds, max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup))))
     n = calibrate_units(wl, Q64, K64, V64, per_step_s)
     rates, times = [], []
     threads = os.cpu_count() or 1

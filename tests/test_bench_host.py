@@ -73,3 +73,19 @@ def test_single_rank_aggregation_and_config():
     for k in ("workload", "global_batch", "seq_len", "parallelism", "l2"):
         assert k in c
     assert bench.FP32_ALU_TFLOPS == pytest.approx(148 * 128 * 2 * 1.965e9 / 1e12)
+
+
+def test_reference_arm_prints_its_contract_line():
+    """``bench.py --impl reference`` times the oracle on the host and prints
+    one JSON line with the reference arm's keys."""
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3", "--workload", "tiny_fp32_prefill", "--cpu-seconds", "0.3"],
+                       capture_output=True, text=True, timeout=600, cwd=bench.ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"] is True
+    for k in ("metric", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
