@@ -2,16 +2,21 @@
 """Benchmark of the block-sparse landmark attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-secondary]
+                    [--workload NAME] [--no-secondary] [--detail FILE]
 
-One step of the headline workload (gated_prefill_32k: B1, Hq 32, Hkv 8, d 128,
-N 32768, block 64, top-16 + sink + local, bf16) is one pass of the prefill
-path through the C ABI: landmarks -> selection -> gated block-sparse prefill.
-``value`` = prefill tokens/s over all ranks (each rank runs its own seeded
-sequence: weak scaling, no collective on the data path).  The same JSON line
-carries the decode workloads (gated_decode_128k: 64 sequences at 128K context;
-hils_decode_1m: hierarchical, 8 sequences at 1M context) and the 256K prefill
-under ``secondary`` at N = 1, each with its own roofline.
+One step of the headline workload (long_prefill_256k: B1, Hq 32, Hkv 8,
+d 128, N 262144, block 128, top-16 + sink + local, bf16, causal) is one pass
+of the prefill path through the C ABI: landmarks -> selection -> gated
+block-sparse prefill.  ``value`` = prefill tokens/s over all ranks (each rank
+runs its own seeded sequence: weak scaling, no collective on the data path).
+
+At N = 1 the same JSON line ends with ``secondary``: a compact summary (value,
+step time, per-kernel times and roofline fractions) of the other workloads --
+the decode at 128K context (gated_decode_128k: 64 sequences, the metric's own
+context length), the hierarchical decode at 1M, the 32K prefills (gated,
+hierarchical, per-query-head lists), the ragged and per-query-head decodes,
+the backward and the flat clustered index.  ``--detail FILE`` writes their
+full records.
 
 Timing: CUDA events on the launching stream around each step and each C call,
 W warm-up steps, K timed steps bracketed by barrier + synchronize, L2 flushed
@@ -249,10 +254,12 @@ def prefill_step(p, t, timer=None):
 
 def prefill_flops(wl, cnt) -> float:
     """Gathered FLOPs of one prefill launch: QK^T and PV over every kept
-    (tile, block) pair, the local block counted whole: 4 * rows * keys * d."""
-    G = wl.Hq // wl.Hkv
+    (tile, block) pair, the local block counted whole: 4 * rows * keys * d,
+    where a list serves G * block query rows (block rows with one list per
+    query head)."""
+    rows = wl.block if wl.per_qhead else (wl.Hq // wl.Hkv) * wl.block
     pairs = float(cnt.sum().item())
-    return pairs * 4.0 * (G * wl.block) * wl.block * wl.d
+    return pairs * 4.0 * rows * wl.block * wl.d
 
 
 def decode_case(wl, device, lens=None):
@@ -322,7 +329,7 @@ def run_timed(step, steps, warmup, ranks, flush_buf):
 # CPU oracle timing (cpu_baseline and --impl reference)
 # ----------------------------------------------------------------------------
 
-def oracle_prefill_sample(wl, Q64, K64, V64, n_units, seed=0):
+def oracle_prefill_sample(wl, Q64, K64, V64, n_units, seed=0, threads=None):
     """Times the oracle on ``n_units`` (batch, kv-head, tile) units drawn from
     the upper tiles (every one with a full top-K list).  Returns (seconds,
     token-equivalents, threads)."""
@@ -330,7 +337,7 @@ def oracle_prefill_sample(wl, Q64, K64, V64, n_units, seed=0):
     rng = np.random.default_rng(seed)
     lo = min(wl.nb - 1, wl.top_k + 2)
     units = [(0, int(rng.integers(0, wl.Hkv)), int(rng.integers(lo, wl.nb))) for _ in range(n_units)]
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     t0 = time.perf_counter()
     oracle.prefill(Q64, K64, V64, wl.block, wl.top_k, wl.flags, round_mode=oracle.ROUND_BF16, units=units,
                    threads=threads)
@@ -365,10 +372,15 @@ def cpu_baseline(wl, target_s):
     Q64, K64, V64 = cpu_inputs(wl)
     n = calibrate_units(wl, Q64, K64, V64, target_s)
     dt, tok, threads = oracle_prefill_sample(wl, Q64, K64, V64, n, seed=1)
+    # the same oracle on one host thread, on a sample about 1/threads as large
+    n1 = max(4, n // max(1, threads))
+    dt1, tok1, _ = oracle_prefill_sample(wl, Q64, K64, V64, n1, seed=2, threads=1)
     return {"value": tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{n} random (kv-head, tile) units of {wl.name} with full top-{wl.top_k} lists "
                       f"(landmarks of the touched kv-heads, selection and gated attention), "
-                      f"{dt:.1f} s on {threads} host threads; tokens counted as block/Hkv per unit"}
+                      f"{dt:.1f} s on {threads} host threads; tokens counted as block/Hkv per unit",
+            "one_core": {"value": tok1 / dt1, "unit": "tokens/s", "cores": 1,
+                         "sample": f"{n1} units, {dt1:.1f} s on 1 thread"}}
 
 
 def run_reference(args, ranks):
@@ -580,7 +592,15 @@ def secondary_decode(name, args, pk, psrc):
         scan_bytes = wl.B * wl.Hkv * ((wl.N - 1) // wl.block + 1) * wl.d * esz
     else:
         scan_bytes = sum(wl.Hkv * ((int(n) - 1) // wl.block + 1) * wl.d * esz for n in lens)
-    gather_bytes = float(cnt.sum().item()) * wl.block * wl.d * esz * 2
+    if wl.per_qhead:
+        # algorithmic bytes: each kv-head's union of the blocks its query heads keep
+        G = wl.Hq // wl.Hkv
+        idx = t["sel"][0].view(wl.B, wl.Hkv, G * (wl.top_k + 2)).to(torch.int64)
+        hit = torch.zeros(wl.B, wl.Hkv, wl.nb + 1, dtype=torch.bool, device=idx.device)
+        hit.scatter_(2, torch.where(idx < 0, wl.nb, idx), True)
+        gather_bytes = float(hit[..., :wl.nb].sum().item()) * wl.block * wl.d * esz * 2
+    else:
+        gather_bytes = float(cnt.sum().item()) * wl.block * wl.d * esz * 2
     ach_dec = gather_bytes / (kms["decode"] / 1e3) / 1e9
     ach_sel = scan_bytes / (kms["select_decode"] / 1e3) / 1e9
     step_ach = (scan_bytes + gather_bytes) / (el / steps / 1e3) / 1e9
@@ -604,6 +624,46 @@ def secondary_decode(name, args, pk, psrc):
     return out
 
 
+def _sig(x, n=3):
+    return None if x is None else float(f"{x:.{n}g}")
+
+
+def compact(rec: dict) -> dict:
+    """The few fields of a secondary record that the summary keeps: value,
+    step time, per-kernel mean times and roofline fractions."""
+    if "error" in rec:
+        return {"error": rec["error"][:120]}
+    unit = {"tokens/s": "tok/s", "queries/s": "q/s"}.get(rec["unit"], rec["unit"])
+    out = {"value": _sig(rec["value"]), "unit": unit, "ms": _sig(rec["ms_per_step"]),
+           "frac": _sig(rec["roofline"]["frac"], 2)}
+    kr = rec.get("kernels_roofline", {})
+    out["kernels"] = {k: ([_sig(v), _sig(kr[k]["frac"], 2)] if k in kr else _sig(v))
+                      for k, v in rec["kernels_ms"].items()}
+    ck = rec.get("clocks") or {}
+    out["mhz"] = ck.get("sm_mhz")
+    if ck.get("reasons"):
+        out["reasons"] = ck["reasons"]
+    return out
+
+
+# secondary workloads at N = 1, in the order they print: the decodes at the
+# metric's 128K context and the 1M hierarchical decode come last, so that they
+# stay in the tail of the line
+SECONDARY = ("long_prefill_256k", "gated_prefill_32k", "hils_prefill_32k", "gated_prefill_32k_perqhead",
+             "gated_prefill_32k_backward", "lsa_decode_32k", "gated_decode_128k_perqhead", "gated_decode_128k_varlen",
+             "hils_decode_1m", "gated_decode_128k")
+
+
+def run_secondary(name, args, pk, psrc):
+    from block_sparse_long_landmark_b200 import inputs
+    if name == "lsa_decode_32k":
+        return secondary_lsa(name, args, pk, psrc)
+    if name.endswith("_backward"):
+        return secondary_backward(name, args, pk, psrc)
+    kind = inputs.WORKLOADS[name.replace("_varlen", "")].kind
+    return (secondary_decode if kind == "decode" else secondary_prefill)(name, args, pk, psrc)
+
+
 def run_ours(args, ranks):
     import block_sparse_long_landmark_b200 as sa
     from block_sparse_long_landmark_b200 import inputs
@@ -613,13 +673,7 @@ def run_ours(args, ranks):
     pk, psrc = peaks()
     if args.only:
         # one workload alone (small profiling cases): a short report, no baselines
-        if args.only == "lsa_decode_32k":
-            fn = secondary_lsa
-        else:
-            kind = inputs.WORKLOADS[args.only.replace("_varlen", "").replace("_backward", "")].kind
-            fn = (secondary_backward if args.only.endswith("_backward") else
-                  secondary_decode if kind == "decode" else secondary_prefill)
-        print(json.dumps({"only": args.only, **fn(args.only, args, pk, psrc)}), flush=True)
+        print(json.dumps({"only": args.only, **run_secondary(args.only, args, pk, psrc)}), flush=True)
         return 0
     base = inputs.WORKLOADS[args.workload]
     wl, p, t = prefill_case(base, "cuda", seed_offset=ranks.rank)
@@ -651,29 +705,24 @@ def run_ours(args, ranks):
         if not args.no_cpu:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
         if not args.no_secondary:
-            sec = {}
-            for name in ("gated_decode_128k", "hils_decode_1m", "long_prefill_256k", "hils_prefill_32k",
-                         "gated_decode_128k_varlen", "gated_prefill_32k_backward", "lsa_decode_32k"):
+            full = {}
+            for name in SECONDARY:
+                if name == wl.name:
+                    continue
                 try:
-                    if name == "lsa_decode_32k":
-                        try:
-                            sec[name] = secondary_lsa(name, args, pk, psrc)
-                        except Exception as e:   # pragma: no cover -- recorded, the headline line still prints
-                            sec[name] = {"error": f"{type(e).__name__}: {e}"}
-                        torch.cuda.empty_cache()
-                        continue
-                    if name.endswith("_backward"):
-                        sec[name] = secondary_backward(name, args, pk, psrc)
-                        torch.cuda.empty_cache()
-                        continue
-                    kind = inputs.WORKLOADS[name.replace("_varlen", "")].kind
-                    sec[name] = (secondary_decode if kind == "decode" else secondary_prefill)(name, args, pk, psrc)
-                except torch.cuda.OutOfMemoryError as e:   # pragma: no cover
-                    sec[name] = {"error": f"out of memory: {e}"}
+                    full[name] = run_secondary(name, args, pk, psrc)
+                except torch.cuda.OutOfMemoryError as e:   # pragma: no cover -- recorded, the line still prints
+                    full[name] = {"error": f"out of memory: {e}"}
+                except sa.SparseAttnError as e:            # pragma: no cover
+                    full[name] = {"error": str(e)}
                 torch.cuda.empty_cache()
-            line["secondary"] = sec
+            if args.detail:
+                with open(args.detail, "w") as f:
+                    json.dump(full, f, indent=1)
+            # last key of the line: what a truncated tail still shows
+            line["secondary"] = {k: compact(v) for k, v in full.items()}
     if ranks.rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps(line, separators=(",", ":")), flush=True)
     return 0
 
 
@@ -683,11 +732,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gated_prefill_32k")
+    ap.add_argument("--workload", default="long_prefill_256k")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--only", default=None, help="measure this one workload alone (profiling)")
+    ap.add_argument("--detail", default=None, help="write the secondary workloads' full records to this file")
     ap.add_argument("--N", type=int, default=0, help="with --only: override the sequence/context length")
     ap.add_argument("--B", type=int, default=0, help="with --only: override the batch")
     args = ap.parse_args(argv)

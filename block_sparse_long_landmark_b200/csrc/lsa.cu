@@ -73,7 +73,8 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_build_kernel(LsaShape s, cons
                 dist += df * df;
             }
             const double na = csize[a], nb = csize[b];
-            const double c = na * nb / (na + nb) * dist;
+            double c = na * nb / (na + nb) * dist;
+            if (!(c <= CUDART_INF)) c = CUDART_INF;      // NaN ranks as +inf: some alive pair always wins
             const int code = a * S + b;
             if (c < best || (c == best && code < bp)) { best = c; bp = code; }
         }
@@ -91,7 +92,9 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_build_kernel(LsaShape s, cons
             }
             __syncthreads();
         }
-        const int a = bpair[0] / S, b = bpair[0] % S;
+        const int bp0 = bpair[0];
+        if (bp0 < 0 || bp0 >= S * S) break;              // no alive pair (cannot happen while live >= 2)
+        const int a = bp0 / S, b = bp0 % S;
         const double na = csize[a], nb = csize[b];
         __syncthreads();
         for (int e = tid; e < D; e += kLsaThreads) cent[a * D + e] = (na * cent[a * D + e] + nb * cent[b * D + e]) / (na + nb);
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_decode_kernel(LsaShape s, con
             bool taken = false;
             for (int x = 0; x < r; ++x) taken |= chosen[x] == c;
             if (taken) continue;
-            const double v = sc[c];
+            const double v = isnan(sc[c]) ? -CUDART_INF : sc[c];   // NaN ranks lowest
             if (v > bv || (v == bv && c < bi)) { bv = v; bi = c; }
         }
         rv[tid] = bv;
@@ -184,9 +187,15 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_decode_kernel(LsaShape s, con
         if (tid == 0) chosen[r] = ri[0];
         __syncthreads();
     }
+    for (int c = tid; c < s.ctotal; c += kLsaThreads)
+        if (isnan(sc[c])) set_status(status, kStatusNaN);
     // kept positions: the chosen clusters' items, the first `sink`, the last `window`
     const int qpos = s.N - 1;
     for (int r = 0; r < ntop; ++r) {
+        if (chosen[r] < 0 || chosen[r] >= s.ctotal) {    // every candidate taken: nothing left to expand
+            if (tid == 0) set_status(status, kStatusBadIndex);
+            continue;
+        }
         const size_t cid = (size_t)bg * s.ctotal + chosen[r];
         const int m = min(max(msize[cid], 0), s.seg);
         for (int x = tid; x < m * s.pool; x += kLsaThreads) {

@@ -166,23 +166,6 @@ __device__ __forceinline__ void reg_fence(float *v) {
 #pragma unroll
     for (int k = 0; k < N; ++k) asm volatile("" : "+f"(v[k]));
 }
-// 2^x on the FMA pipe, for spreading a softmax's exponentials over two
-// pipes.  Range reduction: adding 1.5 * 2^23 rounds x to the nearest integer
-// n, left in the low mantissa bits; f = x - n lies in [-1/2, 1/2].  2^f is a
-// degree-3 polynomial (weighted least-squares fit of 2^f on Chebyshev nodes
-// of [-1/2, 1/2], iteratively reweighted towards equal ripple; relative
-// error below 7.5e-5, far under bf16 rounding), and n is added to its
-// exponent field.  Inputs below -120 (masked logits included) give 0.
-__device__ __forceinline__ float exp2_fma(float x) {
-    const float xc = fmaxf(x, -120.f);
-    const float t = xc + 12582912.f;
-    const float f = xc - (t - 12582912.f);
-    float p = fmaf(0.055171605f, f, 0.24261111f);
-    p = fmaf(p, f, 0.69326097f);
-    p = fmaf(p, f, 0.99992806f);
-    const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-    return x < -120.f ? 0.f : r;
-}
 // max of three floats in one instruction (sm_100); NaN operands are ignored
 // as by fmaxf
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

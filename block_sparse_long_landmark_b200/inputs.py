@@ -46,10 +46,11 @@ class Workload:
     n_plants: int
     alpha: float = 0.5   # key shift along the planted direction
     beta: float | None = None   # query shift; None -> sigma
+    per_qhead: bool = False     # one selection list per query head instead of per kv-head
 
     @property
     def flags(self) -> int:
-        f = F_SINK | F_LOCAL | F_CAUSAL
+        f = F_SINK | F_LOCAL | F_CAUSAL | (F_PER_QHEAD if self.per_qhead else 0)
         return f | (F_HIER if self.hier else F_GATE)
 
     @property
@@ -84,6 +85,11 @@ WORKLOADS = {
     "hils_decode_1m": Workload("hils_decode_1m", "decode", 8, 32, 8, 128, 1048576, 64, 64, "bf16", True,
                                0.5, 4, "per_seq", 64),
 }
+# the same workloads with one list per query head (each head selects its own blocks)
+WORKLOADS["gated_prefill_32k_perqhead"] = WORKLOADS["gated_prefill_32k"].scaled(
+    name="gated_prefill_32k_perqhead", per_qhead=True)
+WORKLOADS["gated_decode_128k_perqhead"] = WORKLOADS["gated_decode_128k"].scaled(
+    name="gated_decode_128k_perqhead", per_qhead=True)
 
 
 def _randn(shape, gen, device, dtype, sigma, chunk=1 << 28):

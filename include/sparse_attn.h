@@ -206,7 +206,11 @@ int sparse_attn_prefill_kernel(const sa_params *p);
 /* Block-sparse decode: the same attention for one query per sequence at
  * position N-1 over the cache K, V [B,Hkv,N,d] (it already holds the query's
  * own key/value); split over the kept blocks, partials merged by
- * log-sum-exp.  q [B,Hq,d] + decode lists -> o [B,Hq,d], lse [B,Hq]. */
+ * log-sum-exp.  q [B,Hq,d] + decode lists -> o [B,Hq,d], lse [B,Hq].
+ * bf16, d = 128, block 64 runs the tensor-core (mma.sync) gather kernel;
+ * every other shape the CUDA-core kernel.  The environment variable
+ * SPARSE_ATTN_DECODE_PATH=simt forces the CUDA-core kernel (a cross-check
+ * hook: both kernels compute the same result). */
 int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
                        const float *score, const int32_t *count, void *o, float *lse, void *ws,
                        size_t ws_bytes, void *stream);

@@ -169,7 +169,10 @@ def decode(q, K, V, pool: int, seg: int, clusters_per_seg: int, top_clusters: in
 
 def build_tree(index: dict, fanout: int) -> list:
     """Levels from the leaves up: level 0 = the flat clusters.  Each level is
-    dict(centres, mass, children) with children = lists of ids one level down."""
+    dict(centres, mass, children) with children = lists of ids one level down.
+    A fan-out below 2 would never shrink a level: it is rejected."""
+    if int(fanout) < 2:
+        raise ValueError(f"fanout must be at least 2, got {fanout}")
     cent = np.asarray(index["centres"], np.float64)
     mass = np.asarray([len(p) for p in index["positions"]], np.float64)
     levels = [{"centres": cent, "mass": mass, "children": [[c] for c in range(len(cent))]}]

@@ -6,7 +6,6 @@ from __future__ import annotations
 import hashlib
 import json
 import os
-import shutil
 
 import pytest
 
@@ -14,31 +13,48 @@ import bench
 from block_sparse_long_landmark_b200 import inputs
 
 
-def test_traffic_is_used_only_for_the_measured_sources(tmp_path, monkeypatch):
-    entry = json.load(open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")))["prefill_gated_prefill_32k"]
-    # the committed counters match the committed sources
-    assert bench.traffic_for("prefill_gated_prefill_32k") == entry["dram_bytes_per_launch"]
-    # a copy of the tree with one source byte changed: the counters no longer apply
-    root = tmp_path / "repo"
-    for rel in entry["sources"] + ["profiles/ncu_traffic.json"]:
+def _fake_tree(root, sources):
+    """A minimal tree with kernel sources and a traffic summary keyed on them."""
+    h = hashlib.sha256()
+    for rel, body in sources.items():
         dst = root / rel
         dst.parent.mkdir(parents=True, exist_ok=True)
-        shutil.copy(os.path.join(bench.ROOT, rel), dst)
+        dst.write_bytes(body)
+        h.update(body)
+    (root / "profiles").mkdir(parents=True, exist_ok=True)
+    entry = {"dram_bytes_per_launch": 123456, "sources": list(sources), "sources_sha256": h.hexdigest()}
+    (root / "profiles" / "ncu_traffic.json").write_text(json.dumps({"prefill_x": entry}))
+    return entry
+
+
+def test_traffic_is_used_only_for_the_measured_sources(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    srcs = {"pkg/csrc/a.cu": b"kernel a\n", "pkg/csrc/b.cuh": b"helpers\n"}
+    entry = _fake_tree(root, srcs)
     monkeypatch.setattr(bench, "ROOT", str(root))
-    assert bench.traffic_for("prefill_gated_prefill_32k") == entry["dram_bytes_per_launch"]
-    src = root / entry["sources"][0]
-    src.write_bytes(src.read_bytes() + b"\n")
-    assert bench.traffic_for("prefill_gated_prefill_32k") is None
+    assert bench.traffic_for("prefill_x") == entry["dram_bytes_per_launch"]
     assert bench.traffic_for("no_such_kernel") is None
+    # any byte of any listed source changed: the counters no longer apply
+    for rel in srcs:
+        f = root / rel
+        f.write_bytes(srcs[rel] + b"\n")
+        assert bench.traffic_for("prefill_x") is None
+        f.write_bytes(srcs[rel])
+        assert bench.traffic_for("prefill_x") == entry["dram_bytes_per_launch"]
+    # a listed source that disappeared, or an entry without its hash, gives no counter
+    (root / "pkg/csrc/b.cuh").unlink()
+    assert bench.traffic_for("prefill_x") is None
 
 
-def test_traffic_hash_covers_every_source():
-    entry = json.load(open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")))["prefill_gated_prefill_32k"]
-    h = hashlib.sha256()
-    for rel in entry["sources"]:
-        h.update(open(os.path.join(bench.ROOT, rel), "rb").read())
-    assert h.hexdigest() == entry["sources_sha256"]
-    assert any(r.endswith("prefill_tc2.cu") for r in entry["sources"])
+def test_committed_traffic_entries_name_existing_sources():
+    d = json.load(open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")))
+    for name, entry in d.items():
+        if not isinstance(entry, dict) or "sources" not in entry:
+            continue
+        assert entry["sources"], name
+        for rel in entry["sources"]:
+            assert os.path.exists(os.path.join(bench.ROOT, rel)), (name, rel)
+        assert len(entry["sources_sha256"]) == 64
 
 
 def test_calibration_ignores_one_time_costs(monkeypatch):

@@ -138,3 +138,11 @@ def test_tree_nodes_are_item_means_and_the_beam_bounds_the_work():
     widest = max(len(ch) for lv in levels[1:] for ch in lv["children"])
     assert comps <= len(levels[-1]["centres"]) + (len(levels) - 1) * beam * widest
     assert comps < leaves
+
+
+@pytest.mark.parametrize("fanout", [1, 0, -3])
+def test_tree_rejects_a_fanout_that_cannot_shrink_a_level(fanout):
+    rng = np.random.default_rng(5)
+    idx = lsa.build_index(rng.standard_normal((256, 8)), 2, 16, 4)
+    with pytest.raises(ValueError):
+        lsa.build_tree(idx, fanout)

@@ -414,3 +414,94 @@ def test_decode_hier_single_block_and_local_partial():
         assert np.abs(out["O"][0, h] - ref).max() <= 1e-12
     # its landmark averages only the 7 keys that exist
     assert np.allclose(out["L"][0, 0, 4], K[0, 0, 64:].mean(axis=0), atol=1e-14, rtol=0)
+
+
+# ----------------------------------------------------------------------------
+# hierarchical weighting with unequal retrieval scores
+# ----------------------------------------------------------------------------
+
+def _hier_closed_form(q_rows, K, V, bs, kept, scores, local, qpos):
+    """HiLS combination written out with torch float64: every kept block is
+    attended on its own (causal inside the local block), and the per-block
+    outputs are mixed with softmax(scores); LSE = logsumexp(scores)."""
+    s = torch.as_tensor(np.asarray(scores, dtype=np.float64))
+    w = torch.softmax(s, dim=0).numpy()
+    out = np.zeros_like(q_rows)
+    for wb, b in zip(w, kept):
+        t0, t1 = b * bs, min((b + 1) * bs, K.shape[0])
+        mask = None
+        if b == local:
+            pos = np.arange(t0, t1)
+            mask = np.where(pos[None, :] <= np.asarray(qpos)[:, None], 0.0, -np.inf)
+        out += wb * sdpa(q_rows, K[t0:t1], V[t0:t1], mask=mask)
+    return out, float(torch.logsumexp(s, dim=0))
+
+
+def _fixed_list(kept, scores, top_k):
+    cap = top_k + 2
+    idx = np.full(cap, -1, dtype=np.int32)
+    sc = np.zeros(cap)
+    idx[:len(kept)] = kept
+    sc[:len(kept)] = scores
+    return {"idx": idx, "sc": sc, "gate": np.zeros(cap), "count": len(kept), "rel_gap": np.inf}
+
+
+@pytest.mark.parametrize("scores", [[0.3, -1.2, 2.0], [0.5, 1.5, 3.0], [-4.0, 0.0, -0.5]])
+def test_hier_unequal_scores_mix_by_softmax_prefill(scores):
+    B, Hq, Hkv, d, bs, N = 1, 2, 1, 8, 16, 80
+    j, kept = 4, [0, 2, 4]
+    Q, K, V = _rand_qkv(31, B, Hq, Hkv, N, d)
+    out = oracle.prefill(Q, K, V, bs, 1, HIER | SINK | LOCAL | CAUSAL, round_mode=oracle.ROUND_NONE,
+                         units=[(0, 0, j)], sel_override=lambda b, s, jj: _fixed_list(kept, scores, 1))
+    rows = slice(j * bs, (j + 1) * bs)
+    qpos = np.arange(j * bs, (j + 1) * bs)
+    for h in range(Hq):
+        ref, lse = _hier_closed_form(Q[0, h, rows], K[0, 0], V[0, 0], bs, kept, scores, j, qpos)
+        assert np.abs(out["O"][0, h, rows] - ref).max() <= 1e-12
+        assert np.abs(out["LSE"][0, h, rows] - lse).max() <= 1e-12
+    if min(scores) > 0:
+        # the linear reading w_b = s_b / sum(s) gives a clearly different output here
+        lin = np.asarray(scores) / np.sum(scores)
+        parts = []
+        for b in kept:
+            t0 = b * bs
+            mask = None if b != j else np.where(np.arange(t0, t0 + bs)[None, :] <= qpos[:, None], 0.0, -np.inf)
+            parts.append(sdpa(Q[0, 0, rows], K[0, 0, t0:t0 + bs], V[0, 0, t0:t0 + bs], mask=mask))
+        alt = sum(wb * p for wb, p in zip(lin, parts))
+        assert np.abs(out["O"][0, 0, rows] - alt).max() > 1e-2
+
+
+def test_hier_unequal_scores_mix_by_softmax_decode():
+    B, Hq, Hkv, d, bs, N = 1, 4, 2, 8, 16, 75          # local block 4 holds 11 keys
+    kept, scores = [0, 1, 3, 4], [1.1, -0.7, 2.4, 0.2]
+    rng = np.random.default_rng(32)
+    q = rng.standard_normal((B, Hq, d))
+    K = rng.standard_normal((B, Hkv, N, d))
+    V = rng.standard_normal((B, Hkv, N, d))
+    out = oracle.decode(q, K, V, bs, 2, HIER | SINK | LOCAL | CAUSAL, round_mode=oracle.ROUND_NONE,
+                        sel_override=lambda b, s: _fixed_list(kept, scores, 2))
+    G = Hq // Hkv
+    for h in range(Hq):
+        g = h // G
+        ref, lse = _hier_closed_form(q[0, h][None], K[0, g], V[0, g], bs, kept, scores, 4, [N - 1])
+        assert np.abs(out["O"][0, h] - ref[0]).max() <= 1e-12
+        assert abs(out["LSE"][0, h] - lse) <= 1e-12
+
+
+def test_hier_own_selection_mixes_by_softmax_of_reported_scores():
+    """With the oracle's own lists (random scores, every tile), the output is
+    the softmax(sc)-weighted sum of per-block attention."""
+    B, Hq, Hkv, d, bs, N = 1, 2, 1, 8, 16, 112
+    Q, K, V = _rand_qkv(33, B, Hq, Hkv, N, d)
+    out = oracle.prefill(Q, K, V, bs, 3, HIER | SINK | LOCAL | CAUSAL, round_mode=oracle.ROUND_NONE)
+    for j in range(N // bs):
+        c = int(out["count"][0, 0, j])
+        kept = [int(x) for x in out["idx"][0, 0, j, :c]]
+        scores = out["sc"][0, 0, j, :c]
+        assert len(set(np.round(scores, 12))) == c or c <= 1
+        rows = slice(j * bs, (j + 1) * bs)
+        qpos = np.arange(j * bs, (j + 1) * bs)
+        for h in range(Hq):
+            ref, lse = _hier_closed_form(Q[0, h, rows], K[0, 0], V[0, 0], bs, kept, scores, j, qpos)
+            assert np.abs(out["O"][0, h, rows] - ref).max() <= 1e-12
+            assert np.abs(out["LSE"][0, h, rows] - lse).max() <= 1e-12
