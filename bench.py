@@ -551,25 +551,75 @@ def secondary_lsa(name, args, pk, psrc):
     build_ms = s0.elapsed_time(s1)
     ws = sa.lsa_workspace(p)
     out = (torch.empty_like(q), torch.empty(c["B"], c["Hq"], dtype=torch.float32, device="cuda"))
+    kept = torch.zeros(c["B"], c["Hkv"], dtype=torch.int32, device="cuda")
 
     def step(tm):
-        (tm or (lambda n, f: f()))("lsa_decode", lambda: sa.lsa_decode(p, q, K, V, index, ws, out=out))
+        (tm or (lambda n, f: f()))("lsa_decode", lambda: sa.lsa_decode(p, q, K, V, index, ws, out=out, kept=kept))
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    steps = 5
+    steps = 10
     el, kms, launches, clocks = run_timed(step, steps, 3, Ranks.single(), flush)
     C = sa.sparse_attn_lsa_clusters(p)
-    per_cluster = c["seg"] * c["pool"]              # upper bound: a cluster holds at most a whole segment
-    kept = min(c["N"], c["sink"] + c["window"] + c["top_clusters"] * per_cluster)
-    nbytes = c["B"] * c["Hkv"] * (C * c["d"] * 8 + kept * c["d"] * 2 * 2)
+    # algorithmic bytes: every centre (fp64) once, the chosen clusters' member
+    # tables, and K and V of every kept position once
+    nkept = int(kept.sum().item())
+    member_bytes = c["B"] * c["Hkv"] * c["top_clusters"] * (c["seg"] + 1) * 4
+    nbytes = c["B"] * c["Hkv"] * C * c["d"] * 8 + member_bytes + nkept * c["d"] * 2 * 2
     hbm = pk["hbm_gbs"]
     ach = nbytes / (kms["lsa_decode"] / 1e3) / 1e9
     return {"metric": "lsa decode queries/s", "value": c["B"] / (el / steps / 1e3), "unit": "queries/s",
             "ms_per_step": el / steps, "kernels_ms": kms, "index_build_ms": build_ms, "config": dict(c),
-            "gpu_launches": launches,
+            "gpu_launches": launches, "kept_positions": nkept,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                         "algorithmic_bytes_upper_bound": nbytes, "traffic": None,
+                         "algorithmic_bytes": nbytes, "traffic": None,
                          "peak_source": psrc + " HBM copy"},
+            "clocks": clocks}
+
+
+LSA_TREE = dict(fanout=4, beam=16)
+
+
+def secondary_lsa_tree(name, args, pk, psrc):
+    """Decode through the tree over the flat index (beam search to the
+    leaves); index and tree are built once, outside the timed region."""
+    import block_sparse_long_landmark_b200 as sa
+    c = LSA_DECODE_32K
+    p = sa.make_lsa_params(**c)
+    g = torch.Generator(device="cuda").manual_seed(21)
+    q = torch.randn(c["B"], c["Hq"], c["d"], generator=g, device="cuda").to(torch.bfloat16)
+    K = torch.randn(c["B"], c["Hkv"], c["N"], c["d"], generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn(c["B"], c["Hkv"], c["N"], c["d"], generator=g, device="cuda").to(torch.bfloat16)
+    index = sa.lsa_build(p, K)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    tree, ws = sa.lsa_tree_build(p, LSA_TREE["fanout"], index)
+    s1.record()
+    torch.cuda.synchronize()
+    build_ms = s0.elapsed_time(s1)
+    out = (torch.empty_like(q), torch.empty(c["B"], c["Hq"], dtype=torch.float32, device="cuda"))
+    kept = torch.zeros(c["B"], c["Hkv"], dtype=torch.int32, device="cuda")
+    comp = torch.zeros_like(kept)
+
+    def step(tm):
+        (tm or (lambda n, f: f()))("lsa_tree_decode", lambda: sa.lsa_tree_decode(
+            p, LSA_TREE["fanout"], LSA_TREE["beam"], q, K, V, index, tree, ws, out=out, kept=kept, compared=comp))
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    steps = 10
+    el, kms, launches, clocks = run_timed(step, steps, 3, Ranks.single(), flush)
+    nkept, ncomp = int(kept.sum().item()), int(comp.sum().item())
+    # algorithmic bytes: every centre compared (fp64), the chosen leaves' member
+    # tables, K and V of every kept position
+    member_bytes = c["B"] * c["Hkv"] * c["top_clusters"] * (c["seg"] + 1) * 4
+    nbytes = ncomp * c["d"] * 8 + member_bytes + nkept * c["d"] * 2 * 2
+    hbm = pk["hbm_gbs"]
+    ach = nbytes / (kms["lsa_tree_decode"] / 1e3) / 1e9
+    return {"metric": "lsa tree decode queries/s", "value": c["B"] / (el / steps / 1e3), "unit": "queries/s",
+            "ms_per_step": el / steps, "kernels_ms": kms, "tree_build_ms": build_ms,
+            "config": dict(c, **LSA_TREE), "gpu_launches": launches, "kept_positions": nkept,
+            "centres_compared": ncomp, "centres_total": c["B"] * c["Hkv"] * sa.sparse_attn_lsa_clusters(p),
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                         "algorithmic_bytes": nbytes, "traffic": None, "peak_source": psrc + " HBM copy"},
             "clocks": clocks}
 
 
@@ -634,23 +684,27 @@ def compact(rec: dict) -> dict:
     if "error" in rec:
         return {"error": rec["error"][:120]}
     unit = {"tokens/s": "tok/s", "queries/s": "q/s"}.get(rec["unit"], rec["unit"])
-    out = {"value": _sig(rec["value"]), "unit": unit, "ms": _sig(rec["ms_per_step"]),
+    out = {"v": _sig(rec["value"]), "u": unit, "ms": _sig(rec["ms_per_step"]),
            "frac": _sig(rec["roofline"]["frac"], 2)}
     kr = rec.get("kernels_roofline", {})
-    out["kernels"] = {k: ([_sig(v), _sig(kr[k]["frac"], 2)] if k in kr else _sig(v))
-                      for k, v in rec["kernels_ms"].items()}
+    out["k"] = {k: ([_sig(v), _sig(kr[k]["frac"], 2)] if k in kr else _sig(v))
+                for k, v in rec["kernels_ms"].items()}
     ck = rec.get("clocks") or {}
     out["mhz"] = ck.get("sm_mhz")
     if ck.get("reasons"):
-        out["reasons"] = ck["reasons"]
+        out["why"] = ck["reasons"]
     return out
 
 
 # secondary workloads at N = 1, in the order they print: the decodes at the
 # metric's 128K context and the 1M hierarchical decode come last, so that they
-# stay in the tail of the line
+# stay in the tail of the line.  Summary keys: v value, u unit, ms step time,
+# frac the roofline fraction of the step (decode) or of the prefill kernel,
+# k per-kernel mean ms (with its own roofline fraction where one is defined),
+# mhz median SM clock, why throttle reasons seen
 SECONDARY = ("long_prefill_256k", "gated_prefill_32k", "hils_prefill_32k", "gated_prefill_32k_perqhead",
-             "gated_prefill_32k_backward", "lsa_decode_32k", "gated_decode_128k_perqhead", "gated_decode_128k_varlen",
+             "gated_prefill_32k_backward", "lsa_decode_32k", "lsa_tree_decode_32k", "gated_decode_128k_perqhead",
+             "gated_decode_128k_varlen",
              "hils_decode_1m", "gated_decode_128k")
 
 
@@ -658,6 +712,8 @@ def run_secondary(name, args, pk, psrc):
     from block_sparse_long_landmark_b200 import inputs
     if name == "lsa_decode_32k":
         return secondary_lsa(name, args, pk, psrc)
+    if name == "lsa_tree_decode_32k":
+        return secondary_lsa_tree(name, args, pk, psrc)
     if name.endswith("_backward"):
         return secondary_backward(name, args, pk, psrc)
     kind = inputs.WORKLOADS[name.replace("_varlen", "")].kind

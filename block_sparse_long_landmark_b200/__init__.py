@@ -34,6 +34,8 @@ EXPORTS = (
     "sparse_attn_landmarks_update", "sparse_attn_select_decode_varlen", "sparse_attn_decode_varlen",
     "sparse_attn_prefill_backward", "sparse_attn_select_backward",
     "sparse_attn_lsa_clusters", "sparse_attn_lsa_workspace_size", "sparse_attn_lsa_build", "sparse_attn_lsa_decode",
+    "sparse_attn_lsa_tree_size", "sparse_attn_lsa_tree_workspace_size", "sparse_attn_lsa_tree_build",
+    "sparse_attn_lsa_tree_decode",
 )
 
 
@@ -117,8 +119,16 @@ def lib() -> ctypes.CDLL:
             L.sparse_attn_lsa_workspace_size.restype = sz
             L.sparse_attn_lsa_build.argtypes = [LP, vp, vp, vp, vp, vp]
             L.sparse_attn_lsa_build.restype = i
-            L.sparse_attn_lsa_decode.argtypes = [LP] + [vp] * 9 + [sz, vp]
+            L.sparse_attn_lsa_decode.argtypes = [LP] + [vp] * 10 + [sz, vp]
             L.sparse_attn_lsa_decode.restype = i
+            L.sparse_attn_lsa_tree_size.argtypes = [LP, i, ctypes.POINTER(ctypes.c_int)]
+            L.sparse_attn_lsa_tree_size.restype = sz
+            L.sparse_attn_lsa_tree_workspace_size.argtypes = [LP, i]
+            L.sparse_attn_lsa_tree_workspace_size.restype = sz
+            L.sparse_attn_lsa_tree_build.argtypes = [LP, i, vp, vp, vp, vp, sz, vp]
+            L.sparse_attn_lsa_tree_build.restype = i
+            L.sparse_attn_lsa_tree_decode.argtypes = [LP, i, i] + [vp] * 12 + [sz, vp]
+            L.sparse_attn_lsa_tree_decode.restype = i
             L.sparse_attn_launch_count.argtypes = []
             L.sparse_attn_launch_count.restype = ctypes.c_ulonglong
             _lib = L
@@ -171,9 +181,30 @@ def sparse_attn_lsa_build(p, K, centres, members, sizes, stream) -> int:
     return lib().sparse_attn_lsa_build(ctypes.byref(p), K, centres, members, sizes, stream)
 
 
-def sparse_attn_lsa_decode(p, q, K, V, centres, members, sizes, o, lse, ws, ws_bytes, stream) -> int:
-    return lib().sparse_attn_lsa_decode(ctypes.byref(p), q, K, V, centres, members, sizes, o, lse, ws, ws_bytes,
-                                        stream)
+def sparse_attn_lsa_decode(p, q, K, V, centres, members, sizes, o, lse, kept, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_lsa_decode(ctypes.byref(p), q, K, V, centres, members, sizes, o, lse, kept, ws,
+                                        ws_bytes, stream)
+
+
+def sparse_attn_lsa_tree_size(p: sa_lsa_params, fanout: int):
+    """(bytes of the tree buffer, levels incl. the leaves); bytes 0 = invalid."""
+    lv = ctypes.c_int(0)
+    n = int(lib().sparse_attn_lsa_tree_size(ctypes.byref(p), fanout, ctypes.byref(lv)))
+    return n, lv.value
+
+
+def sparse_attn_lsa_tree_workspace_size(p: sa_lsa_params, fanout: int) -> int:
+    return int(lib().sparse_attn_lsa_tree_workspace_size(ctypes.byref(p), fanout))
+
+
+def sparse_attn_lsa_tree_build(p, fanout, centres, sizes, tree, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_lsa_tree_build(ctypes.byref(p), fanout, centres, sizes, tree, ws, ws_bytes, stream)
+
+
+def sparse_attn_lsa_tree_decode(p, fanout, beam, q, K, V, centres, members, sizes, tree, o, lse, kept, compared, ws,
+                                ws_bytes, stream) -> int:
+    return lib().sparse_attn_lsa_tree_decode(ctypes.byref(p), fanout, beam, q, K, V, centres, members, sizes, tree, o,
+                                             lse, kept, compared, ws, ws_bytes, stream)
 
 
 def sparse_attn_select_backward(p, Q, L, idx, dscore, count, dQ, dK, ws, ws_bytes, stream) -> int:
@@ -385,8 +416,9 @@ def lsa_workspace(p: sa_lsa_params, device="cuda"):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def lsa_decode(p: sa_lsa_params, q, K, V, index, ws, out=None, stream=None):
-    """Decode through the flat index: (o, lse)."""
+def lsa_decode(p: sa_lsa_params, q, K, V, index, ws, out=None, kept=None, stream=None):
+    """Decode through the flat index: (o, lse).  ``kept``: optional int32
+    [B, Hkv] tensor that receives the number of key positions attended."""
     torch = _torch()
     centres, members, sizes = index
     if out is None:
@@ -395,7 +427,8 @@ def lsa_decode(p: sa_lsa_params, q, K, V, index, ws, out=None, stream=None):
     else:
         o, lse = out
     _check(sparse_attn_lsa_decode(p, _ptr(q), _ptr(K), _ptr(V), _ptr(centres), _ptr(members), _ptr(sizes), _ptr(o),
-                                  _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_lsa_decode")
+                                  _ptr(lse), _ptr(kept), _ptr(ws), ws.numel(), _stream(stream)),
+           "sparse_attn_lsa_decode")
     return o, lse
 
 
@@ -447,3 +480,62 @@ def check_status(ws, stream=None):
     if rc != SA_OK:
         raise SparseAttnError(rc, f"device status bits {detail:#x}")
     return detail
+
+
+def lsa_tree_build(p: sa_lsa_params, fanout: int, index, stream=None):
+    """Tree over the flat index's clusters: (tree buffer uint8, workspace)."""
+    torch = _torch()
+    centres, members, sizes = index
+    nbytes, _ = sparse_attn_lsa_tree_size(p, fanout)
+    if nbytes == 0:
+        raise SparseAttnError(SA_ERR_UNSUPPORTED, "sparse_attn_lsa_tree_size")
+    tree = torch.zeros(nbytes, dtype=torch.uint8, device=centres.device)
+    ws = torch.zeros(sparse_attn_lsa_tree_workspace_size(p, fanout), dtype=torch.uint8, device=centres.device)
+    _check(sparse_attn_lsa_tree_build(p, fanout, _ptr(centres), _ptr(sizes), _ptr(tree), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "sparse_attn_lsa_tree_build")
+    return tree, ws
+
+
+def lsa_tree_decode(p: sa_lsa_params, fanout: int, beam: int, q, K, V, index, tree, ws, out=None, kept=None,
+                    compared=None, stream=None):
+    """Decode through the tree (beam search to the leaves): (o, lse)."""
+    torch = _torch()
+    centres, members, sizes = index
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(p.B, p.Hq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(sparse_attn_lsa_tree_decode(p, fanout, beam, _ptr(q), _ptr(K), _ptr(V), _ptr(centres), _ptr(members),
+                                       _ptr(sizes), _ptr(tree), _ptr(o), _ptr(lse), _ptr(kept), _ptr(compared),
+                                       _ptr(ws), ws.numel(), _stream(stream)), "sparse_attn_lsa_tree_decode")
+    return o, lse
+
+
+def lsa_tree_levels(p: sa_lsa_params, fanout: int, tree):
+    """Views of a built tree buffer, following the layout the header documents:
+    a list over levels of dict(mass [B,Hkv,n], and for levels >= 1 centres
+    [B,Hkv,n,d], first [B,Hkv,n+1], children [B,Hkv,n_below])."""
+    torch = _torch()
+    C = sparse_attn_lsa_clusters(p)
+    n = [C]
+    while n[-1] > fanout:
+        n.append((n[-1] + fanout - 1) // fanout)
+    bgs = p.B * p.Hkv
+
+    def al(x):
+        return (x + 255) & ~255
+
+    off, out = 0, []
+    for lv, nl in enumerate(n):
+        d = {"mass": tree[off:off + bgs * nl * 8].view(torch.float64).view(p.B, p.Hkv, nl)}
+        off += al(bgs * nl * 8)
+        if lv > 0:
+            d["centres"] = tree[off:off + bgs * nl * p.d * 8].view(torch.float64).view(p.B, p.Hkv, nl, p.d)
+            off += al(bgs * nl * p.d * 8)
+            d["first"] = tree[off:off + bgs * (nl + 1) * 4].view(torch.int32).view(p.B, p.Hkv, nl + 1)
+            off += al(bgs * (nl + 1) * 4)
+            d["children"] = tree[off:off + bgs * n[lv - 1] * 4].view(torch.int32).view(p.B, p.Hkv, n[lv - 1])
+            off += al(bgs * n[lv - 1] * 4)
+        out.append(d)
+    return out

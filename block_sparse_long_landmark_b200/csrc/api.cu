@@ -4,6 +4,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "common.cuh"
@@ -252,9 +253,9 @@ int sparse_attn_lsa_clusters(const sa_lsa_params *p) {
 
 size_t sparse_attn_lsa_workspace_size(const sa_lsa_params *p) {
     LsaShape s;
-    if (resolve_lsa(p, s) != SA_OK) return 0;
-    const size_t scores = (size_t)s.B * s.Hkv * (size_t)s.ctotal * sizeof(double);
-    return kStatusBytes + ((scores + 255) & ~(size_t)255);
+    LsaDecPlan pl;
+    if (resolve_lsa(p, s) != SA_OK || !lsa_decode_plan(s, pl)) return 0;
+    return pl.bytes;
 }
 
 int sparse_attn_lsa_build(const sa_lsa_params *p, const void *K, double *centres, int32_t *members, int32_t *sizes,
@@ -269,17 +270,77 @@ int sparse_attn_lsa_build(const sa_lsa_params *p, const void *K, double *centres
 
 int sparse_attn_lsa_decode(const sa_lsa_params *p, const void *q, const void *K, const void *V,
                            const double *centres, const int32_t *members, const int32_t *sizes, void *o, float *lse,
-                           void *ws, size_t ws_bytes, void *stream) {
+                           int32_t *kept, void *ws, size_t ws_bytes, void *stream) {
     LsaShape s;
+    LsaDecPlan pl;
     const int r = resolve_lsa(p, s);
     if (r != SA_OK) return r;
+    if (!lsa_decode_plan(s, pl)) return SA_ERR_UNSUPPORTED;
     if (!q || !K || !V || !o || !lse || !ws) return SA_ERR_ARG;
     if (s.ctotal > 0 && (!centres || !members || !sizes)) return SA_ERR_ARG;
-    if (!aligned16(K) || !aligned16(V) || !aligned16(ws)) return SA_ERR_ARG;
-    if (ws_bytes < sparse_attn_lsa_workspace_size(p)) return SA_ERR_WORKSPACE;
-    double *scores = reinterpret_cast<double *>(static_cast<unsigned char *>(ws) + kStatusBytes);
-    return launch_result(launch_lsa_decode(s, q, K, V, centres, members, sizes, scores, static_cast<unsigned *>(ws),
-                                           o, lse, (cudaStream_t)stream));
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(ws)) return SA_ERR_ARG;
+    if (s.ctotal > 0 && !aligned16(centres)) return SA_ERR_ARG;
+    if (ws_bytes < pl.bytes) return SA_ERR_WORKSPACE;
+    return launch_result(launch_lsa_decode(s, pl, q, K, V, centres, members, sizes, ws, o, lse, kept,
+                                           (cudaStream_t)stream));
+}
+
+static int resolve_tree(const sa_lsa_params *p, int fanout, LsaShape &s, LsaTreePlan &tp) {
+    const int r = resolve_lsa(p, s);
+    if (r != SA_OK) return r;
+    if (fanout < 2) return SA_ERR_ARG;
+    if (!lsa_tree_plan(s, fanout, tp)) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+size_t sparse_attn_lsa_tree_size(const sa_lsa_params *p, int fanout, int *levels) {
+    LsaShape s;
+    LsaTreePlan tp;
+    if (resolve_tree(p, fanout, s, tp) != SA_OK) return 0;
+    if (levels) *levels = tp.L;
+    return tp.bytes;
+}
+
+size_t sparse_attn_lsa_tree_workspace_size(const sa_lsa_params *p, int fanout) {
+    LsaShape s;
+    LsaTreePlan tp;
+    LsaDecPlan pl;
+    if (resolve_tree(p, fanout, s, tp) != SA_OK || !lsa_decode_plan(s, pl, false)) return 0;
+    return pl.bytes + tp.work_bytes;     // the decode's regions, then the build's working centres
+}
+
+int sparse_attn_lsa_tree_build(const sa_lsa_params *p, int fanout, const double *centres, const int32_t *sizes,
+                               void *tree, void *ws, size_t ws_bytes, void *stream) {
+    LsaShape s;
+    LsaTreePlan tp;
+    LsaDecPlan pl;
+    const int r = resolve_tree(p, fanout, s, tp);
+    if (r != SA_OK) return r;
+    if (!lsa_decode_plan(s, pl, false)) return SA_ERR_UNSUPPORTED;
+    if (!centres || !sizes || !tree || !ws) return SA_ERR_ARG;
+    if (!aligned16(centres) || !aligned16(tree) || !aligned16(ws)) return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_lsa_tree_workspace_size(p, fanout)) return SA_ERR_WORKSPACE;
+    double *work = reinterpret_cast<double *>(static_cast<unsigned char *>(ws) + pl.bytes);
+    return launch_result(launch_lsa_tree_build(s, tp, centres, sizes, tree, work, (cudaStream_t)stream));
+}
+
+int sparse_attn_lsa_tree_decode(const sa_lsa_params *p, int fanout, int beam, const void *q, const void *K,
+                                const void *V, const double *centres, const int32_t *members, const int32_t *sizes,
+                                const void *tree, void *o, float *lse, int32_t *kept, int32_t *compared, void *ws,
+                                size_t ws_bytes, void *stream) {
+    LsaShape s;
+    LsaTreePlan tp;
+    LsaDecPlan pl;
+    const int r = resolve_tree(p, fanout, s, tp);
+    if (r != SA_OK) return r;
+    if (beam < 1) return SA_ERR_ARG;
+    if (!lsa_decode_plan(s, pl, false)) return SA_ERR_UNSUPPORTED;
+    if (!q || !K || !V || !centres || !members || !sizes || !tree || !o || !lse || !ws) return SA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(ws) || !aligned16(centres) || !aligned16(tree))
+        return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_lsa_tree_workspace_size(p, fanout)) return SA_ERR_WORKSPACE;
+    return launch_result(launch_lsa_tree_decode(s, pl, tp, beam, q, K, V, centres, members, sizes, tree, ws, o, lse,
+                                                kept, compared, (cudaStream_t)stream));
 }
 
 int sparse_attn_check_status(void *ws, void *stream, int *detail) {

@@ -138,6 +138,13 @@ cudaError_t launch_select(const Shape &s, bool decode, const void *Q, const void
                           int32_t *count, void *ws, size_t ws_bytes, cudaStream_t st);
 size_t select_workspace(const Shape &s, bool decode);
 bool select_tiles_supported(const Shape &s);
+bool select_decode_supported(const Shape &s);
+size_t select_decode_workspace(const Shape &s);
+cudaError_t launch_select_decode(const Shape &s, const void *q, const void *L, int32_t *idx, float *score,
+                                 int32_t *count, void *ws, cudaStream_t st);
+// SPARSE_ATTN_SELECT_PATH=chunked: decode selection by the CTA-per-chunk
+// kernel of select.cu (a cross-check hook; both give the same lists)
+bool select_force_chunked();
 cudaError_t launch_select_tiles(const Shape &s, const void *Q, const void *L, int32_t *idx, float *score,
                                 int32_t *count, unsigned *status, cudaStream_t st);
 cudaError_t launch_prefill_simt(const Shape &s, const void *Q, const void *K, const void *V, const int32_t *idx,
@@ -153,6 +160,7 @@ cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, con
                                cudaStream_t st);
 bool decode_mma_supported(const Shape &s);
 void decode_mma_geometry(const Shape &s, int &S, int &bps);
+size_t decode_mma_partial_bytes(const Shape &s, int S);
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                               const float *score, const int32_t *count, void *o, float *lse, void *ws,
                               cudaStream_t st, int &S_out);

@@ -266,8 +266,13 @@ static void split_geometry(const Shape &s, int &S, int &bps) {
 
 size_t decode_workspace(const Shape &s) {
     int S, bps;
-    if (decode_mma_supported(s)) decode_mma_geometry(s, S, bps);
-    else split_geometry(s, S, bps);
+    if (decode_mma_supported(s)) {
+        decode_mma_geometry(s, S, bps);
+        if (S == 1) return 0;
+        // split partials, then one completion counter per unit
+        return decode_mma_partial_bytes(s, S) + (size_t)s.B * s.Hsel * sizeof(unsigned);
+    }
+    split_geometry(s, S, bps);
     if (S == 1) return 0;
     return (size_t)s.B * s.Hsel * S * s.heads_per * (s.d + 2) * sizeof(float);
 }
@@ -308,13 +313,9 @@ cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const vo
     a.status = (unsigned *)ws;
     a.part = (float *)((char *)ws + kStatusBytes);
     if (decode_mma_supported(s)) {
+        // one launch: the unit's last split merges the partials itself
         int S = 1;
-        cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, o, lse, ws, st, S);
-        if (e != cudaSuccess || S == 1) return e;
-        a.S = S;
-        decode_merge_kernel<__nv_bfloat16><<<(unsigned)(s.B * s.Hsel), kDecThreads, 0, st>>>(a);
-        note_launch();
-        return cudaGetLastError();
+        return launch_decode_mma(s, q, K, V, idx, score, count, o, lse, ws, st, S);
     }
     split_geometry(s, a.S, a.bps);
     return s.dtype == SA_BF16 ? run<__nv_bfloat16>(a, st) : run<float>(a, st);

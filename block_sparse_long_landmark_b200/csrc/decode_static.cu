@@ -19,7 +19,9 @@
 //     them on one stream or serialise them;
 //   * each call clears the status word at the array's start (cudaMemsetAsync
 //     on the call's stream); the split partials need no clearing because
-//     every split writes its own slot before the merge reads it;
+//     every split writes its own slot before the merge reads it, and the
+//     per-unit completion counters behind them start at zero (the array is
+//     zero when the library loads) and are back at zero when a call ends;
 //   * problems whose split partials do not fit return SA_ERR_WORKSPACE before
 //     anything is launched;
 //   * nothing here calls cudaMalloc, cudaFree or an allocating library.

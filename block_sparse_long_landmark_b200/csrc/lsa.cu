@@ -22,11 +22,11 @@
 
 #include "common.cuh"
 #include "lsa.cuh"
+#include "lsa_dev.cuh"
 
 namespace sa {
 namespace {
 
-constexpr int kLsaThreads = 256;
 
 template <typename T>
 __global__ void __launch_bounds__(kLsaThreads) lsa_build_kernel(LsaShape s, const void *Kv, double *centres64,
@@ -129,123 +129,296 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_build_kernel(LsaShape s, cons
     }
 }
 
+// ---------------------------------------------------------------------------
+// Decode through the index
+// ---------------------------------------------------------------------------
+
+// Kernel 2 (flat decode, step 1): one CTA per (batch, kv-head, chunk of
+// centres).  Pooled query of the kv-group's heads (fp64), score of every
+// centre of the chunk, scale * <q, centre> in fp64, the chunk's best
+// min(top, chunk) by (score desc, id asc); the last chunk CTA of a (batch,
+// kv-head) merges the chunks' candidates into the chosen clusters and
+// expands them into key ranges.
 template <typename T>
-__global__ void __launch_bounds__(kLsaThreads) lsa_decode_kernel(LsaShape s, const void *qv, const void *Kv,
-                                                                const void *Vv, const double *centres64,
-                                                                const int32_t *members, const int32_t *msize,
-                                                                double *scores, unsigned *status, void *ov,
-                                                                float *lse) {
-    extern __shared__ unsigned char smraw[];
-    double *qbar = reinterpret_cast<double *>(smraw);                 // [D]
-    double *rv = qbar + s.d;                                          // [kLsaThreads]
-    int *ri = reinterpret_cast<int *>(rv + kLsaThreads);              // [kLsaThreads]
-    int *chosen = ri + kLsaThreads;                                   // [top_clusters]
-    unsigned *keep = reinterpret_cast<unsigned *>(chosen + max(1, s.top_clusters));   // [ceil(N / 32)]
+__global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
+    extern __shared__ __align__(16) unsigned char smraw[];
+    const LsaShape &s = a.s;
+    const LsaDecPlan &pl = a.pl;
+    double *qbar = reinterpret_cast<double *>(smraw);                           // [d]
+    uint64_t *red64 = reinterpret_cast<uint64_t *>(qbar + s.d);                 // [16]
+    int *red = reinterpret_cast<int *>(red64 + 16);                             // [8]
+    int *flag = red + 8;                                                        // [8]
+    uint64_t *keys = reinterpret_cast<uint64_t *>(flag + 8);                    // [max(CH, S*kk)]
+    const int kmax = max(pl.CH, pl.S * pl.kk);
+    int *ids = reinterpret_cast<int *>(keys + kmax);                            // [max(CH, S*kk)]
+    int *pos = ids + kmax;                                                      // [max(CH, S*kk)]
+    int *chosen = pos + kmax;                                                   // [ntop]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bg = blockIdx.x, b = bg / s.Hkv, g = bg % s.Hkv;
+    const int bg = blockIdx.x / pl.S, chunk = blockIdx.x % pl.S;
+    const int b = bg / s.Hkv, g = bg % s.Hkv;
     const int D = s.d;
-    const T *q = (const T *)qv;
+    const T *q = (const T *)a.q;
     for (int e = tid; e < D; e += kLsaThreads) {
         double acc = 0.0;
         for (int h = 0; h < s.G; ++h) acc += (double)to_f(q[((size_t)b * s.Hq + g * s.G + h) * D + e]);
         qbar[e] = acc / s.G;
     }
-    const int nw = (s.N + 31) / 32;
-    for (int x = tid; x < nw; x += kLsaThreads) keep[x] = 0u;
     __syncthreads();
-    // scores of every centre
-    double *sc = scores + (size_t)bg * s.ctotal;
-    const double *cb = centres64 + (size_t)bg * s.ctotal * D;
-    for (int c = tid; c < s.ctotal; c += kLsaThreads) {
-        double acc = 0.0;
-        for (int e = 0; e < D; ++e) acc += cb[(size_t)c * D + e] * qbar[e];
-        sc[c] = (double)s.scale * acc;
-    }
-    __syncthreads();
-    // the best top_clusters, by (score desc, id asc): repeated arg-max
-    const int ntop = min(s.top_clusters, s.ctotal);
-    for (int r = 0; r < ntop; ++r) {
-        double bv = -CUDART_INF;
-        int bi = 0x7fffffff;
-        for (int c = tid; c < s.ctotal; c += kLsaThreads) {
-            bool taken = false;
-            for (int x = 0; x < r; ++x) taken |= chosen[x] == c;
-            if (taken) continue;
-            const double v = isnan(sc[c]) ? -CUDART_INF : sc[c];   // NaN ranks lowest
-            if (v > bv || (v == bv && c < bi)) { bv = v; bi = c; }
+    // scores of the chunk: a warp per centre, 16-byte loads, four centres in flight
+    const int c0 = chunk * pl.CH, n = max(0, min(s.ctotal, c0 + pl.CH) - c0);
+    const double *cb = a.centres + ((size_t)bg * s.ctotal + c0) * D;
+    const int epl = D / 32;                    // doubles per lane: 2 (d 64) or 4 (d 128)
+    bool nan_seen = false;
+    for (int c = warp * 4; c < n; c += 4 * (kLsaThreads / 32)) {
+        double part[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int cc = min(c + u, n - 1);
+            const double *row = cb + (size_t)cc * D + lane * epl;
+            double acc = 0.0;
+            for (int e = 0; e < epl; e += 2) {
+                const double2 v = *reinterpret_cast<const double2 *>(row + e);
+                acc = fma(v.x, qbar[lane * epl + e], acc);
+                acc = fma(v.y, qbar[lane * epl + e + 1], acc);
+            }
+            part[u] = acc;
         }
-        rv[tid] = bv;
-        ri[tid] = bi;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xffffffffu, part[u], o);
+            if (lane == 0 && c + u < n) {
+                const double sc = (double)s.scale * part[u];
+                nan_seen |= isnan(sc);
+                keys[c + u] = ord_key64(sc);
+            }
+        }
+    }
+    if (nan_seen) set_status(a.status, kStatusNaN);
+    __syncthreads();
+    const int nsel = block_topk64(keys, n, pl.kk, pos, red, red64);
+    if (pl.S > 1) {
+        // the chunk's candidates (ascending id) for the merge
+        uint64_t *pk = a.pkey + ((size_t)bg * pl.S + chunk) * pl.kk;
+        int32_t *pi = a.pid + ((size_t)bg * pl.S + chunk) * pl.kk;
+        for (int i = tid; i < nsel; i += kLsaThreads) {
+            pk[i] = keys[pos[i]];
+            pi[i] = c0 + pos[i];
+        }
+        __threadfence();
         __syncthreads();
-        for (int w = kLsaThreads / 2; w > 0; w >>= 1) {
-            if (tid < w && (rv[tid + w] > rv[tid] || (rv[tid + w] == rv[tid] && ri[tid + w] < ri[tid]))) {
-                rv[tid] = rv[tid + w];
-                ri[tid] = ri[tid + w];
-            }
-            __syncthreads();
-        }
-        if (tid == 0) chosen[r] = ri[0];
+        if (tid == 0) flag[0] = atomicAdd(a.done1 + bg, 1u) == (unsigned)(pl.S - 1);
         __syncthreads();
-    }
-    for (int c = tid; c < s.ctotal; c += kLsaThreads)
-        if (isnan(sc[c])) set_status(status, kStatusNaN);
-    // kept positions: the chosen clusters' items, the first `sink`, the last `window`
-    const int qpos = s.N - 1;
-    for (int r = 0; r < ntop; ++r) {
-        if (chosen[r] < 0 || chosen[r] >= s.ctotal) {    // every candidate taken: nothing left to expand
-            if (tid == 0) set_status(status, kStatusBadIndex);
-            continue;
-        }
-        const size_t cid = (size_t)bg * s.ctotal + chosen[r];
-        const int m = min(max(msize[cid], 0), s.seg);
-        for (int x = tid; x < m * s.pool; x += kLsaThreads) {
-            const int item = members[cid * s.seg + x / s.pool];
-            const int t = item * s.pool + x % s.pool;
-            if (item < 0 || t >= s.N) {            // not an index this build wrote: skip, report
-                set_status(status, kStatusBadIndex);
-                continue;
+        if (!flag[0]) return;
+        __threadfence();
+        // merge: chunk c holds min(kk, its centres) candidates, packed in chunk order
+        int ntot = 0;
+        for (int c = 0; c < pl.S; ++c) ntot += min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
+        for (int e = tid; e < pl.S * pl.kk; e += kLsaThreads) {
+            const int c = e / pl.kk, i = e % pl.kk;
+            const int nv = min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
+            if (i < nv) {
+                int base = 0;
+                for (int x = 0; x < c; ++x) base += min(pl.kk, max(0, min(s.ctotal, (x + 1) * pl.CH) - x * pl.CH));
+                const size_t src = ((size_t)bg * pl.S + c) * pl.kk + i;
+                keys[base + i] = __ldcg(reinterpret_cast<const unsigned long long *>(a.pkey) + src);
+                ids[base + i] = __ldcg(a.pid + src);
             }
-            if (t <= qpos) atomicOr(&keep[t >> 5], 1u << (t & 31));
         }
+        __syncthreads();
+        const int nfin = block_topk64(keys, ntot, pl.ntop, pos, red, red64);
+        for (int i = tid; i < nfin; i += kLsaThreads) chosen[i] = ids[pos[i]];
+        if (tid == 0) a.done1[bg] = 0u;
+        __syncthreads();
+        expand_ranges(a, bg, chosen, nfin, red);
+    } else {
+        for (int i = tid; i < nsel; i += kLsaThreads) chosen[i] = c0 + pos[i];
+        __syncthreads();
+        expand_ranges(a, bg, chosen, nsel, red);
     }
-    for (int t = tid; t < s.N; t += kLsaThreads) {
-        if (t < s.sink || (t > qpos - s.window && t <= qpos)) atomicOr(&keep[t >> 5], 1u << (t & 31));
+}
+
+// Kernel 3 (flat decode, step 2): one CTA per (batch, kv-head, slice of the
+// kept positions).  The slice's positions are laid out in shared memory from
+// the ranges; then a VPR-lane group per key row streams K and V with 16-byte
+// loads and keeps an online softmax (fp32, exp2 domain) per query head of
+// the pass.  Lane groups, warps and finally the CTAs of a (batch, kv-head)
+// are merged by log-sum-exp; the last CTA writes o and lse.
+template <typename T, int HG>
+__global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
+    constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
+    constexpr int EPV = 16 / (int)sizeof(T);
+    extern __shared__ __align__(16) unsigned char smraw[];
+    const LsaShape &s = a.s;
+    const LsaDecPlan &pl = a.pl;
+    const int D = s.d, VPR = D / EPV, RPW = 32 / VPR;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int sub = lane / VPR, cv = lane % VPR;
+    const int bg = blockIdx.x / pl.P, pi = blockIdx.x % pl.P;
+    const int b = bg / s.Hkv, g = bg % s.Hkv;
+    int *posv = reinterpret_cast<int *>(smraw);                                // [slice]
+    float *wst = reinterpret_cast<float *>(posv + ((pl.slice + 3) & ~3));      // [8 warps][HG][D + 2]
+    int *misc = reinterpret_cast<int *>(wst + (kLsaThreads / 32) * HG * (D + 2));   // [4]
+
+    const int nr = a.cnt[2 * (size_t)bg], tot = a.cnt[2 * (size_t)bg + 1];
+    const int t0 = (int)((long long)tot * pi / pl.P);
+    int t1 = (int)((long long)tot * (pi + 1) / pl.P);
+    if (t1 - t0 > pl.slice) {      // more positions than a valid index can keep (repeated items): cut, report
+        if (tid == 0) set_status(a.status, kStatusBadIndex);
+        t1 = t0 + pl.slice;
+    }
+    const int32_t *rs = a.rs + (size_t)bg * pl.rmax, *rl = a.rl + (size_t)bg * pl.rmax, *rp = a.rp + (size_t)bg * pl.rmax;
+    if (tid == 0) {
+        // ranges [r0, r1) overlap [t0, t1): rp ascending, every length > 0
+        int lo = 0, hi = nr;                       // first r with rp[r] + rl[r] > t0
+        while (lo < hi) {
+            const int m = (lo + hi) >> 1;
+            if (rp[m] + rl[m] > t0) hi = m; else lo = m + 1;
+        }
+        misc[0] = lo;
+        lo = misc[0];
+        hi = nr;                                   // first r with rp[r] >= t1
+        while (lo < hi) {
+            const int m = (lo + hi) >> 1;
+            if (rp[m] >= t1) hi = m; else lo = m + 1;
+        }
+        misc[1] = lo;
     }
     __syncthreads();
-    // one warp per query head: online softmax over the kept positions (fp32)
-    const T *K = (const T *)Kv + (size_t)bg * s.N * D;
-    const T *V = (const T *)Vv + (size_t)bg * s.N * D;
-    constexpr int kMaxEPT = 4;                       // d <= 128
-    const int ept = D / 32;
-    for (int h = warp; h < s.G; h += kLsaThreads / 32) {
-        const int head = g * s.G + h;
-        float qh[kMaxEPT], o[kMaxEPT];
-        for (int c = 0; c < kMaxEPT; ++c) {
-            qh[c] = c < ept ? to_f(q[((size_t)b * s.Hq + head) * D + lane + 32 * c]) : 0.f;
-            o[c] = 0.f;
+    const int r0 = misc[0], r1 = misc[1];
+    for (int r = r0 + warp; r < r1; r += kLsaThreads / 32) {
+        const int st = rs[r], pre = rp[r], len = rl[r];
+        const int from = max(t0, pre), to = min(t1, pre + len);
+        for (int v = from + lane; v < to; v += 32) posv[v - t0] = st + (v - pre);
+    }
+    __syncthreads();
+    const int np = t1 - t0;
+    const T *Kb = (const T *)a.K + (size_t)bg * s.N * D;
+    const T *Vb = (const T *)a.V + (size_t)bg * s.N * D;
+    const float sl2 = s.scale * kLog2e;
+    for (int h0 = 0; h0 < s.G; h0 += HG) {
+        const int nh = min(HG, s.G - h0);
+        float qf[HG][EPV], acc[HG][EPV], m[HG], l[HG];
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+            if (h < nh) load16((const T *)a.q + ((size_t)b * s.Hq + g * s.G + h0 + h) * D + cv * EPV, qf[h]);
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) {
+                if (h >= nh) qf[h][e] = 0.f;
+                qf[h][e] *= sl2;
+                acc[h][e] = 0.f;
+            }
+            m[h] = -CUDART_INF_F;
+            l[h] = 0.f;
         }
-        float m = -CUDART_INF_F, l = 0.f;
-        for (int w = 0; w < nw; ++w) {
-            unsigned bits = keep[w];
-            while (bits) {
-                const int t = w * 32 + __ffs(bits) - 1;
-                bits &= bits - 1;
-                float dot = 0.f;
-                for (int c = 0; c < ept; ++c) dot += qh[c] * to_f(K[(size_t)t * D + lane + 32 * c]);
-                for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-                const float z = s.scale * dot;
-                const float mn = fmaxf(m, z);
-                const float corr = expf(m - mn), p = expf(z - mn);
-                l = l * corr + p;
-                for (int c = 0; c < ept; ++c) o[c] = o[c] * corr + p * to_f(V[(size_t)t * D + lane + 32 * c]);
-                m = mn;
+        // rows of this lane group: vb + sub + u * RPW * 8 for the warp's bases vb
+        // (the trip count is the same for every lane: the row reductions
+        // shuffle over the whole warp); two rows per group in flight
+        constexpr int U = 2, NW = kLsaThreads / 32;
+        for (int vb = warp * RPW; vb < np; vb += U * RPW * NW) {
+            uint4 kr[U], vr[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = min(vb + sub + u * RPW * NW, np - 1);
+                const size_t row = (size_t)posv[v] * D + cv * EPV;
+                kr[u] = *reinterpret_cast<const uint4 *>(Kb + row);
+                vr[u] = *reinterpret_cast<const uint4 *>(Vb + row);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const bool live = vb + sub + u * RPW * NW < np;   // uniform over the lane group
+                float kf[EPV], vf[EPV];
+                load16(reinterpret_cast<const T *>(&kr[u]), kf);
+                load16(reinterpret_cast<const T *>(&vr[u]), vf);
+#pragma unroll
+                for (int h = 0; h < HG; ++h) {
+                    float z = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e) z = fmaf(qf[h][e], kf[e], z);
+                    for (int o = VPR / 2; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                    if (!live || h >= nh) continue;
+                    const float mn = fmaxf(m[h], z);
+                    const float corr = exp2f(m[h] - mn), p = exp2f(z - mn);
+                    l[h] = l[h] * corr + p;
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e) acc[h][e] = fmaf(acc[h][e], corr, p * vf[e]);
+                    m[h] = mn;
+                }
             }
         }
-        T *oh = (T *)ov + ((size_t)b * s.Hq + head) * D;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        for (int c = 0; c < ept; ++c) from_f(oh[lane + 32 * c], o[c] * inv);
-        if (lane == 0) lse[(size_t)b * s.Hq + head] = l > 0.f ? m + logf(l) : -CUDART_INF_F;
+        // merge the warp's lane groups (lanes VPR apart hold the same columns)
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+            for (int o = VPR; o < 32; o <<= 1) {
+                const float mo = __shfl_xor_sync(0xffffffffu, m[h], o);
+                const float lo = __shfl_xor_sync(0xffffffffu, l[h], o);
+                const float mn = fmaxf(m[h], mo);
+                const float f0 = m[h] == -CUDART_INF_F ? 0.f : exp2f(m[h] - mn);
+                const float f1 = mo == -CUDART_INF_F ? 0.f : exp2f(mo - mn);
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) {
+                    const float ao = __shfl_xor_sync(0xffffffffu, acc[h][e], o);
+                    acc[h][e] = acc[h][e] * f0 + ao * f1;
+                }
+                l[h] = l[h] * f0 + lo * f1;
+                m[h] = mn;
+            }
+            if (sub == 0) {
+                float *w = wst + (warp * HG + h) * (D + 2);
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) w[2 + cv * EPV + e] = acc[h][e];
+                if (cv == 0) {
+                    w[0] = m[h];
+                    w[1] = l[h];
+                }
+            }
+        }
+        __syncthreads();
+        // merge the warps; this CTA's partial per head
+        for (int x = tid; x < nh * (D + 2); x += kLsaThreads) {
+            const int h = x / (D + 2), e = x % (D + 2);
+            float M = -CUDART_INF_F;
+            for (int w = 0; w < kLsaThreads / 32; ++w) M = fmaxf(M, wst[(w * HG + h) * (D + 2)]);
+            float val = 0.f;
+            if (e == 0) {
+                val = M;
+            } else {
+                for (int w = 0; w < kLsaThreads / 32; ++w) {
+                    const float *ww = wst + (w * HG + h) * (D + 2);
+                    if (ww[0] != -CUDART_INF_F) val = fmaf(ww[e], exp2f(ww[0] - M), val);
+                }
+            }
+            a.part[(((size_t)bg * pl.P + pi) * s.G + h0 + h) * (D + 2) + e] = val;
+        }
+        __syncthreads();
     }
+    // the last CTA of this (batch, kv-head) merges the partials
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) misc[2] = atomicAdd(a.done2 + bg, 1u) == (unsigned)(pl.P - 1);
+    __syncthreads();
+    if (!misc[2]) return;
+    __threadfence();
+    for (int x = tid; x < s.G * D; x += kLsaThreads) {
+        const int h = x / D, e = x % D;
+        float M = -CUDART_INF_F;
+        for (int p = 0; p < pl.P; ++p) M = fmaxf(M, __ldcg(a.part + (((size_t)bg * pl.P + p) * s.G + h) * (D + 2)));
+        float L = 0.f, O = 0.f;
+        if (M != -CUDART_INF_F) {
+            for (int p = 0; p < pl.P; ++p) {
+                const float *pp = a.part + (((size_t)bg * pl.P + p) * s.G + h) * (D + 2);
+                const float mp = __ldcg(pp);
+                if (mp == -CUDART_INF_F) continue;
+                const float f = exp2f(mp - M);
+                L = fmaf(__ldcg(pp + 1), f, L);
+                O = fmaf(__ldcg(pp + 2 + e), f, O);
+            }
+        }
+        const size_t oh = (size_t)b * s.Hq + g * s.G + h;
+        from_f(((T *)a.o)[oh * D + e], L > 0.f ? O / L : 0.f);
+        if (e == 0) a.lse[oh] = L > 0.f ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
+    }
+    if (tid == 0) a.done2[bg] = 0u;
 }
 
 }  // namespace
@@ -267,21 +440,128 @@ cudaError_t launch_lsa_build(const LsaShape &s, const void *K, double *centres, 
     return cudaGetLastError();
 }
 
-cudaError_t launch_lsa_decode(const LsaShape &s, const void *q, const void *K, const void *V, const double *centres,
-                              const int32_t *members, const int32_t *sizes, double *scores, unsigned *status, void *o,
-                              float *lse, cudaStream_t st) {
-    const size_t smem = sizeof(double) * ((size_t)s.d + kLsaThreads) +
-                        sizeof(int) * (kLsaThreads + (size_t)max(1, s.top_clusters)) +
-                        sizeof(unsigned) * (((size_t)s.N + 31) / 32);
-    void (*kern)(LsaShape, const void *, const void *, const void *, const double *, const int32_t *, const int32_t *,
-                 double *, unsigned *, void *, float *) =
-        s.dtype == SA_BF16 ? lsa_decode_kernel<__nv_bfloat16> : lsa_decode_kernel<float>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+bool lsa_decode_plan(const LsaShape &s, LsaDecPlan &pl, bool chunks) {
+    const int C = s.ctotal;
+    const int top = s.top_clusters;
+    pl.ntop = min(top, C);
+    if (pl.ntop == 0 || !chunks) {
+        // nothing to choose: one CTA per (batch, kv-head) lays out the sink and the window
+        pl.CH = 0;
+        pl.S = 1;
+    } else {
+        // chunks of 128 centres, grown until the merge's candidates fit one CTA
+        pl.CH = 128;
+        pl.S = max(1, (C + pl.CH - 1) / pl.CH);
+        while (pl.S > 1 && (long long)pl.S * min(top, pl.CH) > 12288 && pl.CH < 8192) {
+            pl.CH *= 2;
+            pl.S = max(1, (C + pl.CH - 1) / pl.CH);
+        }
+    }
+    pl.kk = min(top, pl.CH);
+    if (pl.CH > 8192 || (pl.S > 1 && (long long)pl.S * pl.kk > 12288)) return false;
+    pl.rmax = 2 + pl.ntop * s.seg;
+    const long long sink_n = min(s.sink, s.N);
+    const long long bound = min((long long)s.N, sink_n + (long long)s.window + (long long)pl.ntop * s.seg * s.pool);
+    const int bgs = s.B * s.Hkv;
+    // about two CTAs per SM overall, at least 64 positions and at most 2048 per CTA
+    long long P = (bound + 2047) / 2048;
+    P = max(P, min((296LL + bgs - 1) / bgs, (bound + 63) / 64));
+    pl.P = (int)max(1LL, min(P, 4096LL));
+    pl.slice = (int)max(1LL, (bound + pl.P - 1) / pl.P);
+    pl.HG = s.G >= 8 ? 8 : s.G >= 4 ? 4 : s.G >= 2 ? 2 : 1;
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    size_t off = kStatusBytes;
+    pl.off_key = off;   off += al((size_t)bgs * pl.S * max(1, pl.kk) * 8);
+    pl.off_id = off;    off += al((size_t)bgs * pl.S * max(1, pl.kk) * 4);
+    pl.off_done1 = off; off += al((size_t)bgs * 4);
+    pl.off_rs = off;    off += al((size_t)bgs * pl.rmax * 4);
+    pl.off_rl = off;    off += al((size_t)bgs * pl.rmax * 4);
+    pl.off_rp = off;    off += al((size_t)bgs * pl.rmax * 4);
+    pl.off_cnt = off;   off += al((size_t)bgs * 8);
+    pl.off_part = off;  off += al((size_t)bgs * pl.P * s.G * (s.d + 2) * 4);
+    pl.off_done2 = off; off += al((size_t)bgs * 4);
+    pl.bytes = off;
+    return true;
+}
+
+static size_t select_smem(const LsaShape &s, const LsaDecPlan &pl) {
+    const size_t kmax = (size_t)max(pl.CH, pl.S * pl.kk);
+    return sizeof(double) * s.d + 16 * 8 + 16 * 4 + kmax * (8 + 4 + 4) + (size_t)max(1, pl.ntop) * 4;
+}
+
+static size_t attend_smem(const LsaShape &s, const LsaDecPlan &pl) {
+    return (size_t)((pl.slice + 3) & ~3) * 4 + (size_t)(kLsaThreads / 32) * pl.HG * (s.d + 2) * 4 + 16;
+}
+
+template <typename T>
+static cudaError_t run_lsa_attend(const LsaDecArgs &a, cudaStream_t st) {
+    const LsaShape &s = a.s;
+    const LsaDecPlan &pl = a.pl;
+    void (*k2)(LsaDecArgs) = nullptr;
+    switch (pl.HG) {
+        case 1: k2 = lsa_attend_kernel<T, 1>; break;
+        case 2: k2 = lsa_attend_kernel<T, 2>; break;
+        case 4: k2 = lsa_attend_kernel<T, 4>; break;
+        default: k2 = lsa_attend_kernel<T, 8>; break;
+    }
+    const size_t sm2 = attend_smem(s, pl);
+    cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(s.B * s.Hkv), kLsaThreads, smem, st>>>(s, q, K, V, centres, members, sizes, scores, status, o,
-                                                             lse);
+    k2<<<(unsigned)(s.B * s.Hkv) * pl.P, kLsaThreads, sm2, st>>>(a);
     note_launch();
     return cudaGetLastError();
+}
+
+cudaError_t launch_lsa_attend(const LsaDecArgs &a, cudaStream_t st) {
+    return a.s.dtype == SA_BF16 ? run_lsa_attend<__nv_bfloat16>(a, st) : run_lsa_attend<float>(a, st);
+}
+
+void lsa_bind_workspace(LsaDecArgs &a, void *ws) {
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    const LsaDecPlan &pl = a.pl;
+    a.status = reinterpret_cast<unsigned *>(w);
+    a.pkey = reinterpret_cast<uint64_t *>(w + pl.off_key);
+    a.pid = reinterpret_cast<int32_t *>(w + pl.off_id);
+    a.done1 = reinterpret_cast<unsigned *>(w + pl.off_done1);
+    a.rs = reinterpret_cast<int32_t *>(w + pl.off_rs);
+    a.rl = reinterpret_cast<int32_t *>(w + pl.off_rl);
+    a.rp = reinterpret_cast<int32_t *>(w + pl.off_rp);
+    a.cnt = reinterpret_cast<int32_t *>(w + pl.off_cnt);
+    a.part = reinterpret_cast<float *>(w + pl.off_part);
+    a.done2 = reinterpret_cast<unsigned *>(w + pl.off_done2);
+}
+
+template <typename T>
+static cudaError_t run_lsa_select(const LsaDecArgs &a, cudaStream_t st) {
+    const LsaShape &s = a.s;
+    const LsaDecPlan &pl = a.pl;
+    const size_t sm1 = select_smem(s, pl);
+    cudaError_t e = cudaFuncSetAttribute(lsa_select_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+    if (e != cudaSuccess) return e;
+    lsa_select_kernel<T><<<(unsigned)(s.B * s.Hkv) * pl.S, kLsaThreads, sm1, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lsa_decode(const LsaShape &s, const LsaDecPlan &pl, const void *q, const void *K, const void *V,
+                              const double *centres, const int32_t *members, const int32_t *sizes, void *ws,
+                              void *o, float *lse, int32_t *kept, cudaStream_t st) {
+    LsaDecArgs a{};
+    a.s = s;
+    a.pl = pl;
+    a.q = q;
+    a.K = K;
+    a.V = V;
+    a.centres = centres;
+    a.members = members;
+    a.sizes = sizes;
+    a.o = o;
+    a.lse = lse;
+    a.kept = kept;
+    lsa_bind_workspace(a, ws);
+    cudaError_t e = s.dtype == SA_BF16 ? run_lsa_select<__nv_bfloat16>(a, st) : run_lsa_select<float>(a, st);
+    if (e != cudaSuccess) return e;
+    return launch_lsa_attend(a, st);
 }
 
 }  // namespace sa

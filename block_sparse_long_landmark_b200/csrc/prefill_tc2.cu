@@ -75,9 +75,15 @@ constexpr uint32_t kKOff2 = 2 * kTile2;             // K ring
 constexpr uint32_t kVOff2 = kKOff2 + kStages2 * kTile2;
 constexpr uint32_t kBarOff2 = kVOff2 + kStages2 * kTile2;
 constexpr int kMaxList2 = 258;
-constexpr uint32_t kListOff2 = kBarOff2 + 512;      // [2 slots] blk[kMaxList2], gate[kMaxList2]
-constexpr uint32_t kListBytes = 8 * kMaxList2;
-constexpr uint32_t kSmem2 = kListOff2 + 2 * kListBytes + 64 + 1024;   // + counts + alignment slack
+constexpr int kGateRows = 4;                        // per-head gate rows (lists per query head)
+// [2 slots] blk[kMaxList2], gate[kGateRows][kMaxList2]
+constexpr uint32_t kListOff2 = kBarOff2 + 512;
+constexpr uint32_t kListBytes = 4 * kMaxList2 * (1 + kGateRows);
+// per-query-head lists: the unit's entries before they are merged (blk, gate, head, first)
+constexpr uint32_t kMergeOff2 = kListOff2 + 2 * kListBytes;
+constexpr uint32_t kMergeBytes = 16 * kMaxList2 + 8 * kGateRows;   // + per-head list start and count
+constexpr uint32_t kSmem2 = kMergeOff2 + kMergeBytes + 64 + 1024;   // + counts + alignment slack
+static_assert(kSmem2 <= 227 * 1024, "shared memory");
 
 enum {
     C_Q = 0,                    // Q tiles landed (one phase per unit with work)
@@ -107,6 +113,8 @@ struct Tc2Args {
     int npair;   // units per (batch, kv-head, block)
     int hc;      // query heads per unit
     int units;
+    unsigned long long wait_ns;   // limit of every bounded wait
+    int stall_tile;               // test hook: the K load of this key tile (per CTA) is never issued; -1 = off
 };
 
 struct Unit {
@@ -151,7 +159,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kBarOff2 + 8 * NBAR2);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff2 + 8 * NBAR2 + 4);
-    int *cnt_s = reinterpret_cast<int *>(smem + kListOff2 + 2 * kListBytes);   // [2 slots]
+    int *cnt_s = reinterpret_cast<int *>(smem + kMergeOff2 + kMergeBytes);   // [2 slots]
     auto blk_of = [&](int slot) { return reinterpret_cast<int *>(smem + kListOff2 + slot * kListBytes); };
     auto gate_of = [&](int slot) {
         return reinterpret_cast<float *>(smem + kListOff2 + slot * kListBytes + 4 * kMaxList2);
@@ -186,27 +194,104 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         bool ok = true;
         int gt = 0, nq = 0, ul = 0;   // key tiles, Q loads and units so far
-        int nk = 0, nv = 0;           // K and V tiles issued
+        // copies issued and not yet seen complete: the last Q load (its phase),
+        // and per ring stage the last key tile whose K / V load went out (-1:
+        // none).  A stage is reused only after its previous copy was consumed,
+        // so each barrier has at most this one phase outstanding.
+        int qlast = -1, klast[kStages2], vlast[kStages2];
+        for (int i = 0; i < kStages2; ++i) klast[i] = vlast[i] = -1;
         for (int u = blockIdx.x; u < a.units; u += gridDim.x, ++ul) {
             const Unit w = unit_at(a, u);
             const int slot = ul & 1;
-            if (ul >= 2) ok = mbar_wait(bar(C_LF + slot), ((ul >> 1) - 1) & 1, abort_flag, a.status);
+            if (ul >= 2)
+                ok = mbar_wait(bar(C_LF + slot), ((ul >> 1) - 1) & 1, abort_flag, a.status, a.wait_ns);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             // the unit's list: block ids (bad entries -> -1) and log2-unit gates
-            const int cnt = max(0, min(a.count[w.lu], s.cap));
             int *blk_s = blk_of(slot);
             float *gate_s = gate_of(slot);
-            const int32_t *il = a.idx + w.lu * s.cap;
-            const float *sl = a.score + w.lu * s.cap;
-            const float s_loc = cnt > 0 ? sl[cnt - 1] : 0.f;
-            for (int e = lane; e < cnt; e += 32) {
-                const int blk = il[e];
-                const bool good = blk >= 0 && blk <= w.j && (e == 0 || il[e - 1] < blk);
-                if (!good) set_status(a.status, kStatusBadIndex);
-                blk_s[e] = good ? blk : -1;
-                const bool forced = (blk == w.j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
-                gate_s[e] = kHier ? sl[e] * kLog2e
-                            : ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[e] - s_loc) * kLog2e : 0.f;
+            int cnt;
+            if (!(s.flags & SA_SELECT_PER_QHEAD)) {
+                cnt = max(0, min(a.count[w.lu], s.cap));
+                const int32_t *il = a.idx + w.lu * s.cap;
+                const float *sl = a.score + w.lu * s.cap;
+                const float s_loc = cnt > 0 ? sl[cnt - 1] : 0.f;
+                for (int e = lane; e < cnt; e += 32) {
+                    const int blk = il[e];
+                    const bool good = blk >= 0 && blk <= w.j && (e == 0 || il[e - 1] < blk);
+                    if (!good) set_status(a.status, kStatusBadIndex);
+                    blk_s[e] = good ? blk : -1;
+                    const bool forced = (blk == w.j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
+                    gate_s[e] = kHier ? sl[e] * kLog2e
+                                : ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[e] - s_loc) * kLog2e : 0.f;
+                }
+            } else {
+                // one list per query head: the unit's rows (a.hc heads) read the
+                // union of their heads' lists, ascending; gate row hh holds head
+                // hh's gate of each union entry, -inf where that head did not
+                // keep the block (its keys then drop out of that head's softmax)
+                int *mb = reinterpret_cast<int *>(smem + kMergeOff2);     // entry -> block (-1 bad)
+                float *mg = reinterpret_cast<float *>(mb + kMaxList2);     // entry -> gate
+                int *mh = reinterpret_cast<int *>(mg + kMaxList2);         // entry -> head in unit
+                int *mf = mh + kMaxList2;                                  // entry -> first of its block
+                int *hst = mf + kMaxList2;                                 // head -> first entry
+                int *hcn = hst + kGateRows;                                // head -> entries
+                int cn = 0;                                                // this lane's head count (lane < hc)
+                if (lane < a.hc)
+                    cn = max(0, min(a.count[((size_t)w.b * s.Hq + w.h0 + lane) * s.nb + w.j], s.cap));
+                int start = cn;                                            // exclusive prefix over heads
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, start, o);
+                    if (lane >= o) start += t;
+                }
+                start -= cn;
+                const int E = __shfl_sync(0xffffffffu, start + cn, a.hc - 1);
+                if (lane < a.hc) {
+                    hst[lane] = start;
+                    hcn[lane] = cn;
+                }
+                __syncwarp();
+                for (int f = lane; f < E; f += 32) {
+                    int hh = 0;
+                    for (int x = 1; x < a.hc; ++x) hh += f >= hst[x] ? 1 : 0;
+                    mh[f] = hh;
+                    {
+                        const int st = hst[hh], c = hcn[hh];
+                        const int e = f - st;
+                        const size_t lu = ((size_t)w.b * s.Hq + w.h0 + hh) * s.nb + w.j;
+                        const int32_t *il = a.idx + lu * s.cap;
+                        const float *sl = a.score + lu * s.cap;
+                        const int blk = il[e];
+                        const bool good = blk >= 0 && blk <= w.j && (e == 0 || il[e - 1] < blk);
+                        if (!good) set_status(a.status, kStatusBadIndex);
+                        const bool forced = (blk == w.j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
+                        mb[f] = good ? blk : -1;
+                        mg[f] = ((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[e] - sl[c - 1]) * kLog2e : 0.f;
+                    }
+                }
+                __syncwarp();
+                // first entry of each block (lowest head), then its rank among the distinct blocks
+                for (int f = lane; f < E; f += 32) {
+                    const int blk = mb[f];
+                    bool first = blk >= 0;
+                    for (int x = 0; x < f && first; ++x) first = mb[x] != blk;
+                    mf[f] = first ? 1 : 0;
+                }
+                __syncwarp();
+                int nd = 0;
+                for (int f = lane; f < E; f += 32) nd += mf[f];
+                cnt = __reduce_add_sync(0xffffffffu, nd);
+                for (int x = lane; x < a.hc * kMaxList2; x += 32)
+                    if (x % kMaxList2 < cnt) gate_s[x] = -CUDART_INF_F;
+                __syncwarp();
+                for (int f = lane; f < E; f += 32) {
+                    const int blk = mb[f];
+                    if (blk < 0) continue;
+                    int rank = 0;
+                    for (int x = 0; x < E; ++x) rank += (mf[x] && mb[x] < blk) ? 1 : 0;
+                    if (mf[f]) blk_s[rank] = blk;
+                    gate_s[mh[f] * kMaxList2 + rank] = mg[f];
+                }
             }
             if (lane == 0) cnt_s[slot] = cnt;
             __syncwarp();
@@ -214,8 +299,9 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const int T = key_tiles(s, cnt);
             if (lane == 0 && T > 0) {
                 // Q tiles: rows of heads h0 .. h0+3 (block 64) or h0, h0+1 (block 128)
-                if (nq >= 1) ok = mbar_wait(bar(C_QFREE), (nq - 1) & 1, abort_flag, a.status);
+                if (nq >= 1) ok = mbar_wait(bar(C_QFREE), (nq - 1) & 1, abort_flag, a.status, a.wait_ns);
                 if (ok) {
+                    qlast = nq;
                     mbar_expect_tx(bar(C_Q), 2 * kTile2);
                     for (int q = 0; q < 2; ++q)
                         for (int c = 0; c < 2; ++c)
@@ -239,16 +325,20 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         y0 = kvbase + max(0, blk_s[t]) * 128;
                         y1 = y0 + 64;
                     }
-                    if (gg >= kStages2 && !(ok = mbar_wait(bar(C_KE + st), (use - 1) & 1, abort_flag, a.status)))
+                    if (gg >= kStages2 &&
+                        !(ok = mbar_wait(bar(C_KE + st), (use - 1) & 1, abort_flag, a.status, a.wait_ns)))
                         break;
-                    mbar_expect_tx(bar(C_KF + st), kTile2);
-                    for (int c = 0; c < 2; ++c) {
-                        const uint32_t d = sbase + kKOff2 + st * kTile2 + c * kChunk2;
-                        tma_load_2d(d, &tmK, bar(C_KF + st), 64 * c, y0);
-                        tma_load_2d(d + 8192, &tmK, bar(C_KF + st), 64 * c, y1);
+                    if (gg != a.stall_tile) {
+                        mbar_expect_tx(bar(C_KF + st), kTile2);
+                        for (int c = 0; c < 2; ++c) {
+                            const uint32_t d = sbase + kKOff2 + st * kTile2 + c * kChunk2;
+                            tma_load_2d(d, &tmK, bar(C_KF + st), 64 * c, y0);
+                            tma_load_2d(d + 8192, &tmK, bar(C_KF + st), 64 * c, y1);
+                        }
+                        klast[st] = gg;
                     }
-                    nk = gg + 1;
-                    if (gg >= kStages2 && !(ok = mbar_wait(bar(C_VE + st), (use - 1) & 1, abort_flag, a.status)))
+                    if (gg >= kStages2 &&
+                        !(ok = mbar_wait(bar(C_VE + st), (use - 1) & 1, abort_flag, a.status, a.wait_ns)))
                         break;
                     mbar_expect_tx(bar(C_VF + st), kTile2);
                     for (int c = 0; c < 2; ++c) {
@@ -256,7 +346,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         tma_load_2d(d, &tmV, bar(C_VF + st), 64 * c, y0);
                         tma_load_2d(d + 8192, &tmV, bar(C_VF + st), 64 * c, y1);
                     }
-                    nv = gg + 1;
+                    vlast[st] = gg;
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -267,11 +357,13 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (lane == 0 && *abort_flag) {
             // let the copies in flight land before the CTA exits (bounded)
             volatile int never = 0;
-            if (nq > 0) mbar_wait(bar(C_Q), (nq - 1) & 1, &never, a.status);
-            for (int t = max(0, nk - kStages2); t < nk; ++t)
-                mbar_wait(bar(C_KF + t % kStages2), (t / kStages2) & 1, &never, a.status);
-            for (int t = max(0, nv - kStages2); t < nv; ++t)
-                mbar_wait(bar(C_VF + t % kStages2), (t / kStages2) & 1, &never, a.status);
+            if (qlast >= 0) mbar_wait(bar(C_Q), qlast & 1, &never, a.status, a.wait_ns);
+            for (int st = 0; st < kStages2; ++st) {
+                if (klast[st] >= 0)
+                    mbar_wait(bar(C_KF + st), (klast[st] / kStages2) & 1, &never, a.status, a.wait_ns);
+                if (vlast[st] >= 0)
+                    mbar_wait(bar(C_VF + st), (vlast[st] / kStages2) & 1, &never, a.status, a.wait_ns);
+            }
         }
     } else if (warp == 1) {
         // ---- MMA issuer -----------------------------------------------------
@@ -300,7 +392,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 mma_ts_w(tmem + 256 + q * 128, tmem + q * 128 + 8 * k, db + ((k * 2048) >> 4), idp, acc || k > 0);
         };
         auto wait = [&](int i, int parity) {
-            return __all_sync(0xffffffffu, mbar_wait(bar(i), parity, abort_flag, a.status));
+            return __all_sync(0xffffffffu, mbar_wait(bar(i), parity, abort_flag, a.status, a.wait_ns));
         };
         bool ok = true;
         int gt = 0, nq = 0, ul = 0;
@@ -356,7 +448,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         // (waited on even after an abort: TMEM is freed only after it)
         mma_commit_w(bar(C_END));
         volatile int never = 0;
-        mbar_wait(bar(C_END), 0, &never, a.status);
+        mbar_wait(bar(C_END), 0, &never, a.status, a.wait_ns);
     } else if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow2));
     } else {
@@ -375,15 +467,16 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x, ++ul) {
             const Unit w = unit_at(a, u);
             const int slot = ul & 1;
-            ok = mbar_wait(bar(C_L + slot), (ul >> 1) & 1, abort_flag, a.status);
+            ok = mbar_wait(bar(C_L + slot), (ul >> 1) & 1, abort_flag, a.status, a.wait_ns);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             const int cnt = cnt_s[slot];
             const int *blk_s = blk_of(slot);
-            const float *gate_s = gate_of(slot);
             const int T = key_tiles(s, cnt);
             int head, ri;
             if (s.bs == 64) { head = w.h0 + 2 * q + (r >> 6); ri = r & 63; }
             else { head = w.h0 + q; ri = r; }
+            // per-query-head lists: this row's head has its own gate row
+            const float *gate_s = gate_of(slot) + ((s.flags & SA_SELECT_PER_QHEAD) ? (head - w.h0) * kMaxList2 : 0);
             const int qi = w.j * s.bs + ri;              // query position of this row
             float m_run = -CUDART_INF_F, l = 0.f;
             // hierarchical mode ([HiLS]): every block gets its own softmax and
@@ -396,7 +489,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     if (blk_s[e] >= 0) m_run = fmaxf(m_run, gate_s[e]);
             }
             for (int t = 0; t < T; ++t) {
-                ok = mbar_wait(bar(C_S + q), (gt + t) & 1, abort_flag, a.status);
+                ok = mbar_wait(bar(C_S + q), (gt + t) & 1, abort_flag, a.status, a.wait_ns);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
                 float x[128];
@@ -550,7 +643,7 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (!ok) break;
             // ---- epilogue: O_q / l -> bf16, LSE ----------------------------
             if (T > 0) {
-                ok = mbar_wait(bar(C_OD + q), nq & 1, abort_flag, a.status);
+                ok = mbar_wait(bar(C_OD + q), nq & 1, abort_flag, a.status, a.wait_ns);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
             }
@@ -609,10 +702,12 @@ int sm_count() {
 
 bool prefill_tc2_supported(const Shape &s) {
     if (s.dtype != SA_BF16 || s.d != 128) return false;
-    if (s.flags & SA_SELECT_PER_QHEAD) return false;
     if (s.bs != 64 && s.bs != 128) return false;
     if ((s.G * s.bs) % kRows) return false;
     if (s.cap > kMaxList2) return false;
+    // per-query-head lists: the union of a unit's heads must fit one list (gated or plain mode)
+    if ((s.flags & SA_SELECT_PER_QHEAD) && ((s.flags & SA_HIER) || (kRows / s.bs) * s.cap > kMaxList2))
+        return false;
     const char *e = getenv("SPARSE_ATTN_PREFILL_PATH");
     if (e && (strcmp(e, "simt") == 0 || strcmp(e, "tc1") == 0)) return false;
     return true;
@@ -645,6 +740,17 @@ cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, con
     a.status = status;
     a.hc = kRows / s.bs;
     a.npair = s.G / a.hc;
+    a.wait_ns = tc::kWaitNs;
+    a.stall_tile = -1;
+    // Test hook for the bounded waits: SPARSE_ATTN_TEST_STALL=<t> makes every
+    // CTA skip the K load of its key tile t (nothing is left in flight for
+    // it), so the MMA warp's wait on that tile runs out after 1 ms; the CTA
+    // then records kStatusTimeout, lets its other copies land, frees TMEM
+    // and exits.
+    if (const char *st = getenv("SPARSE_ATTN_TEST_STALL")) {
+        a.stall_tile = atoi(st);
+        a.wait_ns = 1000000ull;
+    }
     a.units = s.B * s.Hkv * s.nb * a.npair;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorNoDevice;

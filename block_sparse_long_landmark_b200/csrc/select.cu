@@ -438,6 +438,7 @@ static void geometry(const Shape &s, bool decode, int &nunits, int &S, int &CH) 
 }
 
 size_t select_workspace(const Shape &s, bool decode) {
+    if (decode && select_decode_supported(s)) return select_decode_workspace(s);
     int nunits, S, CH;
     geometry(s, decode, nunits, S, CH);
     if (S == 1) return 0;
@@ -499,6 +500,9 @@ cudaError_t launch_select(const Shape &s, bool decode, const void *Q, const void
     // prefill: eight tiles per CTA share one landmark scan (select_tiles.cu)
     if (!decode && select_tiles_supported(s))
         return launch_select_tiles(s, Q, L, idx, score, count, (unsigned *)ws, st);
+    // decode: a warp per chunk of candidates (select_decode.cu)
+    if (decode && select_decode_supported(s) && !select_force_chunked())
+        return launch_select_decode(s, Q, L, idx, score, count, ws, st);
     return s.dtype == SA_BF16 ? run<__nv_bfloat16>(s, decode, Q, L, idx, score, count, ws, st)
                               : run<float>(s, decode, Q, L, idx, score, count, ws, st);
 }

@@ -46,16 +46,17 @@ __device__ __forceinline__ unsigned long long gtimer() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Bounded wait: true when the phase completed, false on timeout or abort.
+// Bounded wait: true when the phase completed, false on timeout (after
+// limit_ns) or abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          unsigned *status) {
+                                          unsigned *status, unsigned long long limit_ns = kWaitNs) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = gtimer();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try(bar, parity)) return true;
         if ((it & 63) == 63) {
             if (*abort_flag) return false;
-            if (gtimer() - t0 > kWaitNs) {
+            if (gtimer() - t0 > limit_ns) {
                 *abort_flag = 1;
                 set_status(status, kStatusTimeout);
                 return false;

@@ -308,8 +308,12 @@ typedef struct {
  * SA_ERR_* code for invalid / unsupported parameters. */
 int sparse_attn_lsa_clusters(const sa_lsa_params *p);
 
-/* Workspace bytes for sparse_attn_lsa_decode (status word + scores), 0 when
- * the parameters are invalid. */
+/* Workspace bytes for sparse_attn_lsa_decode, 0 when the parameters are
+ * invalid or unsupported.  Holds the status word, the chunks' candidate
+ * clusters, the kept key ranges, the split attention partials and two
+ * completion counters; zero-fill it once when allocated (the counters are
+ * returned to zero by every call).  Calls sharing a workspace must not
+ * overlap on the GPU. */
 size_t sparse_attn_lsa_workspace_size(const sa_lsa_params *p);
 
 /* Builds the index of every (batch, kv-head) from K [B,Hkv,N,d]:
@@ -321,11 +325,63 @@ int sparse_attn_lsa_build(const sa_lsa_params *p, const void *K, double *centres
 
 /* Decode through the index: q [B,Hq,d], K, V [B,Hkv,N,d] and the index of
  * sparse_attn_lsa_build -> o [B,Hq,d] (dtype of p), lse [B,Hq] (fp32, natural
- * log; -inf when nothing is kept).  A member entry outside the context sets
- * status bit 1 and is skipped. */
+ * log; -inf when nothing is kept), and, when `kept` is not NULL, the number
+ * of key positions each (batch, kv-head) attended to (int32 [B,Hkv]).
+ * Two kernels: centre scores (fp64) in chunks over many CTAs with an exact
+ * top_clusters merge, expanded to key ranges; then the kept keys split over
+ * many CTAs with a log-sum-exp merge.  The merge of the chunks' candidates
+ * runs in one CTA: parameters with top_clusters x ceil(C / 8192) > 12288
+ * (C = clusters per (batch, kv-head)) return SA_ERR_UNSUPPORTED.  A member
+ * entry outside the complete segments sets status bit 1 and is skipped; a
+ * NaN centre score sets bit 2 and ranks below every number. */
 int sparse_attn_lsa_decode(const sa_lsa_params *p, const void *q, const void *K, const void *V,
                            const double *centres, const int32_t *members, const int32_t *sizes, void *o, float *lse,
-                           void *ws, size_t ws_bytes, void *stream);
+                           int32_t *kept, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- Tree over the flat index's clusters (same section of the post: the
+ * clusters are grouped into a hierarchy that a query walks with a beam
+ * search, keeping a few good branches per level, so that it is compared
+ * against far fewer centres than in a flat scan) -------------------------
+ * Construction (the post gives none; this is the reading the library takes):
+ * the flat clusters are the leaves (level 0); every level above is a Ward
+ * clustering of the level below into ceil(n / fanout) nodes, each node
+ * weighted by the key positions it holds, numbered by their first child;
+ * a node's centre is the mass-weighted mean of its children's centres;
+ * levels are added while a level holds more than `fanout` nodes.  Search:
+ * the pooled query is scored against every node of the top level, the
+ * `beam` best of a level by (score desc, id asc) are expanded into their
+ * children, and at the leaves the `top_clusters` best are kept; they are
+ * expanded to key positions, with the sink and window, as in the flat
+ * decode.  Supports 2 <= fanout <= 64 and 1 .. 4096 clusters per (batch,
+ * kv-head); anything else returns SA_ERR_UNSUPPORTED (fanout < 2:
+ * SA_ERR_ARG). */
+
+/* Bytes of the caller-owned tree buffer (0 when invalid or unsupported);
+ * *levels (may be NULL) receives the number of levels, leaves included.
+ * Layout, per level l >= 1 and (batch, kv-head): centres [n_l][d] fp64,
+ * masses [n_l] fp64, first-child offsets [n_l + 1] int32, children
+ * [n_(l-1)] int32 (ascending within each parent); level 0: masses only. */
+size_t sparse_attn_lsa_tree_size(const sa_lsa_params *p, int fanout, int *levels);
+
+/* Workspace bytes for sparse_attn_lsa_tree_build and _tree_decode (one
+ * buffer serves both; zero-fill it once when allocated). */
+size_t sparse_attn_lsa_tree_workspace_size(const sa_lsa_params *p, int fanout);
+
+/* Builds the tree of every (batch, kv-head) from the flat index's centres
+ * and sizes (sparse_attn_lsa_build) into `tree`.  One CTA per (batch,
+ * kv-head) runs Ward's merges level by level in fp64. */
+int sparse_attn_lsa_tree_build(const sa_lsa_params *p, int fanout, const double *centres, const int32_t *sizes,
+                               void *tree, void *ws, size_t ws_bytes, void *stream);
+
+/* Decode through the tree: beam search (beam >= 1) down to the leaves, the
+ * `top_clusters` best leaves expanded to key ranges with the sink and
+ * window, then attention as in sparse_attn_lsa_decode.  Outputs o, lse and,
+ * when not NULL, kept [B,Hkv] (key positions attended) and compared [B,Hkv]
+ * (centres scored on the way down). */
+int sparse_attn_lsa_tree_decode(const sa_lsa_params *p, int fanout, int beam, const void *q, const void *K,
+                                const void *V, const double *centres, const int32_t *members, const int32_t *sizes,
+                                const void *tree, void *o, float *lse, int32_t *kept, int32_t *compared, void *ws,
+                                size_t ws_bytes, void *stream);
 
 /* Synchronises `stream`, returns SA_OK or SA_ERR_DEVICE from the status
  * word in `ws`, and clears it.  *detail (may be NULL) receives the raw bits:

@@ -139,5 +139,36 @@ def test_lsa_entry_points_check_arguments():
     a = 256
     assert sa.sparse_attn_lsa_build(ok, None, a, a, a, None) == sa.SA_ERR_ARG
     assert sa.sparse_attn_lsa_build(ok, a, None, a, a, None) == sa.SA_ERR_ARG
-    assert sa.sparse_attn_lsa_decode(ok, a, a, a, a, a, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
-    assert sa.sparse_attn_lsa_decode(ok, None, a, a, a, a, a, a, a, a, 1 << 20, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_lsa_decode(ok, a, a, a, a, a, a, a, a, None, a, 16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.sparse_attn_lsa_decode(ok, None, a, a, a, a, a, a, a, None, a, 1 << 20, None) == sa.SA_ERR_ARG
+    # the chunk merge of the decode runs in one CTA: too many candidates are refused up front
+    big = sa.make_lsa_params(1, 4, 2, 128, 1 << 20, 1, 64, 64, 4096, 16, 64)
+    assert sa.sparse_attn_lsa_clusters(big) == (1 << 20)
+    assert sa.sparse_attn_lsa_workspace_size(big) == 0
+    assert sa.sparse_attn_lsa_decode(big, a, a, a, a, a, a, a, a, None, a, 1 << 30, None) == sa.SA_ERR_UNSUPPORTED
+
+
+def test_lsa_tree_host_checks():
+    """The tree entry points' host-side checks (no launch happens)."""
+    p = sa.make_lsa_params(1, 4, 2, 128, 8192, 4, 32, 8, 6, 16, 64)      # 512 clusters per kv-head
+    nbytes, levels = sa.sparse_attn_lsa_tree_size(p, 4)
+    assert nbytes > 0 and levels == 5                                       # 512, 128, 32, 8, 2
+    assert sa.sparse_attn_lsa_tree_size(p, 8)[1] == 3                       # 512, 64, 8
+    assert sa.sparse_attn_lsa_tree_size(p, 1)[0] == 0                       # a fan-out below 2 is refused
+    assert sa.sparse_attn_lsa_tree_size(p, 65)[0] == 0
+    ws = sa.sparse_attn_lsa_tree_workspace_size(p, 4)
+    assert ws > sa.sparse_attn_lsa_workspace_size(p)
+    a = 256
+    assert sa.sparse_attn_lsa_tree_build(p, 1, a, a, a, a, ws, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_lsa_tree_build(p, 4, None, a, a, a, ws, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_lsa_tree_build(p, 4, a, a, a, a, 16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.sparse_attn_lsa_tree_decode(p, 4, 0, a, a, a, a, a, a, a, a, a, None, None, a, ws, None) == sa.SA_ERR_ARG
+    assert sa.sparse_attn_lsa_tree_decode(p, 4, 3, None, a, a, a, a, a, a, a, a, None, None, a, ws, None) == \
+        sa.SA_ERR_ARG
+    assert sa.sparse_attn_lsa_tree_decode(p, 4, 3, a, a, a, a, a, a, a, a, a, None, None, a, 16, None) == \
+        sa.SA_ERR_WORKSPACE
+    # more leaves than a tree supports
+    big = sa.make_lsa_params(1, 4, 2, 128, 1 << 17, 1, 16, 8, 6, 16, 64)   # 65536 clusters
+    assert sa.sparse_attn_lsa_tree_size(big, 4)[0] == 0
+    assert sa.sparse_attn_lsa_tree_decode(big, 4, 3, a, a, a, a, a, a, a, a, a, None, None, a, 1 << 30, None) == \
+        sa.SA_ERR_UNSUPPORTED

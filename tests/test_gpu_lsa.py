@@ -25,6 +25,13 @@ CASES = {
                             window=40, dtype="bf16", seed=3),
     "bf16_pool1_everything": dict(B=1, Hq=2, Hkv=1, d=64, N=300, pool=1, seg=20, clusters=5, top=1000, sink=0,
                                   window=0, dtype="bf16", seed=4),
+    # many centre chunks (merge across 6 chunk CTAs), eight query heads per kv-head, overlapping sink and window
+    "bf16_many_chunks_g8": dict(B=1, Hq=16, Hkv=2, d=128, N=6144, pool=2, seg=32, clusters=16, top=40, sink=40,
+                                window=300, dtype="bf16", seed=5),
+    "fp32_g16_two_passes": dict(B=1, Hq=16, Hkv=1, d=64, N=2048, pool=4, seg=16, clusters=4, top=7, sink=3,
+                                window=2100, dtype="fp32", seed=6),
+    "bf16_no_clusters": dict(B=1, Hq=4, Hkv=2, d=128, N=100, pool=4, seg=32, clusters=4, top=8, sink=5,
+                             window=20, dtype="bf16", seed=7),
 }
 
 
@@ -46,9 +53,13 @@ def test_flat_index_matches_oracle(case):
     qd, Kd, Vd = q.cuda(), K.cuda(), V.cuda()
     index = sa.lsa_build(p, Kd)
     ws = sa.lsa_workspace(p)
-    o, lse = sa.lsa_decode(p, qd, Kd, Vd, index, ws)
+    kept = torch.full((c["B"], c["Hkv"]), -1, dtype=torch.int32, device="cuda")
+    o, lse = sa.lsa_decode(p, qd, Kd, Vd, index, ws, kept=kept)
     torch.cuda.synchronize()
     assert sa.check_status(ws) == 0
+    o2, lse2 = sa.lsa_decode(p, qd, Kd, Vd, index, ws)        # a second call: counters were reset
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
     C = sa.sparse_attn_lsa_clusters(p)
     centres, members, sizes = (x.cpu().numpy() for x in index)
     q64, K64, V64 = (x.double().numpy() for x in (q, K, V))
@@ -64,6 +75,9 @@ def test_flat_index_matches_oracle(case):
                 np.testing.assert_allclose(centres[b, g, :C], ref["centres"], rtol=1e-12, atol=1e-12)
     want = lsa.decode(q64, K64, V64, c["pool"], c["seg"], c["clusters"], c["top"], c["sink"], c["window"],
                       scale=float(np.float32(1.0 / np.sqrt(c["d"]))))
+    for b in range(c["B"]):
+        for g in range(c["Hkv"]):
+            assert int(kept[b, g]) == len(want["kept"][(b, g)][1]), (b, g)
     tol = 2e-2 if c["dtype"] == "bf16" else 1e-4
     assert np.abs(o.float().cpu().numpy() - want["O"]).max() <= tol
     assert np.abs(lse.cpu().numpy() - want["LSE"]).max() <= 1e-3

@@ -336,3 +336,35 @@ def test_nan_score_sets_status():
     sa.select(p, Q, L, ws)
     rc, detail = sa.sparse_attn_check_status(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert rc == sa.SA_ERR_DEVICE and detail & 2
+
+
+PERQ_TC_CASES = {
+    # four query heads of a group share a 256-row unit: the union of their four lists
+    "b64_g4": W["gated_prefill_32k_perqhead"].scaled(N=4096, Hq=8, Hkv=2),
+    # two heads of a block-128 tile, ragged end
+    "b128_g2_ragged": W["long_prefill_256k"].scaled(N=3000, Hq=4, Hkv=2, per_qhead=True),
+    # plain (no gate) mode, batch 2
+    "b64_plain_batch2": W["gated_prefill_32k_perqhead"].scaled(B=2, N=2048, Hq=8, Hkv=2),
+}
+
+
+@pytest.mark.parametrize("case", sorted(PERQ_TC_CASES))
+def test_per_qhead_prefill_on_tensor_cores(case, monkeypatch):
+    """One list per query head on the persistent tensor-core kernel: each unit
+    reads the union of its heads' lists and masks, per row, the blocks its
+    head did not keep.  Against the oracle (its own lists) and against the
+    CUDA-core kernel on the same lists."""
+    wl = PERQ_TC_CASES[case]
+    flags = wl.flags & ~inputs.F_GATE if "plain" in case else wl.flags
+    p = sa.params_for(wl, flags=flags)
+    assert sa.sparse_attn_prefill_kernel(p) == 2
+    Q, K, V = _prefill_inputs(wl)
+    ref = _oracle_prefill(wl, Q, K, V, flags=flags)
+    sel = oracle_sel_tensors(ref)
+    _, _, O, lse = run_prefill(p, Q, K, V, sel=sel)
+    _check_outputs(wl, ref, O, lse)
+    monkeypatch.setenv("SPARSE_ATTN_PREFILL_PATH", "simt")
+    assert sa.sparse_attn_prefill_kernel(p) == 0
+    _, _, O2, lse2 = run_prefill(p, Q, K, V, sel=sel)
+    assert (O.float() - O2.float()).abs().max().item() <= 2e-2
+    assert (lse - lse2).abs().max().item() <= 1e-3

@@ -46,6 +46,26 @@ def test_static_decode_matches_workspace_decode(case):
         assert (lse[fin] - lse_ref[fin]).abs().max().item() <= LSE_TOL
 
 
+def test_static_decode_matches_the_oracle():
+    """The same entry point against the CPU oracle on the oracle's own lists."""
+    import oracle
+    wl = CASES["gated"]
+    p = sa.params_for(wl)
+    q, K, V = inputs.make_decode(wl, device="cuda")
+
+    def f64(t):
+        return t.float().cpu().numpy().astype(np.float64)
+
+    ref = oracle.decode(f64(q), f64(K), f64(V), wl.block, wl.top_k, wl.flags, round_mode=oracle.ROUND_BF16)
+    sel = (torch.from_numpy(ref["idx"].astype(np.int32)).cuda(), torch.from_numpy(ref["sc"].astype(np.float32)).cuda(),
+           torch.from_numpy(ref["count"].astype(np.int32)).cuda())
+    for _ in range(2):
+        o, lse = sa.decode_static(p, q, K, V, *sel)
+        torch.cuda.synchronize()
+        assert np.abs(f64(o) - ref["O"]).max() <= O_TOL[wl.dtype]
+        assert np.abs(f64(lse) - ref["LSE"]).max() <= LSE_TOL
+
+
 def test_static_decode_rejects_problems_beyond_the_scratch():
     # 74 units of 16 query heads each, split in 4: 2.46 MB of partials > 2 MiB
     wl = inputs.WORKLOADS["gated_decode_128k"].scaled(B=74, Hq=16, Hkv=1)
