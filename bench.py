@@ -20,7 +20,8 @@ full records.
 
 Timing: CUDA events on the launching stream around each step and each C call,
 W warm-up steps, K timed steps bracketed by barrier + synchronize, L2 flushed
-(a 256 MiB write) before every timed step, max over ranks.  ``--impl
+before every timed step (a 256 MiB write, then a 256 MiB read, so that no
+input and no dirty line is left in L2), max over ranks.  ``--impl
 reference`` times the CPU oracle (a deliberately slow, plain C reference) on a
 bounded sample of the same workload on the host cores.
 """
@@ -222,7 +223,18 @@ class Timer:
 
 
 def flush_l2(buf):
-    buf.fill_(1)
+    """Writes a buffer larger than L2, then reads a second one: every step
+    starts with none of its inputs in L2 and no dirty line left from the
+    flush (otherwise the first kernel of the step pays the flush's own
+    write-back to DRAM)."""
+    w, r = buf
+    w.fill_(1)
+    r.sum(dtype=torch.int32)
+
+
+def flush_buffers(device="cuda"):
+    return (torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device),
+            torch.zeros(L2_FLUSH_BYTES, dtype=torch.uint8, device=device))
 
 
 # ----------------------------------------------------------------------------
@@ -417,7 +429,8 @@ def workload_config(wl, extra=None):
     c = {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "seq_len": wl.N,
          "block": wl.block, "top_k": wl.top_k, "flags": wl.flags, "mode": "hier" if wl.hier else "gated",
          "global_batch": wl.B, "parallelism": "replicas (independent sequences per rank)",
-         "l2": "flushed before every timed step (256 MiB write)"}
+         "l2": "flushed before every timed step (256 MiB written, then 256 MiB read: no input and no dirty "
+               "line in L2)"}
     if extra:
         c.update(extra)
     return c
@@ -465,7 +478,7 @@ def _wl(name, args):
 
 def secondary_prefill(name, args, pk, psrc):
     wl, p, t = prefill_case(_wl(name, args), "cuda")
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = flush_buffers()
     ranks1 = Ranks.single()
     steps = max(2, min(args.steps, 5))
     el, kms, launches, clocks = run_timed(lambda tm: prefill_step(p, t, tm), steps, max(3, args.warmup),
@@ -508,28 +521,35 @@ def secondary_backward(name, args, pk, psrc):
         tmr("select_backward", lambda: sa.select_backward(p, t["Q"], t["L"], t["sel"][0], grads[3], t["sel"][2],
                                                           grads[0], grads[1], t["ws"]))
 
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = flush_buffers()
     steps = 2
     el, kms, launches, clocks = run_timed(step, steps, 3, Ranks.single(), flush)
-    # 10 d FLOP per kept (row, key) pair: z, dO.V, dQ, dK, dV; the forward's count is 4 d per pair
+    # 10 d FLOP per kept (row, key) pair: z, dO.V, dQ, dK, dV (the tensor-core path recomputes
+    # z and dO.V once more for dQ; that extra work is not counted); the forward's count is 4 d
     flops = prefill_flops(wl, t["sel"][2]) * 10 / 4
     ach = flops / (kms["prefill_backward"] / 1e3) / 1e12
+    G = wl.Hq // wl.Hkv
+    tensor = (wl.dtype == "bf16" and wl.d == 128 and wl.block in (64, 128) and (G * wl.block) % 128 == 0
+              and not wl.hier and not wl.per_qhead)
+    if tensor:
+        roof = {"bound": "tensor", "peak": pk["bf16_tflops"], "peak_source": psrc + " bf16 burst"}
+    else:
+        roof = {"bound": "alu", "peak": FP32_ALU_TFLOPS,
+                "peak_source": "derived: 148 SMs x 128 fp32 FMA x 2 x 1.965 GHz"}
+    roof.update({"achieved": ach, "unit": "TFLOP/s", "frac": ach / roof["peak"], "kernel": "prefill_backward",
+                 "algorithmic_flops_per_launch": flops, "traffic": None})
     out = {"metric": "prefill backward tokens/s", "value": wl.N * wl.B / (el / steps / 1e3), "unit": "tokens/s",
            "ms_per_step": el / steps, "kernels_ms": kms, "config": workload_config(wl), "gpu_launches": launches,
-           "roofline": {"bound": "alu", "achieved": ach, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                        "frac": ach / FP32_ALU_TFLOPS, "kernel": "prefill_backward",
-                        "peak_source": "derived: 148 SMs x 128 fp32 FMA x 2 x 1.965 GHz",
-                        "algorithmic_flops_per_launch": flops, "traffic": None},
-           "clocks": clocks}
+           "roofline": roof, "clocks": clocks}
     del t, grads, dO
     torch.cuda.empty_cache()
     return out
 
 
-# flat clustered index (Latent Sparse Attention style): 8 kv-heads of one
-# 32K sequence, 4-key items, 64-item segments of 16 clusters, 64 clusters
-# expanded per query, 64 sink and 1024 window positions
-LSA_DECODE_32K = dict(B=1, Hq=32, Hkv=8, d=128, N=32768, pool=4, seg=64, clusters=16, top_clusters=64, sink=64,
+# flat clustered index (Latent Sparse Attention style): 8 sequences of 32K
+# keys, 8 kv-heads and 32 query heads, 4-key items, 64-item segments of 16
+# clusters, 64 clusters expanded per query, 64 sink and 1024 window positions
+LSA_DECODE_32K = dict(B=8, Hq=32, Hkv=8, d=128, N=32768, pool=4, seg=64, clusters=16, top_clusters=64, sink=64,
                       window=1024)
 
 
@@ -556,7 +576,7 @@ def secondary_lsa(name, args, pk, psrc):
     def step(tm):
         (tm or (lambda n, f: f()))("lsa_decode", lambda: sa.lsa_decode(p, q, K, V, index, ws, out=out, kept=kept))
 
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = flush_buffers()
     steps = 10
     el, kms, launches, clocks = run_timed(step, steps, 3, Ranks.single(), flush)
     C = sa.sparse_attn_lsa_clusters(p)
@@ -604,7 +624,7 @@ def secondary_lsa_tree(name, args, pk, psrc):
         (tm or (lambda n, f: f()))("lsa_tree_decode", lambda: sa.lsa_tree_decode(
             p, LSA_TREE["fanout"], LSA_TREE["beam"], q, K, V, index, tree, ws, out=out, kept=kept, compared=comp))
 
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = flush_buffers()
     steps = 10
     el, kms, launches, clocks = run_timed(step, steps, 3, Ranks.single(), flush)
     nkept, ncomp = int(kept.sum().item()), int(comp.sum().item())
@@ -631,7 +651,7 @@ def secondary_decode(name, args, pk, psrc):
         # ragged batch: lengths uniform in [N/2, N], seeded
         lens = np.random.default_rng(11).integers(wl.N // 2, wl.N + 1, size=wl.B)
     p, t = decode_case(wl, "cuda", lens)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = flush_buffers()
     ranks1 = Ranks.single()
     steps = max(3, args.steps)
     el, kms, launches, clocks = run_timed(lambda tm: decode_step(p, t, tm), steps, max(3, args.warmup),
@@ -733,7 +753,7 @@ def run_ours(args, ranks):
         return 0
     base = inputs.WORKLOADS[args.workload]
     wl, p, t = prefill_case(base, "cuda", seed_offset=ranks.rank)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = flush_buffers()
     el, kms, launches, clocks = run_timed(lambda tm: prefill_step(p, t, tm), args.steps, args.warmup, ranks, flush)
     value, el_max = aggregate(ranks, el, wl.N * wl.B * args.steps)
     flops = prefill_flops(wl, t["sel"][2])

@@ -15,6 +15,27 @@ using namespace sa;
 static std::atomic<unsigned long long> g_launches{0};
 void sa::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+sa::WsLayout sa::ws_layout(const Shape &s) {
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t units = (size_t)s.B * s.Hsel;
+    const size_t ktiles = (size_t)s.B * s.Hkv * ((s.nb * s.bs + 127) / 128);
+    WsLayout L;
+    size_t o = kStatusBytes;
+    L.sel_chunk = o;  o += al(units * s.nb * 4);
+    L.sel_decode = o; o += al(units * 4);
+    L.decode = o;     o += al(units * 4);
+    L.bwd_kv = o;     o += al(ktiles * 8 * 4);
+    L.scratch = o;
+    return L;
+}
+
+int sa::sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
 namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -97,6 +118,30 @@ int launch_result(cudaError_t e) {
 
 }  // namespace
 
+// Decode on a fixed scratch buffer (the no-allocation entry point): the
+// status word, this call's per-unit split counters and its partials, packed
+// from the buffer's start.  The buffer is shared by calls of any shape, so
+// the status word and the counters are cleared on the stream first.
+int sa::decode_on_scratch(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
+                          const float *score, const int32_t *count, void *o, float *lse, void *scratch,
+                          size_t scratch_bytes, size_t *need, cudaStream_t st) {
+    Shape s;
+    const int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t counters = al((size_t)s.B * s.Hsel * sizeof(unsigned));
+    const size_t total = kStatusBytes + counters + al(decode_workspace(s));
+    if (need) *need = total;
+    if (total > scratch_bytes) return SA_ERR_WORKSPACE;
+    if (!q || !K || !V || !idx || !score || !count || !o || !lse || !scratch) return SA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(o) || !aligned16(scratch)) return SA_ERR_ARG;
+    unsigned char *w = static_cast<unsigned char *>(scratch);
+    if (cudaMemsetAsync(w, 0, kStatusBytes + counters, st) != cudaSuccess) return SA_ERR_LAUNCH;
+    return launch_result(launch_decode(s, q, K, V, idx, score, count, o, lse, reinterpret_cast<unsigned *>(w),
+                                       reinterpret_cast<float *>(w + kStatusBytes + counters),
+                                       reinterpret_cast<unsigned *>(w + kStatusBytes), st));
+}
+
 extern "C" {
 
 size_t sparse_attn_workspace_size(const sa_params *p, int op) {
@@ -111,7 +156,7 @@ size_t sparse_attn_workspace_size(const sa_params *p, int op) {
         case SA_OP_SELECT_BACKWARD: extra = select_backward_workspace(s); break;
         default: break;
     }
-    return kStatusBytes + ((extra + 255) & ~(size_t)255);
+    return ws_layout(s).scratch + ((extra + 255) & ~(size_t)255);
 }
 
 int sparse_attn_landmarks(const sa_params *p, const void *K, void *L, void *stream) {
@@ -198,7 +243,11 @@ static int decode_common(const sa_params *p, const void *q, const void *K, const
     if (!q || !K || !V || !idx || !score || !count || !o || !lse || !ws) return SA_ERR_ARG;
     if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(o) || !aligned16(ws)) return SA_ERR_ARG;
     if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_DECODE)) return SA_ERR_WORKSPACE;
-    return launch_result(launch_decode(s, q, K, V, idx, score, count, o, lse, ws, ws_bytes, (cudaStream_t)stream));
+    const WsLayout L = ws_layout(s);
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    return launch_result(launch_decode(s, q, K, V, idx, score, count, o, lse, reinterpret_cast<unsigned *>(w),
+                                       reinterpret_cast<float *>(w + L.scratch), reinterpret_cast<unsigned *>(w + L.decode),
+                                       (cudaStream_t)stream));
 }
 
 int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,

@@ -23,6 +23,9 @@
 // Kernel D: dK += dL_b / n_b for every key.
 #include <math_constants.h>
 
+#include <algorithm>
+
+#include "backward_tc.cuh"
 #include "common.cuh"
 
 namespace sa {
@@ -367,14 +370,20 @@ bool backward_supported(const Shape &s) {
 
 size_t select_backward_workspace(const Shape &s) { return (size_t)s.B * s.Hkv * s.nb * s.d * sizeof(float); }
 
-size_t prefill_backward_workspace(const Shape &s) { return (size_t)s.B * s.Hkv * s.nb * s.cap * sizeof(float); }
+size_t prefill_backward_workspace(const Shape &s) {
+    const size_t simt = (size_t)s.B * s.Hkv * s.nb * s.cap * sizeof(float);
+    // room for either path (SPARSE_ATTN_BACKWARD_PATH=simt selects the CUDA-core one)
+    return backward_tc_shape_ok(s) ? std::max(simt, backward_tc_workspace(s)) : simt;
+}
 
 cudaError_t launch_prefill_backward(const Shape &s, const void *Q, const void *K, const void *V, const void *O,
                                     const float *lse, const void *dO, const int32_t *idx, const float *score,
                                     const int32_t *count, float *dQ, float *dK, float *dV, float *dscore,
                                     void *ws, cudaStream_t st) {
+    if (backward_tc_supported(s))
+        return launch_backward_tc(s, Q, K, V, O, lse, dO, idx, score, count, dQ, dK, dV, dscore, ws, st);
     const size_t kv_bytes = (size_t)s.B * s.Hkv * s.N * s.d * sizeof(float);
-    float *dgate = reinterpret_cast<float *>(static_cast<unsigned char *>(ws) + kStatusBytes);
+    float *dgate = reinterpret_cast<float *>(static_cast<unsigned char *>(ws) + ws_layout(s).scratch);
     const size_t units = (size_t)s.B * s.Hkv * s.nb;
     cudaError_t e;
     if ((e = cudaMemsetAsync(dK, 0, kv_bytes, st)) != cudaSuccess) return e;
@@ -399,7 +408,7 @@ cudaError_t launch_prefill_backward(const Shape &s, const void *Q, const void *K
 cudaError_t launch_select_backward(const Shape &s, const void *Q, const void *L, const int32_t *idx,
                                    const float *dscore, const int32_t *count, float *dQ, float *dK, void *ws,
                                    cudaStream_t st) {
-    float *dL = reinterpret_cast<float *>(static_cast<unsigned char *>(ws) + kStatusBytes);
+    float *dL = reinterpret_cast<float *>(static_cast<unsigned char *>(ws) + ws_layout(s).scratch);
     const size_t units = (size_t)s.B * s.Hkv * s.nb;
     cudaError_t e = cudaMemsetAsync(dL, 0, select_backward_workspace(s), st);
     if (e != cudaSuccess) return e;

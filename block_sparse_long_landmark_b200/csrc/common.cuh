@@ -127,8 +127,30 @@ __device__ __forceinline__ int block_scan_incl(int v, int *tmp, int *total) {
     return v + add;
 }
 
+// Workspace layout shared by every operation of a parameter set: the status
+// word, then one completion-counter array per operation that keeps counters
+// (each returned to zero by the call that uses it, and written by no other
+// operation), then the scratch area that each operation reuses freely.
+struct WsLayout {
+    size_t sel_chunk;    // select.cu: [B * Hsel * nb] chunk CTAs finished per unit
+    size_t sel_decode;   // select_decode.cu: [B * Hsel] CTAs finished per unit
+    size_t decode;       // decode_mma.cu: [B * Hsel] splits finished per unit
+    size_t bwd_kv;       // backward_kv.cu: [B * Hkv * key tiles * 8] splits finished per tile region
+    size_t scratch;      // first byte of the scratch area
+};
+WsLayout ws_layout(const Shape &s);
+
+// Decode with every scratch byte inside `scratch` (see decode_static.cu);
+// *need receives the bytes this shape takes.
+int decode_on_scratch(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
+                      const float *score, const int32_t *count, void *o, float *lse, void *scratch,
+                      size_t scratch_bytes, size_t *need, cudaStream_t st);
+
 // Process-wide count of kernels this library has launched (for reporting).
 void note_launch();
+
+// Streaming multiprocessors of the current device (0 on failure).
+int sm_count();
 
 // ---------------------------------------------------------------------------
 // Internal launchers (return cudaError_t of the launch)
@@ -161,12 +183,14 @@ cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, con
 bool decode_mma_supported(const Shape &s);
 void decode_mma_geometry(const Shape &s, int &S, int &bps);
 size_t decode_mma_partial_bytes(const Shape &s, int S);
+// Decode scratch passed explicitly: the status word, the split partials and
+// the per-unit completion counters (zero before the call, zero after it).
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
-                              const float *score, const int32_t *count, void *o, float *lse, void *ws,
-                              cudaStream_t st, int &S_out);
+                              const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
+                              float *part, unsigned *done, cudaStream_t st, int &S_out);
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
-                          const float *score, const int32_t *count, void *o, float *lse, void *ws,
-                          size_t ws_bytes, cudaStream_t st);
+                          const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
+                          float *part, unsigned *done, cudaStream_t st);
 size_t decode_workspace(const Shape &s);
 bool backward_supported(const Shape &s);
 size_t prefill_backward_workspace(const Shape &s);

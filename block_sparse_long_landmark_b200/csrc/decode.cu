@@ -269,8 +269,8 @@ size_t decode_workspace(const Shape &s) {
     if (decode_mma_supported(s)) {
         decode_mma_geometry(s, S, bps);
         if (S == 1) return 0;
-        // split partials, then one completion counter per unit
-        return decode_mma_partial_bytes(s, S) + (size_t)s.B * s.Hsel * sizeof(unsigned);
+        // split partials (the per-unit completion counters sit in the counter area)
+        return decode_mma_partial_bytes(s, S);
     }
     split_geometry(s, S, bps);
     if (S == 1) return 0;
@@ -297,9 +297,13 @@ static cudaError_t run(DecArgs a, cudaStream_t st) {
 }
 
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
-                          const float *score, const int32_t *count, void *o, float *lse, void *ws,
-                          size_t ws_bytes, cudaStream_t st) {
-    (void)ws_bytes;
+                          const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
+                          float *part, unsigned *done, cudaStream_t st) {
+    if (decode_mma_supported(s)) {
+        // one launch: the unit's last split merges the partials itself
+        int S = 1;
+        return launch_decode_mma(s, q, K, V, idx, score, count, o, lse, status, part, done, st, S);
+    }
     DecArgs a{};
     a.s = s;
     a.q = q;
@@ -310,13 +314,8 @@ cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const vo
     a.count = count;
     a.o = o;
     a.lse = lse;
-    a.status = (unsigned *)ws;
-    a.part = (float *)((char *)ws + kStatusBytes);
-    if (decode_mma_supported(s)) {
-        // one launch: the unit's last split merges the partials itself
-        int S = 1;
-        return launch_decode_mma(s, q, K, V, idx, score, count, o, lse, ws, st, S);
-    }
+    a.status = status;
+    a.part = part;
     split_geometry(s, a.S, a.bps);
     return s.dtype == SA_BF16 ? run<__nv_bfloat16>(a, st) : run<float>(a, st);
 }

@@ -457,8 +457,8 @@ void decode_mma_geometry(const Shape &s, int &S, int &bps) {
 }
 
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
-                              const float *score, const int32_t *count, void *o, float *lse, void *ws,
-                              cudaStream_t st, int &S_out) {
+                              const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
+                              float *part, unsigned *done, cudaStream_t st, int &S_out) {
     std::call_once(g_enc_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult qr;
@@ -488,10 +488,10 @@ cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, cons
     a.count = count;
     a.o = (__nv_bfloat16 *)o;
     a.lse = lse;
-    a.status = (unsigned *)ws;
-    a.part = (float *)((char *)ws + kStatusBytes);
+    a.status = status;
+    a.part = part;
     decode_mma_geometry(s, a.S, a.bps);
-    a.done = (unsigned *)((char *)a.part + decode_mma_partial_bytes(s, a.S));
+    a.done = done;
     S_out = a.S;
     cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemD);
     if (e != cudaSuccess) return e;

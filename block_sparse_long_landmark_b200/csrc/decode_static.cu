@@ -17,11 +17,12 @@
 //   * every call on a device shares the one array, so calls that overlap on
 //     the GPU (different streams, or other host threads) race on it; order
 //     them on one stream or serialise them;
-//   * each call clears the status word at the array's start (cudaMemsetAsync
-//     on the call's stream); the split partials need no clearing because
-//     every split writes its own slot before the merge reads it, and the
-//     per-unit completion counters behind them start at zero (the array is
-//     zero when the library loads) and are back at zero when a call ends;
+//   * each call lays out, from the array's start, the status word, one
+//     completion counter per (sequence, kv-head) and the split partials, and
+//     clears the status word and the counters (cudaMemsetAsync on the call's
+//     stream: calls of other shapes may have left partials there); the
+//     partials need no clearing because every split writes its own slot
+//     before the merge reads it;
 //   * problems whose split partials do not fit return SA_ERR_WORKSPACE before
 //     anything is launched;
 //   * nothing here calls cudaMalloc, cudaFree or an allocating library.
@@ -62,13 +63,14 @@ void *scratch_address() {
 extern "C" int sparse_attn_decode_static(const sa_params *p, const void *q, const void *K, const void *V,
                                          const int32_t *idx, const float *score, const int32_t *count, void *o,
                                          float *lse, void *stream) {
-    const size_t need = sparse_attn_workspace_size(p, SA_OP_DECODE);
-    if (need == 0) return SA_ERR_ARG;                 // invalid parameters
+    // size and argument checks first: too large a problem returns before any set-up or launch
+    size_t need = 0;
+    const int r = sa::decode_on_scratch(p, q, K, V, idx, score, count, o, lse, nullptr, 0, &need, nullptr);
+    if (r != SA_ERR_WORKSPACE) return r;              // invalid parameters
     if (need > kStaticScratchBytes) return SA_ERR_WORKSPACE;
     if (!q || !K || !V || !idx || !score || !count || !o || !lse) return SA_ERR_ARG;
     void *ws = scratch_address();
     if (!ws) return SA_ERR_LAUNCH;
-    cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(ws, 0, sa::kStatusBytes, st) != cudaSuccess) return SA_ERR_LAUNCH;
-    return sparse_attn_decode(p, q, K, V, idx, score, count, o, lse, ws, kStaticScratchBytes, stream);
+    return sa::decode_on_scratch(p, q, K, V, idx, score, count, o, lse, ws, kStaticScratchBytes, nullptr,
+                                 (cudaStream_t)stream);
 }

@@ -691,12 +691,6 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 }
 
 
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    return n;
-}
 
 }  // namespace
 

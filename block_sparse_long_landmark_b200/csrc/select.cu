@@ -443,7 +443,7 @@ size_t select_workspace(const Shape &s, bool decode) {
     geometry(s, decode, nunits, S, CH);
     if (S == 1) return 0;
     return (size_t)nunits * S * s.top_k * (sizeof(uint32_t) + sizeof(int32_t)) + (size_t)nunits * 2 * sizeof(float) +
-           (size_t)nunits * sizeof(unsigned) + 256;
+           256;
 }
 
 template <typename T>
@@ -463,14 +463,13 @@ static cudaError_t run(const Shape &s, bool decode, const void *Q, const void *L
     geometry(s, decode, nunits, a.S, a.CH);
     a.mode = a.S == 1 ? kFinal : kPartial;
     if (a.S > 1) {
-        char *p = (char *)ws + kStatusBytes;
+        char *p = (char *)ws + ws_layout(s).scratch;
         a.part_key = (uint32_t *)p;
         p += (size_t)nunits * a.S * s.top_k * sizeof(uint32_t);
         a.part_idx = (int32_t *)p;
         p += (size_t)nunits * a.S * s.top_k * sizeof(int32_t);
         a.special = (float *)p;
-        p += (size_t)nunits * 2 * sizeof(float);
-        a.done = (unsigned *)p;
+        a.done = (unsigned *)((char *)ws + ws_layout(s).sel_chunk);
     }
     const int vpr = s.d * (int)sizeof(T) / 16;
     const int d = s.d;

@@ -290,7 +290,7 @@ size_t select_decode_workspace(const Shape &s) {
     sd_geometry(s, C);
     if (C == 1) return 0;
     const size_t units = (size_t)s.B * s.Hsel;
-    return units * C * s.top_k * 8 + units * C * 4 + units * 2 * 4 + units * 4 + 4 * 256;
+    return units * C * s.top_k * 8 + units * C * 4 + units * 2 * 4 + 4 * 256;
 }
 
 static size_t sd_smem(const Shape &s, int C) {
@@ -312,7 +312,7 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
     sd_geometry(s, a.C);
     const size_t units = (size_t)s.B * s.Hsel;
     if (a.C > 1) {
-        char *p = (char *)ws + kStatusBytes;
+        char *p = (char *)ws + ws_layout(s).scratch;
         auto take = [&](size_t bytes) {
             char *r = p;
             p += (bytes + 255) & ~(size_t)255;
@@ -322,7 +322,7 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
         a.pidx = (int32_t *)take(units * a.C * s.top_k * 4);
         a.pcnt = (int32_t *)take(units * a.C * 4);
         a.special = (float *)take(units * 2 * 4);
-        a.done = (unsigned *)take(units * 4);
+        a.done = (unsigned *)((char *)ws + ws_layout(s).sel_decode);
     }
     const int vpr = s.d * (int)sizeof(T) / 16;
     void (*kern)(SdArgs) = nullptr;
