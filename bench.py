@@ -728,12 +728,40 @@ SECONDARY = ("long_prefill_256k", "gated_prefill_32k", "hils_prefill_32k", "gate
              "hils_decode_1m", "gated_decode_128k")
 
 
+def secondary_select_only(name, args, pk, psrc):
+    """Decode selection alone (profiling): the workload's query and random
+    landmarks of its context, no KV cache -- the selection reads only these."""
+    import block_sparse_long_landmark_b200 as sa
+    wl = _wl(name[:-len("_select")], args)
+    p = sa.params_for(wl)
+    g = torch.Generator(device="cuda").manual_seed(wl.seed)
+    q = (torch.randn(wl.B, wl.Hq, wl.d, generator=g, device="cuda") * wl.sigma).to(wl.torch_dtype)
+    L = (torch.randn(wl.B, wl.Hkv, wl.nb, wl.d, generator=g, device="cuda") * wl.sigma).to(wl.torch_dtype)
+    ws = sa.workspace(p)
+    sel = sa._sel_out(p, True, "cuda")
+    flush = flush_buffers()
+    steps = max(3, args.steps)
+    el, kms, launches, clocks = run_timed(
+        lambda tm: (tm or (lambda n, f: f()))("select_decode", lambda: sa.select_decode(p, q, L, ws, out=sel)),
+        steps, max(3, args.warmup), Ranks.single(), flush)
+    nbytes = wl.B * wl.Hkv * ((wl.N - 1) // wl.block + 1) * wl.d * L.element_size()
+    ach = nbytes / (kms["select_decode"] / 1e3) / 1e9
+    return {"metric": "decode selection queries/s", "value": wl.B / (el / steps / 1e3), "unit": "queries/s",
+            "ms_per_step": el / steps, "kernels_ms": kms, "config": workload_config(wl), "gpu_launches": launches,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"], "algorithmic_bytes": nbytes, "traffic": None,
+                         "peak_source": psrc + " HBM copy"},
+            "clocks": clocks}
+
+
 def run_secondary(name, args, pk, psrc):
     from block_sparse_long_landmark_b200 import inputs
     if name == "lsa_decode_32k":
         return secondary_lsa(name, args, pk, psrc)
     if name == "lsa_tree_decode_32k":
         return secondary_lsa_tree(name, args, pk, psrc)
+    if name.endswith("_select"):
+        return secondary_select_only(name, args, pk, psrc)
     if name.endswith("_backward"):
         return secondary_backward(name, args, pk, psrc)
     kind = inputs.WORKLOADS[name.replace("_varlen", "")].kind

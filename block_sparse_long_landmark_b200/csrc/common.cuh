@@ -134,7 +134,6 @@ __device__ __forceinline__ int block_scan_incl(int v, int *tmp, int *total) {
 struct WsLayout {
     size_t sel_chunk;    // select.cu: [B * Hsel * nb] chunk CTAs finished per unit
     size_t sel_decode;   // select_decode.cu: [B * Hsel] CTAs finished per unit
-    size_t decode;       // decode_mma.cu: [B * Hsel] splits finished per unit
     size_t bwd_kv;       // backward_kv.cu: [B * Hkv * key tiles * 8] splits finished per tile region
     size_t scratch;      // first byte of the scratch area
 };
@@ -183,14 +182,13 @@ cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, con
 bool decode_mma_supported(const Shape &s);
 void decode_mma_geometry(const Shape &s, int &S, int &bps);
 size_t decode_mma_partial_bytes(const Shape &s, int S);
-// Decode scratch passed explicitly: the status word, the split partials and
-// the per-unit completion counters (zero before the call, zero after it).
+// Decode scratch passed explicitly: the status word and the split partials.
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                               const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                              float *part, unsigned *done, cudaStream_t st, int &S_out);
+                              float *part, cudaStream_t st, int &S_out);
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                          float *part, unsigned *done, cudaStream_t st);
+                          float *part, cudaStream_t st);
 size_t decode_workspace(const Shape &s);
 bool backward_supported(const Shape &s);
 size_t prefill_backward_workspace(const Shape &s);

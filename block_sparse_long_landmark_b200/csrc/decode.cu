@@ -269,7 +269,6 @@ size_t decode_workspace(const Shape &s) {
     if (decode_mma_supported(s)) {
         decode_mma_geometry(s, S, bps);
         if (S == 1) return 0;
-        // split partials (the per-unit completion counters sit in the counter area)
         return decode_mma_partial_bytes(s, S);
     }
     split_geometry(s, S, bps);
@@ -298,12 +297,7 @@ static cudaError_t run(DecArgs a, cudaStream_t st) {
 
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                          float *part, unsigned *done, cudaStream_t st) {
-    if (decode_mma_supported(s)) {
-        // one launch: the unit's last split merges the partials itself
-        int S = 1;
-        return launch_decode_mma(s, q, K, V, idx, score, count, o, lse, status, part, done, st, S);
-    }
+                          float *part, cudaStream_t st) {
     DecArgs a{};
     a.s = s;
     a.q = q;
@@ -316,6 +310,16 @@ cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const vo
     a.lse = lse;
     a.status = status;
     a.part = part;
+    if (decode_mma_supported(s)) {
+        // tensor-core splits, then (when split) one merge CTA per unit
+        int S = 1;
+        cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, o, lse, status, part, st, S);
+        if (e != cudaSuccess || S == 1) return e;
+        a.S = S;
+        decode_merge_kernel<__nv_bfloat16><<<(unsigned)(s.B * s.Hsel), kDecThreads, 0, st>>>(a);
+        note_launch();
+        return cudaGetLastError();
+    }
     split_geometry(s, a.S, a.bps);
     return s.dtype == SA_BF16 ? run<__nv_bfloat16>(a, st) : run<float>(a, st);
 }

@@ -57,7 +57,6 @@ struct DmArgs {
     float *lse;
     unsigned *status;
     float *part;
-    unsigned *done;   // [units] splits finished; the last split merges and puts it back to 0
     int S, bps;
 };
 
@@ -400,36 +399,6 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             }
         }
     }
-    if (a.S == 1) return;
-    // the unit's last split to finish merges the splits' (max, sum, acc) in
-    // split order (partials written and fenced before the count)
-    __shared__ int last_split;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_split = atomicAdd(a.done + u, 1u) == (unsigned)(a.S - 1);
-    __syncthreads();
-    if (!last_split) return;
-    __threadfence();
-    const float *pu = a.part + (size_t)u * a.S * HP * 130;
-    for (int e = tid; e < HP * 128; e += kThreadsD) {
-        const int hh = e >> 7, dim = e & 127;
-        float M = -CUDART_INF_F;
-        for (int sp = 0; sp < a.S; ++sp) M = fmaxf(M, __ldcg(pu + (sp * HP + hh) * 130));
-        float L = 0.f, O = 0.f;
-        if (M != -CUDART_INF_F) {
-            for (int sp = 0; sp < a.S; ++sp) {
-                const float *pp = pu + (sp * HP + hh) * 130;
-                const float mp = __ldcg(pp);
-                if (mp == -CUDART_INF_F) continue;
-                const float w = ex2f(mp - M);
-                L = fmaf(__ldcg(pp + 1), w, L);
-                O = fmaf(__ldcg(pp + 2 + dim), w, O);
-            }
-        }
-        a.o[((size_t)b * s.Hq + h0 + hh) * 128 + dim] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
-        if (dim == 0) a.lse[(size_t)b * s.Hq + h0 + hh] = L > 0.f ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
-    }
-    if (tid == 0) a.done[u] = 0u;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 g_enc = nullptr;
@@ -458,7 +427,7 @@ void decode_mma_geometry(const Shape &s, int &S, int &bps) {
 
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                               const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                              float *part, unsigned *done, cudaStream_t st, int &S_out) {
+                              float *part, cudaStream_t st, int &S_out) {
     std::call_once(g_enc_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult qr;
@@ -491,7 +460,6 @@ cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, cons
     a.status = status;
     a.part = part;
     decode_mma_geometry(s, a.S, a.bps);
-    a.done = done;
     S_out = a.S;
     cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemD);
     if (e != cudaSuccess) return e;

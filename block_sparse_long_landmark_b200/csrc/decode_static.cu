@@ -17,12 +17,10 @@
 //   * every call on a device shares the one array, so calls that overlap on
 //     the GPU (different streams, or other host threads) race on it; order
 //     them on one stream or serialise them;
-//   * each call lays out, from the array's start, the status word, one
-//     completion counter per (sequence, kv-head) and the split partials, and
-//     clears the status word and the counters (cudaMemsetAsync on the call's
-//     stream: calls of other shapes may have left partials there); the
-//     partials need no clearing because every split writes its own slot
-//     before the merge reads it;
+//   * each call lays out, from the array's start, the status word and the
+//     split partials, and clears the status word (cudaMemsetAsync on the
+//     call's stream); the partials need no clearing because every split
+//     writes its own slot before the merge reads it;
 //   * problems whose split partials do not fit return SA_ERR_WORKSPACE before
 //     anything is launched;
 //   * nothing here calls cudaMalloc, cudaFree or an allocating library.

@@ -196,7 +196,13 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     }
     if (nan_seen) set_status(a.status, kStatusNaN);
     __syncthreads();
-    const int nsel = block_topk64(keys, n, pl.kk, pos, red, red64);
+    // the chunk's top-kk by one warp, shared through `flag`
+    if (warp == 0) {
+        const int c = warp_topk64(keys, n, pl.kk, pos);
+        if (lane == 0) flag[1] = c;
+    }
+    __syncthreads();
+    const int nsel = flag[1];
     if (pl.S > 1) {
         // the chunk's candidates (ascending id) for the merge
         uint64_t *pk = a.pkey + ((size_t)bg * pl.S + chunk) * pl.kk;
@@ -226,7 +232,12 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
             }
         }
         __syncthreads();
-        const int nfin = block_topk64(keys, ntot, pl.ntop, pos, red, red64);
+        if (warp == 0) {
+            const int c = warp_topk64(keys, ntot, pl.ntop, pos);
+            if (lane == 0) flag[2] = c;
+        }
+        __syncthreads();
+        const int nfin = flag[2];
         for (int i = tid; i < nfin; i += kLsaThreads) chosen[i] = ids[pos[i]];
         if (tid == 0) a.done1[bg] = 0u;
         __syncthreads();
@@ -238,12 +249,13 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     }
 }
 
-// Kernel 3 (flat decode, step 2): one CTA per (batch, kv-head, slice of the
-// kept positions).  The slice's positions are laid out in shared memory from
-// the ranges; then a VPR-lane group per key row streams K and V with 16-byte
-// loads and keeps an online softmax (fp32, exp2 domain) per query head of
-// the pass.  Lane groups, warps and finally the CTAs of a (batch, kv-head)
-// are merged by log-sum-exp; the last CTA writes o and lse.
+// Kernel 3 (flat decode, step 2): P CTAs per (batch, kv-head), each taking
+// an equal share of the kept positions and walking it in rounds: a round's
+// positions are laid out in shared memory from the ranges, then a VPR-lane
+// group per key row streams K and V with 16-byte loads and keeps an online
+// softmax (fp32, exp2 domain) per query head of the pass.  Lane groups,
+// warps and finally the CTAs of a (batch, kv-head) are merged by
+// log-sum-exp; the last CTA writes o and lse.
 template <typename T, int HG>
 __global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
     constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
@@ -261,38 +273,9 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
     int *misc = reinterpret_cast<int *>(wst + (kLsaThreads / 32) * HG * (D + 2));   // [4]
 
     const int nr = a.cnt[2 * (size_t)bg], tot = a.cnt[2 * (size_t)bg + 1];
-    const int t0 = (int)((long long)tot * pi / pl.P);
-    int t1 = (int)((long long)tot * (pi + 1) / pl.P);
-    if (t1 - t0 > pl.slice) {      // more positions than a valid index can keep (repeated items): cut, report
-        if (tid == 0) set_status(a.status, kStatusBadIndex);
-        t1 = t0 + pl.slice;
-    }
+    // this CTA's share of the kept positions, walked in rounds of pl.slice
+    const int t0 = (int)((long long)tot * pi / pl.P), t1 = (int)((long long)tot * (pi + 1) / pl.P);
     const int32_t *rs = a.rs + (size_t)bg * pl.rmax, *rl = a.rl + (size_t)bg * pl.rmax, *rp = a.rp + (size_t)bg * pl.rmax;
-    if (tid == 0) {
-        // ranges [r0, r1) overlap [t0, t1): rp ascending, every length > 0
-        int lo = 0, hi = nr;                       // first r with rp[r] + rl[r] > t0
-        while (lo < hi) {
-            const int m = (lo + hi) >> 1;
-            if (rp[m] + rl[m] > t0) hi = m; else lo = m + 1;
-        }
-        misc[0] = lo;
-        lo = misc[0];
-        hi = nr;                                   // first r with rp[r] >= t1
-        while (lo < hi) {
-            const int m = (lo + hi) >> 1;
-            if (rp[m] >= t1) hi = m; else lo = m + 1;
-        }
-        misc[1] = lo;
-    }
-    __syncthreads();
-    const int r0 = misc[0], r1 = misc[1];
-    for (int r = r0 + warp; r < r1; r += kLsaThreads / 32) {
-        const int st = rs[r], pre = rp[r], len = rl[r];
-        const int from = max(t0, pre), to = min(t1, pre + len);
-        for (int v = from + lane; v < to; v += 32) posv[v - t0] = st + (v - pre);
-    }
-    __syncthreads();
-    const int np = t1 - t0;
     const T *Kb = (const T *)a.K + (size_t)bg * s.N * D;
     const T *Vb = (const T *)a.V + (size_t)bg * s.N * D;
     const float sl2 = s.scale * kLog2e;
@@ -311,38 +294,65 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
             m[h] = -CUDART_INF_F;
             l[h] = 0.f;
         }
-        // rows of this lane group: vb + sub + u * RPW * 8 for the warp's bases vb
-        // (the trip count is the same for every lane: the row reductions
-        // shuffle over the whole warp); two rows per group in flight
-        constexpr int U = 2, NW = kLsaThreads / 32;
-        for (int vb = warp * RPW; vb < np; vb += U * RPW * NW) {
-            uint4 kr[U], vr[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int v = min(vb + sub + u * RPW * NW, np - 1);
-                const size_t row = (size_t)posv[v] * D + cv * EPV;
-                kr[u] = *reinterpret_cast<const uint4 *>(Kb + row);
-                vr[u] = *reinterpret_cast<const uint4 *>(Vb + row);
+        for (int r0 = t0; r0 < t1; r0 += pl.slice) {
+            const int r1 = min(t1, r0 + pl.slice);
+            __syncthreads();                             // the previous round's positions are read
+            if (tid == 0) {
+                // ranges [q0, q1) overlap [r0, r1): rp ascending, every length > 0
+                int lo = 0, hi = nr;                     // first range with rp + rl > r0
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (rp[mid] + rl[mid] > r0) hi = mid; else lo = mid + 1;
+                }
+                misc[0] = lo;
+                hi = nr;                                 // first range with rp >= r1
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (rp[mid] >= r1) hi = mid; else lo = mid + 1;
+                }
+                misc[1] = lo;
             }
+            __syncthreads();
+            for (int r = misc[0] + warp; r < misc[1]; r += kLsaThreads / 32) {
+                const int st = rs[r], pre = rp[r], len = rl[r];
+                const int from = max(r0, pre), to = min(r1, pre + len);
+                for (int v = from + lane; v < to; v += 32) posv[v - r0] = st + (v - pre);
+            }
+            __syncthreads();
+            const int np = r1 - r0;
+            // rows of this lane group: vb + sub + u * RPW * 8 for the warp's bases vb
+            // (the trip count is the same for every lane: the row reductions
+            // shuffle over the whole warp); two rows per group in flight
+            constexpr int U = 2, NW = kLsaThreads / 32;
+            for (int vb = warp * RPW; vb < np; vb += U * RPW * NW) {
+                uint4 kr[U], vr[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const bool live = vb + sub + u * RPW * NW < np;   // uniform over the lane group
-                float kf[EPV], vf[EPV];
-                load16(reinterpret_cast<const T *>(&kr[u]), kf);
-                load16(reinterpret_cast<const T *>(&vr[u]), vf);
+                for (int u = 0; u < U; ++u) {
+                    const int v = min(vb + sub + u * RPW * NW, np - 1);
+                    const size_t row = (size_t)posv[v] * D + cv * EPV;
+                    kr[u] = *reinterpret_cast<const uint4 *>(Kb + row);
+                    vr[u] = *reinterpret_cast<const uint4 *>(Vb + row);
+                }
 #pragma unroll
-                for (int h = 0; h < HG; ++h) {
-                    float z = 0.f;
+                for (int u = 0; u < U; ++u) {
+                    const bool live = vb + sub + u * RPW * NW < np;   // uniform over the lane group
+                    float kf[EPV], vf[EPV];
+                    load16(reinterpret_cast<const T *>(&kr[u]), kf);
+                    load16(reinterpret_cast<const T *>(&vr[u]), vf);
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e) z = fmaf(qf[h][e], kf[e], z);
-                    for (int o = VPR / 2; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-                    if (!live || h >= nh) continue;
-                    const float mn = fmaxf(m[h], z);
-                    const float corr = exp2f(m[h] - mn), p = exp2f(z - mn);
-                    l[h] = l[h] * corr + p;
+                    for (int h = 0; h < HG; ++h) {
+                        float z = 0.f;
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e) acc[h][e] = fmaf(acc[h][e], corr, p * vf[e]);
-                    m[h] = mn;
+                        for (int e = 0; e < EPV; ++e) z = fmaf(qf[h][e], kf[e], z);
+                        for (int o = VPR / 2; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                        if (!live || h >= nh) continue;
+                        const float mn = fmaxf(m[h], z);
+                        const float corr = exp2f(m[h] - mn), p = exp2f(z - mn);
+                        l[h] = l[h] * corr + p;
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) acc[h][e] = fmaf(acc[h][e], corr, p * vf[e]);
+                        m[h] = mn;
+                    }
                 }
             }
         }
@@ -463,11 +473,12 @@ bool lsa_decode_plan(const LsaShape &s, LsaDecPlan &pl, bool chunks) {
     const long long sink_n = min(s.sink, s.N);
     const long long bound = min((long long)s.N, sink_n + (long long)s.window + (long long)pl.ntop * s.seg * s.pool);
     const int bgs = s.B * s.Hkv;
-    // about two CTAs per SM overall, at least 64 positions and at most 2048 per CTA
-    long long P = (bound + 2047) / 2048;
-    P = max(P, min((296LL + bgs - 1) / bgs, (bound + 63) / 64));
-    pl.P = (int)max(1LL, min(P, 4096LL));
-    pl.slice = (int)max(1LL, (bound + pl.P - 1) / pl.P);
+    // about two CTAs per SM overall, but at least 64 positions per CTA at the bound;
+    // each CTA walks its share in rounds of `slice` positions laid out in shared memory
+    long long P = min(64LL, (296LL + bgs - 1) / bgs);
+    P = min(P, (bound + 63) / 64);
+    pl.P = (int)max(1LL, P);
+    pl.slice = 1024;
     pl.HG = s.G >= 8 ? 8 : s.G >= 4 ? 4 : s.G >= 2 ? 2 : 1;
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
     size_t off = kStatusBytes;

@@ -23,7 +23,7 @@ struct LsaDecPlan {
     int ntop;        // clusters chosen: min(top_clusters, ctotal)
     int rmax;        // key ranges per (batch, kv-head): sink + window + ntop * seg items
     int P;           // attention CTAs per (batch, kv-head)
-    int slice;       // most key positions one attention CTA takes: ceil(bound / P)
+    int slice;       // key positions an attention CTA lays out per round
     int HG;          // query heads per attention pass (1, 2, 4 or 8)
     size_t off_key, off_id, off_done1, off_rs, off_rl, off_rp, off_cnt, off_part, off_done2, bytes;
 };

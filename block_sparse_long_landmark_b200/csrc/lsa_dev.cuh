@@ -18,96 +18,58 @@ __device__ __forceinline__ uint64_t ord_key64(double x) {
     return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// Sum of v over the CTA (kLsaThreads threads); `red` holds 8 ints.
-__device__ __forceinline__ int block_sum(int v, int *red) {
-    v = __reduce_add_sync(0xffffffffu, v);
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    int t = 0;
-#pragma unroll
-    for (int w = 0; w < kLsaThreads / 32; ++w) t += red[w];
-    __syncthreads();                                // red is free again on return
-    return t;
-}
-
-// Positions (ascending) of the top-k of keys[0..n) in shared memory, equal
-// keys to the lower position, written to out[0..); every position when
-// n <= k.  Exact: the k-th largest key T is found bit by bit from the top
-// (bits shared by the largest and smallest key are taken as they are), then
-// a position-ordered compaction takes every key > T and the first keys == T.
-// All threads of the CTA call it; returns the count.
-__device__ inline int block_topk64(const uint64_t *keys, int n, int k, int *out, int *red, uint64_t *red64) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// Positions (ascending) of the top-k of keys[0..n) (shared or global
+// memory), equal keys to the lower position, by one warp (every lane calls
+// it); every position when n <= k.  The k-th largest key T is found bit by
+// bit below the bits the largest and smallest keys share, then an
+// index-ordered ballot compaction takes every key > T and the first keys
+// equal to T.  Returns the count (warp-uniform).
+__device__ inline int warp_topk64(const uint64_t *keys, int n, int k, int *out) {
+    const int lane = threadIdx.x & 31;
     if (k <= 0 || n <= 0) return 0;
     if (n <= k) {
-        for (int i = tid; i < n; i += kLsaThreads) out[i] = i;
-        __syncthreads();
+        for (int i = lane; i < n; i += 32) out[i] = i;
+        __syncwarp();
         return n;
     }
-    uint64_t mx = 0ull, mn = ~0ull;
-    for (int i = tid; i < n; i += kLsaThreads) {
-        mx = max(mx, keys[i]);
-        mn = min(mn, keys[i]);
+    unsigned long long mx = 0ull, mn = ~0ull;
+    for (int i = lane; i < n; i += 32) {
+        mx = max(mx, (unsigned long long)keys[i]);
+        mn = min(mn, (unsigned long long)keys[i]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        mx = max(mx, (uint64_t)__shfl_xor_sync(0xffffffffu, (unsigned long long)mx, o));
-        mn = min(mn, (uint64_t)__shfl_xor_sync(0xffffffffu, (unsigned long long)mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     }
-    __syncthreads();
-    if (lane == 0) {
-        red64[warp] = mx;
-        red64[8 + warp] = mn;
-    }
-    __syncthreads();
-    mx = 0ull;
-    mn = ~0ull;
-#pragma unroll
-    for (int w = 0; w < kLsaThreads / 32; ++w) {
-        mx = max(mx, red64[w]);
-        mn = min(mn, red64[8 + w]);
-    }
-    const uint64_t diff = mx ^ mn;
+    const unsigned long long diff = mx ^ mn;
     const int top = diff ? 63 - __clzll((long long)diff) : -1;
-    const uint64_t low = top >= 0 ? (~0ull >> (63 - top)) : 0ull;
-    uint64_t T = mx & ~low;                        // every key >= T
+    const unsigned long long low = top >= 0 ? (~0ull >> (63 - top)) : 0ull;
+    unsigned long long T = mx & ~low;
     for (int bit = top; bit >= 0; --bit) {
-        const uint64_t c = T | (1ull << bit);
+        const unsigned long long c = T | (1ull << bit);
         int ge = 0;
-        for (int i = tid; i < n; i += kLsaThreads) ge += keys[i] >= c;
-        if (block_sum(ge, red) >= k) T = c;
+        for (int i = lane; i < n; i += 32) ge += keys[i] >= c;
+        if (__reduce_add_sync(0xffffffffu, ge) >= k) T = c;
     }
     int gt = 0;
-    for (int i = tid; i < n; i += kLsaThreads) gt += keys[i] > T;
-    const int take_eq = k - block_sum(gt, red);
-    // compaction in position order: thread t owns positions [i0, i1)
-    const int seg = (n + kLsaThreads - 1) / kLsaThreads;
-    const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
-    int neq = 0;
-    for (int i = i0; i < i1; ++i) neq += keys[i] == T;
-    const int eq_base = block_scan_incl(neq, red, nullptr) - neq;
-    int nsel = 0;
-    {
-        int e = eq_base;
-        for (int i = i0; i < i1; ++i) {
-            const bool take = keys[i] > T || (keys[i] == T && e < take_eq);
-            e += keys[i] == T;
-            nsel += take;
-        }
+    for (int i = lane; i < n; i += 32) gt += keys[i] > T;
+    const int take_eq = k - __reduce_add_sync(0xffffffffu, gt);
+    const unsigned below = (1u << lane) - 1u;
+    int base = 0, eq_before = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const unsigned long long x = i < n ? keys[i] : 0ull;
+        const bool eq = i < n && x == T;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const bool sel = i < n && (x > T || (eq && eq_before + __popc(eqm & below) < take_eq));
+        const unsigned selm = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[base + __popc(selm & below)] = i;
+        base += __popc(selm);
+        eq_before += __popc(eqm);
     }
-    int total;
-    int pos = block_scan_incl(nsel, red, &total) - nsel;
-    {
-        int e = eq_base;
-        for (int i = i0; i < i1; ++i) {
-            const bool take = keys[i] > T || (keys[i] == T && e < take_eq);
-            e += keys[i] == T;
-            if (take) out[pos++] = i;
-        }
-    }
-    __syncthreads();
-    return total;
+    __syncwarp();
+    return base;
 }
 
 // Kept key ranges of one (batch, kv-head) from the chosen clusters (ids

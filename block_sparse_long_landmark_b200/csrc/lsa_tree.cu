@@ -481,7 +481,12 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_tree_select_kernel(TreeSelArg
         compared += nf;
         __syncthreads();
         const int keep = lv > 0 ? ta.beam : min(s.top_clusters, s.ctotal);
-        const int nk = block_topk64(keys, nf, keep, pos, red, red64);
+        if (warp == 0) {
+            const int c = warp_topk64(keys, nf, keep, pos);
+            if (lane == 0) misc[0] = c;
+        }
+        __syncthreads();
+        const int nk = misc[0];
         if (lv == 0) {
             // the chosen leaves (ascending ids) go to the range expansion; `mark` holds them
             for (int i = tid; i < nk; i += kLsaThreads) mark[i] = fr[pos[i]];
