@@ -10,18 +10,23 @@
 //   dK[tile] = scale * sum over kept units u of  dS_u^T Q_u
 //
 // accumulated in tensor memory while the tile's K and V stay in shared memory.
-// Per 128-row tile of a unit the tensor core computes S^T = K Q^T and
-// dP^T = V dO^T (keys in TMEM lanes, rows in columns); two element-wise
-// warpgroups (64 rows each) turn them into P^T and dS^T in bf16 over S^T and
-// dP^T; then dV += P^T dO and dK += dS^T Q.  Tensor memory: S^T [0, 128),
-// dP^T [128, 256), dV [256, 384), dK [384, 512).
+// A 128-row tile of a unit (a "pair") is taken in two halves of 64 rows, each
+// with its own tensor-memory buffer: the tensor core computes S^T = K Q_h^T
+// and dP^T = V dO_h^T for half h, the element-wise warpgroup h turns them into
+// P^T and dS^T in bf16 in place, and dV += P_h^T dO_h, dK += dS_h^T Q_h follow;
+// while one warpgroup works on its half the tensor core serves the other.
+// Tensor memory: half 0 S^T [0, 64) dP^T [64, 128), half 1 [128, 256),
+// dV [256, 384), dK [384, 512).
 //
-// Preparation (no atomics, fixed order): a warp per key tile walks the later
-// blocks' lists (each ascending) and records, in unit order, the units that
-// keep the tile and the list entries of its blocks; a scan turns the counts
-// into offsets.  A tile kept by more than 64 units is split into work items
-// of 64; each split leaves its accumulators in a partial slot, and for each
-// warp's region the split that finishes last sums the slots in split order.
+// Preparation (no atomics in the sums, fixed order): a warp per key tile walks
+// the later blocks' lists (each ascending) and records, in unit order, the
+// units that keep the tile with the gates of its blocks in log2 units; a scan
+// turns the counts into offsets and deals the work items out largest first.
+// A tile kept by more than 64 units is split into work items of 64; each
+// split leaves its accumulators in a partial slot, and for each warp's region
+// the split that finishes last sums the slots in split order.  The per-row
+// LSE and D come from a layout padded to whole blocks, so that each pair's
+// rows are contiguous 16-byte-aligned runs fetched by bulk copies.
 #include <math_constants.h>
 
 #include "backward_tc.cuh"
@@ -39,7 +44,8 @@ constexpr int kUMax = 64;          // units per work item
 struct KvLayout {
     int KT, bpt, tiles, MT;
     size_t pairs_max, items_max, slots_max;
-    size_t off_tcnt, off_toff, off_tsplit, off_tslot, off_ioff, off_tot, off_ent, off_items, off_part, bytes;
+    size_t off_tcnt, off_toff, off_tsplit, off_tslot, off_ioff, off_tot, off_ent, off_items, off_order, off_part,
+        bytes;
 };
 
 KvLayout kv_layout(const Shape &s) {
@@ -62,6 +68,7 @@ KvLayout kv_layout(const Shape &s) {
     L.off_tot = o;    o += 256;
     L.off_ent = o;    o += al(L.pairs_max * 16);
     L.off_items = o;  o += al(L.items_max * 16);
+    L.off_order = o;  o += al(L.items_max * 4);
     L.off_part = o;   o += al(L.slots_max * 2 * 128 * 128 * 4);
     L.bytes = o;
     return L;
@@ -70,8 +77,9 @@ KvLayout kv_layout(const Shape &s) {
 struct InvArgs {
     Shape s;
     const int32_t *idx, *count;
+    const float *score;
     int KT, bpt, tiles;
-    int *tcnt, *toff, *tsplit, *tslot, *ioff, *tot;
+    int *tcnt, *toff, *tsplit, *tslot, *ioff, *tot, *order;
     int4 *ent, *items;
 };
 
@@ -86,8 +94,19 @@ __device__ __forceinline__ int find_entry(const int32_t *il, int cnt, int blk) {
     return (lo < cnt && il[lo] == blk) ? lo : -1;
 }
 
+// Gate of list entry c (block blk) of unit j in log2 units; -inf when the
+// unit does not keep the block.  Forced entries (sink, local) carry no gate.
+__device__ __forceinline__ float entry_gate2(const Shape &s, const float *sl, int cnt, int c, int blk, int j) {
+    if (c < 0) return -CUDART_INF_F;
+    const bool forced = (blk == j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
+    if (!(s.flags & SA_GATE) || forced) return 0.f;
+    return log_sigmoid(sl[c] - sl[cnt - 1]) * kLog2e;
+}
+
 // A warp per key tile: pass 0 counts the units that keep one of its blocks,
-// pass 1 records them (ascending unit) and the tile's work items.
+// pass 1 records them (ascending unit) with their gates, and the tile's work
+// items.  Entry: (unit j, gate of the tile's first block, of its second, 0),
+// gates as float bits.
 __global__ void inv_kernel(InvArgs a, int pass) {
     const int t = (int)(((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
     if (t >= a.tiles) return;
@@ -98,17 +117,24 @@ __global__ void inv_kernel(InvArgs a, int pass) {
     int n = 0;
     for (int j0 = b0; j0 < s.nb; j0 += 32) {          // a unit keeps only blocks up to its own
         const int j = j0 + lane;
-        int c0 = -1, c1 = -1;
+        int c0 = -1, c1 = -1, cnt = 0;
+        size_t lu = 0;
         if (j < s.nb) {
-            const size_t lu = (size_t)bg * s.nb + j;
-            const int cnt = max(0, min(a.count[lu], s.cap));
+            lu = (size_t)bg * s.nb + j;
+            cnt = max(0, min(a.count[lu], s.cap));
             const int32_t *il = a.idx + lu * s.cap;
             c0 = find_entry(il, cnt, b0);
             if (b0 + 1 < b1) c1 = find_entry(il, cnt, b0 + 1);
         }
         const bool keep = c0 >= 0 || c1 >= 0;
         const unsigned m = __ballot_sync(0xffffffffu, keep);
-        if (pass && keep) a.ent[base + n + __popc(m & ((1u << lane) - 1u))] = make_int4(j, c0, c1, 0);
+        if (pass && keep) {
+            const float *sl = a.score + lu * s.cap;
+            const float g0 = entry_gate2(s, sl, cnt, c0, b0, j);
+            const float g1 = a.bpt == 2 ? entry_gate2(s, sl, cnt, c1, b0 + 1, j) : g0;
+            a.ent[base + n + __popc(m & ((1u << lane) - 1u))] =
+                make_int4(j, __float_as_int(g0), __float_as_int(g1), 0);
+        }
         n += __popc(m);
     }
     if (!pass) {
@@ -120,18 +146,27 @@ __global__ void inv_kernel(InvArgs a, int pass) {
         a.items[a.ioff[t] + sp] = make_int4(t, base + sp * kUMax, base + min(n, (sp + 1) * kUMax), sp);
 }
 
-// One CTA: offsets of every tile's units, items and partial slots.
+// One CTA: offsets of every tile's units, items and partial slots, then the
+// order in which the dK/dV kernel takes the items: by size, largest first
+// (items of equal size in any order -- the results do not depend on it).
 __global__ void __launch_bounds__(1024) inv_scan_kernel(InvArgs a) {
     __shared__ int wsum[32][3];
     __shared__ int carry[3];
+    __shared__ int hist[kUMax + 1], cur[kUMax + 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid < 3) carry[tid] = 0;
+    if (tid <= kUMax) hist[tid] = 0;
     __syncthreads();
     for (int t0 = 0; t0 < a.tiles; t0 += 1024) {
         const int t = t0 + tid;
         const int n = t < a.tiles ? a.tcnt[t] : 0;
         const int ns = t < a.tiles ? max(1, (n + kUMax - 1) / kUMax) : 0;
         const int sl = ns > 1 ? ns : 0;
+        if (t < a.tiles) {
+            const int full = n / kUMax, rem = n - full * kUMax;
+            if (full) atomicAdd(&hist[kUMax], full);
+            if (rem || n == 0) atomicAdd(&hist[rem], 1);
+        }
         int v[3] = {n, ns, sl}, incl[3];
 #pragma unroll
         for (int q = 0; q < 3; ++q) {
@@ -166,6 +201,20 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(InvArgs a) {
         a.tot[0] = carry[1];     // work items
         a.tot[1] = carry[0];     // (tile, unit) entries
         a.tot[2] = carry[2];     // partial slots
+        int pos = 0;
+        for (int sz = kUMax; sz >= 0; --sz) {
+            cur[sz] = pos;
+            pos += hist[sz];
+        }
+    }
+    __syncthreads();
+    for (int t = tid; t < a.tiles; t += 1024) {
+        const int n = a.tcnt[t], io = a.ioff[t];
+        const int ns = max(1, (n + kUMax - 1) / kUMax);
+        for (int sp = 0; sp < ns; ++sp) {
+            const int sz = min(kUMax, n - sp * kUMax);
+            a.order[atomicAdd(&cur[sz], 1)] = io + sp;
+        }
     }
 }
 
@@ -180,51 +229,48 @@ constexpr uint32_t kTile = 2 * kChunk;
 constexpr uint32_t kKOff = 0, kVOff = kTile;
 constexpr uint32_t kRingOff = 2 * kTile;           // [2 stages] Q tile, dO tile
 constexpr uint32_t kStageBytes = 2 * kTile;
-constexpr uint32_t kRowOff = kRingOff + 2 * kStageBytes;    // [2 stages] lse2[128], D[128], pos[128]
-constexpr uint32_t kRowBytes = 3 * 128 * 4;
-constexpr uint32_t kInfoOff = kRowOff + 2 * kRowBytes;      // [2 stages] gate[2], blk[2], unit
-constexpr uint32_t kInfoBytes = 32;
-constexpr uint32_t kBarOffKV = kInfoOff + 2 * kInfoBytes + 64;
+constexpr uint32_t kRowOff = kRingOff + 2 * kStageBytes;    // [2 stages] lse2[128], D[128]
+constexpr uint32_t kRowBytes = 2 * 128 * 4;
+constexpr uint32_t kInfoOff = kRowOff + 2 * kRowBytes;      // [2 stages] the pair's entry (int4)
+constexpr uint32_t kInfoBytes = 16;
+constexpr uint32_t kBarOffKV = kInfoOff + 2 * kInfoBytes + 32;
 constexpr uint32_t kSmemKV = kBarOffKV + 512 + 1024;
 static_assert(kSmemKV <= 227 * 1024, "shared memory");
+static_assert(kRowOff % 16 == 0 && kRowBytes % 16 == 0, "bulk copy alignment");
 
 enum {
     B_KVF = 0,          // K, V tiles landed
     B_KVE = 1,          // K, V tiles free
     B_PF = 2,           // [2] pair stage full
     B_PE = 4,           // [2] pair stage free
-    B_ST = 6,           // S^T, dP^T ready
-    B_EW = 7,           // P^T, dS^T written (256 arrivals)
-    B_ACC = 8,          // the item's dV, dK complete
-    B_ACCF = 9,         // dV, dK read out (256 arrivals)
-    B_END = 10,
+    B_ST = 6,           // [2 halves] S^T, dP^T of the half ready
+    B_EW = 8,           // [2 halves] P^T, dS^T of the half written (128 arrivals)
+    B_ACC = 10,         // the item's dV, dK complete
+    B_ACCF = 11,        // dV, dK read out (256 arrivals)
+    B_END = 12,
     NBARKV
 };
 static_assert(8 * NBARKV + 8 <= 512, "barrier area");
 
 struct KvArgs {
     Shape s;
-    const int32_t *idx, *count;
-    const float *score;
-    const float *D, *lse2;
+    const float *D, *lse2;      // [B,Hq,Npad] (Npad = nb * block; rows past N: D 0, lse2 +inf)
     float *dK, *dV;
-    const int *tsplit, *tslot, *tot;
+    const int *tsplit, *tslot, *tot, *order;
     int *rcnt;                  // [tiles][8 regions] splits finished
     const int4 *ent, *items;
     float *part;                // [slots][2][128][128]
     unsigned *status;
-    int KT, MT;
+    int KT, MT, Npad;
     unsigned long long wait_ns;
 };
 
-__device__ __forceinline__ void row_of(const Shape &s, int j, int m, int r, int &hh, int &pos) {
-    if (s.bs == 64) {
-        hh = 2 * m + (r >> 6);
-        pos = j * 64 + (r & 63);
-    } else {
-        hh = m;
-        pos = j * 128 + r;
-    }
+// k-th work item of this CTA, in the snake order over the size-sorted items
+// (round k: CTAs ascending when k is even, descending when odd); -1 when done.
+__device__ __forceinline__ int item_of(const KvArgs &a, int k, int nitems) {
+    const int P = gridDim.x;
+    const int q = k * P + ((k & 1) ? P - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    return q < nitems ? a.order[q] : -1;
 }
 
 __global__ void __launch_bounds__(kThreadsKV, 1)
@@ -240,12 +286,13 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOffKV + 8 * NBARKV + 4);
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
     auto rows_of = [&](int st) { return reinterpret_cast<float *>(smem + kRowOff + st * kRowBytes); };
-    auto info_of = [&](int st) { return reinterpret_cast<float *>(smem + kInfoOff + st * kInfoBytes); };
+    auto info_of = [&](int st) { return reinterpret_cast<int4 *>(smem + kInfoOff + st * kInfoBytes); };
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nitems = a.tot[0];
 
     if (tid == 0) {
-        for (int i = 0; i < NBARKV; ++i) mbar_init(bar(i), (i == B_EW || i == B_ACCF) ? 256 : 1);
+        for (int i = 0; i < NBARKV; ++i)
+            mbar_init(bar(i), (i == B_EW || i == B_EW + 1) ? 128 : i == B_ACCF ? 256 : 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -260,13 +307,15 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---- K/V of the tile, then per (unit, row tile): rows, gates, Q and dO ----
+        // ---- K/V of the tile, then per pair: entry, rows, Q and dO ----------
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLowKV));
         bool ok = true;
         int gp = 0, ni = 0;
         int kvlast = -1;                 // phase of the last K/V load issued
         int plast[2] = {-1, -1};         // last pair issued on each ring stage
-        for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+        for (int k = 0;; ++k) {
+            const int it = item_of(a, k, nitems);
+            if (it < 0) break;
             const int4 item = a.items[it];
             const int np = (item.z - item.y) * a.MT;
             if (np == 0) continue;
@@ -287,55 +336,44 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
+            int4 mine = make_int4(0, 0, 0, 0);
             for (int p = 0; p < np; ++p, ++gp) {
-                const int st = gp & 1;
-                if (gp >= 2) ok = mbar_wait(bar(B_PE + st), ((gp >> 1) - 1) & 1, abort_flag, a.status, a.wait_ns);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                const int4 en = a.ent[item.y + p / a.MT];
-                const int j = en.x, m = p % a.MT;
-                // row data of the 128 rows: lse2 (+inf past the sequence), D, position
-                float *rw = rows_of(st);
-                for (int r = lane; r < 128; r += 32) {
-                    int hh, pos;
-                    row_of(s, j, m, r, hh, pos);
-                    const bool ok_r = pos < s.N;
-                    const size_t grow = ((size_t)b * s.Hq + g * s.G + hh) * s.N + (ok_r ? pos : 0);
-                    rw[r] = ok_r ? a.lse2[grow] : CUDART_INF_F;
-                    rw[128 + r] = ok_r ? a.D[grow] : 0.f;
-                    reinterpret_cast<int *>(rw)[256 + r] = pos;
+                const int st = gp & 1, ui = p / a.MT, m = p % a.MT;
+                if (m == 0 && (ui & 31) == 0) {
+                    const int e = item.y + ui + lane;
+                    mine = e < item.z ? a.ent[e] : make_int4(0, 0, 0, 0);
                 }
+                int4 en;
+                en.x = __shfl_sync(0xffffffffu, mine.x, ui & 31);
+                en.y = __shfl_sync(0xffffffffu, mine.y, ui & 31);
+                en.z = __shfl_sync(0xffffffffu, mine.z, ui & 31);
+                en.w = 0;
                 if (lane == 0) {
-                    // the gate of each 64-key half for this unit (log2 units; -inf: not kept)
-                    const size_t lu = (size_t)bg * s.nb + j;
-                    const int cnt = max(0, min(a.count[lu], s.cap));
-                    const float *sl = a.score + lu * s.cap;
-                    const float s_loc = cnt > 0 ? sl[cnt - 1] : 0.f;
-                    float *inf = info_of(st);
-                    for (int h = 0; h < 2; ++h) {
-                        const int c = (s.bs == 64 && h == 1) ? en.z : en.y;
-                        const int blk = s.bs == 64 ? kt * 2 + h : kt;
-                        const bool forced = (blk == j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
-                        inf[h] = c < 0 ? -CUDART_INF_F
-                                       : (((s.flags & SA_GATE) && !forced) ? log_sigmoid(sl[c] - s_loc) * kLog2e : 0.f);
-                        reinterpret_cast<int *>(inf)[2 + h] = blk;
-                    }
-                    reinterpret_cast<int *>(inf)[4] = j;
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_expect_tx(bar(B_PF + st), 2 * kTile);
-                    const uint32_t qd = sbase + kRingOff + st * kStageBytes, dd = qd + kTile;
-                    for (int e = 0; e < 2; ++e) {
-                        int hh, pos;
-                        row_of(s, j, m, 64 * e, hh, pos);
-                        const int y = (b * s.Hq + g * s.G + hh) * s.N + pos;
-                        for (int c = 0; c < 2; ++c) {
-                            tma_load_2d(qd + c * kChunk + e * 8192, &tmQ, bar(B_PF + st), 64 * c, y);
-                            tma_load_2d(dd + c * kChunk + e * 8192, &tmDO, bar(B_PF + st), 64 * c, y);
+                    if (gp >= 2) ok = mbar_wait(bar(B_PE + st), ((gp >> 1) - 1) & 1, abort_flag, a.status, a.wait_ns);
+                    if (ok) {
+                        const int j = en.x;
+                        *info_of(st) = en;
+                        mbar_expect_tx(bar(B_PF + st), 2 * kTile + kRowBytes);
+                        const uint32_t qd = sbase + kRingOff + st * kStageBytes, dd = qd + kTile;
+                        const uint32_t rw = sbase + kRowOff + st * kRowBytes;
+                        for (int e = 0; e < 2; ++e) {
+                            // rows 64 e .. 64 e + 63: (head, first position)
+                            const int hh = s.bs == 64 ? 2 * m + e : m;
+                            const int pos = s.bs == 64 ? j * 64 : j * 128 + 64 * e;
+                            const int y = (b * s.Hq + g * s.G + hh) * s.N + pos;
+                            for (int c = 0; c < 2; ++c) {
+                                tma_load_2d(qd + c * kChunk + e * 8192, &tmQ, bar(B_PF + st), 64 * c, y);
+                                tma_load_2d(dd + c * kChunk + e * 8192, &tmDO, bar(B_PF + st), 64 * c, y);
+                            }
+                            const size_t rp = (size_t)(b * s.Hq + g * s.G + hh) * a.Npad + pos;
+                            bulk_load(rw + 256 * e, a.lse2 + rp, 256, bar(B_PF + st));
+                            bulk_load(rw + 512 + 256 * e, a.D + rp, 256, bar(B_PF + st));
                         }
+                        plast[st] = gp;
                     }
-                    plast[st] = gp;
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
             }
             if (!ok) break;
             ++ni;
@@ -349,52 +387,76 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     } else if (warp == 1) {
         // ---- MMA issuer -----------------------------------------------------
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLowKV));
-        constexpr uint32_t idk = idesc_bf16(false, 128), idm = idesc_bf16(true, 128);
-        auto gemm_kk = [&](uint32_t dtm, uint32_t aoff, uint32_t boff) {
-            const uint64_t da = desc_k_sw128(sbase + aoff), db = desc_k_sw128(sbase + boff);
+        constexpr uint32_t idh = idesc_bf16(false, 64), idm = idesc_bf16(true, 128);
+        // half h of a pair into buffer h: S^T = K Q_h^T (N = 64 rows), dP^T = V dO_h^T
+        auto sdp = [&](int st, int h) {
+            const uint32_t qo = kRingOff + st * kStageBytes + h * 8192, doo = qo + kTile;
+            const uint64_t dk = desc_k_sw128(sbase + kKOff), dv = desc_k_sw128(sbase + kVOff);
+            const uint64_t dq = desc_k_sw128(sbase + qo), dd = desc_k_sw128(sbase + doo);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const uint32_t off = ((k >> 2) * kChunk + (k & 3) * 32) >> 4;
-                mma_ss_w(dtm, da + off, db + off, idk, k > 0);
+                mma_ss_w(tmem + 128 * h, dk + off, dq + off, idh, k > 0);
             }
-        };
-        // acc += X^T Y: A = X^T in TMEM (bf16, rows 0-63 in columns [a0, a0+32),
-        // rows 64-127 in [a0+64, a0+96)), B = a row tile in shared memory, MN-major
-        auto gemm_tm = [&](uint32_t dtm, uint32_t a0, uint32_t boff, bool acc) {
-            const uint64_t db = desc_mn_sw128(sbase + boff, kChunk);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const uint32_t acol = a0 + (k < 4 ? 8 * k : 64 + 8 * (k - 4));
-                mma_ts_w(dtm, acol, db + ((k * 2048) >> 4), idm, acc || k > 0);
+                const uint32_t off = ((k >> 2) * kChunk + (k & 3) * 32) >> 4;
+                mma_ss_w(tmem + 128 * h + 64, dv + off, dd + off, idh, k > 0);
             }
+        };
+        // dV += P_h^T dO_h, dK += dS_h^T Q_h: A in tensor memory (bf16 pairs of
+        // the half's 64 rows in columns [0, 32) of S^T / dP^T), B = the half's
+        // rows of the stage's tiles, MN-major
+        auto acc_half = [&](int st, int h, bool acc) {
+            const uint32_t qo = kRingOff + st * kStageBytes, doo = qo + kTile;
+            const uint64_t dd = desc_mn_sw128(sbase + doo, kChunk), dq = desc_mn_sw128(sbase + qo, kChunk);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                mma_ts_w(tmem + 256, tmem + 128 * h + 8 * k, dd + (((4 * h + k) * 2048) >> 4), idm, acc || k > 0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                mma_ts_w(tmem + 384, tmem + 128 * h + 64 + 8 * k, dq + (((4 * h + k) * 2048) >> 4), idm,
+                         acc || k > 0);
         };
         auto wait = [&](int i, int parity) {
             return __all_sync(0xffffffffu, mbar_wait(bar(i), parity, abort_flag, a.status, a.wait_ns));
         };
         bool ok = true;
         int gp = 0, ni = 0;
-        for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x) {
+        for (int k = 0; ok; ++k) {
+            const int it = item_of(a, k, nitems);
+            if (it < 0) break;
             const int4 item = a.items[it];
             const int np = (item.z - item.y) * a.MT;
             if (np == 0) continue;
             if (!(ok = wait(B_KVF, ni & 1))) break;
+            if (!(ok = wait(B_PF + (gp & 1), (gp >> 1) & 1))) break;
+            tc_fence_after();
+            sdp(gp & 1, 0);
+            mma_commit_w(bar(B_ST));
+            sdp(gp & 1, 1);
+            mma_commit_w(bar(B_ST + 1));
             for (int p = 0; ok && p < np; ++p, ++gp) {
                 const int st = gp & 1;
-                const uint32_t qo = kRingOff + st * kStageBytes, doo = qo + kTile;
-                if (!(ok = wait(B_PF + st, (gp >> 1) & 1))) break;
-                tc_fence_after();
-                gemm_kk(tmem + 0, kKOff, qo);        // S^T = K Q^T
-                gemm_kk(tmem + 128, kVOff, doo);     // dP^T = V dO^T
-                mma_commit_w(bar(B_ST));
-                if (!(ok = wait(B_EW, gp & 1))) break;
-                tc_fence_after();
-                if (p == 0 && ni > 0) {
-                    if (!(ok = wait(B_ACCF, (ni - 1) & 1))) break;
+                const bool more = p + 1 < np;
+                for (int h = 0; h < 2; ++h) {
+                    if (!(ok = wait(B_EW + h, gp & 1))) break;
                     tc_fence_after();
+                    if (p == 0 && h == 0 && ni > 0) {
+                        // the previous item's accumulators must have been read out
+                        if (!(ok = wait(B_ACCF, (ni - 1) & 1))) break;
+                        tc_fence_after();
+                    }
+                    acc_half(st, h, p > 0 || h > 0);
+                    if (h == 1) mma_commit_w(bar(B_PE + st));
+                    if (more) {
+                        // the next pair's half h into the buffer just read (the MMAs run in order)
+                        if (h == 0 && !(ok = wait(B_PF + (st ^ 1), ((gp + 1) >> 1) & 1))) break;
+                        tc_fence_after();
+                        sdp(st ^ 1, h);
+                        mma_commit_w(bar(B_ST + h));
+                    }
                 }
-                gemm_tm(tmem + 256, tmem + 0, doo, p > 0);     // dV += P^T dO
-                gemm_tm(tmem + 384, tmem + 128, qo, p > 0);    // dK += dS^T Q
-                mma_commit_w(bar(B_PE + st));
             }
             if (!ok) break;
             mma_commit_w(bar(B_ACC));
@@ -408,20 +470,26 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLowKV));
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHighKV));
-        // ---- element-wise warpgroups: wg 0 rows 0-63, wg 1 rows 64-127 -----
+        // ---- element-wise warpgroups: wg h takes half h (rows 64 h .. 64 h + 63)
+        // of every pair; for the accumulators, columns 64 wg .. 64 wg + 63 ----
         const int wg = (warp - 4) >> 2, qq = warp & 3, ew = warp - 4;
         const int kl = 32 * qq + lane;                   // key lane of the tile
         const uint32_t lane_off = (uint32_t)(32 * qq) << 16;
+        const uint32_t tb = tmem + lane_off + 128 * wg;  // this half's buffer
         const bool causal = s.flags & SA_CAUSAL;
         const float sc2 = s.scale * kLog2e;
         bool ok = true;
         int gp = 0, ni = 0;
-        for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x) {
+        for (int k = 0; ok; ++k) {
+            const int it = item_of(a, k, nitems);
+            if (it < 0) break;
             const int4 item = a.items[it];
             const int np = (item.z - item.y) * a.MT;
             const int bg = item.x / a.KT, kt = item.x % a.KT;
             const int key = kt * 128 + kl;
             const bool key_ok = key < s.N;
+            const int hk = s.bs == 64 ? (kl >> 6) : 0;             // the key's block within the tile
+            const int blk = s.bs == 64 ? kt * 2 + hk : kt;
             float *dkrow = a.dK + ((size_t)bg * s.N + (key_ok ? key : 0)) * 128 + 64 * wg;
             float *dvrow = a.dV + ((size_t)bg * s.N + (key_ok ? key : 0)) * 128 + 64 * wg;
             if (np == 0) {
@@ -435,53 +503,58 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             for (int p = 0; p < np; ++p, ++gp) {
                 const int st = gp & 1;
-                ok = mbar_wait(bar(B_ST), gp & 1, abort_flag, a.status, a.wait_ns);
+                ok = mbar_wait(bar(B_ST + wg), gp & 1, abort_flag, a.status, a.wait_ns) &&
+                     mbar_wait(bar(B_PF + st), (gp >> 1) & 1, abort_flag, a.status, a.wait_ns);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
-                const float *rw = rows_of(st);
-                const int *rpos = reinterpret_cast<const int *>(rw) + 256;
-                const float *inf = info_of(st);
-                const int h = s.bs == 64 ? (kl >> 6) : 0;
-                const float gl = inf[h];
-                const int blk = reinterpret_cast<const int *>(inf)[2 + h];
-                const int j = reinterpret_cast<const int *>(inf)[4];
+                const float *rw = rows_of(st) + 64 * wg;
+                const int4 en = *info_of(st);
+                const int j = en.x;
+                const float gl = __int_as_float(hk ? en.z : en.y);
                 const bool kvis = key_ok && gl != -CUDART_INF_F;
-                const bool local = causal && blk == j;
-                // this warpgroup's 64 rows in two halves of 32 (S^T, dP^T in, P^T, dS^T out);
-                // each half's bf16 output lands in columns the other half does not read
+                // first position of this half's rows; in the unit's own block, row r
+                // (position pos0 + r) sees the key only when r >= key - pos0
+                const int pos0 = s.bs == 64 ? j * 64 : j * 128 + 64 * wg;
+                const int lim = (causal && blk == j) ? key - pos0 : -1;
                 float x[32], y[32];
                 uint32_t pp[16], pd[16];
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    tmem_ld32(tmem + lane_off + 64 * wg + 32 * hf, x);
-                    tmem_ld32(tmem + lane_off + 128 + 64 * wg + 32 * hf, y);
+                    tmem_ld32(tb + 32 * hf, x);
+                    tmem_ld32(tb + 64 + 32 * hf, y);
                     tmem_wait_ld();
                     reg_fence<32>(x);
                     reg_fence<32>(y);
 #pragma unroll
-                    for (int k = 0; k < 32; k += 2) {
-                        float pv[2], dv[2];
+                    for (int k4 = 0; k4 < 32; k4 += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(rw + 32 * hf + k4);
+                        const float4 d4 = *reinterpret_cast<const float4 *>(rw + 128 + 32 * hf + k4);
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float pv[4], dv[4];
 #pragma unroll
-                        for (int q2 = 0; q2 < 2; ++q2) {
-                            const int r = 64 * wg + 32 * hf + k + q2;
-                            const bool vis = kvis && !(local && key > rpos[r]);
-                            const float p = vis ? ex2(fmaf(x[k + q2], sc2, gl - rw[r])) : 0.f;
-                            pv[q2] = p;
-                            dv[q2] = p * (y[k + q2] - rw[128 + r]);
+                        for (int q = 0; q < 4; ++q) {
+                            const int r = 32 * hf + k4 + q;
+                            const bool vis = kvis && r >= lim;
+                            const float p = vis ? ex2(fmaf(x[k4 + q], sc2, gl - lv[q])) : 0.f;
+                            pv[q] = p;
+                            dv[q] = p * (y[k4 + q] - dvv[q]);
                         }
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(pv[0], pv[1]);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(dv[0], dv[1]);
-                        pp[k >> 1] = *reinterpret_cast<uint32_t *>(&h1);
-                        pd[k >> 1] = *reinterpret_cast<uint32_t *>(&h2);
+#pragma unroll
+                        for (int q = 0; q < 4; q += 2) {
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(pv[q], pv[q + 1]);
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(dv[q], dv[q + 1]);
+                            pp[(k4 + q) >> 1] = *reinterpret_cast<uint32_t *>(&h1);
+                            pd[(k4 + q) >> 1] = *reinterpret_cast<uint32_t *>(&h2);
+                        }
                     }
-                    // half hf of 32 rows -> 16 bf16-pair columns at 64 wg + 16 hf: below
-                    // column 64 wg + 32 hf, the first one half 1 reads
-                    tmem_st16(tmem + lane_off + 64 * wg + 16 * hf, pp);
-                    tmem_st16(tmem + lane_off + 128 + 64 * wg + 16 * hf, pd);
+                    // rows 32 hf .. 32 hf + 31 -> 16 bf16-pair columns at 16 hf: below
+                    // column 32 hf, the first one the second half reads
+                    tmem_st16(tb + 16 * hf, pp);
+                    tmem_st16(tb + 64 + 16 * hf, pd);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar(B_EW));
+                mbar_arrive(bar(B_EW + wg));
             }
             if (!ok) break;
             // ---- the item's accumulators: this warp's 32 keys x 64 columns ----
@@ -565,6 +638,7 @@ cudaError_t launch_backward_kv(const Shape &s, const void *Q, const void *K, con
     ia.s = s;
     ia.idx = idx;
     ia.count = count;
+    ia.score = score;
     ia.KT = L.KT;
     ia.bpt = L.bpt;
     ia.tiles = L.tiles;
@@ -574,6 +648,7 @@ cudaError_t launch_backward_kv(const Shape &s, const void *Q, const void *K, con
     ia.tslot = reinterpret_cast<int *>(w + L.off_tslot);
     ia.ioff = reinterpret_cast<int *>(w + L.off_ioff);
     ia.tot = reinterpret_cast<int *>(w + L.off_tot);
+    ia.order = reinterpret_cast<int *>(w + L.off_order);
     ia.ent = reinterpret_cast<int4 *>(w + L.off_ent);
     ia.items = reinterpret_cast<int4 *>(w + L.off_items);
     const unsigned wgrid = (unsigned)(((size_t)L.tiles * 32 + 255) / 256);
@@ -594,11 +669,9 @@ cudaError_t launch_backward_kv(const Shape &s, const void *Q, const void *K, con
     if (!make_map_d128(&mq, Q, qrows, 64) || !make_map_d128(&mk, K, krows, 64) || !make_map_d128(&mv, V, krows, 64) ||
         !make_map_d128(&mdo, dO, qrows, 64))
         return cudaErrorInvalidValue;
+    if ((reinterpret_cast<uintptr_t>(D) | reinterpret_cast<uintptr_t>(lse2)) & 15) return cudaErrorInvalidValue;
     KvArgs a{};
     a.s = s;
-    a.idx = idx;
-    a.count = count;
-    a.score = score;
     a.D = D;
     a.lse2 = lse2;
     a.dK = dK;
@@ -606,6 +679,7 @@ cudaError_t launch_backward_kv(const Shape &s, const void *Q, const void *K, con
     a.tsplit = ia.tsplit;
     a.tslot = ia.tslot;
     a.tot = ia.tot;
+    a.order = ia.order;
     a.rcnt = rcnt;
     a.ent = ia.ent;
     a.items = ia.items;
@@ -613,6 +687,7 @@ cudaError_t launch_backward_kv(const Shape &s, const void *Q, const void *K, con
     a.status = status;
     a.KT = L.KT;
     a.MT = L.MT;
+    a.Npad = s.nb * s.bs;
     a.wait_ns = kWaitNs;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorNoDevice;

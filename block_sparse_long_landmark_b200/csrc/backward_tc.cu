@@ -43,28 +43,33 @@ using namespace tc;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------
-// Row preparation: D = <dO, O> (fp32) and LSE * log2(e) per query row; rows
-// past the sequence get lse2 = +inf (so P = 0) and D = 0.
+// Row preparation: D = <dO, O> (fp32) and LSE * log2(e) per query row, in a
+// layout padded to whole blocks ([B,Hq,Npad], Npad = nb * block): padded rows
+// and empty rows get lse2 = +inf (so P = 0) and D = 0.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) bwd_rowprep_kernel(Shape s, const __nv_bfloat16 *O,
                                                           const __nv_bfloat16 *dO, const float *lse, float *D,
-                                                          float *lse2, long long rows) {
+                                                          float *lse2, long long rows_pad, int Npad) {
     // 16 lanes per 128-element row (16-byte loads), two rows per warp
     const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
     const int cv = threadIdx.x & 15;
+    const long long bh = r / Npad;
+    const int pos = (int)(r - bh * Npad);
+    const bool real = r < rows_pad && pos < s.N;
+    const long long src = bh * s.N + pos;
     float acc = 0.f;
-    if (r < rows) {
+    if (real) {
         float a[8], b[8];
-        load16(O + r * 128 + cv * 8, a);
-        load16(dO + r * 128 + cv * 8, b);
+        load16(O + src * 128 + cv * 8, a);
+        load16(dO + src * 128 + cv * 8, b);
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc = fmaf(a[i], b[i], acc);
     }
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (r < rows && cv == 0) {
+    if (r < rows_pad && cv == 0) {
         D[r] = acc;
-        const float l = lse[r];
+        const float l = real ? lse[src] : -CUDART_INF_F;
         lse2[r] = l == -CUDART_INF_F ? CUDART_INF_F : l * kLog2e;   // an empty row: P = 0
     }
 }
@@ -113,11 +118,12 @@ struct DqArgs {
     const int32_t *idx;
     const float *score;
     const int32_t *count;
-    const float *D, *lse2;      // [B,Hq,N]
+    const float *D, *lse2;      // [B,Hq,Npad], padded to whole blocks
     float *dQ;                  // [B,Hq,N,d] fp32, overwritten
     float *dgp;                 // [units][MT][cap][8 warps] gate-gradient partials
     unsigned *status;
     int MT;                     // 128-row tiles per unit: G * block / 128
+    int Npad;                   // nb * block
     int items;                  // units * MT
     unsigned long long wait_ns;
 };
@@ -239,15 +245,42 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                 }
                 const int kvbase = (w.b * s.Hkv + w.g) * s.N;
-                for (int t = 0; ok && t < T; ++t) {
-                    const int gg = gt + t, st = gg % kStages, use = gg / kStages;
-                    int y0, y1;
+                auto rows_of_tile = [&](int t, int &y0, int &y1) {
                     if (s.bs == 64) {
                         y0 = kvbase + max(0, blk_s[2 * t]) * 64;
                         y1 = kvbase + max(0, blk_s[min(2 * t + 1, cnt - 1)]) * 64;
                     } else {
                         y0 = kvbase + max(0, blk_s[t]) * 128;
                         y1 = y0 + 64;
+                    }
+                };
+                if (ok && it + (int)gridDim.x < a.items) {
+                    // the next item's Q and dO rows into L2 while this one runs
+                    const Item nx = item_at(a, it + gridDim.x);
+                    for (int e = 0; e < 2; ++e) {
+                        int hh, pos;
+                        row_of(s, nx.j, nx.m, 64 * e, hh, pos);
+                        const int y = (nx.b * s.Hq + nx.g * s.G + hh) * s.N + pos;
+                        for (int c = 0; c < 2; ++c) {
+                            tma_prefetch_2d(&tmQ, 64 * c, y);
+                            tma_prefetch_2d(&tmDO, 64 * c, y);
+                        }
+                    }
+                }
+                for (int t = 0; ok && t < T; ++t) {
+                    const int gg = gt + t, st = gg % kStages, use = gg / kStages;
+                    int y0, y1;
+                    rows_of_tile(t, y0, y1);
+                    if (t + kStages < T) {
+                        // the tile after the ring's depth into L2 ahead of its load
+                        int p0, p1;
+                        rows_of_tile(t + kStages, p0, p1);
+                        for (int c = 0; c < 2; ++c) {
+                            tma_prefetch_2d(&tmK, 64 * c, p0);
+                            tma_prefetch_2d(&tmK, 64 * c, p1);
+                            tma_prefetch_2d(&tmV, 64 * c, p0);
+                            tma_prefetch_2d(&tmV, 64 * c, p1);
+                        }
                     }
                     if (gg >= kStages &&
                         !(ok = mbar_wait(bar(Q_KE + st), (use - 1) & 1, abort_flag, a.status, a.wait_ns)))
@@ -394,8 +427,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const int head = w.g * s.G + hh;
             const bool row_ok = qi < s.N;
             const size_t grow = ((size_t)w.b * s.Hq + head) * s.N + (row_ok ? qi : 0);
-            const float l2 = row_ok ? a.lse2[grow] : CUDART_INF_F;
-            const float Dr = row_ok ? a.D[grow] : 0.f;
+            const size_t prow = ((size_t)w.b * s.Hq + head) * a.Npad + qi;    // +inf, 0 past the sequence
+            const float l2 = a.lse2[prow];
+            const float Dr = a.D[prow];
             float *dgp = a.dgp + ((size_t)w.unit * a.MT + w.m) * s.cap * 8;   // [entry][8 warps]
             for (int t = 0; t < T; ++t) {
                 const int gg = gt + t;
@@ -426,6 +460,12 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 const float gl = (blk >= 0 && e < cnt) ? gate_s[e] : 0.f;
                 const float bias = gl - l2;
+                // keys t0 + k with k < lim are visible to this row
+                int lim = 0;
+                if (row_ok && blk >= 0) {
+                    lim = min(64, s.N - t0);
+                    if (causal && blk == w.j) lim = min(lim, qi - t0 + 1);
+                }
                 float dsum = 0.f;
                 uint32_t pk[32];
 #pragma unroll
@@ -433,9 +473,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     float ds2[2];
 #pragma unroll
                     for (int q2 = 0; q2 < 2; ++q2) {
-                        const int key = t0 + k + q2;
-                        const bool vis = row_ok && blk >= 0 && key < s.N && !(causal && blk == w.j && key > qi);
-                        const float p = vis ? ex2(fmaf(x[k + q2], sc2, bias)) : 0.f;
+                        const float p = k + q2 < lim ? ex2(fmaf(x[k + q2], sc2, bias)) : 0.f;
                         ds2[q2] = p * (y[k + q2] - Dr);
                         dsum += ds2[q2];
                     }
@@ -552,7 +590,7 @@ bool backward_tc_supported(const Shape &s) {
 }
 
 size_t backward_tc_workspace(const Shape &s) {
-    const size_t rows = (size_t)s.B * s.Hq * s.N;
+    const size_t rows = (size_t)s.B * s.Hq * s.nb * s.bs;
     const size_t units = (size_t)s.B * s.Hkv * s.nb;
     const int MT = s.G * s.bs / 128;
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -564,7 +602,8 @@ cudaError_t launch_backward_tc(const Shape &s, const void *Q, const void *K, con
                                const int32_t *count, float *dQ, float *dK, float *dV, float *dscore, void *ws,
                                cudaStream_t st) {
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    const size_t rows = (size_t)s.B * s.Hq * s.N;
+    const int Npad = s.nb * s.bs;
+    const size_t rows = (size_t)s.B * s.Hq * Npad;
     const size_t units = (size_t)s.B * s.Hkv * s.nb;
     const int MT = s.G * s.bs / 128;
     unsigned char *w = static_cast<unsigned char *>(ws) + ws_layout(s).scratch;
@@ -577,7 +616,7 @@ cudaError_t launch_backward_tc(const Shape &s, const void *Q, const void *K, con
     unsigned *status = static_cast<unsigned *>(ws);
 
     bwd_rowprep_kernel<<<(unsigned)((rows * 16 + 255) / 256), 256, 0, st>>>(
-        s, (const __nv_bfloat16 *)O, (const __nv_bfloat16 *)dO, lse, D, lse2, (long long)rows);
+        s, (const __nv_bfloat16 *)O, (const __nv_bfloat16 *)dO, lse, D, lse2, (long long)rows, Npad);
     note_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -602,6 +641,7 @@ cudaError_t launch_backward_tc(const Shape &s, const void *Q, const void *K, con
     a.dgp = dgp;
     a.status = status;
     a.MT = MT;
+    a.Npad = Npad;
     a.items = (int)(units * MT);
     a.wait_ns = kWaitNs;
     const int sms = sm_count();

@@ -128,7 +128,14 @@ typedef struct {
  * status word).  The workspace must be zero-filled once when allocated; the
  * library leaves the status word zero unless a device-side problem occurs,
  * and returns every completion counter it keeps there to zero by the end of
- * each call.  Calls that share a workspace must not overlap on the GPU.  */
+ * each call.  Calls that share a workspace must not overlap on the GPU.
+ * Layout: the status word, then one counter region per operation that keeps
+ * counters (prefill selection, decode selection, backward key tiles), then
+ * scratch shared by all operations.  The regions are sized from the
+ * parameters, so a workspace serves the operations of the parameter set it
+ * was sized for (any op, the largest size over the ops used); one sized for
+ * another set must not be reused unless it is at least as large for every op
+ * with the same geometry (same B, Hq, Hkv, N, block).  */
 size_t sparse_attn_workspace_size(const sa_params *p, int op);
 
 /* Landmarks (first step of the path; [HiLS] landmark, [LSA] keys pooled
