@@ -10,6 +10,24 @@
 
 namespace sa {
 
+// Launch that may start before the previous kernel on the stream has finished
+// (programmatic dependent launch); the kernel waits for its inputs on the
+// device (griddepcontrol.wait) before it reads what that kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // Status word at the start of every workspace: bit 1 = index list entry out
 // of range, bit 2 = NaN score, bit 4 = bounded wait expired.
 constexpr unsigned kStatusBadIndex = 1u;
@@ -182,10 +200,12 @@ cudaError_t launch_prefill_tc2(const Shape &s, const void *Q, const void *K, con
 bool decode_mma_supported(const Shape &s);
 void decode_mma_geometry(const Shape &s, int &S, int &bps);
 size_t decode_mma_partial_bytes(const Shape &s, int S);
-// Decode scratch passed explicitly: the status word and the split partials.
+int decode_mma_records(int S);
+// Decode scratch passed explicitly: the status word and the partial records
+// (R_out per unit, merged by the caller's merge launch).
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
-                              const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                              float *part, cudaStream_t st, int &S_out);
+                              const float *score, const int32_t *count, unsigned *status, float *part,
+                              cudaStream_t st, int &R_out);
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
                           float *part, cudaStream_t st);

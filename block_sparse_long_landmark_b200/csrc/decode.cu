@@ -236,6 +236,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_merge_kernel(DecArgs a) {
     const int u = blockIdx.x;
     const int hs = u % s.Hsel, b = u / s.Hsel;
     const int h0 = (s.flags & SA_SELECT_PER_QHEAD) ? hs : hs * s.G;
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // the records of the launch before this one
     const float *pp = a.part + (size_t)u * a.S * HP * (d + 2);
     for (int e = threadIdx.x; e < HP * d; e += kDecThreads) {
         const int hh = e / d, dim = e % d;
@@ -268,7 +269,6 @@ size_t decode_workspace(const Shape &s) {
     int S, bps;
     if (decode_mma_supported(s)) {
         decode_mma_geometry(s, S, bps);
-        if (S == 1) return 0;
         return decode_mma_partial_bytes(s, S);
     }
     split_geometry(s, S, bps);
@@ -311,14 +311,14 @@ cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const vo
     a.status = status;
     a.part = part;
     if (decode_mma_supported(s)) {
-        // tensor-core splits, then (when split) one merge CTA per unit
-        int S = 1;
-        cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, o, lse, status, part, st, S);
-        if (e != cudaSuccess || S == 1) return e;
-        a.S = S;
-        decode_merge_kernel<__nv_bfloat16><<<(unsigned)(s.B * s.Hsel), kDecThreads, 0, st>>>(a);
+        // tensor-core item records, then one merge CTA per unit
+        int R = 1;
+        cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, status, part, st, R);
+        if (e != cudaSuccess) return e;
+        a.S = R;
+        e = launch_pdl(decode_merge_kernel<__nv_bfloat16>, dim3((unsigned)(s.B * s.Hsel)), dim3(kDecThreads), 0, st, a);
         note_launch();
-        return cudaGetLastError();
+        return e != cudaSuccess ? e : cudaGetLastError();
     }
     split_geometry(s, a.S, a.bps);
     return s.dtype == SA_BF16 ? run<__nv_bfloat16>(a, st) : run<float>(a, st);
