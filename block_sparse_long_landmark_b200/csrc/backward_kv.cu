@@ -348,6 +348,20 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 en.y = __shfl_sync(0xffffffffu, mine.y, ui & 31);
                 en.z = __shfl_sync(0xffffffffu, mine.z, ui & 31);
                 en.w = 0;
+                // the Q and dO rows of the pair two ahead into L2 (its unit's entry is
+                // in this batch of 32 unless it starts the next one)
+                const int pa = p + 2, ua = pa / a.MT;
+                const int ja = __shfl_sync(0xffffffffu, mine.x, ua & 31);
+                if (lane < 2 && pa < np && (ua >> 5) == (ui >> 5)) {
+                    const int ma = pa % a.MT, e = lane;
+                    const int hh = s.bs == 64 ? 2 * ma + e : ma;
+                    const int pos = s.bs == 64 ? ja * 64 : ja * 128 + 64 * e;
+                    const int y = (b * s.Hq + g * s.G + hh) * s.N + pos;
+                    for (int c = 0; c < 2; ++c) {
+                        tma_prefetch_2d(&tmQ, 64 * c, y);
+                        tma_prefetch_2d(&tmDO, 64 * c, y);
+                    }
+                }
                 if (lane == 0) {
                     if (gp >= 2) ok = mbar_wait(bar(B_PE + st), ((gp >> 1) - 1) & 1, abort_flag, a.status, a.wait_ns);
                     if (ok) {

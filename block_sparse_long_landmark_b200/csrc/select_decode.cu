@@ -6,31 +6,36 @@
 // перебирать весь контекст"): the start of the context is always added.
 //
 // Decode scans every landmark of a sequence once per step, so the step is a
-// stream of landmarks from HBM.  Here each warp owns a chunk of 256
-// candidate blocks of one (batch, selection head): it averages the unit's
-// query heads (every lane its own 16-byte slice), streams the chunk's
-// landmarks with 16-byte loads (a VPR-lane group per row, eight rows per
-// group in flight), scores them in fp32 and takes the chunk's top-K with
-// the warp-level bitwise select (warp_select.cuh) -- no block-wide barrier,
-// so one warp's selection overlaps the other warps' streaming.  Warp 0 then
-// merges the CTA's eight chunk lists; when a unit spans several CTAs, each
-// leaves its list in the workspace and the unit's last CTA to finish merges
-// them.  The candidates sit in index order throughout and every select takes
-// equal keys at the lower position, so the result is the exact top-K by
-// (score desc, index asc) whatever the split.
+// stream of landmarks from HBM.  A CTA owns 2048 consecutive candidate blocks
+// of one (batch, selection head): a producer warp streams their landmarks in
+// 32 KB stages through a three-stage ring of bulk copies in shared memory, and
+// eight scoring warps each take an eighth of every stage.  Each lane holds a
+// 16-byte slice of the unit's pooled query and scores eight 16-byte slices per
+// stage; the partial dots are summed by a reduce-scatter across the lanes of
+// a row, so every lane ends with one full score.  Each warp then takes the
+// top-K of its 256 candidates with the warp-level bitwise select
+// (warp_select.cuh), warp 0 merges the CTA's eight lists, and when a unit spans
+// several CTAs each leaves its list in the workspace and the unit's last CTA to
+// finish merges them.  The candidates sit in index order throughout and every
+// select takes equal keys at the lower position, so the result is the exact
+// top-K by (score desc, index asc) whatever the split.
 #include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 #include "warp_select.cuh"
 
 namespace sa {
 namespace {
 
-constexpr int kSdThreads = 256;
-constexpr int kSdWarps = kSdThreads / 32;
-constexpr int kSdChunk = 256;        // candidates per warp
+constexpr int kSdWarps = 8;          // scoring warps; warp 8 streams
+constexpr int kSdThreads = 32 * (kSdWarps + 1);
+constexpr int kSdChunk = 256;        // candidates per scoring warp (its top-K)
 constexpr int kSdMaxMerge = 4096;    // candidates the cross-CTA merge holds in shared memory
+constexpr int kSdStage = 32768;      // bytes per ring stage: eight 16-byte slices per scoring lane
+constexpr int kSdStages = 3;
+constexpr uint32_t kSdRingBytes = (uint32_t)kSdStages * kSdStage;
 
 struct SdArgs {
     Shape s;
@@ -51,8 +56,17 @@ struct SdArgs {
 struct SdSmem {
     float s_special[2];
     int nv[kSdWarps];
-    int last;
+    int abort_flag;
+    uint64_t full[kSdStages], empty[kSdStages];
 };
+
+// Shared memory: header, keys [8][256], the ring [stages][32 KB], the CTA
+// merge area [8 * top_k] keys + ids, [top_k] positions.  Once the stream is
+// over the ring serves the warps' top-K positions, the final list and the
+// cross-CTA merge.
+__host__ __device__ constexpr size_t sd_off_keys() { return (sizeof(SdSmem) + 127) & ~(size_t)127; }
+__host__ __device__ constexpr size_t sd_off_ring() { return sd_off_keys() + (size_t)kSdWarps * kSdChunk * 4; }
+__host__ __device__ constexpr size_t sd_off_merge() { return sd_off_ring() + kSdRingBytes; }
 
 // Final list of unit u: [0 (sink)] + selected (ascending) + [local].
 __device__ void write_list(const SdArgs &a, int u, int local, const int *sel_idx, const uint32_t *sel_key, int nsel,
@@ -78,20 +92,42 @@ __device__ void write_list(const SdArgs &a, int u, int local, const int *sel_idx
     if ((threadIdx.x & 31) == 0) a.count[u] = cnt;
 }
 
+// fp32 slice of a 16-byte group of elements
+__device__ __forceinline__ void slice_f32(const uint4 &u, const __nv_bfloat16 *, float *f) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void slice_f32(const uint4 &u, const float *, float *f) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
+}
+
 template <typename T, int VPR>
-__global__ void __launch_bounds__(kSdThreads, 4) select_decode_kernel(SdArgs a) {
+__global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) {
+    using namespace tc;
     constexpr int EPV = Vec<T>::n;
-    constexpr int RPW = 32 / VPR;            // rows per warp step
-    constexpr int U = 8;                     // steps in flight
+    constexpr int RB = VPR * 16;                    // bytes per row
+    constexpr int RPL = 32 / VPR;                   // rows per 16-byte load step of the warp
+    constexpr int ROWS = kSdStage / RB;             // rows per stage
+    constexpr int RW = ROWS / kSdWarps;             // rows per scoring warp per stage
+    constexpr int NL = RW / RPL;                    // load steps (partial dots) per lane per stage
+    constexpr int SPAN = VPR / NL;                  // lanes that end with the same row's score
+    static_assert(NL == 8 && SPAN >= 1, "stage geometry");
     const Shape &s = a.s;
     const int D = VPR * EPV;
-    extern __shared__ __align__(16) unsigned char smraw[];
+    extern __shared__ __align__(128) unsigned char smraw[];
     SdSmem &sm = *reinterpret_cast<SdSmem *>(smraw);
-    uint32_t *keys = reinterpret_cast<uint32_t *>(smraw + ((sizeof(SdSmem) + 15) & ~15));   // [8][256]
-    int *wpos = reinterpret_cast<int *>(keys + kSdWarps * kSdChunk);                          // [8][256]
-    uint32_t *mkey = reinterpret_cast<uint32_t *>(wpos + kSdWarps * kSdChunk);                // [merge]
-    int *midx = reinterpret_cast<int *>(mkey + max(kSdWarps, a.C) * s.top_k);                // [merge]
-    int *mpos = midx + max(kSdWarps, a.C) * s.top_k;                                          // [top_k]
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smraw + sd_off_keys());      // [2048]
+    unsigned char *ring = smraw + sd_off_ring();                                // [stages][32 KB]
+    uint32_t *mkey = reinterpret_cast<uint32_t *>(smraw + sd_off_merge());     // [8 * top_k]
+    int *midx = reinterpret_cast<int *>(mkey + kSdWarps * s.top_k);            // [8 * top_k]
+    int *mpos = midx + kSdWarps * s.top_k;                                      // [top_k]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.x / a.C, cta = blockIdx.x % a.C;
@@ -101,61 +137,118 @@ __global__ void __launch_bounds__(kSdThreads, 4) select_decode_kernel(SdArgs a) 
     const int hq0 = perq ? hs : hs * s.G;
     const int local = (seq_n(s, b) - 1) / s.bs;
     const int first = (s.flags & SA_SINK) ? 1 : 0;
-    const int ncand = max(0, local - first);
-    const int c0 = first + (cta * kSdWarps + warp) * kSdChunk;      // this warp's first candidate
-    const int n = max(0, min(local, c0 + kSdChunk) - c0);
+    const int cc0 = first + cta * kSdWarps * kSdChunk;              // the CTA's first candidate
+    const int ncta = max(0, min(local, cc0 + kSdWarps * kSdChunk) - cc0);
+    const int wsel = min(warp, kSdWarps - 1);
+    const int c0 = cc0 + wsel * kSdChunk;                           // a scoring warp's first candidate
+    const int n = max(0, min(ncta - wsel * kSdChunk, kSdChunk));
 
-    // the unit's pooled query: lane group member cv holds elements cv*EPV ..
-    const int sub = lane / VPR, cv = lane % VPR;
-    float qv[EPV];
-#pragma unroll
-    for (int i = 0; i < EPV; ++i) qv[i] = 0.f;
-    for (int hh = 0; hh < s.heads_per; ++hh) {
-        float f[EPV];
-        load16((const T *)a.q + ((size_t)b * s.Hq + hq0 + hh) * D + cv * EPV, f);
-#pragma unroll
-        for (int i = 0; i < EPV; ++i) qv[i] += f[i];
+    // the attention launch that follows may start as this grid's CTAs are placed
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kSdStages; ++i) {
+            mbar_init(smem_u32(&sm.full[i]), 1);
+            mbar_init(smem_u32(&sm.empty[i]), kSdWarps);
+        }
+        sm.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-#pragma unroll
-    for (int i = 0; i < EPV; ++i) qv[i] /= (float)s.heads_per;
-    const T *Lg = (const T *)a.L + ((size_t)b * s.Hkv + g) * s.nb * D;
+    __syncthreads();
 
-    // ---- this warp's chunk: scores, then its top-K -------------------------
-    uint32_t *kw = keys + warp * kSdChunk;
-    int *pw = wpos + warp * kSdChunk;
+    const T *Lg = (const T *)a.L + ((size_t)b * s.Hkv + g) * s.nb * D;
+    const size_t cbytes = (size_t)ncta * RB;                        // the CTA's landmark bytes
+    const int nst = (int)((cbytes + kSdStage - 1) / kSdStage);
+    uint32_t *kw = keys + wsel * kSdChunk;
     bool nan_seen = false;
-    for (int r0 = 0; r0 < n; r0 += RPW * U) {
-        uint4 raw[U];
+    float qv[EPV];
+    const int sub = lane / VPR, cv = lane % VPR;
+    if (warp == kSdWarps) {
+        // ---- producer: the CTA's landmarks, stage by stage --------------------
+        if (lane == 0) {
+            const unsigned char *src = reinterpret_cast<const unsigned char *>(Lg + (size_t)cc0 * D);
+            int issued = 0;
+            for (int i = 0; i < nst; ++i) {
+                const int st = i % kSdStages;
+                if (i >= kSdStages &&
+                    !mbar_wait(smem_u32(&sm.empty[st]), ((i / kSdStages) - 1) & 1, &sm.abort_flag, a.status))
+                    break;
+                const uint32_t bytes = (uint32_t)min((size_t)kSdStage, cbytes - (size_t)i * kSdStage);
+                mbar_expect_tx(smem_u32(&sm.full[st]), bytes);
+                bulk_load(smem_u32(ring + st * kSdStage), src + (size_t)i * kSdStage, bytes, smem_u32(&sm.full[st]));
+                issued = i + 1;
+            }
+            if (sm.abort_flag) {
+                // let the copies in flight land before the ring is reused
+                volatile int never = 0;
+                for (int i = max(0, issued - kSdStages); i < issued; ++i)
+                    mbar_wait(smem_u32(&sm.full[i % kSdStages]), (i / kSdStages) & 1, &never, a.status);
+            }
+        }
+    } else {
+        // ---- scoring warps -------------------------------------------------------
+        // the unit's pooled query: lane group member cv holds elements cv*EPV ..
 #pragma unroll
-        for (int uu = 0; uu < U; ++uu) {
-            const int r = min(r0 + sub + RPW * uu, n - 1);
-            raw[uu] = *reinterpret_cast<const uint4 *>(Lg + (size_t)(c0 + r) * D + cv * EPV);
+        for (int i = 0; i < EPV; ++i) qv[i] = 0.f;
+        for (int hh = 0; hh < s.heads_per; ++hh) {
+            float f[EPV];
+            load16((const T *)a.q + ((size_t)b * s.Hq + hq0 + hh) * D + cv * EPV, f);
+#pragma unroll
+            for (int i = 0; i < EPV; ++i) qv[i] += f[i];
         }
 #pragma unroll
-        for (int uu = 0; uu < U; ++uu) {
-            float f[EPV];
-            load16(reinterpret_cast<const T *>(&raw[uu]), f);
-            float dot = 0.f;
+        for (int i = 0; i < EPV; ++i) qv[i] /= (float)s.heads_per;
+        for (int i = 0; i < nst; ++i) {
+            const int st = i % kSdStages;
+            const bool ok = mbar_wait(smem_u32(&sm.full[st]), (i / kSdStages) & 1, &sm.abort_flag, a.status);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const unsigned char *stg = ring + st * kSdStage + warp * RW * RB;
+            float v[NL];
 #pragma unroll
-            for (int i = 0; i < EPV; ++i) dot = fmaf(qv[i], f[i], dot);
+            for (int l = 0; l < NL; ++l) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(stg + (l * RPL + sub) * RB + cv * 16);
+                float f[EPV];
+                slice_f32(raw, (const T *)nullptr, f);
+                float dot = 0.f;
 #pragma unroll
-            for (int o = VPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            const int r = r0 + sub + RPW * uu;
-            if (cv == 0 && r < n) {
-                const float sc = s.scale * dot;
+                for (int e = 0; e < EPV; ++e) dot = fmaf(qv[e], f[e], dot);
+                v[l] = dot;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.empty[st]));
+            // reduce-scatter over the VPR lanes of a row: each halving step keeps
+            // half of the rows and adds the partner's partials for them
+#pragma unroll
+            for (int m = VPR / 2, cnt = NL; cnt > 1; m >>= 1, cnt >>= 1) {
+                const bool upper = cv & m;
+#pragma unroll
+                for (int k = 0; k < cnt / 2; ++k) {
+                    const float send = upper ? v[k] : v[k + cnt / 2];
+                    const float keep = upper ? v[k + cnt / 2] : v[k];
+                    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+#pragma unroll
+            for (int m = SPAN / 2; m > 0; m >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+            // the row this lane's score belongs to, as an offset in the CTA's candidates
+            const int r = i * ROWS + warp * RW + (cv / SPAN) * RPL + sub;
+            if (cv % SPAN == 0 && r < ncta) {
+                const float sc = s.scale * v[0];
                 nan_seen |= isnan(sc);
-                kw[r] = ord_key(sc);
+                keys[r] = ord_key(sc);
             }
         }
     }
-    __syncwarp();
-    const int nsel = warp_topk_positions<8>(kw, n, s.top_k, pw);
-    // the warp's list (ascending block ids) into the CTA's merge area
-    for (int i = lane; i < nsel; i += 32) {
-        mkey[warp * s.top_k + i] = kw[pw[i]];
-        midx[warp * s.top_k + i] = c0 + pw[i];
+    __syncthreads();
+    if (warp < kSdWarps) {
+        int *pw = reinterpret_cast<int *>(ring) + warp * kSdChunk;  // the warp's positions (the ring is free)
+        const int nsel = warp_topk_positions<8>(kw, n, s.top_k, pw);
+        // the warp's list (ascending block ids) into the CTA's merge area
+        for (int i = lane; i < nsel; i += 32) {
+            mkey[warp * s.top_k + i] = kw[pw[i]];
+            midx[warp * s.top_k + i] = c0 + pw[i];
+        }
+        if (lane == 0) sm.nv[warp] = nsel;
     }
-    if (lane == 0) sm.nv[warp] = nsel;
     // the sink and local scores (one warp of the unit's first CTA)
     if (cta == 0 && warp == 0) {
 #pragma unroll
@@ -202,10 +295,11 @@ __global__ void __launch_bounds__(kSdThreads, 4) select_decode_kernel(SdArgs a) 
         ntot += m;
     }
     const int nc = warp_topk_positions<8>(mkey, ntot, s.top_k, mpos);
+    // the final list's staging: the keys area is free once the warp lists are merged
+    uint32_t *sel_key = keys;
+    int *sel_idx = reinterpret_cast<int *>(keys + kSdChunk);
     if (a.C == 1) {
         // one CTA per unit: its list is the unit's
-        int *sel_idx = wpos;                    // reuse: this CTA's other buffers are free now
-        uint32_t *sel_key = keys;
         for (int i = lane; i < nc; i += 32) {
             sel_idx[i] = midx[mpos[i]];
             sel_key[i] = mkey[mpos[i]];
@@ -237,29 +331,30 @@ __global__ void __launch_bounds__(kSdThreads, 4) select_decode_kernel(SdArgs a) 
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
     __threadfence();
+    // the unit's C lists into the ring space (every stream of this CTA is over)
+    uint32_t *xkey = reinterpret_cast<uint32_t *>(ring);            // [C * top_k]
+    int *xidx = reinterpret_cast<int *>(xkey + (size_t)a.C * s.top_k);
+    int *xpos = xidx + (size_t)a.C * s.top_k;                        // [top_k]
     ntot = 0;
     for (int c = 0; c < a.C; ++c) {
         const int m = __ldcg(a.pcnt + (size_t)u * a.C + c);
         for (int i = lane; i < m; i += 32) {
             const size_t src = ((size_t)u * a.C + c) * s.top_k + i;
-            mkey[ntot + i] = __ldcg(a.pkey + src);
-            midx[ntot + i] = __ldcg(a.pidx + src);
+            xkey[ntot + i] = __ldcg(a.pkey + src);
+            xidx[ntot + i] = __ldcg(a.pidx + src);
         }
         ntot += m;
     }
     __syncwarp();
-    const int nf = warp_topk_positions<0>(mkey, ntot, s.top_k, mpos);
-    int *sel_idx = wpos;
-    uint32_t *sel_key = keys;
+    const int nf = warp_topk_positions<0>(xkey, ntot, s.top_k, xpos);
     for (int i = lane; i < nf; i += 32) {
-        sel_idx[i] = midx[mpos[i]];
-        sel_key[i] = mkey[mpos[i]];
+        sel_idx[i] = xidx[xpos[i]];
+        sel_key[i] = xkey[xpos[i]];
     }
     __syncwarp();
     write_list(a, u, local, sel_idx, sel_key, nf, __ldcg(a.special + (size_t)u * 2),
                __ldcg(a.special + (size_t)u * 2 + 1));
     if (lane == 0) a.done[u] = 0u;
-    (void)ncand;
 }
 
 }  // namespace
@@ -293,9 +388,9 @@ size_t select_decode_workspace(const Shape &s) {
     return units * C * s.top_k * 8 + units * C * 4 + units * 2 * 4 + 4 * 256;
 }
 
-static size_t sd_smem(const Shape &s, int C) {
-    const size_t merge = (size_t)max(kSdWarps, C) * s.top_k;
-    return ((sizeof(SdSmem) + 15) & ~(size_t)15) + (size_t)kSdWarps * kSdChunk * 8 + merge * 8 + (size_t)s.top_k * 4;
+static size_t sd_smem(const Shape &s) {
+    static_assert((size_t)kSdMaxMerge * 8 + kSdChunk * 4 <= kSdRingBytes, "cross-CTA merge fits the ring space");
+    return sd_off_merge() + (size_t)kSdWarps * s.top_k * 8 + (size_t)s.top_k * 4;
 }
 
 template <typename T>
@@ -332,7 +427,7 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
         case 32: kern = select_decode_kernel<T, 32>; break;
         default: return cudaErrorInvalidValue;
     }
-    const size_t smem = sd_smem(s, a.C);
+    const size_t smem = sd_smem(s);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(units * a.C), kSdThreads, smem, st>>>(a);
