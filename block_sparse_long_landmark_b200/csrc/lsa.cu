@@ -135,24 +135,26 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_build_kernel(LsaShape s, cons
 
 // Kernel 2 (flat decode, step 1): one CTA per (batch, kv-head, chunk of
 // centres).  Pooled query of the kv-group's heads (fp64), score of every
-// centre of the chunk, scale * <q, centre> in fp64, the chunk's best
-// min(top, chunk) by (score desc, id asc); the last chunk CTA of a (batch,
-// kv-head) merges the chunks' candidates into the chosen clusters and
-// expands them into key ranges.
+// centre of the chunk, scale * <q, centre> in fp64; the chunk passes all its
+// scores to the merge, or, when the merge could not hold every centre, its
+// best kk by (score desc, id asc).  The last chunk CTA of a (batch, kv-head)
+// takes the top_clusters best of the candidates with a block-wide radix
+// select and expands them into the flat list of kept key positions.
 template <typename T>
 __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     extern __shared__ __align__(16) unsigned char smraw[];
     const LsaShape &s = a.s;
     const LsaDecPlan &pl = a.pl;
     double *qbar = reinterpret_cast<double *>(smraw);                           // [d]
-    uint64_t *red64 = reinterpret_cast<uint64_t *>(qbar + s.d);                 // [16]
-    int *red = reinterpret_cast<int *>(red64 + 16);                             // [8]
+    int *red = reinterpret_cast<int *>(qbar + s.d);                             // [8]
     int *flag = red + 8;                                                        // [8]
-    uint64_t *keys = reinterpret_cast<uint64_t *>(flag + 8);                    // [max(CH, S*kk)]
+    int *hist = flag + 8;                                                       // [264]
+    uint64_t *keys = reinterpret_cast<uint64_t *>(hist + 264);                  // [max(CH, S*kk)]
     const int kmax = max(pl.CH, pl.S * pl.kk);
     int *ids = reinterpret_cast<int *>(keys + kmax);                            // [max(CH, S*kk)]
     int *pos = ids + kmax;                                                      // [max(CH, S*kk)]
     int *chosen = pos + kmax;                                                   // [ntop]
+    int *off = chosen + pl.ntop;                                                // [ntop + 1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bg = blockIdx.x / pl.S, chunk = blockIdx.x % pl.S;
     const int b = bg / s.Hkv, g = bg % s.Hkv;
@@ -196,66 +198,62 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     }
     if (nan_seen) set_status(a.status, kStatusNaN);
     __syncthreads();
-    // the chunk's top-kk by one warp, shared through `flag`
-    if (warp == 0) {
-        const int c = warp_topk64(keys, n, pl.kk, pos);
-        if (lane == 0) flag[1] = c;
-    }
-    __syncthreads();
-    const int nsel = flag[1];
-    if (pl.S > 1) {
-        // the chunk's candidates (ascending id) for the merge
-        uint64_t *pk = a.pkey + ((size_t)bg * pl.S + chunk) * pl.kk;
-        int32_t *pi = a.pid + ((size_t)bg * pl.S + chunk) * pl.kk;
-        for (int i = tid; i < nsel; i += kLsaThreads) {
-            pk[i] = keys[pos[i]];
-            pi[i] = c0 + pos[i];
-        }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) flag[0] = atomicAdd(a.done1 + bg, 1u) == (unsigned)(pl.S - 1);
-        __syncthreads();
-        if (!flag[0]) return;
-        __threadfence();
-        // merge: chunk c holds min(kk, its centres) candidates, packed in chunk order
-        int ntot = 0;
-        for (int c = 0; c < pl.S; ++c) ntot += min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
-        for (int e = tid; e < pl.S * pl.kk; e += kLsaThreads) {
-            const int c = e / pl.kk, i = e % pl.kk;
-            const int nv = min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
-            if (i < nv) {
-                int base = 0;
-                for (int x = 0; x < c; ++x) base += min(pl.kk, max(0, min(s.ctotal, (x + 1) * pl.CH) - x * pl.CH));
-                const size_t src = ((size_t)bg * pl.S + c) * pl.kk + i;
-                keys[base + i] = __ldcg(reinterpret_cast<const unsigned long long *>(a.pkey) + src);
-                ids[base + i] = __ldcg(a.pid + src);
-            }
-        }
-        __syncthreads();
-        if (warp == 0) {
-            const int c = warp_topk64(keys, ntot, pl.ntop, pos);
-            if (lane == 0) flag[2] = c;
-        }
-        __syncthreads();
-        const int nfin = flag[2];
-        for (int i = tid; i < nfin; i += kLsaThreads) chosen[i] = ids[pos[i]];
-        if (tid == 0) a.done1[bg] = 0u;
-        __syncthreads();
-        expand_ranges(a, bg, chosen, nfin, red);
-    } else {
+    if (pl.S == 1) {
+        const int nsel = block_topk64(keys, n, pl.ntop, pos, hist, red);
         for (int i = tid; i < nsel; i += kLsaThreads) chosen[i] = c0 + pos[i];
         __syncthreads();
-        expand_ranges(a, bg, chosen, nsel, red);
+        expand_positions(a, bg, chosen, nsel, off, red);
+        return;
     }
+    // the chunk's candidates (ascending id) for the merge: every score, or its best kk
+    int nsel = n;
+    if (pl.kk < pl.CH) {
+        nsel = block_topk64(keys, n, pl.kk, pos, hist, red);
+    } else {
+        for (int i = tid; i < n; i += kLsaThreads) pos[i] = i;
+        __syncthreads();
+    }
+    uint64_t *pk = a.pkey + ((size_t)bg * pl.S + chunk) * pl.kk;
+    int32_t *pi = a.pid + ((size_t)bg * pl.S + chunk) * pl.kk;
+    for (int i = tid; i < nsel; i += kLsaThreads) {
+        pk[i] = keys[pos[i]];
+        pi[i] = c0 + pos[i];
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) flag[0] = atomicAdd(a.done1 + bg, 1u) == (unsigned)(pl.S - 1);
+    __syncthreads();
+    if (!flag[0]) return;
+    __threadfence();
+    // merge: chunk c holds min(kk, its centres) candidates, packed in chunk order
+    int ntot = 0;
+    for (int c = 0; c < pl.S; ++c) ntot += min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
+    for (int e = tid; e < pl.S * pl.kk; e += kLsaThreads) {
+        const int c = e / pl.kk, i = e % pl.kk;
+        const int nv = min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
+        if (i < nv) {
+            // chunks before the last are full: c * min(kk, CH) candidates precede chunk c
+            const int base = c * min(pl.kk, pl.CH);
+            const size_t src = ((size_t)bg * pl.S + c) * pl.kk + i;
+            keys[base + i] = __ldcg(reinterpret_cast<const unsigned long long *>(a.pkey) + src);
+            ids[base + i] = __ldcg(a.pid + src);
+        }
+    }
+    __syncthreads();
+    const int nfin = block_topk64(keys, ntot, pl.ntop, pos, hist, red);
+    for (int i = tid; i < nfin; i += kLsaThreads) chosen[i] = ids[pos[i]];
+    if (tid == 0) a.done1[bg] = 0u;
+    __syncthreads();
+    expand_positions(a, bg, chosen, nfin, off, red);
 }
 
 // Kernel 3 (flat decode, step 2): P CTAs per (batch, kv-head), each taking
 // an equal share of the kept positions and walking it in rounds: a round's
-// positions are laid out in shared memory from the ranges, then a VPR-lane
-// group per key row streams K and V with 16-byte loads and keeps an online
-// softmax (fp32, exp2 domain) per query head of the pass.  Lane groups,
-// warps and finally the CTAs of a (batch, kv-head) are merged by
-// log-sum-exp; the last CTA writes o and lse.
+// positions are staged in shared memory from the flat list, then a VPR-lane
+// group per key row streams K and V with 16-byte loads (four rows per group
+// in flight) and keeps an online softmax (fp32, exp2 domain) per query head of
+// the pass.  Lane groups, warps and finally the CTAs of a (batch, kv-head) are
+// merged by log-sum-exp; the last CTA writes o and lse.
 template <typename T, int HG>
 __global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
     constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
@@ -272,10 +270,10 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
     float *wst = reinterpret_cast<float *>(posv + ((pl.slice + 3) & ~3));      // [8 warps][HG][D + 2]
     int *misc = reinterpret_cast<int *>(wst + (kLsaThreads / 32) * HG * (D + 2));   // [4]
 
-    const int nr = a.cnt[2 * (size_t)bg], tot = a.cnt[2 * (size_t)bg + 1];
+    const int tot = a.cnt[2 * (size_t)bg + 1];
     // this CTA's share of the kept positions, walked in rounds of pl.slice
     const int t0 = (int)((long long)tot * pi / pl.P), t1 = (int)((long long)tot * (pi + 1) / pl.P);
-    const int32_t *rs = a.rs + (size_t)bg * pl.rmax, *rl = a.rl + (size_t)bg * pl.rmax, *rp = a.rp + (size_t)bg * pl.rmax;
+    const int32_t *plist = a.pos + (size_t)bg * pl.pmax;
     const T *Kb = (const T *)a.K + (size_t)bg * s.N * D;
     const T *Vb = (const T *)a.V + (size_t)bg * s.N * D;
     const float sl2 = s.scale * kLog2e;
@@ -297,33 +295,13 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
         for (int r0 = t0; r0 < t1; r0 += pl.slice) {
             const int r1 = min(t1, r0 + pl.slice);
             __syncthreads();                             // the previous round's positions are read
-            if (tid == 0) {
-                // ranges [q0, q1) overlap [r0, r1): rp ascending, every length > 0
-                int lo = 0, hi = nr;                     // first range with rp + rl > r0
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (rp[mid] + rl[mid] > r0) hi = mid; else lo = mid + 1;
-                }
-                misc[0] = lo;
-                hi = nr;                                 // first range with rp >= r1
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (rp[mid] >= r1) hi = mid; else lo = mid + 1;
-                }
-                misc[1] = lo;
-            }
-            __syncthreads();
-            for (int r = misc[0] + warp; r < misc[1]; r += kLsaThreads / 32) {
-                const int st = rs[r], pre = rp[r], len = rl[r];
-                const int from = max(r0, pre), to = min(r1, pre + len);
-                for (int v = from + lane; v < to; v += 32) posv[v - r0] = st + (v - pre);
-            }
+            for (int i = tid; i < r1 - r0; i += kLsaThreads) posv[i] = plist[r0 + i];
             __syncthreads();
             const int np = r1 - r0;
             // rows of this lane group: vb + sub + u * RPW * 8 for the warp's bases vb
             // (the trip count is the same for every lane: the row reductions
             // shuffle over the whole warp); two rows per group in flight
-            constexpr int U = 2, NW = kLsaThreads / 32;
+            constexpr int U = 4, NW = kLsaThreads / 32;
             for (int vb = warp * RPW; vb < np; vb += U * RPW * NW) {
                 uint4 kr[U], vr[U];
 #pragma unroll
@@ -458,25 +436,33 @@ bool lsa_decode_plan(const LsaShape &s, LsaDecPlan &pl, bool chunks) {
         // nothing to choose: one CTA per (batch, kv-head) lays out the sink and the window
         pl.CH = 0;
         pl.S = 1;
+        pl.kk = 0;
     } else {
-        // chunks of 128 centres, grown until the merge's candidates fit one CTA
+        // chunks of 128 centres; the merge takes every score when it can hold
+        // them all (C <= 4096), else each chunk passes its best min(top, CH),
+        // the chunks grown until the merge's candidates fit one CTA
         pl.CH = 128;
         pl.S = max(1, (C + pl.CH - 1) / pl.CH);
-        while (pl.S > 1 && (long long)pl.S * min(top, pl.CH) > 12288 && pl.CH < 8192) {
-            pl.CH *= 2;
-            pl.S = max(1, (C + pl.CH - 1) / pl.CH);
+        if (C <= 4096) {
+            pl.kk = pl.CH;
+        } else {
+            while (pl.S > 1 && (long long)pl.S * min(top, pl.CH) > 12288 && pl.CH < 8192) {
+                pl.CH *= 2;
+                pl.S = max(1, (C + pl.CH - 1) / pl.CH);
+            }
+            pl.kk = min(top, pl.CH);
         }
     }
-    pl.kk = min(top, pl.CH);
     if (pl.CH > 8192 || (pl.S > 1 && (long long)pl.S * pl.kk > 12288)) return false;
-    pl.rmax = 2 + pl.ntop * s.seg;
     const long long sink_n = min(s.sink, s.N);
-    const long long bound = min((long long)s.N, sink_n + (long long)s.window + (long long)pl.ntop * s.seg * s.pool);
+    // what the expansion can write even for an index whose clusters share items
+    const long long bound = sink_n + min((long long)s.window, (long long)s.N) + (long long)pl.ntop * s.seg * s.pool;
+    if (bound > (1LL << 30)) return false;
+    pl.pmax = (int)max(1LL, bound);
     const int bgs = s.B * s.Hkv;
-    // about two CTAs per SM overall, but at least 64 positions per CTA at the bound;
-    // each CTA walks its share in rounds of `slice` positions laid out in shared memory
-    long long P = min(64LL, (296LL + bgs - 1) / bgs);
-    P = min(P, (bound + 63) / 64);
+    // about four CTAs per SM overall, but at least 32 positions per CTA at the bound
+    long long P = min(64LL, (4LL * 148 + bgs - 1) / bgs);
+    P = min(P, (bound + 31) / 32);
     pl.P = (int)max(1LL, P);
     pl.slice = 1024;
     pl.HG = s.G >= 8 ? 8 : s.G >= 4 ? 4 : s.G >= 2 ? 2 : 1;
@@ -485,9 +471,7 @@ bool lsa_decode_plan(const LsaShape &s, LsaDecPlan &pl, bool chunks) {
     pl.off_key = off;   off += al((size_t)bgs * pl.S * max(1, pl.kk) * 8);
     pl.off_id = off;    off += al((size_t)bgs * pl.S * max(1, pl.kk) * 4);
     pl.off_done1 = off; off += al((size_t)bgs * 4);
-    pl.off_rs = off;    off += al((size_t)bgs * pl.rmax * 4);
-    pl.off_rl = off;    off += al((size_t)bgs * pl.rmax * 4);
-    pl.off_rp = off;    off += al((size_t)bgs * pl.rmax * 4);
+    pl.off_pos = off;   off += al((size_t)bgs * pl.pmax * 4);
     pl.off_cnt = off;   off += al((size_t)bgs * 8);
     pl.off_part = off;  off += al((size_t)bgs * pl.P * s.G * (s.d + 2) * 4);
     pl.off_done2 = off; off += al((size_t)bgs * 4);
@@ -497,7 +481,7 @@ bool lsa_decode_plan(const LsaShape &s, LsaDecPlan &pl, bool chunks) {
 
 static size_t select_smem(const LsaShape &s, const LsaDecPlan &pl) {
     const size_t kmax = (size_t)max(pl.CH, pl.S * pl.kk);
-    return sizeof(double) * s.d + 16 * 8 + 16 * 4 + kmax * (8 + 4 + 4) + (size_t)max(1, pl.ntop) * 4;
+    return sizeof(double) * s.d + (8 + 8 + 264) * 4 + kmax * (8 + 4 + 4) + (2 * (size_t)pl.ntop + 1) * 4;
 }
 
 static size_t attend_smem(const LsaShape &s, const LsaDecPlan &pl) {
@@ -534,9 +518,7 @@ void lsa_bind_workspace(LsaDecArgs &a, void *ws) {
     a.pkey = reinterpret_cast<uint64_t *>(w + pl.off_key);
     a.pid = reinterpret_cast<int32_t *>(w + pl.off_id);
     a.done1 = reinterpret_cast<unsigned *>(w + pl.off_done1);
-    a.rs = reinterpret_cast<int32_t *>(w + pl.off_rs);
-    a.rl = reinterpret_cast<int32_t *>(w + pl.off_rl);
-    a.rp = reinterpret_cast<int32_t *>(w + pl.off_rp);
+    a.pos = reinterpret_cast<int32_t *>(w + pl.off_pos);
     a.cnt = reinterpret_cast<int32_t *>(w + pl.off_cnt);
     a.part = reinterpret_cast<float *>(w + pl.off_part);
     a.done2 = reinterpret_cast<unsigned *>(w + pl.off_done2);

@@ -19,13 +19,14 @@ struct LsaShape {
 struct LsaDecPlan {
     int S;           // centre-score chunks per (batch, kv-head)
     int CH;          // centres per chunk
-    int kk;          // candidates a chunk keeps: min(top_clusters, CH)
+    int kk;          // candidates a chunk passes to the merge: CH when the merge holds every
+                     // centre, else min(top_clusters, CH)
     int ntop;        // clusters chosen: min(top_clusters, ctotal)
-    int rmax;        // key ranges per (batch, kv-head): sink + window + ntop * seg items
+    int pmax;        // kept key positions per (batch, kv-head), at most
     int P;           // attention CTAs per (batch, kv-head)
-    int slice;       // key positions an attention CTA lays out per round
+    int slice;       // key positions an attention CTA stages per round
     int HG;          // query heads per attention pass (1, 2, 4 or 8)
-    size_t off_key, off_id, off_done1, off_rs, off_rl, off_rp, off_cnt, off_part, off_done2, bytes;
+    size_t off_key, off_id, off_done1, off_pos, off_cnt, off_part, off_done2, bytes;
 };
 
 struct LsaDecArgs {
@@ -38,8 +39,8 @@ struct LsaDecArgs {
     uint64_t *pkey;       // [B*Hkv][S][kk] chunk candidates (keys)
     int32_t *pid;         // [B*Hkv][S][kk] chunk candidates (cluster ids)
     unsigned *done1;      // [B*Hkv] score chunks finished; back to 0 by the merging CTA
-    int32_t *rs, *rl, *rp;   // [B*Hkv][rmax] key ranges: start, length, exclusive prefix of lengths
-    int32_t *cnt;         // [B*Hkv][2]: ranges, kept positions
+    int32_t *pos;         // [B*Hkv][pmax] kept key positions
+    int32_t *cnt;         // [B*Hkv][2]: kept positions (twice)
     float *part;          // [B*Hkv][P][G][d + 2] attention partials (m, l, acc)
     unsigned *done2;      // [B*Hkv] attention CTAs finished; back to 0 by the merging CTA
     void *o;
@@ -77,7 +78,7 @@ cudaError_t launch_lsa_tree_decode(const LsaShape &s, const LsaDecPlan &pl, cons
 
 cudaError_t launch_lsa_build(const LsaShape &s, const void *K, double *centres, int32_t *members, int32_t *sizes,
                              cudaStream_t st);
-// Step 2 of a decode through the index: attention over the key ranges that
+// Step 2 of a decode through the index: attention over the key positions that
 // step 1 (flat scan or tree search) left in the workspace.
 cudaError_t launch_lsa_attend(const LsaDecArgs &a, cudaStream_t st);
 // Workspace pointers of a decode (layout of `pl`) filled into `a`.

@@ -11,7 +11,7 @@
 // node's centre is the mass-weighted mean of its children's centres.  The
 // search keeps the `beam` best nodes of a level by (score desc, id asc),
 // descends into their children, and at the leaves keeps the `top_clusters`
-// best, which are then expanded to key ranges exactly as in the flat decode.
+// best, which are then expanded to key positions exactly as in the flat decode.
 //
 // Build: one CTA per (batch, kv-head), level by level.  Ward's merges run in
 // fp64 with a cached nearest neighbour per node: the all-pairs start stages
@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_tree_build_kernel(TreeArgs a)
 
 // Beam search of one (batch, kv-head): the pooled query scored against the
 // top level's nodes, the `beam` best of each level expanded into their
-// children, the `top_clusters` best leaves expanded to key ranges.
+// children, the `top_clusters` best leaves expanded to key positions.
 struct TreeSelArgs {
     LsaDecArgs d;
     LsaTreePlan tp;
@@ -441,13 +441,14 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_tree_select_kernel(TreeSelArg
     const LsaTreePlan &tp = ta.tp;
     const int F = tp.maxfront;
     double *qbar = reinterpret_cast<double *>(smraw);                 // [d]
-    uint64_t *red64 = reinterpret_cast<uint64_t *>(qbar + s.d);       // [16]
-    int *red = reinterpret_cast<int *>(red64 + 16);                   // [8]
+    int *red = reinterpret_cast<int *>(qbar + s.d);                   // [8]
     int *misc = red + 8;                                              // [8]
-    uint64_t *keys = reinterpret_cast<uint64_t *>(misc + 8);          // [F]
+    int *hist = misc + 8;                                             // [264]
+    uint64_t *keys = reinterpret_cast<uint64_t *>(hist + 264);        // [F]
     int *fr = reinterpret_cast<int *>(keys + F);                      // [F] frontier, ascending ids
     int *pos = fr + F;                                                // [F]
     int *mark = pos + F;                                              // [F]
+    int *off = mark + F;                                              // [F + 1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bg = blockIdx.x, b = bg / s.Hkv, g = bg % s.Hkv;
     const int D = s.d;
@@ -467,31 +468,35 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_tree_select_kernel(TreeSelArg
         const double *cen = lv == 0 ? a.centres + (size_t)bg * s.ctotal * D
                                     : reinterpret_cast<const double *>(ta.tree + tp.off_cent[lv]) +
                                           (size_t)bg * tp.n[lv] * D;
-        for (int i = warp; i < nf; i += kLsaThreads / 32) {
-            const double *row = cen + (size_t)fr[i] * D;
-            double acc = 0.0;
-            for (int e = lane; e < D; e += 32) acc = fma(row[e], qbar[e], acc);
-            acc = warp_total(acc);
-            if (lane == 0) {
-                const double sc = (double)s.scale * acc;
-                nan_seen |= isnan(sc);
-                keys[i] = ord_key64(sc);
+        // a warp per centre, four centres of the frontier in flight per warp
+        for (int i0 = warp * 4; i0 < nf; i0 += 4 * (kLsaThreads / 32)) {
+            double part[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const double *row = cen + (size_t)fr[min(i0 + u, nf - 1)] * D;
+                double acc = 0.0;
+                for (int e = lane; e < D; e += 32) acc = fma(row[e], qbar[e], acc);
+                part[u] = acc;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const double acc = warp_total(part[u]);
+                if (lane == 0 && i0 + u < nf) {
+                    const double sc = (double)s.scale * acc;
+                    nan_seen |= isnan(sc);
+                    keys[i0 + u] = ord_key64(sc);
+                }
             }
         }
         compared += nf;
         __syncthreads();
         const int keep = lv > 0 ? ta.beam : min(s.top_clusters, s.ctotal);
-        if (warp == 0) {
-            const int c = warp_topk64(keys, nf, keep, pos);
-            if (lane == 0) misc[0] = c;
-        }
-        __syncthreads();
-        const int nk = misc[0];
+        const int nk = block_topk64(keys, nf, keep, pos, hist, red);
         if (lv == 0) {
-            // the chosen leaves (ascending ids) go to the range expansion; `mark` holds them
+            // the chosen leaves (ascending ids) go to the position expansion; `mark` holds them
             for (int i = tid; i < nk; i += kLsaThreads) mark[i] = fr[pos[i]];
             __syncthreads();
-            expand_ranges(a, bg, mark, nk, red);
+            expand_positions(a, bg, mark, nk, off, red);
             break;
         }
         // next frontier: the children of the kept nodes, in ascending id order
@@ -565,7 +570,7 @@ static size_t tree_build_smem(const LsaShape &s, const LsaTreePlan &tp) {
 }
 
 static size_t tree_select_smem(const LsaShape &s, const LsaTreePlan &tp) {
-    return (size_t)s.d * 8 + 16 * 8 + 16 * 4 + (size_t)tp.maxfront * (8 + 4 + 4 + 4);
+    return (size_t)s.d * 8 + (8 + 8 + 264) * 4 + (size_t)tp.maxfront * (8 + 4 + 4 + 4 + 4) + 4;
 }
 
 cudaError_t launch_lsa_tree_build(const LsaShape &s, const LsaTreePlan &tp, const double *centres,

@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
         }
         ntot += m;
     }
-    const int nc = warp_topk_positions<8>(mkey, ntot, s.top_k, mpos);
+    const int nc = warp_topk_positions<16>(mkey, ntot, s.top_k, mpos);
     // the final list's staging: the keys area is free once the warp lists are merged
     uint32_t *sel_key = keys;
     int *sel_idx = reinterpret_cast<int *>(keys + kSdChunk);
@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
         ntot += m;
     }
     __syncwarp();
-    const int nf = warp_topk_positions<0>(xkey, ntot, s.top_k, xpos);
+    const int nf = warp_topk_positions<16>(xkey, ntot, s.top_k, xpos);
     for (int i = lane; i < nf; i += 32) {
         sel_idx[i] = xidx[xpos[i]];
         sel_key[i] = xkey[xpos[i]];

@@ -317,8 +317,8 @@ int sparse_attn_lsa_clusters(const sa_lsa_params *p);
 
 /* Workspace bytes for sparse_attn_lsa_decode, 0 when the parameters are
  * invalid or unsupported.  Holds the status word, the chunks' candidate
- * clusters, the kept key ranges, the split attention partials and two
- * completion counters; zero-fill it once when allocated (the counters are
+ * clusters, the list of kept key positions, the split attention partials and
+ * two completion counters; zero-fill it once when allocated (the counters are
  * returned to zero by every call).  Calls sharing a workspace must not
  * overlap on the GPU. */
 size_t sparse_attn_lsa_workspace_size(const sa_lsa_params *p);
@@ -335,8 +335,9 @@ int sparse_attn_lsa_build(const sa_lsa_params *p, const void *K, double *centres
  * log; -inf when nothing is kept), and, when `kept` is not NULL, the number
  * of key positions each (batch, kv-head) attended to (int32 [B,Hkv]).
  * Two kernels: centre scores (fp64) in chunks over many CTAs with an exact
- * top_clusters merge, expanded to key ranges; then the kept keys split over
- * many CTAs with a log-sum-exp merge.  The merge of the chunks' candidates
+ * top_clusters merge (a block-wide radix select), expanded to the list of
+ * kept key positions; then the kept keys split over many CTAs with a
+ * log-sum-exp merge.  The merge of the chunks' candidates
  * runs in one CTA: parameters with top_clusters x ceil(C / 8192) > 12288
  * (C = clusters per (batch, kv-head)) return SA_ERR_UNSUPPORTED.  A member
  * entry outside the complete segments sets status bit 1 and is skipped; a
@@ -381,7 +382,7 @@ int sparse_attn_lsa_tree_build(const sa_lsa_params *p, int fanout, const double 
                                void *tree, void *ws, size_t ws_bytes, void *stream);
 
 /* Decode through the tree: beam search (beam >= 1) down to the leaves, the
- * `top_clusters` best leaves expanded to key ranges with the sink and
+ * `top_clusters` best leaves expanded to key positions with the sink and
  * window, then attention as in sparse_attn_lsa_decode.  Outputs o, lse and,
  * when not NULL, kept [B,Hkv] (key positions attended) and compared [B,Hkv]
  * (centres scored on the way down). */
