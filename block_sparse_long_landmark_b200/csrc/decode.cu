@@ -228,33 +228,68 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecArgs a) {
     }
 }
 
+// One CTA per unit: the unit's R = a.S partial records (m, l, acc[d] per
+// head) combined by log-sum-exp.  (m, l) of every record go to shared memory
+// first, then per head the max M and the sum L, then each record's weight
+// 2^(m - M); the accumulators are read with independent loads.
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads) decode_merge_kernel(DecArgs a) {
     constexpr float kLn2 = 0.6931471805599453f;
+    extern __shared__ float msm[];               // [R][HP] m, [R][HP] l, [HP] M, [HP] L
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // the records of the launch before this one
     const Shape &s = a.s;
-    const int d = s.d, HP = s.heads_per;
+    const int d = s.d, HP = s.heads_per, R = a.S;
     const int u = blockIdx.x;
     const int hs = u % s.Hsel, b = u / s.Hsel;
     const int h0 = (s.flags & SA_SELECT_PER_QHEAD) ? hs : hs * s.G;
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // the records of the launch before this one
-    const float *pp = a.part + (size_t)u * a.S * HP * (d + 2);
+    const float *pp = a.part + (size_t)u * R * HP * (d + 2);
+    float *wm = msm, *wl = wm + R * HP, *Mh = wl + R * HP, *Lh = Mh + HP;
+    for (int i = threadIdx.x; i < R * HP; i += kDecThreads) {
+        wm[i] = pp[(size_t)i * (d + 2)];
+        wl[i] = pp[(size_t)i * (d + 2) + 1];
+    }
+    __syncthreads();
+    for (int hh = threadIdx.x; hh < HP; hh += kDecThreads) {
+        float M = -CUDART_INF_F, L = 0.f;
+        for (int r = 0; r < R; ++r) M = fmaxf(M, wm[r * HP + hh]);
+        if (M != -CUDART_INF_F)
+            for (int r = 0; r < R; ++r)
+                if (wm[r * HP + hh] != -CUDART_INF_F) L = fmaf(wl[r * HP + hh], exp2f(wm[r * HP + hh] - M), L);
+        Mh[hh] = M;
+        Lh[hh] = L;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < R * HP; i += kDecThreads) {
+        const float M = Mh[i % HP];
+        wm[i] = (wm[i] == -CUDART_INF_F || M == -CUDART_INF_F) ? 0.f : exp2f(wm[i] - M);
+    }
+    __syncthreads();
     for (int e = threadIdx.x; e < HP * d; e += kDecThreads) {
         const int hh = e / d, dim = e % d;
-        float M = -CUDART_INF_F;
-        for (int sp = 0; sp < a.S; ++sp) M = fmaxf(M, pp[(sp * HP + hh) * (d + 2)]);
-        float L = 0.f, O = 0.f;
-        if (M != -CUDART_INF_F) {
-            for (int sp = 0; sp < a.S; ++sp) {
-                const float *q = pp + (sp * HP + hh) * (d + 2);
-                if (q[0] == -CUDART_INF_F) continue;
-                const float w = exp2f(q[0] - M);
-                L = fmaf(q[1], w, L);
-                O = fmaf(q[2 + dim], w, O);
-            }
-        }
+        float O = 0.f;
+#pragma unroll 4
+        for (int r = 0; r < R; ++r) O = fmaf(pp[((size_t)r * HP + hh) * (d + 2) + 2 + dim], wm[r * HP + hh], O);
+        const float L = Lh[hh];
         from_f(((T *)a.o)[((size_t)b * s.Hq + h0 + hh) * d + dim], L > 0.f ? O / L : 0.f);
-        if (dim == 0) a.lse[(size_t)b * s.Hq + h0 + hh] = L > 0.f ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
+        if (dim == 0) a.lse[(size_t)b * s.Hq + h0 + hh] = L > 0.f ? (Mh[hh] + log2f(L)) * kLn2 : -CUDART_INF_F;
     }
+}
+
+static size_t merge_smem(const Shape &s, int R) { return (2 * (size_t)R * s.heads_per + 2 * (size_t)s.heads_per) * 4; }
+
+template <typename T>
+static cudaError_t launch_merge(const DecArgs &a, cudaStream_t st, bool pdl) {
+    const size_t smem = merge_smem(a.s, a.S);
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(decode_merge_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const unsigned units = (unsigned)(a.s.B * a.s.Hsel);
+    cudaError_t e = pdl ? launch_pdl(decode_merge_kernel<T>, dim3(units), dim3(kDecThreads), smem, st, a)
+                        : (decode_merge_kernel<T><<<units, kDecThreads, smem, st>>>(a), cudaSuccess);
+    note_launch();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 static void split_geometry(const Shape &s, int &S, int &bps) {
@@ -290,9 +325,7 @@ static cudaError_t run(DecArgs a, cudaStream_t st) {
     note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess || a.S == 1) return e;
-    decode_merge_kernel<T><<<units, kDecThreads, 0, st>>>(a);
-    note_launch();
-    return cudaGetLastError();
+    return launch_merge<T>(a, st, false);
 }
 
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
@@ -316,9 +349,7 @@ cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const vo
         cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, status, part, st, R);
         if (e != cudaSuccess) return e;
         a.S = R;
-        e = launch_pdl(decode_merge_kernel<__nv_bfloat16>, dim3((unsigned)(s.B * s.Hsel)), dim3(kDecThreads), 0, st, a);
-        note_launch();
-        return e != cudaSuccess ? e : cudaGetLastError();
+        return launch_merge<__nv_bfloat16>(a, st, true);
     }
     split_geometry(s, a.S, a.bps);
     return s.dtype == SA_BF16 ? run<__nv_bfloat16>(a, st) : run<float>(a, st);

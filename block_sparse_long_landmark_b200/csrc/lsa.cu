@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
 // the pass.  Lane groups, warps and finally the CTAs of a (batch, kv-head) are
 // merged by log-sum-exp; the last CTA writes o and lse.
 template <typename T, int HG>
-__global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
+__global__ void __launch_bounds__(kLsaThreads, 2) lsa_attend_kernel(LsaDecArgs a) {
     constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
     constexpr int EPV = 16 / (int)sizeof(T);
     extern __shared__ __align__(16) unsigned char smraw[];
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
     const int b = bg / s.Hkv, g = bg % s.Hkv;
     int *posv = reinterpret_cast<int *>(smraw);                                // [slice]
     float *wst = reinterpret_cast<float *>(posv + ((pl.slice + 3) & ~3));      // [8 warps][HG][D + 2]
-    int *misc = reinterpret_cast<int *>(wst + (kLsaThreads / 32) * HG * (D + 2));   // [4]
+    int *misc = reinterpret_cast<int *>(wst + max((kLsaThreads / 32) * HG * (D + 2), 2 * pl.P * s.G + 2 * s.G));   // [4]
 
     const int tot = a.cnt[2 * (size_t)bg + 1];
     // this CTA's share of the kept positions, walked in rounds of pl.slice
@@ -387,21 +387,37 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_attend_kernel(LsaDecArgs a) {
     __syncthreads();
     if (!misc[2]) return;
     __threadfence();
+    // the P partials: (m, l) of each into shared memory, per head the max M and
+    // the sum L, then each partial's weight 2^(m - M); the accumulators are then
+    // read with independent loads
+    const float *pb = a.part + (size_t)bg * pl.P * s.G * (D + 2);
+    float *wm = wst, *wl = wm + pl.P * s.G, *Mh = wl + pl.P * s.G, *Lh = Mh + s.G;
+    for (int i = tid; i < pl.P * s.G; i += kLsaThreads) {
+        wm[i] = __ldcg(pb + (size_t)i * (D + 2));
+        wl[i] = __ldcg(pb + (size_t)i * (D + 2) + 1);
+    }
+    __syncthreads();
+    for (int h = tid; h < s.G; h += kLsaThreads) {
+        float M = -CUDART_INF_F, L = 0.f;
+        for (int p = 0; p < pl.P; ++p) M = fmaxf(M, wm[p * s.G + h]);
+        if (M != -CUDART_INF_F)
+            for (int p = 0; p < pl.P; ++p)
+                if (wm[p * s.G + h] != -CUDART_INF_F) L = fmaf(wl[p * s.G + h], exp2f(wm[p * s.G + h] - M), L);
+        Mh[h] = M;
+        Lh[h] = L;
+    }
+    __syncthreads();
+    for (int i = tid; i < pl.P * s.G; i += kLsaThreads) {
+        const float M = Mh[i % s.G];
+        wm[i] = (wm[i] == -CUDART_INF_F || M == -CUDART_INF_F) ? 0.f : exp2f(wm[i] - M);
+    }
+    __syncthreads();
     for (int x = tid; x < s.G * D; x += kLsaThreads) {
         const int h = x / D, e = x % D;
-        float M = -CUDART_INF_F;
-        for (int p = 0; p < pl.P; ++p) M = fmaxf(M, __ldcg(a.part + (((size_t)bg * pl.P + p) * s.G + h) * (D + 2)));
-        float L = 0.f, O = 0.f;
-        if (M != -CUDART_INF_F) {
-            for (int p = 0; p < pl.P; ++p) {
-                const float *pp = a.part + (((size_t)bg * pl.P + p) * s.G + h) * (D + 2);
-                const float mp = __ldcg(pp);
-                if (mp == -CUDART_INF_F) continue;
-                const float f = exp2f(mp - M);
-                L = fmaf(__ldcg(pp + 1), f, L);
-                O = fmaf(__ldcg(pp + 2 + e), f, O);
-            }
-        }
+        float O = 0.f;
+#pragma unroll 8
+        for (int p = 0; p < pl.P; ++p) O = fmaf(__ldcg(pb + ((size_t)p * s.G + h) * (D + 2) + 2 + e), wm[p * s.G + h], O);
+        const float M = Mh[h], L = Lh[h];
         const size_t oh = (size_t)b * s.Hq + g * s.G + h;
         from_f(((T *)a.o)[oh * D + e], L > 0.f ? O / L : 0.f);
         if (e == 0) a.lse[oh] = L > 0.f ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
@@ -460,12 +476,13 @@ bool lsa_decode_plan(const LsaShape &s, LsaDecPlan &pl, bool chunks) {
     if (bound > (1LL << 30)) return false;
     pl.pmax = (int)max(1LL, bound);
     const int bgs = s.B * s.Hkv;
-    // about four CTAs per SM overall, but at least 32 positions per CTA at the bound
-    long long P = min(64LL, (4LL * 148 + bgs - 1) / bgs);
+    // one wave of the attention kernel (two CTAs per SM), but at least 32
+    // positions per CTA at the bound
+    long long P = min(64LL, max(1LL, 2LL * 148 / bgs));
     P = min(P, (bound + 31) / 32);
     pl.P = (int)max(1LL, P);
     pl.slice = 1024;
-    pl.HG = s.G >= 8 ? 8 : s.G >= 4 ? 4 : s.G >= 2 ? 2 : 1;
+    pl.HG = s.G >= 4 ? 4 : s.G >= 2 ? 2 : 1;     // query heads per pass (more would cost occupancy)
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
     size_t off = kStatusBytes;
     pl.off_key = off;   off += al((size_t)bgs * pl.S * max(1, pl.kk) * 8);
@@ -485,7 +502,9 @@ static size_t select_smem(const LsaShape &s, const LsaDecPlan &pl) {
 }
 
 static size_t attend_smem(const LsaShape &s, const LsaDecPlan &pl) {
-    return (size_t)((pl.slice + 3) & ~3) * 4 + (size_t)(kLsaThreads / 32) * pl.HG * (s.d + 2) * 4 + 16;
+    // the warps' states, or the last CTA's merge weights (2 P G + 2 G floats), whichever is larger
+    const size_t wst = max((size_t)(kLsaThreads / 32) * pl.HG * (s.d + 2), 2 * (size_t)pl.P * s.G + 2 * (size_t)s.G);
+    return (size_t)((pl.slice + 3) & ~3) * 4 + wst * 4 + 16;
 }
 
 template <typename T>
@@ -496,8 +515,7 @@ static cudaError_t run_lsa_attend(const LsaDecArgs &a, cudaStream_t st) {
     switch (pl.HG) {
         case 1: k2 = lsa_attend_kernel<T, 1>; break;
         case 2: k2 = lsa_attend_kernel<T, 2>; break;
-        case 4: k2 = lsa_attend_kernel<T, 4>; break;
-        default: k2 = lsa_attend_kernel<T, 8>; break;
+        default: k2 = lsa_attend_kernel<T, 4>; break;
     }
     const size_t sm2 = attend_smem(s, pl);
     cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);

@@ -25,7 +25,7 @@ struct LsaDecPlan {
     int pmax;        // kept key positions per (batch, kv-head), at most
     int P;           // attention CTAs per (batch, kv-head)
     int slice;       // key positions an attention CTA stages per round
-    int HG;          // query heads per attention pass (1, 2, 4 or 8)
+    int HG;          // query heads per attention pass (1, 2 or 4)
     size_t off_key, off_id, off_done1, off_pos, off_cnt, off_part, off_done2, bytes;
 };
 

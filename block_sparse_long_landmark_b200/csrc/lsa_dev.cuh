@@ -34,6 +34,25 @@ __device__ inline int block_topk64(const uint64_t *keys, int n, int k, int *out,
         __syncthreads();
         return n;
     }
+    if (n <= kLsaThreads) {
+        // a key per thread, ranked by the keys above it (equal keys: the lower
+        // position first); the k lowest ranks, compacted in position order
+        int sel = 0;
+        if (tid < n) {
+            const unsigned long long x = keys[tid];
+            int r = 0;
+            for (int j = 0; j < n; ++j) {
+                const unsigned long long y = keys[j];
+                r += (y > x) || (y == x && j < tid);
+            }
+            sel = r < k;
+        }
+        int tot;
+        const int at = block_scan_incl(sel, red, &tot) - sel;
+        if (sel) out[at] = tid;
+        __syncthreads();
+        return tot;
+    }
     int *misc = hist + 256;
     unsigned long long prefix = 0ull, mask = 0ull;
     int kr = k;                                    // rank of T among the keys matching `prefix`

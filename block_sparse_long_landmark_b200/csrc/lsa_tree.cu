@@ -503,6 +503,38 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_tree_select_kernel(TreeSelArg
         const int nb = tp.n[lv - 1];
         const int32_t *cs = reinterpret_cast<const int32_t *>(ta.tree + tp.off_cs[lv]) + (size_t)bg * (tp.n[lv] + 1);
         const int32_t *ci = reinterpret_cast<const int32_t *>(ta.tree + tp.off_ci[lv]) + (size_t)bg * nb;
+        if (nk <= kLsaThreads) {
+            // few kept nodes: gather their children, then place each by its rank
+            int c0 = 0, cn = 0;
+            if (tid < nk) {
+                const int p = fr[pos[tid]];
+                c0 = cs[p];
+                cn = max(0, cs[p + 1] - c0);
+            }
+            int nc;
+            const int at = block_scan_incl(cn, red, &nc) - cn;
+            if (nc <= min(kLsaThreads, F)) {
+                for (int c = 0; c < cn; ++c) {
+                    const int x = ci[c0 + c];
+                    mark[at + c] = (x >= 0 && x < nb) ? x : -1;
+                }
+                __syncthreads();
+                int x = -1, r = 0;
+                if (tid < nc) {
+                    x = mark[tid];
+                    for (int j = 0; j < nc; ++j) {
+                        const int y = mark[j];
+                        r += y >= 0 && (y < x || (y == x && j < tid));
+                    }
+                }
+                int nv;
+                block_scan_incl(x >= 0 ? 1 : 0, red, &nv);
+                if (x >= 0) fr[r] = x;
+                nf = nv;
+                __syncthreads();
+                continue;
+            }
+        }
         for (int x = tid; x < nb; x += kLsaThreads) mark[x] = 0;
         __syncthreads();
         for (int i = warp; i < nk; i += kLsaThreads / 32) {

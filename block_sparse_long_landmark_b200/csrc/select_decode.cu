@@ -31,11 +31,12 @@ namespace {
 
 constexpr int kSdWarps = 8;          // scoring warps; warp 8 streams
 constexpr int kSdThreads = 32 * (kSdWarps + 1);
-constexpr int kSdChunk = 256;        // candidates per scoring warp (its top-K)
+constexpr int kSdChunk = 256;        // candidates per scoring warp (its top-K), or twice that
 constexpr int kSdMaxMerge = 4096;    // candidates the cross-CTA merge holds in shared memory
 constexpr int kSdStage = 32768;      // bytes per ring stage: eight 16-byte slices per scoring lane
-constexpr int kSdStages = 3;
-constexpr uint32_t kSdRingBytes = (uint32_t)kSdStages * kSdStage;
+constexpr int kSdStages = 3;        // ring stages with 256 candidates per warp; 2 with 512
+__host__ __device__ constexpr int sd_stages(int CH) { return CH == kSdChunk ? kSdStages : 2; }
+__host__ __device__ constexpr uint32_t sd_ring_bytes(int CH) { return (uint32_t)sd_stages(CH) * kSdStage; }
 
 struct SdArgs {
     Shape s;
@@ -65,8 +66,8 @@ struct SdSmem {
 // over the ring serves the warps' top-K positions, the final list and the
 // cross-CTA merge.
 __host__ __device__ constexpr size_t sd_off_keys() { return (sizeof(SdSmem) + 127) & ~(size_t)127; }
-__host__ __device__ constexpr size_t sd_off_ring() { return sd_off_keys() + (size_t)kSdWarps * kSdChunk * 4; }
-__host__ __device__ constexpr size_t sd_off_merge() { return sd_off_ring() + kSdRingBytes; }
+__host__ __device__ constexpr size_t sd_off_ring(int CH) { return sd_off_keys() + (size_t)kSdWarps * CH * 4; }
+__host__ __device__ constexpr size_t sd_off_merge(int CH) { return sd_off_ring(CH) + sd_ring_bytes(CH); }
 
 // Final list of unit u: [0 (sink)] + selected (ascending) + [local].
 __device__ void write_list(const SdArgs &a, int u, int local, const int *sel_idx, const uint32_t *sel_key, int nsel,
@@ -108,8 +109,9 @@ __device__ __forceinline__ void slice_f32(const uint4 &u, const float *, float *
     f[3] = __uint_as_float(u.w);
 }
 
-template <typename T, int VPR>
+template <typename T, int VPR, int CH>
 __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) {
+    constexpr int NST = sd_stages(CH);
     using namespace tc;
     constexpr int EPV = Vec<T>::n;
     constexpr int RB = VPR * 16;                    // bytes per row
@@ -123,9 +125,9 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     const int D = VPR * EPV;
     extern __shared__ __align__(128) unsigned char smraw[];
     SdSmem &sm = *reinterpret_cast<SdSmem *>(smraw);
-    uint32_t *keys = reinterpret_cast<uint32_t *>(smraw + sd_off_keys());      // [2048]
-    unsigned char *ring = smraw + sd_off_ring();                                // [stages][32 KB]
-    uint32_t *mkey = reinterpret_cast<uint32_t *>(smraw + sd_off_merge());     // [8 * top_k]
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smraw + sd_off_keys());      // [8 * CH]
+    unsigned char *ring = smraw + sd_off_ring(CH);                              // [stages][32 KB]
+    uint32_t *mkey = reinterpret_cast<uint32_t *>(smraw + sd_off_merge(CH));   // [8 * top_k]
     int *midx = reinterpret_cast<int *>(mkey + kSdWarps * s.top_k);            // [8 * top_k]
     int *mpos = midx + kSdWarps * s.top_k;                                      // [top_k]
 
@@ -137,16 +139,16 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     const int hq0 = perq ? hs : hs * s.G;
     const int local = (seq_n(s, b) - 1) / s.bs;
     const int first = (s.flags & SA_SINK) ? 1 : 0;
-    const int cc0 = first + cta * kSdWarps * kSdChunk;              // the CTA's first candidate
-    const int ncta = max(0, min(local, cc0 + kSdWarps * kSdChunk) - cc0);
+    const int cc0 = first + cta * kSdWarps * CH;                    // the CTA's first candidate
+    const int ncta = max(0, min(local, cc0 + kSdWarps * CH) - cc0);
     const int wsel = min(warp, kSdWarps - 1);
-    const int c0 = cc0 + wsel * kSdChunk;                           // a scoring warp's first candidate
-    const int n = max(0, min(ncta - wsel * kSdChunk, kSdChunk));
+    const int c0 = cc0 + wsel * CH;                                 // a scoring warp's first candidate
+    const int n = max(0, min(ncta - wsel * CH, CH));
 
     // the attention launch that follows may start as this grid's CTAs are placed
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kSdStages; ++i) {
+        for (int i = 0; i < NST; ++i) {
             mbar_init(smem_u32(&sm.full[i]), 1);
             mbar_init(smem_u32(&sm.empty[i]), kSdWarps);
         }
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     const T *Lg = (const T *)a.L + ((size_t)b * s.Hkv + g) * s.nb * D;
     const size_t cbytes = (size_t)ncta * RB;                        // the CTA's landmark bytes
     const int nst = (int)((cbytes + kSdStage - 1) / kSdStage);
-    uint32_t *kw = keys + wsel * kSdChunk;
+    uint32_t *kw = keys + wsel * CH;
     bool nan_seen = false;
     float qv[EPV];
     const int sub = lane / VPR, cv = lane % VPR;
@@ -168,9 +170,9 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
             const unsigned char *src = reinterpret_cast<const unsigned char *>(Lg + (size_t)cc0 * D);
             int issued = 0;
             for (int i = 0; i < nst; ++i) {
-                const int st = i % kSdStages;
-                if (i >= kSdStages &&
-                    !mbar_wait(smem_u32(&sm.empty[st]), ((i / kSdStages) - 1) & 1, &sm.abort_flag, a.status))
+                const int st = i % NST;
+                if (i >= NST &&
+                    !mbar_wait(smem_u32(&sm.empty[st]), ((i / NST) - 1) & 1, &sm.abort_flag, a.status))
                     break;
                 const uint32_t bytes = (uint32_t)min((size_t)kSdStage, cbytes - (size_t)i * kSdStage);
                 mbar_expect_tx(smem_u32(&sm.full[st]), bytes);
@@ -180,8 +182,8 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
             if (sm.abort_flag) {
                 // let the copies in flight land before the ring is reused
                 volatile int never = 0;
-                for (int i = max(0, issued - kSdStages); i < issued; ++i)
-                    mbar_wait(smem_u32(&sm.full[i % kSdStages]), (i / kSdStages) & 1, &never, a.status);
+                for (int i = max(0, issued - NST); i < issued; ++i)
+                    mbar_wait(smem_u32(&sm.full[i % NST]), (i / NST) & 1, &never, a.status);
             }
         }
     } else {
@@ -198,8 +200,8 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
 #pragma unroll
         for (int i = 0; i < EPV; ++i) qv[i] /= (float)s.heads_per;
         for (int i = 0; i < nst; ++i) {
-            const int st = i % kSdStages;
-            const bool ok = mbar_wait(smem_u32(&sm.full[st]), (i / kSdStages) & 1, &sm.abort_flag, a.status);
+            const int st = i % NST;
+            const bool ok = mbar_wait(smem_u32(&sm.full[st]), (i / NST) & 1, &sm.abort_flag, a.status);
             if (!__all_sync(0xffffffffu, ok)) break;
             const unsigned char *stg = ring + st * kSdStage + warp * RW * RB;
             float v[NL];
@@ -240,8 +242,8 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     }
     __syncthreads();
     if (warp < kSdWarps) {
-        int *pw = reinterpret_cast<int *>(ring) + warp * kSdChunk;  // the warp's positions (the ring is free)
-        const int nsel = warp_topk_positions<8>(kw, n, s.top_k, pw);
+        int *pw = reinterpret_cast<int *>(ring) + warp * CH;        // the warp's positions (the ring is free)
+        const int nsel = warp_topk_positions<CH / 32>(kw, n, s.top_k, pw);
         // the warp's list (ascending block ids) into the CTA's merge area
         for (int i = lane; i < nsel; i += 32) {
             mkey[warp * s.top_k + i] = kw[pw[i]];
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     const int nc = warp_topk_positions<16>(mkey, ntot, s.top_k, mpos);
     // the final list's staging: the keys area is free once the warp lists are merged
     uint32_t *sel_key = keys;
-    int *sel_idx = reinterpret_cast<int *>(keys + kSdChunk);
+    int *sel_idx = reinterpret_cast<int *>(keys + kSdChunk);   // top_k <= 256
     if (a.C == 1) {
         // one CTA per unit: its list is the unit's
         for (int i = lane; i < nc; i += 32) {
@@ -359,13 +361,16 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
 
 }  // namespace
 
-// Geometry: warp-chunks per unit cover the largest candidate count (the
-// full context), grouped eight to a CTA.
-static void sd_geometry(const Shape &s, int &C) {
+// Geometry: scoring-warp chunks of 256 candidates (512 when that turns more
+// than one wave of CTAs -- two per SM -- into one) cover the largest candidate
+// count (the full context), grouped eight to a CTA.
+static void sd_geometry(const Shape &s, int &C, int &CH) {
     const int first = (s.flags & SA_SINK) ? 1 : 0;
     const int ncand = max(1, (s.N - 1) / s.bs - first);
-    const int W = (ncand + kSdChunk - 1) / kSdChunk;
-    C = (W + kSdWarps - 1) / kSdWarps;
+    const long long units = (long long)s.B * s.Hsel, slots = 2LL * 148;
+    auto ctas = [&](int ch) { return (ncand + kSdWarps * ch - 1) / (kSdWarps * ch); };
+    CH = (units * ctas(kSdChunk) > slots && units * ctas(2 * kSdChunk) <= slots) ? 2 * kSdChunk : kSdChunk;
+    C = ctas(CH);
 }
 
 bool select_force_chunked() {
@@ -375,22 +380,24 @@ bool select_force_chunked() {
 
 bool select_decode_supported(const Shape &s) {
     if (s.top_k < 1 || s.top_k > kSdChunk) return false;
-    int C;
-    sd_geometry(s, C);
+    int C, CH;
+    sd_geometry(s, C, CH);
     return C == 1 || (long long)C * s.top_k <= kSdMaxMerge;
 }
 
 size_t select_decode_workspace(const Shape &s) {
-    int C;
-    sd_geometry(s, C);
+    int C, CH;
+    sd_geometry(s, C, CH);
     if (C == 1) return 0;
     const size_t units = (size_t)s.B * s.Hsel;
     return units * C * s.top_k * 8 + units * C * 4 + units * 2 * 4 + 4 * 256;
 }
 
-static size_t sd_smem(const Shape &s) {
-    static_assert((size_t)kSdMaxMerge * 8 + kSdChunk * 4 <= kSdRingBytes, "cross-CTA merge fits the ring space");
-    return sd_off_merge() + (size_t)kSdWarps * s.top_k * 8 + (size_t)s.top_k * 4;
+static size_t sd_smem(const Shape &s, int CH) {
+    static_assert((size_t)kSdMaxMerge * 8 + kSdChunk * 4 <= sd_ring_bytes(2 * kSdChunk),
+                  "cross-CTA merge fits the ring space");
+    static_assert((size_t)kSdWarps * 2 * kSdChunk * 4 <= sd_ring_bytes(2 * kSdChunk), "positions fit the ring space");
+    return sd_off_merge(CH) + (size_t)kSdWarps * s.top_k * 8 + (size_t)s.top_k * 4;
 }
 
 template <typename T>
@@ -404,7 +411,8 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
     a.score = score;
     a.count = count;
     a.status = (unsigned *)ws;
-    sd_geometry(s, a.C);
+    int CH;
+    sd_geometry(s, a.C, CH);
     const size_t units = (size_t)s.B * s.Hsel;
     if (a.C > 1) {
         char *p = (char *)ws + ws_layout(s).scratch;
@@ -422,12 +430,12 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
     const int vpr = s.d * (int)sizeof(T) / 16;
     void (*kern)(SdArgs) = nullptr;
     switch (vpr) {
-        case 8: kern = select_decode_kernel<T, 8>; break;
-        case 16: kern = select_decode_kernel<T, 16>; break;
-        case 32: kern = select_decode_kernel<T, 32>; break;
+        case 8: kern = CH == kSdChunk ? select_decode_kernel<T, 8, kSdChunk> : select_decode_kernel<T, 8, 2 * kSdChunk>; break;
+        case 16: kern = CH == kSdChunk ? select_decode_kernel<T, 16, kSdChunk> : select_decode_kernel<T, 16, 2 * kSdChunk>; break;
+        case 32: kern = CH == kSdChunk ? select_decode_kernel<T, 32, kSdChunk> : select_decode_kernel<T, 32, 2 * kSdChunk>; break;
         default: return cudaErrorInvalidValue;
     }
-    const size_t smem = sd_smem(s);
+    const size_t smem = sd_smem(s, CH);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(units * a.C), kSdThreads, smem, st>>>(a);
