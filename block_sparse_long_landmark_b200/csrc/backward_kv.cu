@@ -21,7 +21,11 @@
 // Preparation (no atomics in the sums, fixed order): a warp per key tile walks
 // the later blocks' lists (each ascending) and records, in unit order, the
 // units that keep the tile with the gates of its blocks in log2 units; a scan
-// turns the counts into offsets and deals the work items out largest first.
+// turns the counts into offsets, and the work items are ordered group by group
+// ((batch, kv-head)), largest first within a group.  The CTAs claim items in
+// that order from a global counter, so a CTA that finishes early takes more
+// and the CTAs work on one or two groups at a time: the Q and dO rows they
+// re-read (those of the units that keep each tile) stay in L2.
 // A tile kept by more than 64 units is split into work items of 64; each
 // split leaves its accumulators in a partial slot, and for each warp's region
 // the split that finishes last sums the slots in split order.  The per-row
@@ -146,27 +150,18 @@ __global__ void inv_kernel(InvArgs a, int pass) {
         a.items[a.ioff[t] + sp] = make_int4(t, base + sp * kUMax, base + min(n, (sp + 1) * kUMax), sp);
 }
 
-// One CTA: offsets of every tile's units, items and partial slots, then the
-// order in which the dK/dV kernel takes the items: by size, largest first
-// (items of equal size in any order -- the results do not depend on it).
+// One CTA: offsets of every tile's units, items and partial slots.
 __global__ void __launch_bounds__(1024) inv_scan_kernel(InvArgs a) {
     __shared__ int wsum[32][3];
     __shared__ int carry[3];
-    __shared__ int hist[kUMax + 1], cur[kUMax + 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid < 3) carry[tid] = 0;
-    if (tid <= kUMax) hist[tid] = 0;
     __syncthreads();
     for (int t0 = 0; t0 < a.tiles; t0 += 1024) {
         const int t = t0 + tid;
         const int n = t < a.tiles ? a.tcnt[t] : 0;
         const int ns = t < a.tiles ? max(1, (n + kUMax - 1) / kUMax) : 0;
         const int sl = ns > 1 ? ns : 0;
-        if (t < a.tiles) {
-            const int full = n / kUMax, rem = n - full * kUMax;
-            if (full) atomicAdd(&hist[kUMax], full);
-            if (rem || n == 0) atomicAdd(&hist[rem], 1);
-        }
         int v[3] = {n, ns, sl}, incl[3];
 #pragma unroll
         for (int q = 0; q < 3; ++q) {
@@ -201,14 +196,33 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(InvArgs a) {
         a.tot[0] = carry[1];     // work items
         a.tot[1] = carry[0];     // (tile, unit) entries
         a.tot[2] = carry[2];     // partial slots
-        int pos = 0;
+        a.tot[3] = 0;            // the dK/dV kernel's claim counter
+    }
+}
+
+// A CTA per (batch, kv-head): the order of that group's items -- largest first
+// (items of equal size in any order; the results do not depend on it).
+__global__ void __launch_bounds__(1024) inv_order_kernel(InvArgs a) {
+    __shared__ int hist[kUMax + 1], cur[kUMax + 1];
+    const int tid = threadIdx.x, bg = blockIdx.x;
+    const int t0 = bg * a.KT, t1 = t0 + a.KT;
+    if (tid <= kUMax) hist[tid] = 0;
+    __syncthreads();
+    for (int t = t0 + tid; t < t1; t += blockDim.x) {
+        const int n = a.tcnt[t], full = n / kUMax, rem = n - full * kUMax;
+        if (full) atomicAdd(&hist[kUMax], full);
+        if (rem || n == 0) atomicAdd(&hist[rem], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int pos = a.ioff[t0];           // the group's items start here
         for (int sz = kUMax; sz >= 0; --sz) {
             cur[sz] = pos;
             pos += hist[sz];
         }
     }
     __syncthreads();
-    for (int t = tid; t < a.tiles; t += 1024) {
+    for (int t = t0 + tid; t < t1; t += blockDim.x) {
         const int n = a.tcnt[t], io = a.ioff[t];
         const int ns = max(1, (n + kUMax - 1) / kUMax);
         for (int sp = 0; sp < ns; ++sp) {
@@ -233,7 +247,8 @@ constexpr uint32_t kRowOff = kRingOff + 2 * kStageBytes;    // [2 stages] lse2[1
 constexpr uint32_t kRowBytes = 2 * 128 * 4;
 constexpr uint32_t kInfoOff = kRowOff + 2 * kRowBytes;      // [2 stages] the pair's entry (int4)
 constexpr uint32_t kInfoBytes = 16;
-constexpr uint32_t kBarOffKV = kInfoOff + 2 * kInfoBytes + 32;
+constexpr uint32_t kItemOff = kInfoOff + 2 * kInfoBytes;    // [4] claimed item ids (-1: no more)
+constexpr uint32_t kBarOffKV = kItemOff + 16 + 32;
 constexpr uint32_t kSmemKV = kBarOffKV + 512 + 1024;
 static_assert(kSmemKV <= 227 * 1024, "shared memory");
 static_assert(kRowOff % 16 == 0 && kRowBytes % 16 == 0, "bulk copy alignment");
@@ -248,7 +263,9 @@ enum {
     B_ACC = 10,         // the item's dV, dK complete
     B_ACCF = 11,        // dV, dK read out (256 arrivals)
     B_END = 12,
-    NBARKV
+    B_IF = 13,          // [4] item slot published
+    B_IE = 17,          // [4] item slot read (the MMA warp and the 8 element-wise warps)
+    NBARKV = 21
 };
 static_assert(8 * NBARKV + 8 <= 512, "barrier area");
 
@@ -256,7 +273,8 @@ struct KvArgs {
     Shape s;
     const float *D, *lse2;      // [B,Hq,Npad] (Npad = nb * block; rows past N: D 0, lse2 +inf)
     float *dK, *dV;
-    const int *tsplit, *tslot, *tot, *order;
+    const int *tsplit, *tslot, *order;
+    int *tot;                   // [0] items; [3] the claim counter (zero at launch)
     int *rcnt;                  // [tiles][8 regions] splits finished
     const int4 *ent, *items;
     float *part;                // [slots][2][128][128]
@@ -265,12 +283,16 @@ struct KvArgs {
     unsigned long long wait_ns;
 };
 
-// k-th work item of this CTA, in the snake order over the size-sorted items
-// (round k: CTAs ascending when k is even, descending when odd); -1 when done.
-__device__ __forceinline__ int item_of(const KvArgs &a, int k, int nitems) {
-    const int P = gridDim.x;
-    const int q = k * P + ((k & 1) ? P - 1 - (int)blockIdx.x : (int)blockIdx.x);
-    return q < nitems ? a.order[q] : -1;
+// The CTA's k-th work item, published by warp 0 in item slot k % 4: warps
+// 1 and 4..11 wait for it, and one lane of each tells the slot is read.
+__device__ __forceinline__ int item_read(const KvArgs &a, const volatile int *itq, uint32_t bar_if, uint32_t bar_ie,
+                                         int k, volatile int *abort_flag, bool &ok) {
+    ok = tc::mbar_wait(bar_if, (k >> 2) & 1, abort_flag, a.status, a.wait_ns);
+    ok = __all_sync(0xffffffffu, ok);
+    const int it = ok ? itq[k & 3] : -1;
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) tc::mbar_arrive(bar_ie);
+    return it;
 }
 
 __global__ void __launch_bounds__(kThreadsKV, 1)
@@ -287,12 +309,13 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
     auto rows_of = [&](int st) { return reinterpret_cast<float *>(smem + kRowOff + st * kRowBytes); };
     auto info_of = [&](int st) { return reinterpret_cast<int4 *>(smem + kInfoOff + st * kInfoBytes); };
+    volatile int *itq = reinterpret_cast<volatile int *>(smem + kItemOff);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nitems = a.tot[0];
 
     if (tid == 0) {
         for (int i = 0; i < NBARKV; ++i)
-            mbar_init(bar(i), (i == B_EW || i == B_EW + 1) ? 128 : i == B_ACCF ? 256 : 1);
+            mbar_init(bar(i), (i == B_EW || i == B_EW + 1) ? 128 : i == B_ACCF ? 256 : (i >= B_IE) ? 9 : 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -313,9 +336,25 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         int gp = 0, ni = 0;
         int kvlast = -1;                 // phase of the last K/V load issued
         int plast[2] = {-1, -1};         // last pair issued on each ring stage
+        // claims run one item ahead of the item being loaded
+        int nxt = 0;
+        if (lane == 0) nxt = atomicAdd(a.tot + 3, 1);
         for (int k = 0;; ++k) {
-            const int it = item_of(a, k, nitems);
-            if (it < 0) break;
+            int it = -1;
+            if (lane == 0) {
+                if (ok && nxt < nitems) {
+                    it = a.order[nxt];
+                    nxt = atomicAdd(a.tot + 3, 1);
+                }
+                // publish it in slot k % 4 once the slot's previous item has been read
+                if (k >= 4 && !mbar_wait(bar(B_IE + (k & 3)), ((k >> 2) - 1) & 1, abort_flag, a.status, a.wait_ns))
+                    ok = false;
+                itq[k & 3] = ok ? it : -1;
+                mbar_arrive(bar(B_IF + (k & 3)));
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            it = __shfl_sync(0xffffffffu, it, 0);
+            if (!ok || it < 0) break;
             const int4 item = a.items[it];
             const int np = (item.z - item.y) * a.MT;
             if (np == 0) continue;
@@ -438,8 +477,8 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         int gp = 0, ni = 0;
         for (int k = 0; ok; ++k) {
-            const int it = item_of(a, k, nitems);
-            if (it < 0) break;
+            const int it = item_read(a, itq, bar(B_IF + (k & 3)), bar(B_IE + (k & 3)), k, abort_flag, ok);
+            if (!ok || it < 0) break;
             const int4 item = a.items[it];
             const int np = (item.z - item.y) * a.MT;
             if (np == 0) continue;
@@ -495,8 +534,8 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         int gp = 0, ni = 0;
         for (int k = 0; ok; ++k) {
-            const int it = item_of(a, k, nitems);
-            if (it < 0) break;
+            const int it = item_read(a, itq, bar(B_IF + (k & 3)), bar(B_IE + (k & 3)), k, abort_flag, ok);
+            if (!ok || it < 0) break;
             const int4 item = a.items[it];
             const int np = (item.z - item.y) * a.MT;
             const int bg = item.x / a.KT, kt = item.x % a.KT;
@@ -671,6 +710,8 @@ cudaError_t launch_backward_kv(const Shape &s, const void *Q, const void *K, con
     inv_scan_kernel<<<1, 1024, 0, st>>>(ia);
     note_launch();
     inv_kernel<<<wgrid, 256, 0, st>>>(ia, 1);
+    note_launch();
+    inv_order_kernel<<<(unsigned)(s.B * s.Hkv), 1024, 0, st>>>(ia);
     note_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

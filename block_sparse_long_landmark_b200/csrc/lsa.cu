@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     const int b = bg / s.Hkv, g = bg % s.Hkv;
     const int D = s.d;
     const T *q = (const T *)a.q;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the attention may start early
     for (int e = tid; e < D; e += kLsaThreads) {
         double acc = 0.0;
         for (int h = 0; h < s.G; ++h) acc += (double)to_f(q[((size_t)b * s.Hq + g * s.G + h) * D + e]);
@@ -228,6 +229,7 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     // merge: chunk c holds min(kk, its centres) candidates, packed in chunk order
     int ntot = 0;
     for (int c = 0; c < pl.S; ++c) ntot += min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
+#pragma unroll 4
     for (int e = tid; e < pl.S * pl.kk; e += kLsaThreads) {
         const int c = e / pl.kk, i = e % pl.kk;
         const int nv = min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
@@ -270,6 +272,7 @@ __global__ void __launch_bounds__(kLsaThreads, 2) lsa_attend_kernel(LsaDecArgs a
     float *wst = reinterpret_cast<float *>(posv + ((pl.slice + 3) & ~3));      // [8 warps][HG][D + 2]
     int *misc = reinterpret_cast<int *>(wst + max((kLsaThreads / 32) * HG * (D + 2), 2 * pl.P * s.G + 2 * s.G));   // [4]
 
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // the list comes from the launch before this one
     const int tot = a.cnt[2 * (size_t)bg + 1];
     // this CTA's share of the kept positions, walked in rounds of pl.slice
     const int t0 = (int)((long long)tot * pi / pl.P), t1 = (int)((long long)tot * (pi + 1) / pl.P);
@@ -311,26 +314,53 @@ __global__ void __launch_bounds__(kLsaThreads, 2) lsa_attend_kernel(LsaDecArgs a
                     kr[u] = *reinterpret_cast<const uint4 *>(Kb + row);
                     vr[u] = *reinterpret_cast<const uint4 *>(Vb + row);
                 }
+                // the U rows' scores for every head of the pass (summed over the lane group)
+                float z[U][HG];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const bool live = vb + sub + u * RPW * NW < np;   // uniform over the lane group
-                    float kf[EPV], vf[EPV];
+                    float kf[EPV];
                     load16(reinterpret_cast<const T *>(&kr[u]), kf);
-                    load16(reinterpret_cast<const T *>(&vr[u]), vf);
 #pragma unroll
                     for (int h = 0; h < HG; ++h) {
-                        float z = 0.f;
+                        float t = 0.f;
 #pragma unroll
-                        for (int e = 0; e < EPV; ++e) z = fmaf(qf[h][e], kf[e], z);
-                        for (int o = VPR / 2; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-                        if (!live || h >= nh) continue;
-                        const float mn = fmaxf(m[h], z);
-                        const float corr = exp2f(m[h] - mn), p = exp2f(z - mn);
-                        l[h] = l[h] * corr + p;
-#pragma unroll
-                        for (int e = 0; e < EPV; ++e) acc[h][e] = fmaf(acc[h][e], corr, p * vf[e]);
-                        m[h] = mn;
+                        for (int e = 0; e < EPV; ++e) t = fmaf(qf[h][e], kf[e], t);
+                        for (int o = VPR / 2; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+                        // rows past the round (uniform over the lane group) and padded heads take no part
+                        z[u][h] = (vb + sub + u * RPW * NW < np && h < nh) ? t : -CUDART_INF_F;
                     }
+                }
+                // one online-softmax step per head for the U rows: a single rescale
+#pragma unroll
+                for (int h = 0; h < HG; ++h) {
+                    float mn = m[h];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) mn = fmaxf(mn, z[u][h]);
+                    if (mn == -CUDART_INF_F) {
+#pragma unroll
+                        for (int u = 0; u < U; ++u) z[u][h] = 0.f;
+                        continue;
+                    }
+                    const float corr = m[h] == -CUDART_INF_F ? 0.f : exp2f(m[h] - mn);
+                    float ps = 0.f;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        z[u][h] = exp2f(z[u][h] - mn);      // -inf rows give 0
+                        ps += z[u][h];
+                    }
+                    l[h] = l[h] * corr + ps;
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e) acc[h][e] *= corr;
+                    m[h] = mn;
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    float vf[EPV];
+                    load16(reinterpret_cast<const T *>(&vr[u]), vf);
+#pragma unroll
+                    for (int h = 0; h < HG; ++h)
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) acc[h][e] = fmaf(z[u][h], vf[e], acc[h][e]);
                 }
             }
         }
@@ -454,10 +484,13 @@ bool lsa_decode_plan(const LsaShape &s, LsaDecPlan &pl, bool chunks) {
         pl.S = 1;
         pl.kk = 0;
     } else {
-        // chunks of 128 centres; the merge takes every score when it can hold
-        // them all (C <= 4096), else each chunk passes its best min(top, CH),
-        // the chunks grown until the merge's candidates fit one CTA
+        // chunks of 128 centres or more, so that the grid is one wave (four
+        // CTAs per SM); the merge takes every score when it can hold them all
+        // (C <= 4096), else each chunk passes its best min(top, CH), the chunks
+        // grown until the merge's candidates fit one CTA
+        const long long bgs = (long long)s.B * s.Hkv;
         pl.CH = 128;
+        while (pl.CH < 4096 && bgs * ((C + pl.CH - 1) / pl.CH) > 4 * 148) pl.CH *= 2;
         pl.S = max(1, (C + pl.CH - 1) / pl.CH);
         if (C <= 4096) {
             pl.kk = pl.CH;
@@ -520,9 +553,9 @@ static cudaError_t run_lsa_attend(const LsaDecArgs &a, cudaStream_t st) {
     const size_t sm2 = attend_smem(s, pl);
     cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
     if (e != cudaSuccess) return e;
-    k2<<<(unsigned)(s.B * s.Hkv) * pl.P, kLsaThreads, sm2, st>>>(a);
+    e = launch_pdl(k2, dim3((unsigned)(s.B * s.Hkv) * pl.P), dim3(kLsaThreads), sm2, st, a);
     note_launch();
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_lsa_attend(const LsaDecArgs &a, cudaStream_t st) {

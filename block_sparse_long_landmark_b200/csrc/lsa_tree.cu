@@ -453,6 +453,7 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_tree_select_kernel(TreeSelArg
     const int bg = blockIdx.x, b = bg / s.Hkv, g = bg % s.Hkv;
     const int D = s.d;
     const T *q = (const T *)a.q;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the attention may start early
     for (int e = tid; e < D; e += kLsaThreads) {
         double acc = 0.0;
         for (int h = 0; h < s.G; ++h) acc += (double)to_f(q[((size_t)b * s.Hq + g * s.G + h) * D + e]);
