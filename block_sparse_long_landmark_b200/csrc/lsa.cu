@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     const int c0 = chunk * pl.CH, n = max(0, min(s.ctotal, c0 + pl.CH) - c0);
     const double *cb = a.centres + ((size_t)bg * s.ctotal + c0) * D;
     const int epl = D / 32;                    // doubles per lane: 2 (d 64) or 4 (d 128)
+    double qv[4];                              // this lane's slice of the pooled query
+#pragma unroll
+    for (int e = 0; e < 4; ++e) qv[e] = e < epl ? qbar[lane * epl + e] : 0.0;
     bool nan_seen = false;
     for (int c = warp * 4; c < n; c += 4 * (kLsaThreads / 32)) {
         double part[4];
@@ -179,10 +182,13 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
             const int cc = min(c + u, n - 1);
             const double *row = cb + (size_t)cc * D + lane * epl;
             double acc = 0.0;
-            for (int e = 0; e < epl; e += 2) {
-                const double2 v = *reinterpret_cast<const double2 *>(row + e);
-                acc = fma(v.x, qbar[lane * epl + e], acc);
-                acc = fma(v.y, qbar[lane * epl + e + 1], acc);
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                if (e < epl) {
+                    const double2 v = *reinterpret_cast<const double2 *>(row + e);
+                    acc = fma(v.x, qv[e], acc);
+                    acc = fma(v.y, qv[e + 1], acc);
+                }
             }
             part[u] = acc;
         }
