@@ -24,7 +24,10 @@ SA_OP_LANDMARKS, SA_OP_SELECT, SA_OP_SELECT_DECODE, SA_OP_PREFILL, SA_OP_DECODE 
 SA_OP_PREFILL_BACKWARD, SA_OP_SELECT_BACKWARD = 5, 6
 SA_OK, SA_ERR_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_LAUNCH, SA_ERR_DEVICE = 0, -1, -2, -3, -4, -5
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libsparse_attn.so")
+# SPARSE_ATTN_LIB selects another build of the same library (for example the
+# address-checking one, lib/libsparse_attn_bounds.so)
+LIB_PATH = os.environ.get("SPARSE_ATTN_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib",
+                                                               "libsparse_attn.so")
 
 EXPORTS = (
     "sparse_attn_workspace_size", "sparse_attn_landmarks", "sparse_attn_select", "sparse_attn_select_decode",

@@ -34,6 +34,7 @@
 #include <math_constants.h>
 
 #include "backward_tc.cuh"
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -365,6 +366,7 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 if (ok) {
                     mbar_expect_tx(bar(B_KVF), 2 * kTile);
                     const int y = bg * s.N + kt * 128;
+                    SA_CHECK_START(a.status, kt * 128, s.N);
                     for (int c = 0; c < 2; ++c)
                         for (int e = 0; e < 2; ++e) {
                             tma_load_2d(sbase + kKOff + c * kChunk + e * 8192, &tmK, bar(B_KVF), 64 * c, y + 64 * e);
@@ -414,6 +416,8 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                             const int hh = s.bs == 64 ? 2 * m + e : m;
                             const int pos = s.bs == 64 ? j * 64 : j * 128 + 64 * e;
                             const int y = (b * s.Hq + g * s.G + hh) * s.N + pos;
+                            SA_CHECK_START(a.status, hh, s.G);
+                            SA_CHECK_SPAN(a.status, pos, 64, a.Npad);
                             for (int c = 0; c < 2; ++c) {
                                 tma_load_2d(qd + c * kChunk + e * 8192, &tmQ, bar(B_PF + st), 64 * c, y);
                                 tma_load_2d(dd + c * kChunk + e * 8192, &tmDO, bar(B_PF + st), 64 * c, y);

@@ -32,6 +32,7 @@
 #include <cstring>
 
 #include "backward_tc.cuh"
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -238,6 +239,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         int hh, pos;
                         row_of(s, w.j, w.m, 64 * e, hh, pos);
                         const int y = (w.b * s.Hq + w.g * s.G + hh) * s.N + pos;
+                        SA_CHECK_START(a.status, hh, s.G);
+                        SA_CHECK_SPAN(a.status, pos, 64, s.nb * s.bs);
                         for (int c = 0; c < 2; ++c) {
                             tma_load_2d(sbase + kQOff + c * kChunk + e * 8192, &tmQ, bar(Q_Q), 64 * c, y);
                             tma_load_2d(sbase + kDOOff + c * kChunk + e * 8192, &tmDO, bar(Q_Q), 64 * c, y);
@@ -271,6 +274,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const int gg = gt + t, st = gg % kStages, use = gg / kStages;
                     int y0, y1;
                     rows_of_tile(t, y0, y1);
+                    SA_CHECK_START(a.status, y0 - kvbase, s.N);
+                    SA_CHECK_START(a.status, y1 - kvbase, s.bs == 64 ? s.N : s.nb * s.bs);   // a block's second half: padded extent
                     if (t + kStages < T) {
                         // the tile after the ring's depth into L2 ahead of its load
                         int p0, p1;

@@ -15,6 +15,7 @@
 // log-sum-exp.  All query heads of a kv-head group share the blocks they read.
 #include <math_constants.h>
 
+#include "bounds.cuh"
 #include "common.cuh"
 
 namespace sa {
@@ -86,6 +87,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecArgs a) {
         const bool forced = (blk == local && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
         const float gate = (gate_on && !forced) ? log_sigmoid(sc[c] - s_local) * kLog2e : 0.f;
         const int t0 = blk * bs, nk = min(bs, nseq - t0);
+        SA_CHECK_START(a.status, t0, nseq);
         __syncthreads();
         {
             constexpr int EPV = Vec<T>::n;

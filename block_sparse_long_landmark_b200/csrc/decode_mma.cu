@@ -33,6 +33,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "bounds.cuh"
 #include "common.cuh"
 
 namespace sa {
@@ -225,6 +226,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full),
                                          "r"(kStageBytes) : "memory");
                             const int y = kvbase + max(0, blk) * 64;
+                            SA_CHECK_START(a.status, max(0, blk) * 64, s.N);
                             const uint32_t dst = sb + st * kStageBytes;
 #pragma unroll
                             for (int ch = 0; ch < 2; ++ch) {

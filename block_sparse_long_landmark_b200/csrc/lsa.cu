@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "lsa.cuh"
+#include "bounds.cuh"
 #include "lsa_dev.cuh"
 
 namespace sa {
@@ -304,7 +305,10 @@ __global__ void __launch_bounds__(kLsaThreads, 2) lsa_attend_kernel(LsaDecArgs a
         for (int r0 = t0; r0 < t1; r0 += pl.slice) {
             const int r1 = min(t1, r0 + pl.slice);
             __syncthreads();                             // the previous round's positions are read
-            for (int i = tid; i < r1 - r0; i += kLsaThreads) posv[i] = plist[r0 + i];
+            for (int i = tid; i < r1 - r0; i += kLsaThreads) {
+                posv[i] = plist[r0 + i];
+                SA_CHECK_START(a.status, posv[i], s.N);
+            }
             __syncthreads();
             const int np = r1 - r0;
             // rows of this lane group: vb + sub + u * RPW * 8 for the warp's bases vb

@@ -17,6 +17,7 @@
 // shuffle reduction across the row's threads, one online-softmax update.
 #include <math_constants.h>
 
+#include "bounds.cuh"
 #include "common.cuh"
 
 namespace sa {
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(kRows *TPR) prefill_simt_kernel(PrefArgs a) {
         const bool forced = (blk == j && (s.flags & SA_LOCAL)) || (blk == 0 && (s.flags & SA_SINK));
         const float gate = (gate_on && !forced) ? log_sigmoid(sc[c] - s_local) * kLog2e : 0.f;
         const int t0 = blk * s.bs, nk = min(s.bs, s.N - t0);
+        SA_CHECK_START(a.status, t0, s.N);
         __syncthreads();
         {
             const int nvec = nk * D / Vec<T>::n;

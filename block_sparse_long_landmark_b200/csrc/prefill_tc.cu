@@ -37,6 +37,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -164,6 +165,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     // block 64: rows of heads h0 and h0+1; block 128: rows 0-63 and 64-127 of head h0
                     const int y = s.bs == 64 ? ((b * s.Hq + h0 + e) * s.N) + j * 64
                                              : ((b * s.Hq + h0) * s.N) + j * 128 + 64 * e;
+                    SA_CHECK_START(a.status, s.bs == 64 ? h0 + e : h0, s.Hq);
+                    SA_CHECK_START(a.status, j * s.bs, s.nb * s.bs);
                     tma_load_2d(sbase + kQOff + c * kQChunk + e * 8192, &tmQ, bar(B_Q), 64 * c, y);
                 }
             const int kvbase = (b * s.Hkv + g) * s.N;
@@ -172,6 +175,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 const int st = t % kStages, use = t / kStages;
                 const int blk = max(0, blk_s[t / sub]);
                 const int y = kvbase + blk * s.bs + (t % sub) * 64;
+                SA_CHECK_START(a.status, blk * s.bs, s.N);
                 if (t >= kStages && !mbar_wait(bar(B_KE + st), (use - 1) & 1, abort_flag, a.status)) break;
                 mbar_expect_tx(bar(B_KF + st), kKTile);
                 for (int ch = 0; ch < 2; ++ch)

@@ -55,6 +55,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -308,6 +309,8 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                             for (int e = 0; e < 2; ++e) {
                                 const int y = s.bs == 64 ? (w.b * s.Hq + w.h0 + 2 * q + e) * s.N + w.j * 64
                                                          : (w.b * s.Hq + w.h0 + q) * s.N + w.j * 128 + 64 * e;
+                                SA_CHECK_START(a.status, s.bs == 64 ? w.h0 + 2 * q + e : w.h0 + q, s.Hq);
+                                SA_CHECK_START(a.status, s.bs == 64 ? w.j * 64 : w.j * 128 + 64 * e, s.nb * s.bs);
                                 tma_load_2d(sbase + kQOff2 + q * kTile2 + c * kChunk2 + e * 8192, &tmQ, bar(C_Q),
                                             64 * c, y);
                             }
@@ -328,6 +331,8 @@ prefill_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     if (gg >= kStages2 &&
                         !(ok = mbar_wait(bar(C_KE + st), (use - 1) & 1, abort_flag, a.status, a.wait_ns)))
                         break;
+                    SA_CHECK_START(a.status, y0 - kvbase, s.N);
+                    SA_CHECK_START(a.status, y1 - kvbase, s.bs == 64 ? s.N : s.nb * s.bs);   // a block's second half: padded extent
                     if (gg != a.stall_tile) {
                         mbar_expect_tx(bar(C_KF + st), kTile2);
                         for (int c = 0; c < 2; ++c) {

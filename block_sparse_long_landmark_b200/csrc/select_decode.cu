@@ -22,6 +22,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "warp_select.cuh"
@@ -175,6 +176,7 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
                     !mbar_wait(smem_u32(&sm.empty[st]), ((i / NST) - 1) & 1, &sm.abort_flag, a.status))
                     break;
                 const uint32_t bytes = (uint32_t)min((size_t)kSdStage, cbytes - (size_t)i * kSdStage);
+                SA_CHECK_SPAN(a.status, (long long)cc0 * RB + (long long)i * kSdStage, bytes, (long long)s.nb * RB);
                 mbar_expect_tx(smem_u32(&sm.full[st]), bytes);
                 bulk_load(smem_u32(ring + st * kSdStage), src + (size_t)i * kSdStage, bytes, smem_u32(&sm.full[st]));
                 issued = i + 1;

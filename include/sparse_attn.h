@@ -42,9 +42,10 @@
  *     besides CUDA's own per-device kernel images, a launch counter and the
  *     static scratch array of sparse_attn_decode_static.
  *   - Device-side problems (an index list entry out of range, a NaN score, a
- *     bounded wait that expired) never trap: the kernel skips the bad item
- *     and records a code in the workspace's status word, which
- *     sparse_attn_check_status() returns and clears.
+ *     bounded wait that expired, and in the address-checking build a gather
+ *     outside its slab) never trap: the kernel skips the bad item and records
+ *     a code in the workspace's status word, which sparse_attn_check_status()
+ *     returns and clears.
  *   - Layouts.  Q, O: [B, Hq, N, d]; K, V: [B, Hkv, N, d]; landmarks L:
  *     [B, Hkv, nb, d] with nb = ceil(N / block); decode query q and output o:
  *     [B, Hq, d]; LSE: [B, Hq, N] (prefill) or [B, Hq] (decode), fp32.
@@ -393,7 +394,10 @@ int sparse_attn_lsa_tree_decode(const sa_lsa_params *p, int fanout, int beam, co
 
 /* Synchronises `stream`, returns SA_OK or SA_ERR_DEVICE from the status
  * word in `ws`, and clears it.  *detail (may be NULL) receives the raw bits:
- * 1 index list entry out of range, 2 NaN score, 4 bounded wait expired. */
+ * 1 index list entry out of range, 2 NaN score, 4 bounded wait expired, 8 a
+ * gather whose first row lies outside the slab it means to read (only in the
+ * address-checking build, libsparse_attn_bounds.so, compiled with
+ * -DSA_DEBUG_BOUNDS; the release build makes no such check). */
 int sparse_attn_check_status(void *ws, void *stream, int *detail);
 
 /* Static string for a return code. */

@@ -36,6 +36,14 @@ def test_every_declared_symbol_is_exported():
     assert set(sa.EXPORTS) >= names
 
 
+def test_the_address_checking_build_exports_the_same_symbols():
+    from block_sparse_long_landmark_b200 import build
+    path = build.build(bounds=True)
+    lib = ctypes.CDLL(path)
+    for n in declared_symbols():
+        assert hasattr(lib, n), n
+
+
 def test_version_and_strings():
     assert sa.sparse_attn_version() >= 100
     for code in (0, -1, -2, -3, -4, -5):
