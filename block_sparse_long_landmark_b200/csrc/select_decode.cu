@@ -6,34 +6,34 @@
 // перебирать весь контекст"): the start of the context is always added.
 //
 // Decode scans every landmark of a sequence once per step, so the step is a
-// stream of landmarks from HBM.  A CTA owns 2048 consecutive candidate blocks
-// of one (batch, selection head): a producer warp streams their landmarks in
-// 32 KB stages through a three-stage ring of bulk copies in shared memory, and
-// eight scoring warps each take an eighth of every stage.  Each lane holds a
-// 16-byte slice of the unit's pooled query and scores eight 16-byte slices per
-// stage; the partial dots are summed by a reduce-scatter across the lanes of
-// a row, so every lane ends with one full score.  Each warp then takes the
-// top-K of its 256 candidates with the warp-level bitwise select
-// (warp_select.cuh), warp 0 merges the CTA's eight lists, and when a unit spans
-// several CTAs each leaves its list in the workspace and the unit's last CTA to
-// finish merges them.  The candidates sit in index order throughout and every
-// select takes equal keys at the lower position, so the result is the exact
-// top-K by (score desc, index asc) whatever the split.
+// stream of landmarks from HBM.  A CTA owns 2048 (or 4096) consecutive
+// candidate blocks of one (batch, selection head): a producer warp streams
+// their landmarks in 32 KB stages through a ring of bulk copies in shared
+// memory, and eight scoring warps each take an eighth of every stage.  Each
+// lane holds a 16-byte slice of the unit's pooled query and scores eight
+// 16-byte slices per stage; the partial dots are summed by a reduce-scatter
+// across the lanes of a row, so every lane ends with one full score.  Once the
+// stream is over the eight warps take the CTA's top-K together with a
+// byte-wise radix select (block_select.cuh); when a unit spans several CTAs
+// each leaves its list in the workspace and the unit's last CTA to finish
+// selects again over the lists.  The candidates sit in index order throughout
+// and every select takes equal keys at the lower position, so the result is
+// the exact top-K by (score desc, index asc) whatever the split.
 #include <cstdlib>
 #include <cstring>
 
+#include "block_select.cuh"
 #include "bounds.cuh"
 #include "common.cuh"
 #include "tc_ptx.cuh"
-#include "warp_select.cuh"
 
 namespace sa {
 namespace {
 
 constexpr int kSdWarps = 8;          // scoring warps; warp 8 streams
 constexpr int kSdThreads = 32 * (kSdWarps + 1);
-constexpr int kSdChunk = 256;        // candidates per scoring warp (its top-K), or twice that
-constexpr int kSdMaxMerge = 4096;    // candidates the cross-CTA merge holds in shared memory
+constexpr int kSdChunk = 256;        // candidates per scoring warp, or twice that
+constexpr int kSdMaxMerge = 4096;    // candidates the cross-CTA merge holds (16 per scoring thread)
 constexpr int kSdStage = 32768;      // bytes per ring stage: eight 16-byte slices per scoring lane
 constexpr int kSdStages = 3;        // ring stages with 256 candidates per warp; 2 with 512
 __host__ __device__ constexpr int sd_stages(int CH) { return CH == kSdChunk ? kSdStages : 2; }
@@ -49,7 +49,6 @@ struct SdArgs {
     unsigned *status;
     uint32_t *pkey;       // [units][C][top_k] per-CTA candidates (keys)
     int32_t *pidx;        // [units][C][top_k] per-CTA candidates (block ids)
-    int32_t *pcnt;        // [units][C] candidates per CTA
     float *special;       // [units][2]: s_0, s_local
     unsigned *done;       // [units] CTAs finished; back to 0 by the merging CTA
     int C;                // CTAs per unit
@@ -57,18 +56,27 @@ struct SdArgs {
 
 struct SdSmem {
     float s_special[2];
-    int nv[kSdWarps];
     int abort_flag;
+    int last;
     uint64_t full[kSdStages], empty[kSdStages];
 };
 
-// Shared memory: header, keys [8][256], the ring [stages][32 KB], the CTA
-// merge area [8 * top_k] keys + ids, [top_k] positions.  Once the stream is
-// over the ring serves the warps' top-K positions, the final list and the
-// cross-CTA merge.
+// Shared memory: header, keys [8 * CH], the ring [stages][32 KB].  Once the
+// stream is over the ring holds the select's state, the positions it returns,
+// the final list and the cross-CTA merge's keys and block ids.
 __host__ __device__ constexpr size_t sd_off_keys() { return (sizeof(SdSmem) + 127) & ~(size_t)127; }
 __host__ __device__ constexpr size_t sd_off_ring(int CH) { return sd_off_keys() + (size_t)kSdWarps * CH * 4; }
-__host__ __device__ constexpr size_t sd_off_merge(int CH) { return sd_off_ring(CH) + sd_ring_bytes(CH); }
+__host__ __device__ constexpr size_t sd_smem_bytes(int CH) { return sd_off_ring(CH) + sd_ring_bytes(CH); }
+// offsets inside the ring once the stream is over
+constexpr size_t kSdXKey = 0;                                   // [kSdMaxMerge] keys
+constexpr size_t kSdXIdx = kSdXKey + (size_t)kSdMaxMerge * 4;   // [kSdMaxMerge] block ids
+constexpr size_t kSdBs = kSdXIdx + (size_t)kSdMaxMerge * 4;     // BsSmem
+constexpr size_t kSdPos = kSdBs + ((sizeof(BsSmem) + 15) & ~(size_t)15);   // [kSdChunk] positions
+constexpr size_t kSdSelKey = kSdPos + (size_t)kSdChunk * 4;     // [kSdChunk] final keys
+constexpr size_t kSdSelIdx = kSdSelKey + (size_t)kSdChunk * 4;  // [kSdChunk] final block ids
+constexpr size_t kSdAfter = kSdSelIdx + (size_t)kSdChunk * 4;
+static_assert(kSdAfter <= sd_ring_bytes(2 * kSdChunk) && kSdAfter <= sd_ring_bytes(kSdChunk),
+              "the select's state fits the ring");
 
 // Final list of unit u: [0 (sink)] + selected (ascending) + [local].
 __device__ void write_list(const SdArgs &a, int u, int local, const int *sel_idx, const uint32_t *sel_key, int nsel,
@@ -128,9 +136,6 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     SdSmem &sm = *reinterpret_cast<SdSmem *>(smraw);
     uint32_t *keys = reinterpret_cast<uint32_t *>(smraw + sd_off_keys());      // [8 * CH]
     unsigned char *ring = smraw + sd_off_ring(CH);                              // [stages][32 KB]
-    uint32_t *mkey = reinterpret_cast<uint32_t *>(smraw + sd_off_merge(CH));   // [8 * top_k]
-    int *midx = reinterpret_cast<int *>(mkey + kSdWarps * s.top_k);            // [8 * top_k]
-    int *mpos = midx + kSdWarps * s.top_k;                                      // [top_k]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.x / a.C, cta = blockIdx.x % a.C;
@@ -142,9 +147,6 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     const int first = (s.flags & SA_SINK) ? 1 : 0;
     const int cc0 = first + cta * kSdWarps * CH;                    // the CTA's first candidate
     const int ncta = max(0, min(local, cc0 + kSdWarps * CH) - cc0);
-    const int wsel = min(warp, kSdWarps - 1);
-    const int c0 = cc0 + wsel * CH;                                 // a scoring warp's first candidate
-    const int n = max(0, min(ncta - wsel * CH, CH));
 
     // the attention launch that follows may start as this grid's CTAs are placed
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -161,7 +163,6 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     const T *Lg = (const T *)a.L + ((size_t)b * s.Hkv + g) * s.nb * D;
     const size_t cbytes = (size_t)ncta * RB;                        // the CTA's landmark bytes
     const int nst = (int)((cbytes + kSdStage - 1) / kSdStage);
-    uint32_t *kw = keys + wsel * CH;
     bool nan_seen = false;
     float qv[EPV];
     const int sub = lane / VPR, cv = lane % VPR;
@@ -201,6 +202,25 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
         }
 #pragma unroll
         for (int i = 0; i < EPV; ++i) qv[i] /= (float)s.heads_per;
+        // the sink and local scores (warp 0 of the unit's first CTA, while the
+        // first stage is in flight)
+        if (cta == 0 && warp == 0) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int blk = e == 0 ? 0 : local;
+                float f[EPV];
+                load16(Lg + (size_t)blk * D + cv * EPV, f);
+                float dot = 0.f;
+#pragma unroll
+                for (int i = 0; i < EPV; ++i) dot = fmaf(qv[i], f[i], dot);
+#pragma unroll
+                for (int o = VPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                if (lane == 0) {
+                    sm.s_special[e] = s.scale * dot;
+                    nan_seen |= isnan(s.scale * dot);
+                }
+            }
+        }
         for (int i = 0; i < nst; ++i) {
             const int st = i % NST;
             const bool ok = mbar_wait(smem_u32(&sm.full[st]), (i / NST) & 1, &sm.abort_flag, a.status);
@@ -242,123 +262,71 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
             }
         }
     }
-    __syncthreads();
-    if (warp < kSdWarps) {
-        int *pw = reinterpret_cast<int *>(ring) + warp * CH;        // the warp's positions (the ring is free)
-        const int nsel = warp_topk_positions<CH / 32>(kw, n, s.top_k, pw);
-        // the warp's list (ascending block ids) into the CTA's merge area
-        for (int i = lane; i < nsel; i += 32) {
-            mkey[warp * s.top_k + i] = kw[pw[i]];
-            midx[warp * s.top_k + i] = c0 + pw[i];
-        }
-        if (lane == 0) sm.nv[warp] = nsel;
-    }
-    // the sink and local scores (one warp of the unit's first CTA)
-    if (cta == 0 && warp == 0) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int blk = e == 0 ? 0 : local;
-            float f[EPV];
-            load16(Lg + (size_t)blk * D + cv * EPV, f);
-            float dot = 0.f;
-#pragma unroll
-            for (int i = 0; i < EPV; ++i) dot = fmaf(qv[i], f[i], dot);
-#pragma unroll
-            for (int o = VPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            if (lane == 0) {
-                sm.s_special[e] = s.scale * dot;
-                nan_seen |= isnan(s.scale * dot);
-            }
-        }
-    }
     if (nan_seen) set_status(a.status, kStatusNaN);
     __syncthreads();
-
-    // ---- warp 0: the CTA's list, then the unit's ---------------------------
-    if (warp != 0) return;
-    // pack the lists in warp (= index) order; a list only moves down (the
-    // lists before it hold at most top_k entries each), read before written
-    int ntot = 0;
-    for (int w = 0; w < kSdWarps; ++w) {
-        const int m = sm.nv[w];
-        for (int i0 = 0; i0 < m; i0 += 32) {
-            const int i = i0 + lane;
-            uint32_t k = 0u;
-            int id = 0;
-            if (i < m) {
-                k = mkey[w * s.top_k + i];
-                id = midx[w * s.top_k + i];
-            }
-            __syncwarp();
-            if (i < m) {
-                mkey[ntot + i] = k;
-                midx[ntot + i] = id;
-            }
-            __syncwarp();
-        }
-        ntot += m;
-    }
-    const int nc = warp_topk_positions<16>(mkey, ntot, s.top_k, mpos);
-    // the final list's staging: the keys area is free once the warp lists are merged
-    uint32_t *sel_key = keys;
-    int *sel_idx = reinterpret_cast<int *>(keys + kSdChunk);   // top_k <= 256
+    // ---- the CTA's top-K: the eight scoring warps together ------------------
+    // (the producer leaves; the rest synchronise on named barrier 1)
+    if (warp == kSdWarps) return;
+    constexpr int NT = kSdWarps * 32;
+    BsSmem &bs = *reinterpret_cast<BsSmem *>(ring + kSdBs);
+    int *pos = reinterpret_cast<int *>(ring + kSdPos);
+    uint32_t *sel_key = reinterpret_cast<uint32_t *>(ring + kSdSelKey);
+    int *sel_idx = reinterpret_cast<int *>(ring + kSdSelIdx);
+    const int nc = block_topk32<kSdWarps, CH / 32>(keys, ncta, s.top_k, pos, bs, 1);
     if (a.C == 1) {
         // one CTA per unit: its list is the unit's
-        for (int i = lane; i < nc; i += 32) {
-            sel_idx[i] = midx[mpos[i]];
-            sel_key[i] = mkey[mpos[i]];
+        for (int i = threadIdx.x; i < nc; i += NT) {
+            sel_idx[i] = cc0 + pos[i];
+            sel_key[i] = keys[pos[i]];
         }
-        __syncwarp();
-        write_list(a, u, local, sel_idx, sel_key, nc, sm.s_special[0], sm.s_special[1]);
+        named_bar_sync<NT>(1);
+        if (warp == 0) write_list(a, u, local, sel_idx, sel_key, nc, sm.s_special[0], sm.s_special[1]);
         return;
     }
     {
         uint32_t *pk = a.pkey + ((size_t)u * a.C + cta) * s.top_k;
         int32_t *pi = a.pidx + ((size_t)u * a.C + cta) * s.top_k;
-        for (int i = lane; i < nc; i += 32) {
-            pk[i] = mkey[mpos[i]];
-            pi[i] = midx[mpos[i]];
+        for (int i = threadIdx.x; i < nc; i += NT) {
+            pk[i] = keys[pos[i]];
+            pi[i] = cc0 + pos[i];
         }
-        if (lane == 0) {
-            a.pcnt[(size_t)u * a.C + cta] = nc;
-            if (cta == 0) {
-                a.special[(size_t)u * 2] = sm.s_special[0];
-                a.special[(size_t)u * 2 + 1] = sm.s_special[1];
-            }
+        if (cta == 0 && threadIdx.x == 0) {
+            a.special[(size_t)u * 2] = sm.s_special[0];
+            a.special[(size_t)u * 2 + 1] = sm.s_special[1];
         }
     }
-    // the unit's last CTA to finish merges (writes fenced before the count)
+    // the unit's last CTA to finish merges (every thread's writes fenced
+    // before the count)
     __threadfence();
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) last = atomicAdd(a.done + u, 1u) == (unsigned)(a.C - 1);
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) return;
+    named_bar_sync<NT>(1);
+    if (threadIdx.x == 0) sm.last = atomicAdd(a.done + u, 1u) == (unsigned)(a.C - 1);
+    named_bar_sync<NT>(1);
+    if (!sm.last) return;
     __threadfence();
-    // the unit's C lists into the ring space (every stream of this CTA is over)
-    uint32_t *xkey = reinterpret_cast<uint32_t *>(ring);            // [C * top_k]
-    int *xidx = reinterpret_cast<int *>(xkey + (size_t)a.C * s.top_k);
-    int *xpos = xidx + (size_t)a.C * s.top_k;                        // [top_k]
-    ntot = 0;
-    for (int c = 0; c < a.C; ++c) {
-        const int m = __ldcg(a.pcnt + (size_t)u * a.C + c);
-        for (int i = lane; i < m; i += 32) {
-            const size_t src = ((size_t)u * a.C + c) * s.top_k + i;
-            xkey[ntot + i] = __ldcg(a.pkey + src);
-            xidx[ntot + i] = __ldcg(a.pidx + src);
-        }
-        ntot += m;
+    // Every CTA before the unit's last non-empty one owns 8 * CH > top_k
+    // candidates and left a full list, so the lists lie end to end in the
+    // workspace in candidate order: [full lists] + [min(rest, top_k)].
+    const int ncand = max(0, local - first), per = kSdWarps * CH;
+    const int ntot = (ncand / per) * s.top_k + min(ncand % per, s.top_k);
+    uint32_t *xkey = reinterpret_cast<uint32_t *>(ring + kSdXKey);
+    int *xidx = reinterpret_cast<int *>(ring + kSdXIdx);
+    const size_t src0 = (size_t)u * a.C * s.top_k;
+    for (int i = threadIdx.x; i < ntot; i += NT) {
+        xkey[i] = __ldcg(a.pkey + src0 + i);
+        xidx[i] = __ldcg(a.pidx + src0 + i);
     }
-    __syncwarp();
-    const int nf = warp_topk_positions<16>(xkey, ntot, s.top_k, xpos);
-    for (int i = lane; i < nf; i += 32) {
-        sel_idx[i] = xidx[xpos[i]];
-        sel_key[i] = xkey[xpos[i]];
+    named_bar_sync<NT>(1);
+    const int nf = block_topk32<kSdWarps, kSdMaxMerge / NT>(xkey, ntot, s.top_k, pos, bs, 1);
+    for (int i = threadIdx.x; i < nf; i += NT) {
+        sel_idx[i] = xidx[pos[i]];
+        sel_key[i] = xkey[pos[i]];
     }
-    __syncwarp();
-    write_list(a, u, local, sel_idx, sel_key, nf, __ldcg(a.special + (size_t)u * 2),
-               __ldcg(a.special + (size_t)u * 2 + 1));
-    if (lane == 0) a.done[u] = 0u;
+    named_bar_sync<NT>(1);
+    if (warp == 0) {
+        write_list(a, u, local, sel_idx, sel_key, nf, __ldcg(a.special + (size_t)u * 2),
+                   __ldcg(a.special + (size_t)u * 2 + 1));
+        if (lane == 0) a.done[u] = 0u;
+    }
 }
 
 }  // namespace
@@ -392,15 +360,10 @@ size_t select_decode_workspace(const Shape &s) {
     sd_geometry(s, C, CH);
     if (C == 1) return 0;
     const size_t units = (size_t)s.B * s.Hsel;
-    return units * C * s.top_k * 8 + units * C * 4 + units * 2 * 4 + 4 * 256;
+    return units * C * s.top_k * 8 + units * 2 * 4 + 3 * 256;
 }
 
-static size_t sd_smem(const Shape &s, int CH) {
-    static_assert((size_t)kSdMaxMerge * 8 + kSdChunk * 4 <= sd_ring_bytes(2 * kSdChunk),
-                  "cross-CTA merge fits the ring space");
-    static_assert((size_t)kSdWarps * 2 * kSdChunk * 4 <= sd_ring_bytes(2 * kSdChunk), "positions fit the ring space");
-    return sd_off_merge(CH) + (size_t)kSdWarps * s.top_k * 8 + (size_t)s.top_k * 4;
-}
+static size_t sd_smem(int CH) { return sd_smem_bytes(CH); }
 
 template <typename T>
 static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t *idx, float *score, int32_t *count,
@@ -425,7 +388,6 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
         };
         a.pkey = (uint32_t *)take(units * a.C * s.top_k * 4);
         a.pidx = (int32_t *)take(units * a.C * s.top_k * 4);
-        a.pcnt = (int32_t *)take(units * a.C * 4);
         a.special = (float *)take(units * 2 * 4);
         a.done = (unsigned *)((char *)ws + ws_layout(s).sel_decode);
     }
@@ -437,7 +399,7 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
         case 32: kern = CH == kSdChunk ? select_decode_kernel<T, 32, kSdChunk> : select_decode_kernel<T, 32, 2 * kSdChunk>; break;
         default: return cudaErrorInvalidValue;
     }
-    const size_t smem = sd_smem(s, CH);
+    const size_t smem = sd_smem(CH);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(units * a.C), kSdThreads, smem, st>>>(a);
