@@ -281,7 +281,7 @@ def decode_case(wl, device, lens=None):
     from block_sparse_long_landmark_b200 import inputs
     p = sa.params_for(wl)
     q, K, V = inputs.make_decode(wl, device=device)
-    ws = sa.workspace(p, device=device)
+    ws = sa.workspace(p, device=device, ops=sa.DECODE_OPS)
     t = dict(q=q, K=K, V=V, ws=ws)
     if lens is None:
         t["L"] = sa.landmarks(p, K)
@@ -746,7 +746,7 @@ def secondary_select_only(name, args, pk, psrc):
     g = torch.Generator(device="cuda").manual_seed(wl.seed)
     q = (torch.randn(wl.B, wl.Hq, wl.d, generator=g, device="cuda") * wl.sigma).to(wl.torch_dtype)
     L = (torch.randn(wl.B, wl.Hkv, wl.nb, wl.d, generator=g, device="cuda") * wl.sigma).to(wl.torch_dtype)
-    ws = sa.workspace(p)
+    ws = sa.workspace(p, ops=sa.DECODE_OPS)
     sel = sa._sel_out(p, True, "cuda")
     flush = flush_buffers()
     steps = max(3, args.steps)

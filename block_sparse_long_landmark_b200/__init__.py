@@ -302,10 +302,17 @@ def _hsel(p):
     return p.Hq if p.flags & SA_SELECT_PER_QHEAD else p.Hkv
 
 
-def workspace(p: sa_params, device="cuda"):
-    """A zero-filled workspace large enough for every operation of `p`."""
+DECODE_OPS = (SA_OP_LANDMARKS, SA_OP_SELECT_DECODE, SA_OP_DECODE)
+FORWARD_OPS = (SA_OP_LANDMARKS, SA_OP_SELECT, SA_OP_SELECT_DECODE, SA_OP_PREFILL, SA_OP_DECODE)
+
+
+def workspace(p: sa_params, device="cuda", ops=None):
+    """A zero-filled workspace large enough for the operations `ops` of `p`
+    (SA_OP_* codes; every operation when None).  The backward's workspace
+    grows with B * Hq * N, so a decode-only caller passes DECODE_OPS."""
     torch = _torch()
-    n = max(sparse_attn_workspace_size(p, op) for op in range(7))
+    ops = range(7) if ops is None else ops
+    n = max(sparse_attn_workspace_size(p, op) for op in ops)
     if n == 0:
         raise SparseAttnError(SA_ERR_ARG, "workspace_size")
     return torch.zeros(n, dtype=torch.uint8, device=device)

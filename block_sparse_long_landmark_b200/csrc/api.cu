@@ -23,6 +23,7 @@ sa::WsLayout sa::ws_layout(const Shape &s) {
     size_t o = kStatusBytes;
     L.sel_chunk = o;  o += al(units * s.nb * 4);
     L.sel_decode = o; o += al(units * 4);
+    L.dec = o;        o += al(units * 8);
     L.bwd_kv = o;     o += al(ktiles * 8 * 4);
     L.scratch = o;
     return L;
@@ -118,9 +119,10 @@ int launch_result(cudaError_t e) {
 }  // namespace
 
 // Decode on a fixed scratch buffer (the no-allocation entry point): the
-// status word and this call's split partials, packed from the buffer's
-// start.  The status word is cleared on the stream first; the partials need
-// no clearing (every split writes its own slot before the merge reads it).
+// status word, the per-unit completion counters and this call's split
+// partials, packed from the buffer's start.  The status word and the
+// counters are cleared on the stream first; the partials need no clearing
+// (every split writes its own slot before the merge reads it).
 int sa::decode_on_scratch(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, void *scratch,
                           size_t scratch_bytes, size_t *need, cudaStream_t st) {
@@ -128,15 +130,17 @@ int sa::decode_on_scratch(const sa_params *p, const void *q, const void *K, cons
     const int r = resolve(p, s);
     if (r != SA_OK) return r;
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    const size_t total = kStatusBytes + al(decode_workspace(s));
+    const size_t cnt_bytes = al((size_t)s.B * s.Hsel * 8);
+    const size_t total = kStatusBytes + cnt_bytes + al(decode_workspace(s));
     if (need) *need = total;
     if (total > scratch_bytes) return SA_ERR_WORKSPACE;
     if (!q || !K || !V || !idx || !score || !count || !o || !lse || !scratch) return SA_ERR_ARG;
     if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(o) || !aligned16(scratch)) return SA_ERR_ARG;
     unsigned char *w = static_cast<unsigned char *>(scratch);
-    if (cudaMemsetAsync(w, 0, kStatusBytes, st) != cudaSuccess) return SA_ERR_LAUNCH;
+    if (cudaMemsetAsync(w, 0, kStatusBytes + cnt_bytes, st) != cudaSuccess) return SA_ERR_LAUNCH;
     return launch_result(launch_decode(s, q, K, V, idx, score, count, o, lse, reinterpret_cast<unsigned *>(w),
-                                       reinterpret_cast<float *>(w + kStatusBytes), st));
+                                       reinterpret_cast<unsigned *>(w + kStatusBytes),
+                                       reinterpret_cast<float *>(w + kStatusBytes + cnt_bytes), st));
 }
 
 extern "C" {
@@ -243,6 +247,7 @@ static int decode_common(const sa_params *p, const void *q, const void *K, const
     const WsLayout L = ws_layout(s);
     unsigned char *w = static_cast<unsigned char *>(ws);
     return launch_result(launch_decode(s, q, K, V, idx, score, count, o, lse, reinterpret_cast<unsigned *>(w),
+                                       reinterpret_cast<unsigned *>(w + L.dec),
                                        reinterpret_cast<float *>(w + L.scratch), (cudaStream_t)stream));
 }
 

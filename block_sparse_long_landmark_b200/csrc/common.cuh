@@ -152,6 +152,7 @@ __device__ __forceinline__ int block_scan_incl(int v, int *tmp, int *total) {
 struct WsLayout {
     size_t sel_chunk;    // select.cu: [B * Hsel * nb] chunk CTAs finished per unit
     size_t sel_decode;   // select_decode.cu: [B * Hsel] CTAs finished per unit
+    size_t dec;          // decode.cu: [B * Hsel] partial records written, [B * Hsel] merge CTAs done
     size_t bwd_kv;       // backward_kv.cu: [B * Hkv * key tiles * 8] splits finished per tile region
     size_t scratch;      // first byte of the scratch area
 };
@@ -201,14 +202,15 @@ bool decode_mma_supported(const Shape &s);
 void decode_mma_geometry(const Shape &s, int &S, int &bps);
 size_t decode_mma_partial_bytes(const Shape &s, int S);
 int decode_mma_records(int S);
-// Decode scratch passed explicitly: the status word and the partial records
-// (R_out per unit, merged by the caller's merge launch).
+// Decode scratch passed explicitly: the status word, two completion counters
+// per unit (zero on entry, zero again on exit) and the partial records
+// (R_out per unit, combined by the caller's merge launch).
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
-                              const float *score, const int32_t *count, unsigned *status, float *part,
-                              cudaStream_t st, int &R_out);
+                              const float *score, const int32_t *count, unsigned *status, unsigned *ucnt,
+                              float *part, cudaStream_t st, int &R_out);
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                          float *part, cudaStream_t st);
+                          unsigned *ucnt, float *part, cudaStream_t st);
 size_t decode_workspace(const Shape &s);
 bool backward_supported(const Shape &s);
 size_t prefill_backward_workspace(const Shape &s);

@@ -33,6 +33,9 @@ struct DecArgs {
     float *lse;
     unsigned *status;
     float *part;   // [units][S][HP][d + 2]
+    // tensor-core records: [units] records written (the merge waits until a
+    // unit's count reaches S), [units] merge CTAs done; null otherwise
+    unsigned *ucnt, *mcnt;
     int S, bps;
 };
 
@@ -230,66 +233,114 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecArgs a) {
     }
 }
 
-// One CTA per unit: the unit's R = a.S partial records (m, l, acc[d] per
-// head) combined by log-sum-exp.  (m, l) of every record go to shared memory
-// first, then per head the max M and the sum L, then each record's weight
-// 2^(m - M); the accumulators are read with independent loads.
+// One CTA per (unit, query head of the unit): the unit's R = a.S partial
+// records of that head (m, l, acc[d]) combined by log-sum-exp.  Each thread
+// takes whole output dimensions: the max M over the records' m, then L and O
+// weighted by 2^(m - M), empty records (m = -inf) skipped; up to 16 records
+// are read in one round of independent loads.
+// Records of the tensor-core decode come with a per-unit count: the launch
+// starts while the decode still runs and each CTA waits (bounded) only for
+// its own unit's R records; the unit's last merge CTA clears both counters.
+// Otherwise the CTA waits for the whole previous launch.
+constexpr int kMergeThreads = 128;
+constexpr int kMergeRegR = 16;        // records held in registers (more: two passes over them)
+constexpr unsigned long long kMergeWaitNs = 2000000000ull;
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kDecThreads) decode_merge_kernel(DecArgs a) {
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecArgs a) {
     constexpr float kLn2 = 0.6931471805599453f;
-    extern __shared__ float msm[];               // [R][HP] m, [R][HP] l, [HP] M, [HP] L
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // the records of the launch before this one
+    __shared__ int gave_up;
     const Shape &s = a.s;
     const int d = s.d, HP = s.heads_per, R = a.S;
-    const int u = blockIdx.x;
+    const int u = blockIdx.x / HP, hh = blockIdx.x % HP;   // a unit's heads side by side
+    if (a.ucnt) {
+        if (threadIdx.x == 0) {
+            gave_up = 0;
+            unsigned long long t0, t;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+            while (ld_acquire_u32(a.ucnt + u) < (unsigned)R) {
+                // the decode gave up (its own wait ran out): no records will come
+                if (*(volatile unsigned *)a.status & kStatusTimeout) { gave_up = 1; break; }
+                asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+                if (t - t0 > kMergeWaitNs) {
+                    set_status(a.status, kStatusTimeout);
+                    gave_up = 1;
+                    break;
+                }
+                __nanosleep(256);
+            }
+        }
+        __syncthreads();
+        if (gave_up) return;
+    } else {
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // the records of the launch before this one
+    }
     const int hs = u % s.Hsel, b = u / s.Hsel;
     const int h0 = (s.flags & SA_SELECT_PER_QHEAD) ? hs : hs * s.G;
-    const float *pp = a.part + (size_t)u * R * HP * (d + 2);
-    float *wm = msm, *wl = wm + R * HP, *Mh = wl + R * HP, *Lh = Mh + HP;
-    for (int i = threadIdx.x; i < R * HP; i += kDecThreads) {
-        wm[i] = pp[(size_t)i * (d + 2)];
-        wl[i] = pp[(size_t)i * (d + 2) + 1];
-    }
-    __syncthreads();
-    for (int hh = threadIdx.x; hh < HP; hh += kDecThreads) {
-        float M = -CUDART_INF_F, L = 0.f;
-        for (int r = 0; r < R; ++r) M = fmaxf(M, wm[r * HP + hh]);
-        if (M != -CUDART_INF_F)
-            for (int r = 0; r < R; ++r)
-                if (wm[r * HP + hh] != -CUDART_INF_F) L = fmaf(wl[r * HP + hh], exp2f(wm[r * HP + hh] - M), L);
-        Mh[hh] = M;
-        Lh[hh] = L;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < R * HP; i += kDecThreads) {
-        const float M = Mh[i % HP];
-        wm[i] = (wm[i] == -CUDART_INF_F || M == -CUDART_INF_F) ? 0.f : exp2f(wm[i] - M);
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < HP * d; e += kDecThreads) {
-        const int hh = e / d, dim = e % d;
-        float O = 0.f;
+    const size_t rs = (size_t)HP * (d + 2);                  // record stride
+    const float *pp = a.part + (size_t)u * R * rs + (size_t)hh * (d + 2);
+    T *orow = (T *)a.o + ((size_t)b * s.Hq + h0 + hh) * d;
+    for (int dim = threadIdx.x; dim < d; dim += kMergeThreads) {
+        float M = -CUDART_INF_F, L = 0.f, O = 0.f;
+        if (R <= kMergeRegR) {
+            // every record's (m, l, acc[dim]) in one round of independent loads
+            float mr[kMergeRegR], lr[kMergeRegR], ar[kMergeRegR];
+#pragma unroll
+            for (int r = 0; r < kMergeRegR; ++r) {
+                mr[r] = r < R ? __ldcg(pp + r * rs) : -CUDART_INF_F;
+                lr[r] = r < R ? __ldcg(pp + r * rs + 1) : 0.f;
+                ar[r] = r < R ? __ldcg(pp + r * rs + 2 + dim) : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < kMergeRegR; ++r) M = fmaxf(M, mr[r]);
+            if (M != -CUDART_INF_F) {
+#pragma unroll
+                for (int r = 0; r < kMergeRegR; ++r)
+                    if (mr[r] != -CUDART_INF_F) {
+                        const float w = exp2f(mr[r] - M);
+                        L = fmaf(lr[r], w, L);
+                        O = fmaf(ar[r], w, O);
+                    }
+            }
+        } else {
+            for (int r = 0; r < R; ++r) M = fmaxf(M, __ldcg(pp + r * rs));
+            if (M != -CUDART_INF_F) {
 #pragma unroll 4
-        for (int r = 0; r < R; ++r) O = fmaf(pp[((size_t)r * HP + hh) * (d + 2) + 2 + dim], wm[r * HP + hh], O);
-        const float L = Lh[hh];
-        from_f(((T *)a.o)[((size_t)b * s.Hq + h0 + hh) * d + dim], L > 0.f ? O / L : 0.f);
-        if (dim == 0) a.lse[(size_t)b * s.Hq + h0 + hh] = L > 0.f ? (Mh[hh] + log2f(L)) * kLn2 : -CUDART_INF_F;
+                for (int r = 0; r < R; ++r) {
+                    const float m = __ldcg(pp + r * rs);
+                    if (m != -CUDART_INF_F) {
+                        const float w = exp2f(m - M);
+                        L = fmaf(__ldcg(pp + r * rs + 1), w, L);
+                        O = fmaf(__ldcg(pp + r * rs + 2 + dim), w, O);
+                    }
+                }
+            }
+        }
+        from_f(orow[dim], L > 0.f ? O / L : 0.f);
+        if (dim == 0) a.lse[(size_t)b * s.Hq + h0 + hh] = L > 0.f ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
+    }
+    if (a.ucnt) {
+        // every read of this CTA is done; the unit's last merge CTA clears the counters
+        __syncthreads();
+        if (threadIdx.x == 0 && atomicAdd(a.mcnt + u, 1u) == (unsigned)HP - 1) {
+            a.ucnt[u] = 0u;
+            a.mcnt[u] = 0u;
+        }
     }
 }
 
-static size_t merge_smem(const Shape &s, int R) { return (2 * (size_t)R * s.heads_per + 2 * (size_t)s.heads_per) * 4; }
 
 template <typename T>
 static cudaError_t launch_merge(const DecArgs &a, cudaStream_t st, bool pdl) {
-    const size_t smem = merge_smem(a.s, a.S);
-    if (smem > 48 * 1024) {
-        const cudaError_t e = cudaFuncSetAttribute(decode_merge_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    const unsigned units = (unsigned)(a.s.B * a.s.Hsel);
-    cudaError_t e = pdl ? launch_pdl(decode_merge_kernel<T>, dim3(units), dim3(kDecThreads), smem, st, a)
-                        : (decode_merge_kernel<T><<<units, kDecThreads, smem, st>>>(a), cudaSuccess);
+    const dim3 grid((unsigned)(a.s.B * a.s.Hsel * a.s.heads_per));
+    cudaError_t e = pdl ? launch_pdl(decode_merge_kernel<T>, grid, dim3(kMergeThreads), 0, st, a)
+                        : (decode_merge_kernel<T><<<grid, kMergeThreads, 0, st>>>(a), cudaSuccess);
     note_launch();
     return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -332,7 +383,7 @@ static cudaError_t run(DecArgs a, cudaStream_t st) {
 
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                          float *part, cudaStream_t st) {
+                          unsigned *ucnt, float *part, cudaStream_t st) {
     DecArgs a{};
     a.s = s;
     a.q = q;
@@ -346,11 +397,14 @@ cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const vo
     a.status = status;
     a.part = part;
     if (decode_mma_supported(s)) {
-        // tensor-core item records, then one merge CTA per unit
+        // tensor-core item records, counted per unit; the merge launch starts
+        // early and takes each unit as soon as its records are in
         int R = 1;
-        cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, status, part, st, R);
+        cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, status, ucnt, part, st, R);
         if (e != cudaSuccess) return e;
         a.S = R;
+        a.ucnt = ucnt;
+        a.mcnt = ucnt + (size_t)s.B * s.Hsel;
         return launch_merge<__nv_bfloat16>(a, st, true);
     }
     split_geometry(s, a.S, a.bps);

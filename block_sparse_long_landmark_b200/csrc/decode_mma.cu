@@ -21,10 +21,12 @@
 //   O[16 x 128] += P[16 x 64] V_b      (P straight from S's registers)
 // keeping an online softmax; at its last block of an item it leaves (max,
 // sum, acc) per head in the item's partial record, and the producer marks
-// the records of warps that got no block of an item empty.  A merge kernel
-// combines the kNW x splits records of each unit.  Both launches may start
-// early (programmatic dependent launch) and wait for their inputs on the
-// device.
+// the records of warps that got no block of an item empty.  Every record
+// written is counted towards its unit (after a fence), so the merge launch
+// that follows, started early, combines each unit's kNW x splits records as
+// soon as the count is complete, while other units still stream.  The launch
+// may start early too (programmatic dependent launch) and waits for the
+// lists on the device.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -67,6 +69,7 @@ struct DmArgs {
     const int32_t *count;
     unsigned *status;
     float *part;                // [units][S][kNW][heads_per][kRec]
+    unsigned *ucnt;             // [units] records written (the merge launch waits on it, then clears it)
     int S, bps, items;
 };
 
@@ -128,6 +131,14 @@ __device__ __forceinline__ uint32_t swz(int row, int u) { return row * 128 + ((u
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Counts n records of unit u as written (the warp's own writes fenced first).
+__device__ __forceinline__ void count_records(const DmArgs &a, int u, int n) {
+    __threadfence();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) atomicAdd(a.ucnt + u, (unsigned)n);
+    __syncwarp();
+}
 
 __global__ void __launch_bounds__(kThreadsD, 3)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DmArgs a) {
@@ -252,13 +263,16 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             if (!ok) break;
             if (n < kNW) {
                 // consumer warps that get no block of this item: empty records
+                int nempty = 0;
                 for (int w = 0; w < kNW; ++w) {
                     bool covered = false;
                     for (int c = 0; c < n; ++c) covered |= (gi0 + c) % kNW == w;
                     if (covered) continue;
+                    ++nempty;
                     float *rec = a.part + (((size_t)item * kNW + w) * HP) * kRec;
                     for (int hh = lane; hh < HP; hh += 32) rec[(size_t)hh * kRec] = -CUDART_INF_F;
                 }
+                count_records(a, u, nempty);
             }
         }
         // one end record per consumer warp (no data: a plain arrival completes the stage)
@@ -450,6 +464,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                 for (int nd = 0; nd < 16; ++nd)
                     *reinterpret_cast<float2 *>(rh + 2 + 8 * nd + 2 * tq) = make_float2(oacc[nd][2 * rr], oacc[nd][2 * rr + 1]);
             }
+            count_records(a, u, 1);
         }
     }
 }
@@ -465,11 +480,12 @@ bool decode_mma_supported(const Shape &s) {
     return !(e && strcmp(e, "simt") == 0);
 }
 
+int decode_mma_records(int S) { return S * kNW; }
+
 size_t decode_mma_partial_bytes(const Shape &s, int S) {
     return (((size_t)s.B * s.Hsel * S * kNW * s.heads_per * kRec * sizeof(float)) + 255) & ~(size_t)255;
 }
 
-int decode_mma_records(int S) { return S * kNW; }
 
 // Items as large as possible (fewer partial records to write and merge) while
 // the grid still fills three quarters of the slots (three CTAs per SM), with
@@ -493,8 +509,8 @@ void decode_mma_geometry(const Shape &s, int &S, int &bps) {
 }
 
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
-                              const float *score, const int32_t *count, unsigned *status, float *part,
-                              cudaStream_t st, int &R_out) {
+                              const float *score, const int32_t *count, unsigned *status, unsigned *ucnt,
+                              float *part, cudaStream_t st, int &R_out) {
     std::call_once(g_enc_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult qr;
@@ -524,6 +540,7 @@ cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, cons
     a.count = count;
     a.status = status;
     a.part = part;
+    a.ucnt = ucnt;
     decode_mma_geometry(s, a.S, a.bps);
     a.items = s.B * s.Hsel * a.S;
     const int grid = dm_grid(a.items, sm_count());

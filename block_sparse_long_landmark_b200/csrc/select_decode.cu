@@ -14,7 +14,7 @@
 // 16-byte slices per stage; the partial dots are summed by a reduce-scatter
 // across the lanes of a row, so every lane ends with one full score.  Once the
 // stream is over the eight warps take the CTA's top-K together with a
-// byte-wise radix select (block_select.cuh); when a unit spans several CTAs
+// radix select (block_select.cuh); when a unit spans several CTAs
 // each leaves its list in the workspace and the unit's last CTA to finish
 // selects again over the lists.  The candidates sit in index order throughout
 // and every select takes equal keys at the lower position, so the result is
@@ -303,6 +303,12 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     named_bar_sync<NT>(1);
     if (!sm.last) return;
     __threadfence();
+    // the sink and local scores, loaded before the lists so the loads overlap
+    float sp0 = 0.f, sp1 = 0.f;
+    if (warp == 0) {
+        sp0 = __ldcg(a.special + (size_t)u * 2);
+        sp1 = __ldcg(a.special + (size_t)u * 2 + 1);
+    }
     // Every CTA before the unit's last non-empty one owns 8 * CH > top_k
     // candidates and left a full list, so the lists lie end to end in the
     // workspace in candidate order: [full lists] + [min(rest, top_k)].
@@ -323,8 +329,7 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     }
     named_bar_sync<NT>(1);
     if (warp == 0) {
-        write_list(a, u, local, sel_idx, sel_key, nf, __ldcg(a.special + (size_t)u * 2),
-                   __ldcg(a.special + (size_t)u * 2 + 1));
+        write_list(a, u, local, sel_idx, sel_key, nf, sp0, sp1);
         if (lane == 0) a.done[u] = 0u;
     }
 }

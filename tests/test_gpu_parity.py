@@ -200,6 +200,32 @@ def test_decode_mma_matches_cuda_core(case, monkeypatch):
     assert (lse - lse2).abs().max().item() <= 1e-3
 
 
+@pytest.mark.parametrize("case", ["gated_wide", "hier_16k", "gated_ragged"])
+def test_decode_steps_reuse_one_workspace(case):
+    """Decode steps on one workspace with alternating queries: the kernel
+    counts each unit's partial records in the workspace and the CTA that
+    completes a unit merges it, returning the counter to zero, so every step
+    must give the oracle's output for its own query (a counter left behind
+    would merge a later step's unit early or never)."""
+    wl = DECODE_CASES[case]
+    p = sa.params_for(wl)
+    q, K, V = inputs.make_decode(wl, device="cuda")
+    q2 = inputs.make_decode(wl.scaled(seed=wl.seed + 7), device="cuda")[0]
+    ws = sa.workspace(p, ops=sa.DECODE_OPS)
+    L = sa.landmarks(p, K)
+    refs = {}
+    for step in range(4):
+        qs = q if step % 2 == 0 else q2
+        key = step % 2
+        if key not in refs:
+            refs[key] = _oracle_decode(wl, qs, K, V)
+        sel = oracle_sel_tensors(refs[key])
+        o, lse = sa.decode(p, qs, K, V, *sel, ws)
+        torch.cuda.synchronize()
+        assert sa.check_status(ws) == 0
+        _check_outputs(wl, refs[key], o, lse)
+
+
 @pytest.mark.parametrize("flags", [inputs.F_SINK | inputs.F_LOCAL | inputs.F_CAUSAL,
                                    inputs.F_LOCAL | inputs.F_GATE | inputs.F_CAUSAL,
                                    inputs.F_SINK | inputs.F_LOCAL | inputs.F_GATE | inputs.F_PER_QHEAD,
