@@ -4,29 +4,27 @@
 //
 // Each thread holds KPT keys in registers; warp w owns the contiguous
 // positions [w * 32 * KPT, (w + 1) * 32 * KPT), lane l the positions
-// w * 32 * KPT + j * 32 + l.  Positions at or past n hold key 0, the smallest
-// key: they lie after every real position, so they never displace one (a
-// real key equal to 0 -- a NaN score -- comes first in position order).
+// w * 32 * KPT + j * 32 + l.  The result is the top-k by (key desc, position
+// asc), positions ascending.
 //
-// Up to 2 * 32 * NW keys, each thread ranks its keys against all of them
+// Up to 2 * 32 * NW keys: each thread ranks its keys against all of them
 // (keys above, plus equal keys at a lower position) and keeps ranks below k.
 // Longer lists:
-//   1. A histogram of the top 12 bits of the keys (sign, exponent and three
-//      mantissa bits of the score; the wide digit spreads typical scores over
-//      many bins, so few lanes of a warp add to the same counter) gives the
-//      digit of the k-th largest key T and how many keys lie above it.
-//      Counters are 16 bits, two to a word (n < 65536).
-//   2. When at most 32 * NW keys share T's digit (the usual case: the top-k
-//      of a few thousand scores ends in a thin bin), they are gathered and
-//      ranked among themselves, which gives T.  Otherwise two more passes of
-//      12 and 8 bits, each over the keys that match the digits found so far,
-//      give T's remaining bits.
-//   3. A compaction in position order takes every key > T and the first
-//      (k - #keys > T) keys equal to T, so equal scores go to the lower
-//      position, as the selection rule requires; positions come out
-//      ascending.  Each warp counts its segment with ballots, one barrier
-//      publishes the warps' counts, and each key's output slot is
-//      (#keys > T before it) + min(#keys == T before it, k - #keys > T).
+//   1. A lower bound L of the k-th largest key: warp w takes the
+//      ceil(k / NW)-th largest of its lanes' maxima, L is the least of these.
+//      Each warp then holds at least ceil(k / NW) keys >= L (the maxima of
+//      those lanes), so at least k keys are >= L and the top-k all are.
+//   2. The keys >= L -- typically a few per cent of the list -- are gathered
+//      in position order (ballots and one prefix over the warps) and ranked
+//      among themselves; ranks below k are the result.
+//   3. When more than kBsCand keys pass L (heavy ties, or keys that rise
+//      along the list), a radix select instead: a histogram of the top 12
+//      bits of the keys gives the digit of the k-th largest key T and how
+//      many keys lie above it; the keys of that digit, when few, are ranked
+//      among themselves for T, else two more passes of 12 and 8 bits give the
+//      rest of T.  A compaction in position order then takes every key > T
+//      and the first (k - #keys > T) keys equal to T.  Counters are 16 bits,
+//      two to a word (n < 65536).
 #pragma once
 
 #include "common.cuh"
@@ -35,14 +33,16 @@ namespace sa {
 
 constexpr int kBsMaxWarps = 16;
 constexpr int kBsBins = 4096;   // widest digit: 12 bits
-
-constexpr int kBsCand = 32 * kBsMaxWarps;   // keys of T's digit ranked directly
+constexpr int kBsCand = 512;    // keys gathered and ranked directly
 
 struct BsSmem {
-    uint32_t hist[2][kBsBins / 2];   // 16-bit counters, bin b in half (b & 1) of word b >> 1
-    int misc[2][3];                  // per pass: T's digit, keys above that digit, keys of that digit
-    int wcnt[kBsMaxWarps][2];        // per warp: scan totals; keys > T, keys == T
-    uint32_t cand[kBsCand];          // keys of T's first digit
+    uint32_t hist[2][kBsBins / 2];    // 16-bit counters, bin b in half (b & 1) of word b >> 1
+    alignas(16) uint32_t cand[kBsCand];   // gathered keys (position order)
+    int cpos[kBsCand];                // their positions
+    int misc[2][3];                   // per pass: T's digit, keys above that digit, keys of that digit
+    int wcnt[kBsMaxWarps][2];         // per warp: counts for the prefixes
+    int wsel[kBsCand / 32 + kBsMaxWarps];   // per rank round and warp: selected candidates
+    uint32_t wlow[kBsMaxWarps];       // per warp: its bound
     int ncand;
     uint32_t T;
     int take;
@@ -53,15 +53,51 @@ __device__ __forceinline__ void named_bar_sync(int id) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(NT) : "memory");
 }
 
+// The kw-th largest (1 <= kw <= 32) of the 32 lanes' values, bit by bit
+// below the bits all lanes share.
+__device__ __forceinline__ uint32_t warp_kth_largest(uint32_t v, int kw) {
+    const uint32_t hi = __reduce_max_sync(0xffffffffu, v), lo = __reduce_min_sync(0xffffffffu, v);
+    const uint32_t diff = hi ^ lo;
+    if (diff == 0u) return hi;
+    int b = 31 - __clz(diff);
+    uint32_t T = b == 31 ? 0u : (hi & ~((2u << b) - 1u));
+    for (; b >= 0; --b) {
+        const uint32_t c = T | (1u << b);
+        if (__popc(__ballot_sync(0xffffffffu, v >= c)) >= kw) T = c;
+    }
+    return T;
+}
+
+// Rank of key x at index c among list[0..m): keys above it plus equal keys at
+// a lower index.  list is 16-byte aligned; four keys per shared load.
+__device__ __forceinline__ int rank_in(const uint32_t *list, int m, uint32_t x, int c) {
+    const uint4 *l4 = reinterpret_cast<const uint4 *>(list);
+    int r0 = 0, r1 = 0;
+    const int m4 = (reinterpret_cast<uintptr_t>(list) & 15u) ? 0 : m >> 2;
+#pragma unroll 4
+    for (int i4 = 0; i4 < m4; ++i4) {
+        const uint4 y = l4[i4];
+        const int i = i4 << 2;
+        r0 += (y.x > x) | ((y.x == x) & (i < c));
+        r1 += (y.y > x) | ((y.y == x) & (i + 1 < c));
+        r0 += (y.z > x) | ((y.z == x) & (i + 2 < c));
+        r1 += (y.w > x) | ((y.w == x) & (i + 3 < c));
+    }
+    for (int i = m4 << 2; i < m; ++i) r0 += (list[i] > x) | ((list[i] == x) & (i < c));
+    return r0 + r1;
+}
+
 // Positions (ascending) of the top-k keys of keys[0..n) into out[0..k):
-// every position when n <= k.  n <= NW * 32 * KPT < 65536.  Called by the
-// threads 0 .. NW*32-1 of the CTA together; returns the count (uniform).
+// every position when n <= k.  n <= NW * 32 * KPT < 65536, k <= 32 * NW.
+// Called by the threads 0 .. NW*32-1 of the CTA together; returns the count
+// (uniform).
 template <int NW, int KPT>
 __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem &bs, int bar_id) {
     static_assert(NW <= kBsMaxWarps && NW * 32 * KPT < 65536, "shape");
     constexpr int NT = NW * 32;
     constexpr int WPT = kBsBins / 2 / NT;      // histogram words per thread in the scan
     static_assert(WPT * NT * 2 == kBsBins, "scan split");
+    constexpr int RR = (kBsCand + NT - 1) / NT;   // rank rounds over the gathered keys
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (k <= 0 || n <= 0) return 0;
     if (n <= k) {
@@ -77,15 +113,7 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
         for (int h = 0; h < 2; ++h) {
             const int p = h * NT + tid;
             if (h * NT >= n) break;                       // uniform
-            if (p < n) {
-                const uint32_t x = keys[p];
-                int rk = 0;
-                for (int i = 0; i < n; ++i) {
-                    const uint32_t y = keys[i];
-                    rk += (y > x) | ((y == x) & (i < p));
-                }
-                sel[h] = rk < k;
-            }
+            if (p < n) sel[h] = rank_in(keys, n, keys[p], p) < k;
         }
         const unsigned m0 = __ballot_sync(0xffffffffu, sel[0]), m1 = __ballot_sync(0xffffffffu, sel[1]);
         if (lane == 0) {
@@ -116,11 +144,84 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
         r[j] = v ? keys[p0 + j * 32] : 0u;
         valid |= (v ? 1u : 0u) << j;
     }
+
+    // ---- 1. the lower bound L ------------------------------------------------
+    {
+        uint32_t tmax = 0u;
+#pragma unroll
+        for (int j = 0; j < KPT; ++j)
+            if ((valid >> j) & 1u) tmax = max(tmax, r[j]);
+        const uint32_t lw = warp_kth_largest(tmax, (k + NW - 1) / NW);
+        if (lane == 0) bs.wlow[warp] = lw;
+    }
+    named_bar_sync<NT>(bar_id);
+    uint32_t L = 0xffffffffu;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) L = min(L, bs.wlow[w]);
+
+    // ---- 2. the keys >= L, gathered in position order and ranked ------------
+    unsigned bal[KPT];
+    {
+        int W = 0;
+#pragma unroll
+        for (int j = 0; j < KPT; ++j) {
+            bal[j] = __ballot_sync(0xffffffffu, ((valid >> j) & 1u) && r[j] >= L);
+            W += __popc(bal[j]);
+        }
+        if (lane == 0) bs.wcnt[warp][0] = W;
+    }
+    named_bar_sync<NT>(bar_id);
+    int base = 0, m = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const int c = bs.wcnt[w][0];
+        if (w < warp) base += c;
+        m += c;
+    }
+    if (m <= kBsCand) {
+#pragma unroll
+        for (int j = 0; j < KPT; ++j) {
+            if ((bal[j] >> lane) & 1u) {
+                const int at = base + __popc(bal[j] & below);
+                bs.cand[at] = r[j];
+                bs.cpos[at] = p0 + j * 32;
+            }
+            base += __popc(bal[j]);
+        }
+        named_bar_sync<NT>(bar_id);
+        unsigned sb[RR];
+#pragma unroll
+        for (int rr = 0; rr < RR; ++rr) {
+            const int c = rr * NT + tid;
+            bool sel = false;
+            if (rr * NT < m && c < m) sel = rank_in(bs.cand, m, bs.cand[c], c) < k;
+            sb[rr] = __ballot_sync(0xffffffffu, sel);
+            if (lane == 0) bs.wsel[rr * NW + warp] = __popc(sb[rr]);
+        }
+        named_bar_sync<NT>(bar_id);
+        int ob = 0;
+#pragma unroll
+        for (int rr = 0; rr < RR; ++rr) {
+            int before = 0, tot = 0;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const int c = bs.wsel[rr * NW + w];
+                if (w < warp) before += c;
+                tot += c;
+            }
+            if ((sb[rr] >> lane) & 1u) out[ob + before + __popc(sb[rr] & below)] = bs.cpos[rr * NT + tid];
+            ob += tot;
+        }
+        named_bar_sync<NT>(bar_id);
+        return ob;
+    }
+
+    // ---- 3. radix select ----------------------------------------------------
     for (int i = tid; i < kBsBins / 2; i += NT) bs.hist[0][i] = 0u;
     if (tid == 0) bs.ncand = 0;
     named_bar_sync<NT>(bar_id);
 
-    // ---- 1. T's first digit; 2. T from its digit's keys, or two more digits
+    // T's first digit; then T from the keys of that digit, or two more digits
     uint32_t prefix = 0u, mask = 0u;
     int kr = k;   // rank of T among the keys that match `prefix`
     uint32_t T = 0u;
@@ -210,7 +311,7 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
         }
     }
 
-    // ---- 3. compaction in position order -----------------------------------
+    // compaction in position order: keys > T, then the first keys equal to T
     unsigned gtm[KPT], eqm[KPT];
     int G = 0, E = 0;
 #pragma unroll
