@@ -296,8 +296,15 @@ def decode_case(wl, device, lens=None):
 
 
 def decode_step(p, t, timer=None):
+    """One decode step.  Timed: the library's decode-step call (selection and
+    decode launches overlapped); attribution (with a timer): the two calls
+    one after the other, each between events."""
     import block_sparse_long_landmark_b200 as sa
-    tm = timer or (lambda n, f: f())
+    if timer is None:
+        sa.decode_step(p, t["q"], t["L"], t["K"], t["V"], t["ws"], seq_len=t.get("sl"), sel=t["sel"],
+                       out=(t["o"], t["lse"]))
+        return
+    tm = timer
     if "sl" in t:
         tm("select_decode", lambda: sa.select_decode_varlen(p, t["q"], t["L"], t["sl"], t["ws"], out=t["sel"]))
         tm("decode", lambda: sa.decode_varlen(p, t["q"], t["K"], t["V"], t["sl"], *t["sel"], t["ws"],

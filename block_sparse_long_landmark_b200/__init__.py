@@ -35,7 +35,7 @@ EXPORTS = (
     "sparse_attn_version", "sparse_attn_launch_count", "sparse_attn_decode_static",
     "sparse_attn_prefill_kernel", "sparse_attn_last_cuda_error", "sparse_attn_cuda_error_string",
     "sparse_attn_landmarks_update", "sparse_attn_select_decode_varlen", "sparse_attn_decode_varlen",
-    "sparse_attn_prefill_backward", "sparse_attn_select_backward",
+    "sparse_attn_decode_step", "sparse_attn_prefill_backward", "sparse_attn_select_backward",
     "sparse_attn_lsa_clusters", "sparse_attn_lsa_workspace_size", "sparse_attn_lsa_build", "sparse_attn_lsa_decode",
     "sparse_attn_lsa_tree_size", "sparse_attn_lsa_tree_workspace_size", "sparse_attn_lsa_tree_build",
     "sparse_attn_lsa_tree_decode",
@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
             L.sparse_attn_select_decode_varlen.restype = i
             L.sparse_attn_decode_varlen.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
             L.sparse_attn_decode_varlen.restype = i
+            L.sparse_attn_decode_step.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
+            L.sparse_attn_decode_step.restype = i
             L.sparse_attn_last_cuda_error.argtypes = []
             L.sparse_attn_last_cuda_error.restype = i
             L.sparse_attn_cuda_error_string.argtypes = [i]
@@ -235,6 +237,11 @@ def sparse_attn_select_decode_varlen(p, q, L, seq_len, idx, score, count, ws, ws
 def sparse_attn_decode_varlen(p, q, K, V, seq_len, idx, score, count, o, lse, ws, ws_bytes, stream) -> int:
     return lib().sparse_attn_decode_varlen(ctypes.byref(p), q, K, V, seq_len, idx, score, count, o, lse, ws,
                                            ws_bytes, stream)
+
+
+def sparse_attn_decode_step(p, q, L, K, V, seq_len, idx, score, count, o, lse, ws, ws_bytes, stream) -> int:
+    return lib().sparse_attn_decode_step(ctypes.byref(p), q, L, K, V, seq_len, idx, score, count, o, lse, ws,
+                                         ws_bytes, stream)
 
 
 def sparse_attn_check_status(ws, stream):
@@ -482,6 +489,24 @@ def decode_varlen(p, q, K, V, seq_len, idx, sc, cnt, ws, out=None, stream=None):
                                      _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "sparse_attn_decode_varlen")
     return o, lse
+
+
+def decode_step(p, q, L, K, V, ws, seq_len=None, sel=None, out=None, stream=None):
+    """One decode step: the selection into `sel` (idx, score, count) and the
+    decode into `out` (o, lse), the two launches overlapped when the kernels
+    allow it.  `ws` must cover SA_OP_SELECT_DECODE and SA_OP_DECODE."""
+    torch = _torch()
+    idx, sc, cnt = sel if sel is not None else _sel_out(p, True, q.device)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(p.B, p.Hq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    sl = _ptr(seq_len) if seq_len is not None else None
+    _check(sparse_attn_decode_step(p, _ptr(q), _ptr(L), _ptr(K), _ptr(V), sl, _ptr(idx), _ptr(sc), _ptr(cnt),
+                                   _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "sparse_attn_decode_step")
+    return (idx, sc, cnt), (o, lse)
 
 
 def check_status(ws, stream=None):

@@ -23,6 +23,7 @@ sa::WsLayout sa::ws_layout(const Shape &s) {
     size_t o = kStatusBytes;
     L.sel_chunk = o;  o += al(units * s.nb * 4);
     L.sel_decode = o; o += al(units * 4);
+    L.sel_ready = o;  o += al(units * 4);
     L.dec = o;        o += al(units * 8);
     L.bwd_kv = o;     o += al(ktiles * 8 * 4);
     L.scratch = o;
@@ -39,6 +40,16 @@ int sa::sm_count() {
 namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Numbers that tell one decode step's published lists from every earlier
+// step's (never 0, the value of a fresh workspace).
+std::atomic<unsigned> g_epoch{0};
+unsigned next_epoch() {
+    unsigned e;
+    do e = g_epoch.fetch_add(1u, std::memory_order_relaxed) + 1u;
+    while (e == 0u);
+    return e;
+}
 
 // Resolves and checks a parameter block.  Returns SA_OK or an error code.
 int resolve(const sa_params *p, Shape &s) {
@@ -255,6 +266,34 @@ int sparse_attn_decode(const sa_params *p, const void *q, const void *K, const v
                        const float *score, const int32_t *count, void *o, float *lse, void *ws, size_t ws_bytes,
                        void *stream) {
     return decode_common(p, q, K, V, nullptr, idx, score, count, o, lse, ws, ws_bytes, stream);
+}
+
+int sparse_attn_decode_step(const sa_params *p, const void *q, const void *L, const void *K, const void *V,
+                            const int32_t *seq_len, int32_t *idx, float *score, int32_t *count, void *o,
+                            float *lse, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    int r = resolve(p, s);
+    if (r != SA_OK) return r;
+    s.seq_len = seq_len;
+    if (!q || !L || !K || !V || !idx || !score || !count || !o || !lse || !ws) return SA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(L) || !aligned16(K) || !aligned16(V) || !aligned16(o) || !aligned16(ws))
+        return SA_ERR_ARG;
+    if (ws_bytes < sparse_attn_workspace_size(p, SA_OP_SELECT_DECODE) ||
+        ws_bytes < sparse_attn_workspace_size(p, SA_OP_DECODE))
+        return SA_ERR_WORKSPACE;
+    const WsLayout Lw = ws_layout(s);
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    const cudaStream_t st = (cudaStream_t)stream;
+    // overlap when the selection publishes lists and the decode can wait on them
+    const bool overlap = select_decode_supported(s) && !select_force_chunked() && decode_mma_supported(s);
+    unsigned *ready = overlap ? reinterpret_cast<unsigned *>(w + Lw.sel_ready) : nullptr;
+    const unsigned epoch = overlap ? next_epoch() : 0u;
+    const cudaError_t e = overlap ? launch_select_decode(s, q, L, idx, score, count, ws, st, ready, epoch)
+                                  : launch_select(s, true, q, L, idx, score, count, ws, ws_bytes, st);
+    if (e != cudaSuccess) return launch_result(e);
+    return launch_result(launch_decode(s, q, K, V, idx, score, count, o, lse, reinterpret_cast<unsigned *>(w),
+                                       reinterpret_cast<unsigned *>(w + Lw.dec),
+                                       reinterpret_cast<float *>(w + Lw.scratch), st, ready, epoch));
 }
 
 int sparse_attn_decode_varlen(const sa_params *p, const void *q, const void *K, const void *V, const int32_t *seq_len,

@@ -152,6 +152,7 @@ __device__ __forceinline__ int block_scan_incl(int v, int *tmp, int *total) {
 struct WsLayout {
     size_t sel_chunk;    // select.cu: [B * Hsel * nb] chunk CTAs finished per unit
     size_t sel_decode;   // select_decode.cu: [B * Hsel] CTAs finished per unit
+    size_t sel_ready;    // select_decode.cu -> decode_mma.cu: [B * Hsel] epoch of the unit's latest list
     size_t dec;          // decode.cu: [B * Hsel] partial records written, [B * Hsel] merge CTAs done
     size_t bwd_kv;       // backward_kv.cu: [B * Hkv * key tiles * 8] splits finished per tile region
     size_t scratch;      // first byte of the scratch area
@@ -180,8 +181,11 @@ size_t select_workspace(const Shape &s, bool decode);
 bool select_tiles_supported(const Shape &s);
 bool select_decode_supported(const Shape &s);
 size_t select_decode_workspace(const Shape &s);
+// With `ready` (the decode step's overlap), each unit's final list is
+// published by storing `epoch` into ready[unit] once it is written.
 cudaError_t launch_select_decode(const Shape &s, const void *q, const void *L, int32_t *idx, float *score,
-                                 int32_t *count, void *ws, cudaStream_t st);
+                                 int32_t *count, void *ws, cudaStream_t st, unsigned *ready = nullptr,
+                                 unsigned epoch = 0);
 // SPARSE_ATTN_SELECT_PATH=chunked: decode selection by the CTA-per-chunk
 // kernel of select.cu (a cross-check hook; both give the same lists)
 bool select_force_chunked();
@@ -205,12 +209,16 @@ int decode_mma_records(int S);
 // Decode scratch passed explicitly: the status word, two completion counters
 // per unit (zero on entry, zero again on exit) and the partial records
 // (R_out per unit, combined by the caller's merge launch).
+// With `ready` the launch does not wait for the previous launch as a whole:
+// each item waits (bounded) until ready[unit] holds `epoch`.
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                               const float *score, const int32_t *count, unsigned *status, unsigned *ucnt,
-                              float *part, cudaStream_t st, int &R_out);
+                              float *part, cudaStream_t st, int &R_out, const unsigned *ready = nullptr,
+                              unsigned epoch = 0);
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                          unsigned *ucnt, float *part, cudaStream_t st);
+                          unsigned *ucnt, float *part, cudaStream_t st, const unsigned *ready = nullptr,
+                          unsigned epoch = 0);
 size_t decode_workspace(const Shape &s);
 bool backward_supported(const Shape &s);
 size_t prefill_backward_workspace(const Shape &s);

@@ -383,7 +383,7 @@ static cudaError_t run(DecArgs a, cudaStream_t st) {
 
 cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                           const float *score, const int32_t *count, void *o, float *lse, unsigned *status,
-                          unsigned *ucnt, float *part, cudaStream_t st) {
+                          unsigned *ucnt, float *part, cudaStream_t st, const unsigned *ready, unsigned epoch) {
     DecArgs a{};
     a.s = s;
     a.q = q;
@@ -400,7 +400,7 @@ cudaError_t launch_decode(const Shape &s, const void *q, const void *K, const vo
         // tensor-core item records, counted per unit; the merge launch starts
         // early and takes each unit as soon as its records are in
         int R = 1;
-        cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, status, ucnt, part, st, R);
+        cudaError_t e = launch_decode_mma(s, q, K, V, idx, score, count, status, ucnt, part, st, R, ready, epoch);
         if (e != cudaSuccess) return e;
         a.S = R;
         a.ucnt = ucnt;

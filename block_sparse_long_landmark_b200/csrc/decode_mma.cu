@@ -26,7 +26,9 @@
 // that follows, started early, combines each unit's kNW x splits records as
 // soon as the count is complete, while other units still stream.  The launch
 // may start early too (programmatic dependent launch) and waits for the
-// lists on the device.
+// lists on the device: for the whole selection launch, or, in a decode step,
+// for each item's own unit (the selection publishes each list with the
+// step's epoch), so items of early units stream while later ones are chosen.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -70,6 +72,8 @@ struct DmArgs {
     unsigned *status;
     float *part;                // [units][S][kNW][heads_per][kRec]
     unsigned *ucnt;             // [units] records written (the merge launch waits on it, then clears it)
+    const unsigned *ready;      // [units] epoch of the unit's latest list, or null (wait for the whole launch)
+    unsigned epoch;
     int S, bps, items;
 };
 
@@ -166,7 +170,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     }
     __syncthreads();
     pdl_launch();
-    pdl_wait();               // the lists come from the launch before this one
+    if (!a.ready) pdl_wait();   // the lists come from the launch before this one
 
     if (warp == 0) {
         // ---- producer: every item's kept blocks, in order ------------------
@@ -180,6 +184,33 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         auto preload = [&](int item) {
             if (item >= a.items) return;
             const int u = item / a.S, c0 = (item % a.S) * a.bps;
+            if (a.ready) {
+                // this unit's list of this step: bounded wait on its epoch
+                int gave_up = 0;
+                if (lane == 0) {
+                    const unsigned long long t0 = now_ns();
+                    unsigned v;
+                    for (;;) {
+                        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.ready + u) : "memory");
+                        if (v == a.epoch) break;
+                        if (*abort_flag || now_ns() - t0 > kWaitNsD) {
+                            if (!*abort_flag) set_status(a.status, kStatusTimeout);
+                            *abort_flag = 1;
+                            gave_up = 1;
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, gave_up, 0)) {
+                    p_cnt = 0;
+                    return;
+                }
+                // every lane reads the list below: each takes the acquire itself
+                unsigned v;
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.ready + u) : "memory");
+                (void)v;
+            }
             p_cnt = a.count[u];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
@@ -198,7 +229,6 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
             const int cnt = max(0, min(p_cnt, s.cap));
             const int c_il[2] = {p_il[0], p_il[1]}, c_ilm[2] = {p_ilm[0], p_ilm[1]};
             const float c_sl[2] = {p_sl[0], p_sl[1]};
-            preload(item + gridDim.x);
             const int local = (seq_n(s, b) - 1) / 64;
             const int c0 = sp * a.bps;
             const int n = max(0, min(cnt, c0 + a.bps) - c0);
@@ -261,6 +291,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                 }
             }
             if (!ok) break;
+            // the next item's list, while this item's last blocks are in flight
+            preload(item + gridDim.x);
             if (n < kNW) {
                 // consumer warps that get no block of this item: empty records
                 int nempty = 0;
@@ -510,7 +542,7 @@ void decode_mma_geometry(const Shape &s, int &S, int &bps) {
 
 cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, const void *V, const int32_t *idx,
                               const float *score, const int32_t *count, unsigned *status, unsigned *ucnt,
-                              float *part, cudaStream_t st, int &R_out) {
+                              float *part, cudaStream_t st, int &R_out, const unsigned *ready, unsigned epoch) {
     std::call_once(g_enc_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult qr;
@@ -541,6 +573,8 @@ cudaError_t launch_decode_mma(const Shape &s, const void *q, const void *K, cons
     a.status = status;
     a.part = part;
     a.ucnt = ucnt;
+    a.ready = ready;
+    a.epoch = epoch;
     decode_mma_geometry(s, a.S, a.bps);
     a.items = s.B * s.Hsel * a.S;
     const int grid = dm_grid(a.items, sm_count());

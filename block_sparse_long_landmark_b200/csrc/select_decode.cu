@@ -51,6 +51,8 @@ struct SdArgs {
     int32_t *pidx;        // [units][C][top_k] per-CTA candidates (block ids)
     float *special;       // [units][2]: s_0, s_local
     unsigned *done;       // [units] CTAs finished; back to 0 by the merging CTA
+    unsigned *ready;      // [units] epoch of the latest list, or null (not published)
+    unsigned epoch;
     int C;                // CTAs per unit
 };
 
@@ -100,6 +102,16 @@ __device__ void write_list(const SdArgs &a, int u, int local, const int *sel_idx
         sc[i] = sv;
     }
     if ((threadIdx.x & 31) == 0) a.count[u] = cnt;
+}
+
+// The unit's list is written (by the calling warp): store the call's epoch
+// with release order, for a decode step that waits on it unit by unit.
+__device__ __forceinline__ void publish_list(const SdArgs &a, int u) {
+    if (!a.ready) return;
+    __threadfence();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0)
+        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.ready + u), "r"(a.epoch) : "memory");
 }
 
 // fp32 slice of a 16-byte group of elements
@@ -280,7 +292,10 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
             sel_key[i] = keys[pos[i]];
         }
         named_bar_sync<NT>(1);
-        if (warp == 0) write_list(a, u, local, sel_idx, sel_key, nc, sm.s_special[0], sm.s_special[1]);
+        if (warp == 0) {
+            write_list(a, u, local, sel_idx, sel_key, nc, sm.s_special[0], sm.s_special[1]);
+            publish_list(a, u);
+        }
         return;
     }
     {
@@ -330,6 +345,7 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     named_bar_sync<NT>(1);
     if (warp == 0) {
         write_list(a, u, local, sel_idx, sel_key, nf, sp0, sp1);
+        publish_list(a, u);
         if (lane == 0) a.done[u] = 0u;
     }
 }
@@ -372,7 +388,7 @@ static size_t sd_smem(int CH) { return sd_smem_bytes(CH); }
 
 template <typename T>
 static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t *idx, float *score, int32_t *count,
-                          void *ws, cudaStream_t st) {
+                          void *ws, cudaStream_t st, unsigned *ready, unsigned epoch) {
     SdArgs a{};
     a.s = s;
     a.q = q;
@@ -381,6 +397,8 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
     a.score = score;
     a.count = count;
     a.status = (unsigned *)ws;
+    a.ready = ready;
+    a.epoch = epoch;
     int CH;
     sd_geometry(s, a.C, CH);
     const size_t units = (size_t)s.B * s.Hsel;
@@ -413,9 +431,9 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
 }
 
 cudaError_t launch_select_decode(const Shape &s, const void *q, const void *L, int32_t *idx, float *score,
-                                 int32_t *count, void *ws, cudaStream_t st) {
-    return s.dtype == SA_BF16 ? run_sd<__nv_bfloat16>(s, q, L, idx, score, count, ws, st)
-                              : run_sd<float>(s, q, L, idx, score, count, ws, st);
+                                 int32_t *count, void *ws, cudaStream_t st, unsigned *ready, unsigned epoch) {
+    return s.dtype == SA_BF16 ? run_sd<__nv_bfloat16>(s, q, L, idx, score, count, ws, st, ready, epoch)
+                              : run_sd<float>(s, q, L, idx, score, count, ws, st, ready, epoch);
 }
 
 }  // namespace sa

@@ -248,6 +248,21 @@ int sparse_attn_decode_varlen(const sa_params *p, const void *q, const void *K, 
                               const int32_t *idx, const float *score, const int32_t *count, void *o, float *lse,
                               void *ws, size_t ws_bytes, void *stream);
 
+/* One decode step: sparse_attn_select_decode (or its _varlen form when
+ * seq_len is not NULL) followed by sparse_attn_decode on the lists it
+ * writes into idx/score/count, with the same results as those two calls.
+ * When both run their tensor-core / bulk-copy kernels (bf16, d = 128, block
+ * 64, no SPARSE_ATTN_*_PATH override) the two launches overlap: the
+ * selection publishes each (batch, selection head)'s list as soon as it is
+ * final (a per-call number stored into the workspace), and the decode's
+ * work for that list starts then instead of after the whole selection, so
+ * the cache gather of early lists overlaps the end of the selection.  Uses
+ * a workspace at least as large as both SA_OP_SELECT_DECODE and
+ * SA_OP_DECODE need. */
+int sparse_attn_decode_step(const sa_params *p, const void *q, const void *L, const void *K, const void *V,
+                            const int32_t *seq_len, int32_t *idx, float *score, int32_t *count, void *o,
+                            float *lse, void *ws, size_t ws_bytes, void *stream);
+
 /* Backward of the gated (or plain) block-sparse prefill -- [SAS] "Как это
  * применить": the selector's score enters the softmax as the gate
  * g_c = log_sigmoid(s_c - s_local), which is how the loss reaches the
