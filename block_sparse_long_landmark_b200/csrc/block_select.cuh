@@ -2,21 +2,24 @@
 // 32-bit score keys by NW warps of one CTA, synchronised on a named barrier
 // (other warps of the CTA may have left).
 //
-// Each thread holds KPT keys in registers; warp w owns the contiguous
-// positions [w * 32 * KPT, (w + 1) * 32 * KPT), lane l the positions
-// w * 32 * KPT + j * 32 + l.  The result is the top-k by (key desc, position
-// asc), positions ascending.
+// Each thread holds kpt <= KPT keys in registers; warp w owns the contiguous
+// positions [w * 32 * kpt, (w + 1) * 32 * kpt), lane l the positions
+// w * 32 * kpt + j * 32 + l.  The result is the top-k by (key desc,
+// position asc), positions ascending.
 //
-// Up to 2 * 32 * NW keys: each thread ranks its keys against all of them
-// (keys above, plus equal keys at a lower position) and keeps ranks below k.
-// Longer lists:
+// Up to 16 * NW keys: each thread ranks its key against all of them (keys
+// above, plus equal keys at a lower position) and keeps ranks below k.
+// Longer lists (the bound below is tight when every warp holds keys: the
+// caller picks kpt so that the list spreads over all of them):
 //   1. A lower bound L of the k-th largest key: warp w takes the
-//      ceil(k / NW)-th largest of its lanes' maxima, L is the least of these.
+//      ceil(k / NW)-th largest of its lanes' maxima (each lane ranks its
+//      maximum against the warp's), L is the least of these.
 //      Each warp then holds at least ceil(k / NW) keys >= L (the maxima of
 //      those lanes), so at least k keys are >= L and the top-k all are.
 //   2. The keys >= L -- typically a few per cent of the list -- are gathered
 //      in position order (ballots and one prefix over the warps) and ranked
-//      among themselves; ranks below k are the result.
+//      among themselves (up to four threads per key, each over a slice);
+//      ranks below k are the result.
 //   3. When more than kBsCand keys pass L (heavy ties, or keys that rise
 //      along the list), a radix select instead: a histogram of the top 12
 //      bits of the keys gives the digit of the k-th largest key T and how
@@ -53,29 +56,30 @@ __device__ __forceinline__ void named_bar_sync(int id) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(NT) : "memory");
 }
 
-// The kw-th largest (1 <= kw <= 32) of the 32 lanes' values, bit by bit
-// below the bits all lanes share.
+// The kw-th largest (1 <= kw <= 32) of the 32 lanes' values: each lane ranks
+// its value against every lane's (32 independent shuffles; equal values in
+// lane order), and the lane of rank kw - 1 holds the answer.
 __device__ __forceinline__ uint32_t warp_kth_largest(uint32_t v, int kw) {
-    const uint32_t hi = __reduce_max_sync(0xffffffffu, v), lo = __reduce_min_sync(0xffffffffu, v);
-    const uint32_t diff = hi ^ lo;
-    if (diff == 0u) return hi;
-    int b = 31 - __clz(diff);
-    uint32_t T = b == 31 ? 0u : (hi & ~((2u << b) - 1u));
-    for (; b >= 0; --b) {
-        const uint32_t c = T | (1u << b);
-        if (__popc(__ballot_sync(0xffffffffu, v >= c)) >= kw) T = c;
+    const int lane = threadIdx.x & 31;
+    int rk = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const uint32_t x = __shfl_sync(0xffffffffu, v, j);
+        rk += (x > v) | ((x == v) & (j < lane));
     }
-    return T;
+    const unsigned at = __ballot_sync(0xffffffffu, rk == kw - 1);
+    return __shfl_sync(0xffffffffu, v, __ffs(at) - 1);
 }
 
-// Rank of key x at index c among list[0..m): keys above it plus equal keys at
-// a lower index.  list is 16-byte aligned; four keys per shared load.
-__device__ __forceinline__ int rank_in(const uint32_t *list, int m, uint32_t x, int c) {
+// Rank of key x at index c counted over list[lo..hi): keys above it plus
+// equal keys at a lower index.  lo a multiple of 4; four keys per shared
+// load when list is 16-byte aligned.
+__device__ __forceinline__ int rank_range(const uint32_t *list, int lo, int hi, uint32_t x, int c) {
     const uint4 *l4 = reinterpret_cast<const uint4 *>(list);
     int r0 = 0, r1 = 0;
-    const int m4 = (reinterpret_cast<uintptr_t>(list) & 15u) ? 0 : m >> 2;
+    const int e4 = (reinterpret_cast<uintptr_t>(list) & 15u) ? lo >> 2 : hi >> 2;
 #pragma unroll 4
-    for (int i4 = 0; i4 < m4; ++i4) {
+    for (int i4 = lo >> 2; i4 < e4; ++i4) {
         const uint4 y = l4[i4];
         const int i = i4 << 2;
         r0 += (y.x > x) | ((y.x == x) & (i < c));
@@ -83,16 +87,21 @@ __device__ __forceinline__ int rank_in(const uint32_t *list, int m, uint32_t x, 
         r0 += (y.z > x) | ((y.z == x) & (i + 2 < c));
         r1 += (y.w > x) | ((y.w == x) & (i + 3 < c));
     }
-    for (int i = m4 << 2; i < m; ++i) r0 += (list[i] > x) | ((list[i] == x) & (i < c));
+    for (int i = max(lo, e4 << 2); i < hi; ++i) r0 += (list[i] > x) | ((list[i] == x) & (i < c));
     return r0 + r1;
+}
+__device__ __forceinline__ int rank_in(const uint32_t *list, int m, uint32_t x, int c) {
+    return rank_range(list, 0, m, x, c);
 }
 
 // Positions (ascending) of the top-k keys of keys[0..n) into out[0..k):
-// every position when n <= k.  n <= NW * 32 * KPT < 65536, k <= 32 * NW.
+// every position when n <= k.  n <= NW * 32 * kpt, kpt <= KPT,
+// NW * 32 * KPT < 65536, k <= 32 * NW;
+// keys 16-byte aligned for the wide loads of the ranking (else one by one).
 // Called by the threads 0 .. NW*32-1 of the CTA together; returns the count
 // (uniform).
 template <int NW, int KPT>
-__device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem &bs, int bar_id) {
+__device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem &bs, int bar_id, int kpt) {
     static_assert(NW <= kBsMaxWarps && NW * 32 * KPT < 65536, "shape");
     constexpr int NT = NW * 32;
     constexpr int WPT = kBsBins / 2 / NT;      // histogram words per thread in the scan
@@ -106,41 +115,26 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
         return n;
     }
     const unsigned below = (1u << lane) - 1u;
-    if (n <= 2 * NT) {
+    if (n <= NT / 2) {
         // rank every key: keys above it, plus equal keys at a lower position
-        bool sel[2] = {false, false};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int p = h * NT + tid;
-            if (h * NT >= n) break;                       // uniform
-            if (p < n) sel[h] = rank_in(keys, n, keys[p], p) < k;
-        }
-        const unsigned m0 = __ballot_sync(0xffffffffu, sel[0]), m1 = __ballot_sync(0xffffffffu, sel[1]);
-        if (lane == 0) {
-            bs.wcnt[warp][0] = __popc(m0);
-            bs.wcnt[warp][1] = __popc(m1);
-        }
+        const bool sel = tid < n && rank_in(keys, n, keys[tid], tid) < k;
+        const unsigned m0 = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) bs.wcnt[warp][0] = __popc(m0);
         named_bar_sync<NT>(bar_id);
-        int b0 = 0, t0 = 0, b1 = 0;
+        int b0 = 0;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            t0 += bs.wcnt[w][0];
-            if (w < warp) {
-                b0 += bs.wcnt[w][0];
-                b1 += bs.wcnt[w][1];
-            }
-        }
-        if (sel[0]) out[b0 + __popc(m0 & below)] = tid;
-        if (sel[1]) out[t0 + b1 + __popc(m1 & below)] = NT + tid;
+        for (int w = 0; w < NW; ++w)
+            if (w < warp) b0 += bs.wcnt[w][0];
+        if (sel) out[b0 + __popc(m0 & below)] = tid;
         named_bar_sync<NT>(bar_id);
         return k;
     }
-    const int p0 = warp * 32 * KPT + lane;
+    const int p0 = warp * 32 * kpt + lane;
     uint32_t r[KPT];
     unsigned valid = 0u;
 #pragma unroll
     for (int j = 0; j < KPT; ++j) {
-        const bool v = p0 + j * 32 < n;
+        const bool v = j < kpt && p0 + j * 32 < n;
         r[j] = v ? keys[p0 + j * 32] : 0u;
         valid |= (v ? 1u : 0u) << j;
     }
@@ -189,13 +183,20 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
             base += __popc(bal[j]);
         }
         named_bar_sync<NT>(bar_id);
+        // tpc adjacent threads rank one candidate, each over a slice of the list
+        const int tpc = m <= NT / 4 ? 4 : (m <= NT / 2 ? 2 : 1);
+        const int per = ((m + tpc - 1) / tpc + 3) & ~3;
         unsigned sb[RR];
 #pragma unroll
         for (int rr = 0; rr < RR; ++rr) {
-            const int c = rr * NT + tid;
-            bool sel = false;
-            if (rr * NT < m && c < m) sel = rank_in(bs.cand, m, bs.cand[c], c) < k;
-            sb[rr] = __ballot_sync(0xffffffffu, sel);
+            const int t = rr * NT + tid, c = t / tpc, part = t % tpc;
+            int rk = 0;
+            if (c < m) {
+                const int lo = part * per, hi = min(m, lo + per);
+                if (lo < hi) rk = rank_range(bs.cand, lo, hi, bs.cand[c], c);
+            }
+            for (int o = 1; o < tpc; o <<= 1) rk += __shfl_xor_sync(0xffffffffu, rk, o);
+            sb[rr] = __ballot_sync(0xffffffffu, part == 0 && c < m && rk < k);
             if (lane == 0) bs.wsel[rr * NW + warp] = __popc(sb[rr]);
         }
         named_bar_sync<NT>(bar_id);
@@ -209,7 +210,7 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
                 if (w < warp) before += c;
                 tot += c;
             }
-            if ((sb[rr] >> lane) & 1u) out[ob + before + __popc(sb[rr] & below)] = bs.cpos[rr * NT + tid];
+            if ((sb[rr] >> lane) & 1u) out[ob + before + __popc(sb[rr] & below)] = bs.cpos[(rr * NT + tid) / tpc];
             ob += tot;
         }
         named_bar_sync<NT>(bar_id);

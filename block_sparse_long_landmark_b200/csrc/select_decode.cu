@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     int *pos = reinterpret_cast<int *>(ring + kSdPos);
     uint32_t *sel_key = reinterpret_cast<uint32_t *>(ring + kSdSelKey);
     int *sel_idx = reinterpret_cast<int *>(ring + kSdSelIdx);
-    const int nc = block_topk32<kSdWarps, CH / 32>(keys, ncta, s.top_k, pos, bs, 1);
+    const int nc = block_topk32<kSdWarps, CH / 32>(keys, ncta, s.top_k, pos, bs, 1, CH / 32);
     if (a.C == 1) {
         // one CTA per unit: its list is the unit's
         for (int i = threadIdx.x; i < nc; i += NT) {
@@ -337,7 +337,10 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
         xidx[i] = __ldcg(a.pidx + src0 + i);
     }
     named_bar_sync<NT>(1);
-    const int nf = block_topk32<kSdWarps, kSdMaxMerge / NT>(xkey, ntot, s.top_k, pos, bs, 1);
+    // one list entry per thread when they fit: every warp then takes part in the bound
+    const int nf = ntot <= NT ? block_topk32<kSdWarps, 1>(xkey, ntot, s.top_k, pos, bs, 1, 1)
+                              : block_topk32<kSdWarps, kSdMaxMerge / NT>(xkey, ntot, s.top_k, pos, bs, 1,
+                                                                         (ntot + NT - 1) / NT);
     for (int i = threadIdx.x; i < nf; i += NT) {
         sel_idx[i] = xidx[pos[i]];
         sel_key[i] = xkey[pos[i]];
