@@ -94,25 +94,77 @@ __device__ __forceinline__ int rank_in(const uint32_t *list, int m, uint32_t x, 
     return rank_range(list, 0, m, x, c);
 }
 
-// Positions (ascending) of the top-k keys of keys[0..n) into out[0..k):
-// every position when n <= k.  n <= NW * 32 * kpt, kpt <= KPT,
-// NW * 32 * KPT < 65536, k <= 32 * NW;
-// keys 16-byte aligned for the wide loads of the ranking (else one by one).
-// Called by the threads 0 .. NW*32-1 of the CTA together; returns the count
-// (uniform).
+// Result of block_select_core: either the keys >= a lower bound of the k-th
+// largest key, gathered in position order into bs.cand (keys) and bs.cpos
+// (positions), or -- when too many pass the bound, or the list is short --
+// the exact top-k positions (ascending) in `out`.  Either way at least k keys
+// (counting the whole list) are >= bound when the list has k keys (bound 0
+// makes no claim), and the keys handed back hold the top-k.
+struct BsResult {
+    int n;            // keys gathered, or positions in out
+    bool gathered;
+    uint32_t bound;
+};
+
+// Ranks the m gathered keys cand[0..m) (16-byte aligned, in position order)
+// by (key desc, index asc) and writes the indices of the top k, ascending,
+// to out.  Returns the count (uniform).
+template <int NW>
+__device__ int block_rank_gathered(const uint32_t *cand, int m, int k, int *out, BsSmem &bs, int bar_id) {
+    constexpr int NT = NW * 32;
+    constexpr int RR = (kBsCand + NT - 1) / NT;   // rank rounds over the gathered keys
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    // tpc adjacent threads rank one candidate, each over a slice of the list
+    const int tpc = m <= NT / 4 ? 4 : (m <= NT / 2 ? 2 : 1);
+    const int per = ((m + tpc - 1) / tpc + 3) & ~3;
+    unsigned sb[RR];
+#pragma unroll
+    for (int rr = 0; rr < RR; ++rr) {
+        const int t = rr * NT + tid, c = t / tpc, part = t % tpc;
+        int rk = 0;
+        if (c < m) {
+            const int lo = part * per, hi = min(m, lo + per);
+            if (lo < hi) rk = rank_range(cand, lo, hi, cand[c], c);
+        }
+        for (int o = 1; o < tpc; o <<= 1) rk += __shfl_xor_sync(0xffffffffu, rk, o);
+        sb[rr] = __ballot_sync(0xffffffffu, part == 0 && c < m && rk < k);
+        if (lane == 0) bs.wsel[rr * NW + warp] = __popc(sb[rr]);
+    }
+    named_bar_sync<NT>(bar_id);
+    int ob = 0;
+#pragma unroll
+    for (int rr = 0; rr < RR; ++rr) {
+        int before = 0, tot = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const int c = bs.wsel[rr * NW + w];
+            if (w < warp) before += c;
+            tot += c;
+        }
+        if ((sb[rr] >> lane) & 1u) out[ob + before + __popc(sb[rr] & below)] = (rr * NT + tid) / tpc;
+        ob += tot;
+    }
+    named_bar_sync<NT>(bar_id);
+    return ob;
+}
+
+// Steps 1 and 2 (gather only) or the short-list / radix paths; n <= NW * 32 *
+// kpt, kpt <= KPT, NW * 32 * KPT < 65536, k <= 32 * NW, keys 16-byte aligned
+// for the wide loads of the short-list ranking.
 template <int NW, int KPT>
-__device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem &bs, int bar_id, int kpt) {
+__device__ BsResult block_select_core(const uint32_t *keys, int n, int k, int *out, BsSmem &bs, int bar_id,
+                                      int kpt) {
     static_assert(NW <= kBsMaxWarps && NW * 32 * KPT < 65536, "shape");
     constexpr int NT = NW * 32;
     constexpr int WPT = kBsBins / 2 / NT;      // histogram words per thread in the scan
     static_assert(WPT * NT * 2 == kBsBins, "scan split");
-    constexpr int RR = (kBsCand + NT - 1) / NT;   // rank rounds over the gathered keys
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (k <= 0 || n <= 0) return 0;
+    if (k <= 0 || n <= 0) return BsResult{0, false, 0u};
     if (n <= k) {
         for (int i = tid; i < n; i += NT) out[i] = i;
         named_bar_sync<NT>(bar_id);
-        return n;
+        return BsResult{n, false, 0u};
     }
     const unsigned below = (1u << lane) - 1u;
     if (n <= NT / 2) {
@@ -127,7 +179,7 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
             if (w < warp) b0 += bs.wcnt[w][0];
         if (sel) out[b0 + __popc(m0 & below)] = tid;
         named_bar_sync<NT>(bar_id);
-        return k;
+        return BsResult{k, false, 0u};
     }
     const int p0 = warp * 32 * kpt + lane;
     uint32_t r[KPT];
@@ -153,7 +205,7 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
 #pragma unroll
     for (int w = 0; w < NW; ++w) L = min(L, bs.wlow[w]);
 
-    // ---- 2. the keys >= L, gathered in position order and ranked ------------
+    // ---- 2. the keys >= L, gathered in position order -----------------------
     unsigned bal[KPT];
     {
         int W = 0;
@@ -183,38 +235,7 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
             base += __popc(bal[j]);
         }
         named_bar_sync<NT>(bar_id);
-        // tpc adjacent threads rank one candidate, each over a slice of the list
-        const int tpc = m <= NT / 4 ? 4 : (m <= NT / 2 ? 2 : 1);
-        const int per = ((m + tpc - 1) / tpc + 3) & ~3;
-        unsigned sb[RR];
-#pragma unroll
-        for (int rr = 0; rr < RR; ++rr) {
-            const int t = rr * NT + tid, c = t / tpc, part = t % tpc;
-            int rk = 0;
-            if (c < m) {
-                const int lo = part * per, hi = min(m, lo + per);
-                if (lo < hi) rk = rank_range(bs.cand, lo, hi, bs.cand[c], c);
-            }
-            for (int o = 1; o < tpc; o <<= 1) rk += __shfl_xor_sync(0xffffffffu, rk, o);
-            sb[rr] = __ballot_sync(0xffffffffu, part == 0 && c < m && rk < k);
-            if (lane == 0) bs.wsel[rr * NW + warp] = __popc(sb[rr]);
-        }
-        named_bar_sync<NT>(bar_id);
-        int ob = 0;
-#pragma unroll
-        for (int rr = 0; rr < RR; ++rr) {
-            int before = 0, tot = 0;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const int c = bs.wsel[rr * NW + w];
-                if (w < warp) before += c;
-                tot += c;
-            }
-            if ((sb[rr] >> lane) & 1u) out[ob + before + __popc(sb[rr] & below)] = bs.cpos[(rr * NT + tid) / tpc];
-            ob += tot;
-        }
-        named_bar_sync<NT>(bar_id);
-        return ob;
+        return BsResult{m, true, L};
     }
 
     // ---- 3. radix select ----------------------------------------------------
@@ -344,7 +365,20 @@ __device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem
         eb += __popc(eqm[j]);
     }
     named_bar_sync<NT>(bar_id);
-    return k;
+    return BsResult{k, false, T};
+}
+
+// Positions (ascending) of the top-k keys of keys[0..n) into out[0..k):
+// every position when n <= k.  Shapes as block_select_core.  Returns the
+// count (uniform).
+template <int NW, int KPT>
+__device__ int block_topk32(const uint32_t *keys, int n, int k, int *out, BsSmem &bs, int bar_id, int kpt) {
+    const BsResult r = block_select_core<NW, KPT>(keys, n, k, out, bs, bar_id, kpt);
+    if (!r.gathered) return r.n;
+    const int nc = block_rank_gathered<NW>(bs.cand, r.n, k, out, bs, bar_id);
+    for (int i = threadIdx.x; i < nc; i += NW * 32) out[i] = bs.cpos[out[i]];
+    named_bar_sync<NW * 32>(bar_id);
+    return nc;
 }
 
 }  // namespace sa

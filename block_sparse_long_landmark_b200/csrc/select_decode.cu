@@ -14,11 +14,13 @@
 // 16-byte slices per stage; the partial dots are summed by a reduce-scatter
 // across the lanes of a row, so every lane ends with one full score.  Once the
 // stream is over the eight warps take the CTA's top-K together with a
-// radix select (block_select.cuh); when a unit spans several CTAs
-// each leaves its list in the workspace and the unit's last CTA to finish
-// selects again over the lists.  The candidates sit in index order throughout
-// and every select takes equal keys at the lower position, so the result is
-// the exact top-K by (score desc, index asc) whatever the split.
+// bounded-candidate select (block_select.cuh).  When a unit spans several
+// CTAs, each leaves its top-K in the workspace ordered by (key desc, block
+// asc); the unit's last CTA to finish ranks every entry in the unit by its
+// index in its own list plus a binary search in each other list, keeps ranks
+// below K and orders them by block.  Every select takes equal keys at the
+// lower block, so the result is the exact top-K by (score desc, index asc)
+// whatever the split.
 #include <cstdlib>
 #include <cstring>
 
@@ -33,7 +35,8 @@ namespace {
 constexpr int kSdWarps = 8;          // scoring warps; warp 8 streams
 constexpr int kSdThreads = 32 * (kSdWarps + 1);
 constexpr int kSdChunk = 256;        // candidates per scoring warp, or twice that
-constexpr int kSdMaxMerge = 4096;    // candidates the cross-CTA merge holds (16 per scoring thread)
+constexpr int kSdMaxMerge = 4096;    // list entries the cross-CTA merge holds
+constexpr int kSdMaxC = 64;          // CTAs per unit, at most
 constexpr int kSdStage = 32768;      // bytes per ring stage: eight 16-byte slices per scoring lane
 constexpr int kSdStages = 3;        // ring stages with 256 candidates per warp; 2 with 512
 __host__ __device__ constexpr int sd_stages(int CH) { return CH == kSdChunk ? kSdStages : 2; }
@@ -47,8 +50,9 @@ struct SdArgs {
     float *score;
     int32_t *count;
     unsigned *status;
-    uint32_t *pkey;       // [units][C][top_k] per-CTA candidates (keys)
-    int32_t *pidx;        // [units][C][top_k] per-CTA candidates (block ids)
+    uint32_t *pkey;       // [units][C][top_k] each CTA's top-K keys, by (key desc, block asc)
+    int32_t *pidx;        // [units][C][top_k] their block ids
+    int32_t *pcnt;        // [units][C] how many
     float *special;       // [units][2]: s_0, s_local
     unsigned *done;       // [units] CTAs finished; back to 0 by the merging CTA
     unsigned *ready;      // [units] epoch of the latest list, or null (not published)
@@ -60,6 +64,8 @@ struct SdSmem {
     float s_special[2];
     int abort_flag;
     int last;
+    int ccnt[kSdMaxC];          // the unit's CTAs: list lengths
+    int coff[kSdMaxC + 1];      // and where each list starts
     uint64_t full[kSdStages], empty[kSdStages];
 };
 
@@ -299,15 +305,26 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
         return;
     }
     {
+        // several CTAs per unit: this CTA's list into the workspace, ordered by
+        // (key desc, block asc) -- each entry's rank among the list's entries
         uint32_t *pk = a.pkey + ((size_t)u * a.C + cta) * s.top_k;
         int32_t *pi = a.pidx + ((size_t)u * a.C + cta) * s.top_k;
         for (int i = threadIdx.x; i < nc; i += NT) {
-            pk[i] = keys[pos[i]];
-            pi[i] = cc0 + pos[i];
+            const uint32_t x = keys[pos[i]];
+            int rk = 0;
+            for (int j = 0; j < nc; ++j) {
+                const uint32_t y = keys[pos[j]];
+                rk += (y > x) | ((y == x) & (j < i));
+            }
+            pk[rk] = x;
+            pi[rk] = cc0 + pos[i];
         }
-        if (cta == 0 && threadIdx.x == 0) {
-            a.special[(size_t)u * 2] = sm.s_special[0];
-            a.special[(size_t)u * 2 + 1] = sm.s_special[1];
+        if (threadIdx.x == 0) {
+            a.pcnt[(size_t)u * a.C + cta] = nc;
+            if (cta == 0) {
+                a.special[(size_t)u * 2] = sm.s_special[0];
+                a.special[(size_t)u * 2 + 1] = sm.s_special[1];
+            }
         }
     }
     // the unit's last CTA to finish merges (every thread's writes fenced
@@ -324,27 +341,66 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
         sp0 = __ldcg(a.special + (size_t)u * 2);
         sp1 = __ldcg(a.special + (size_t)u * 2 + 1);
     }
-    // Every CTA before the unit's last non-empty one owns 8 * CH > top_k
-    // candidates and left a full list, so the lists lie end to end in the
-    // workspace in candidate order: [full lists] + [min(rest, top_k)].
-    const int ncand = max(0, local - first), per = kSdWarps * CH;
-    const int ntot = (ncand / per) * s.top_k + min(ncand % per, s.top_k);
+    // The unit's lists, end to end in CTA order, each by (key desc, block asc).
+    // An entry's rank in the unit is its index in its own list plus, in every
+    // other list, the entries above it: keys > x, and keys == x too in the
+    // lists of earlier CTAs (lower blocks) -- a binary search per list.
     uint32_t *xkey = reinterpret_cast<uint32_t *>(ring + kSdXKey);
     int *xidx = reinterpret_cast<int *>(ring + kSdXIdx);
-    const size_t src0 = (size_t)u * a.C * s.top_k;
-    for (int i = threadIdx.x; i < ntot; i += NT) {
-        xkey[i] = __ldcg(a.pkey + src0 + i);
-        xidx[i] = __ldcg(a.pidx + src0 + i);
+    if (threadIdx.x < a.C) sm.ccnt[threadIdx.x] = __ldcg(a.pcnt + (size_t)u * a.C + threadIdx.x);
+    named_bar_sync<NT>(1);
+    if (threadIdx.x == 0) {
+        int o = 0;
+        for (int c = 0; c < a.C; ++c) {
+            sm.coff[c] = o;
+            o += sm.ccnt[c];
+        }
+        sm.coff[a.C] = o;
     }
     named_bar_sync<NT>(1);
-    // one list entry per thread when they fit: every warp then takes part in the bound
-    const int nf = ntot <= NT ? block_topk32<kSdWarps, 1>(xkey, ntot, s.top_k, pos, bs, 1, 1)
-                              : block_topk32<kSdWarps, kSdMaxMerge / NT>(xkey, ntot, s.top_k, pos, bs, 1,
-                                                                         (ntot + NT - 1) / NT);
-    for (int i = threadIdx.x; i < nf; i += NT) {
-        sel_idx[i] = xidx[pos[i]];
-        sel_key[i] = xkey[pos[i]];
+    const int total = sm.coff[a.C];
+    for (int e = threadIdx.x; e < total; e += NT) {
+        int c = 0;
+        while (sm.coff[c + 1] <= e) ++c;
+        const size_t src = ((size_t)u * a.C + c) * s.top_k + (e - sm.coff[c]);
+        xkey[e] = __ldcg(a.pkey + src);
+        xidx[e] = __ldcg(a.pidx + src);
     }
+    named_bar_sync<NT>(1);
+    for (int e = threadIdx.x; e < total; e += NT) {
+        int c = 0;
+        while (sm.coff[c + 1] <= e) ++c;
+        const uint32_t x = xkey[e];
+        int rk = e - sm.coff[c];
+        for (int c2 = 0; c2 < a.C && rk < s.top_k; ++c2) {
+            if (c2 == c) continue;
+            // first entry of list c2 not above x (descending keys)
+            int lo = sm.coff[c2], hi = sm.coff[c2 + 1];
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                const uint32_t y = xkey[mid];
+                if (y > x || (c2 < c && y == x)) lo = mid + 1;
+                else hi = mid;
+            }
+            rk += lo - sm.coff[c2];
+        }
+        if (rk < s.top_k) {       // the unit's top-K, slot = rank
+            sel_key[rk] = x;
+            pos[rk] = xidx[e];
+        }
+    }
+    named_bar_sync<NT>(1);
+    // the kept entries by ascending block
+    const int nf = min(total, s.top_k);
+    for (int i = threadIdx.x; i < nf; i += NT) {
+        const int b = pos[i];
+        int at = 0;
+        for (int j = 0; j < nf; ++j) at += pos[j] < b;
+        sel_idx[at] = b;
+        xkey[at] = sel_key[i];
+    }
+    named_bar_sync<NT>(1);
+    for (int i = threadIdx.x; i < nf; i += NT) sel_key[i] = xkey[i];
     named_bar_sync<NT>(1);
     if (warp == 0) {
         write_list(a, u, local, sel_idx, sel_key, nf, sp0, sp1);
@@ -376,7 +432,7 @@ bool select_decode_supported(const Shape &s) {
     if (s.top_k < 1 || s.top_k > kSdChunk) return false;
     int C, CH;
     sd_geometry(s, C, CH);
-    return C == 1 || (long long)C * s.top_k <= kSdMaxMerge;
+    return C == 1 || (C <= kSdMaxC && (long long)C * s.top_k <= kSdMaxMerge);
 }
 
 size_t select_decode_workspace(const Shape &s) {
@@ -384,7 +440,7 @@ size_t select_decode_workspace(const Shape &s) {
     sd_geometry(s, C, CH);
     if (C == 1) return 0;
     const size_t units = (size_t)s.B * s.Hsel;
-    return units * C * s.top_k * 8 + units * 2 * 4 + 3 * 256;
+    return units * C * s.top_k * 8 + units * C * 4 + units * 2 * 4 + 4 * 256;
 }
 
 static size_t sd_smem(int CH) { return sd_smem_bytes(CH); }
@@ -414,6 +470,7 @@ static cudaError_t run_sd(const Shape &s, const void *q, const void *L, int32_t 
         };
         a.pkey = (uint32_t *)take(units * a.C * s.top_k * 4);
         a.pidx = (int32_t *)take(units * a.C * s.top_k * 4);
+        a.pcnt = (int32_t *)take(units * a.C * 4);
         a.special = (float *)take(units * 2 * 4);
         a.done = (unsigned *)((char *)ws + ws_layout(s).sel_decode);
     }
