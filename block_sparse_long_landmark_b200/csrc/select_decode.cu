@@ -120,6 +120,21 @@ __device__ __forceinline__ void publish_list(const SdArgs &a, int u) {
         asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.ready + u), "r"(a.epoch) : "memory");
 }
 
+// How many of list[0..n) (16-byte aligned) are below x; four per shared load.
+__device__ __forceinline__ int count_below(const int *list, int n, int x) {
+    const int4 *l4 = reinterpret_cast<const int4 *>(list);
+    int c0 = 0, c1 = 0;
+    const int n4 = n >> 2;
+#pragma unroll 4
+    for (int i4 = 0; i4 < n4; ++i4) {
+        const int4 y = l4[i4];
+        c0 += (y.x < x) + (y.z < x);
+        c1 += (y.y < x) + (y.w < x);
+    }
+    for (int i = n4 << 2; i < n; ++i) c0 += list[i] < x;
+    return c0 + c1;
+}
+
 // fp32 slice of a 16-byte group of elements
 __device__ __forceinline__ void slice_f32(const uint4 &u, const __nv_bfloat16 *, float *f) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -309,13 +324,11 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
         // (key desc, block asc) -- each entry's rank among the list's entries
         uint32_t *pk = a.pkey + ((size_t)u * a.C + cta) * s.top_k;
         int32_t *pi = a.pidx + ((size_t)u * a.C + cta) * s.top_k;
+        for (int i = threadIdx.x; i < nc; i += NT) sel_key[i] = keys[pos[i]];
+        named_bar_sync<NT>(1);
         for (int i = threadIdx.x; i < nc; i += NT) {
-            const uint32_t x = keys[pos[i]];
-            int rk = 0;
-            for (int j = 0; j < nc; ++j) {
-                const uint32_t y = keys[pos[j]];
-                rk += (y > x) | ((y == x) & (j < i));
-            }
+            const uint32_t x = sel_key[i];
+            const int rk = rank_in(sel_key, nc, x, i);
             pk[rk] = x;
             pi[rk] = cc0 + pos[i];
         }
@@ -345,57 +358,46 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     // An entry's rank in the unit is its index in its own list plus, in every
     // other list, the entries above it: keys > x, and keys == x too in the
     // lists of earlier CTAs (lower blocks) -- a binary search per list.
-    uint32_t *xkey = reinterpret_cast<uint32_t *>(ring + kSdXKey);
+    uint32_t *xkey = reinterpret_cast<uint32_t *>(ring + kSdXKey);     // [C][top_k]
     int *xidx = reinterpret_cast<int *>(ring + kSdXIdx);
+    // every list slot and every count in one round of loads
+    const int K = s.top_k, slots = a.C * K;
     if (threadIdx.x < a.C) sm.ccnt[threadIdx.x] = __ldcg(a.pcnt + (size_t)u * a.C + threadIdx.x);
-    named_bar_sync<NT>(1);
-    if (threadIdx.x == 0) {
-        int o = 0;
-        for (int c = 0; c < a.C; ++c) {
-            sm.coff[c] = o;
-            o += sm.ccnt[c];
-        }
-        sm.coff[a.C] = o;
+    for (int e = threadIdx.x; e < slots; e += NT) {
+        xkey[e] = __ldcg(a.pkey + (size_t)u * slots + e);
+        xidx[e] = __ldcg(a.pidx + (size_t)u * slots + e);
     }
     named_bar_sync<NT>(1);
-    const int total = sm.coff[a.C];
-    for (int e = threadIdx.x; e < total; e += NT) {
-        int c = 0;
-        while (sm.coff[c + 1] <= e) ++c;
-        const size_t src = ((size_t)u * a.C + c) * s.top_k + (e - sm.coff[c]);
-        xkey[e] = __ldcg(a.pkey + src);
-        xidx[e] = __ldcg(a.pidx + src);
-    }
-    named_bar_sync<NT>(1);
-    for (int e = threadIdx.x; e < total; e += NT) {
-        int c = 0;
-        while (sm.coff[c + 1] <= e) ++c;
+    int total = 0;
+    for (int c = 0; c < a.C; ++c) total += sm.ccnt[c];
+    for (int e = threadIdx.x; e < slots; e += NT) {
+        const int c = e / K, i0 = e - c * K;
+        if (i0 >= sm.ccnt[c]) continue;
         const uint32_t x = xkey[e];
-        int rk = e - sm.coff[c];
-        for (int c2 = 0; c2 < a.C && rk < s.top_k; ++c2) {
+        int rk = i0;
+        for (int c2 = 0; c2 < a.C && rk < K; ++c2) {
             if (c2 == c) continue;
             // first entry of list c2 not above x (descending keys)
-            int lo = sm.coff[c2], hi = sm.coff[c2 + 1];
+            int lo = c2 * K, hi = c2 * K + sm.ccnt[c2];
             while (lo < hi) {
                 const int mid = (lo + hi) >> 1;
                 const uint32_t y = xkey[mid];
                 if (y > x || (c2 < c && y == x)) lo = mid + 1;
                 else hi = mid;
             }
-            rk += lo - sm.coff[c2];
+            rk += lo - c2 * K;
         }
-        if (rk < s.top_k) {       // the unit's top-K, slot = rank
+        if (rk < K) {       // the unit's top-K, slot = rank
             sel_key[rk] = x;
             pos[rk] = xidx[e];
         }
     }
     named_bar_sync<NT>(1);
     // the kept entries by ascending block
-    const int nf = min(total, s.top_k);
+    const int nf = min(total, K);
     for (int i = threadIdx.x; i < nf; i += NT) {
         const int b = pos[i];
-        int at = 0;
-        for (int j = 0; j < nf; ++j) at += pos[j] < b;
+        const int at = count_below(pos, nf, b);
         sel_idx[at] = b;
         xkey[at] = sel_key[i];
     }
