@@ -32,6 +32,12 @@ CASES = {
                                 window=2100, dtype="fp32", seed=6),
     "bf16_no_clusters": dict(B=1, Hq=4, Hkv=2, d=128, N=100, pool=4, seg=32, clusters=4, top=8, sink=5,
                              window=20, dtype="bf16", seed=7),
+    # more than 16 centre chunks: the block radix merge (every score passed: 18 chunks; each
+    # chunk's best passed: 36 chunks); 2..16 chunks take the ordered lists and binary searches
+    "bf16_radix_merge_all": dict(B=1, Hq=4, Hkv=1, d=64, N=4608, pool=1, seg=32, clusters=16, top=24, sink=8,
+                                 window=64, dtype="bf16", seed=8),
+    "bf16_radix_merge_best": dict(B=1, Hq=4, Hkv=1, d=64, N=9216, pool=1, seg=32, clusters=16, top=24, sink=8,
+                                  window=64, dtype="bf16", seed=9),
 }
 
 
