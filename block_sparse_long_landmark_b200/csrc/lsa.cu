@@ -141,6 +141,116 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_build_kernel(LsaShape s, cons
 // best kk by (score desc, id asc).  The last chunk CTA of a (batch, kv-head)
 // takes the top_clusters best of the candidates with a block-wide radix
 // select and expands them into the flat list of kept key positions.
+// The kw-th largest (1 <= kw <= 32) of the 32 lanes' 64-bit values: each
+// lane ranks its value against every lane's (equal values in lane order).
+__device__ __forceinline__ uint64_t warp_kth_largest64(uint64_t v, int kw) {
+    const int lane = threadIdx.x & 31;
+    int rk = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const uint64_t x = __shfl_sync(0xffffffffu, v, j);
+        rk += (x > v) | ((x == v) & (j < lane));
+    }
+    const unsigned at = __ballot_sync(0xffffffffu, rk == kw - 1);
+    return __shfl_sync(0xffffffffu, v, __ffs(at) - 1);
+}
+
+// The merge's top-k (k <= 256) of keys[0..n) (n <= 16 * threads): a lower
+// bound L of the k-th largest key (warp w's ceil(k/8)-th largest lane
+// maximum, the least over the warps, so that at least k keys are >= L), the
+// keys >= L and their ids copied in list order into `scratch` (1536 ints,
+// 8-byte aligned), ranked among themselves; the ids of ranks below k, in
+// list order, into chosen.  Returns the count, or -1 (nothing written) when
+// more than 512 keys pass.  `hist` holds 16 + 16 * 8 + 2 * 8 ints.
+__device__ int merge_bounded(const uint64_t *keys, const int *ids, int n, int k, int *scratch, int *chosen,
+                             int *hist) {
+    constexpr int NW = kLsaThreads / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    const int J = (n + kLsaThreads - 1) / kLsaThreads;
+    uint64_t *wlow = reinterpret_cast<uint64_t *>(hist);      // [8]
+    int *cnt = hist + 16;                                     // [16][8]
+    int *rcnt = hist + 16 + 16 * NW;                          // [2][8]
+    uint64_t tmax = 0ull;
+    for (int j = 0; j < J; ++j) {
+        const int i = j * kLsaThreads + tid;
+        if (i < n) tmax = max(tmax, keys[i]);
+    }
+    const uint64_t lw = warp_kth_largest64(tmax, (k + NW - 1) / NW);
+    if (lane == 0) wlow[warp] = lw;
+    __syncthreads();
+    uint64_t L = ~0ull;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) L = min(L, wlow[w]);
+    for (int j = 0; j < J; ++j) {
+        const int i = j * kLsaThreads + tid;
+        const unsigned bal = __ballot_sync(0xffffffffu, i < n && keys[i] >= L);
+        if (lane == 0) cnt[j * NW + warp] = __popc(bal);
+    }
+    __syncthreads();
+    int m = 0;
+    for (int x = 0; x < J * NW; ++x) m += cnt[x];
+    if (m > 512) {
+        __syncthreads();          // every thread has read the counts before hist is reused
+        return -1;
+    }
+    uint64_t *ckey = reinterpret_cast<uint64_t *>(scratch);  // [512]
+    int *cid = scratch + 1024;                                // [512]
+    int base = 0;
+    for (int j = 0; j < J; ++j) {
+        const int i = j * kLsaThreads + tid;
+        const bool p = i < n && keys[i] >= L;
+        const unsigned bal = __ballot_sync(0xffffffffu, p);
+        int before = 0, tot = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const int c = cnt[j * NW + w];
+            if (w < warp) before += c;
+            tot += c;
+        }
+        if (p) {
+            const int at = base + before + __popc(bal & below);
+            ckey[at] = keys[i];
+            cid[at] = ids[i];
+        }
+        base += tot;
+    }
+    __syncthreads();
+    unsigned sb[2];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int c = rr * kLsaThreads + tid;
+        bool sel = false;
+        if (c < m) {
+            const uint64_t x = ckey[c];
+            int rk = 0;
+            for (int jj = 0; jj < m; ++jj) {
+                const uint64_t y = ckey[jj];
+                rk += (y > x) | ((y == x) & (jj < c));
+            }
+            sel = rk < k;
+        }
+        sb[rr] = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) rcnt[rr * NW + warp] = __popc(sb[rr]);
+    }
+    __syncthreads();
+    int ob = 0;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        int before = 0, tot = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const int c = rcnt[rr * NW + w];
+            if (w < warp) before += c;
+            tot += c;
+        }
+        if ((sb[rr] >> lane) & 1u) chosen[ob + before + __popc(sb[rr] & below)] = cid[rr * kLsaThreads + tid];
+        ob += tot;
+    }
+    __syncthreads();
+    return ob;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     extern __shared__ __align__(16) unsigned char smraw[];
@@ -249,8 +359,15 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
         }
     }
     __syncthreads();
-    const int nfin = block_topk64(keys, ntot, pl.ntop, pos, hist, red);
-    for (int i = tid; i < nfin; i += kLsaThreads) chosen[i] = ids[pos[i]];
+    // most lists: a bound, then a few hundred keys ranked; else the radix select
+    int nfin = -1;
+    if (ntot >= 1024 && ntot <= 16 * kLsaThreads && pl.ntop <= 256 && kmax >= 1536 &&
+        (reinterpret_cast<uintptr_t>(pos) & 7u) == 0)
+        nfin = merge_bounded(keys, ids, ntot, pl.ntop, pos, chosen, hist);
+    if (nfin < 0) {
+        nfin = block_topk64(keys, ntot, pl.ntop, pos, hist, red);
+        for (int i = tid; i < nfin; i += kLsaThreads) chosen[i] = ids[pos[i]];
+    }
     if (tid == 0) a.done1[bg] = 0u;
     __syncthreads();
     expand_positions(a, bg, chosen, nfin, off, red);
