@@ -346,17 +346,32 @@ __global__ void __launch_bounds__(kLsaThreads) lsa_select_kernel(LsaDecArgs a) {
     // merge: chunk c holds min(kk, its centres) candidates, packed in chunk order
     int ntot = 0;
     for (int c = 0; c < pl.S; ++c) ntot += min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
-#pragma unroll 4
-    for (int e = tid; e < pl.S * pl.kk; e += kLsaThreads) {
-        const int c = e / pl.kk, i = e % pl.kk;
-        const int nv = min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
-        if (i < nv) {
-            // chunks before the last are full: c * min(kk, CH) candidates precede chunk c
-            const int base = c * min(pl.kk, pl.CH);
-            const size_t src = ((size_t)bg * pl.S + c) * pl.kk + i;
-            keys[base + i] = __ldcg(reinterpret_cast<const unsigned long long *>(a.pkey) + src);
-            ids[base + i] = __ldcg(a.pid + src);
+    // (eight entries per thread loaded before any is stored: one round of loads)
+    for (int e0 = 0; e0 < pl.S * pl.kk; e0 += 8 * kLsaThreads) {
+        unsigned long long kv[8];
+        int iv[8], dst[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * kLsaThreads + tid;
+            dst[u] = -1;
+            if (e < pl.S * pl.kk) {
+                const int c = e / pl.kk, i = e % pl.kk;
+                const int nv = min(pl.kk, max(0, min(s.ctotal, (c + 1) * pl.CH) - c * pl.CH));
+                if (i < nv) {
+                    // chunks before the last are full: c * min(kk, CH) candidates precede chunk c
+                    dst[u] = c * min(pl.kk, pl.CH) + i;
+                    const size_t src = ((size_t)bg * pl.S + c) * pl.kk + i;
+                    kv[u] = __ldcg(reinterpret_cast<const unsigned long long *>(a.pkey) + src);
+                    iv[u] = __ldcg(a.pid + src);
+                }
+            }
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (dst[u] >= 0) {
+                keys[dst[u]] = kv[u];
+                ids[dst[u]] = iv[u];
+            }
     }
     __syncthreads();
     // most lists: a bound, then a few hundred keys ranked; else the radix select
