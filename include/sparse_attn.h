@@ -131,8 +131,11 @@ typedef struct {
  * and returns every completion counter it keeps there to zero by the end of
  * each call.  Calls that share a workspace must not overlap on the GPU.
  * Layout: the status word, then one counter region per operation that keeps
- * counters (prefill selection, decode selection, backward key tiles), then
- * scratch shared by all operations.  The regions are sized from the
+ * counters (prefill selection, decode selection, decode records and merge
+ * CTAs, backward key tiles), the per-list publication words of
+ * sparse_attn_decode_step (a number per call, never reset), then scratch
+ * shared by all operations.  After a call that reported a device-side
+ * timeout, zero-fill the workspace again.  The regions are sized from the
  * parameters, so a workspace serves the operations of the parameter set it
  * was sized for (any op, the largest size over the ops used); one sized for
  * another set must not be reused unless it is at least as large for every op
