@@ -396,9 +396,9 @@ __global__ void __launch_bounds__(kSdThreads, 2) select_decode_kernel(SdArgs a) 
     // the kept entries by ascending block
     const int nf = min(total, K);
     for (int i = threadIdx.x; i < nf; i += NT) {
-        const int b = pos[i];
-        const int at = count_below(pos, nf, b);
-        sel_idx[at] = b;
+        const int blk = pos[i];
+        const int at = count_below(pos, nf, blk);
+        sel_idx[at] = blk;
         xkey[at] = sel_key[i];
     }
     named_bar_sync<NT>(1);
