@@ -24,7 +24,7 @@ def round_mode(dtype: str) -> int:
 
 def run_prefill(p, Q, K, V, sel=None):
     """GPU landmarks -> select -> prefill.  ``sel`` = (idx, sc, cnt) overrides selection."""
-    ws = sa.workspace(p)
+    ws = sa.workspace(p, ops=sa.FORWARD_OPS)
     L = sa.landmarks(p, K)
     if sel is None:
         sel = sa.select(p, Q, L, ws)
@@ -35,7 +35,7 @@ def run_prefill(p, Q, K, V, sel=None):
 
 
 def run_decode(p, q, K, V, sel=None):
-    ws = sa.workspace(p)
+    ws = sa.workspace(p, ops=sa.DECODE_OPS)
     L = sa.landmarks(p, K)
     if sel is None:
         sel = sa.select_decode(p, q, L, ws)

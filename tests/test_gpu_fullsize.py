@@ -5,7 +5,9 @@ of its kv-head, selection, attention).
 
 Samples: gated_prefill_32k -- every unit; gated_decode_128k -- 8 of the 64
 sequences, all kv-heads; long_prefill_256k -- all kv-heads of 24 random tiles
-plus every 64th tile of kv-head 0; hils_decode_1m -- 2 of the 8 sequences."""
+plus every 64th tile of kv-head 0; hils_decode_1m -- 2 of the 8 sequences.
+The decodes run as one decode-step call (selection and decode overlapped),
+as the benchmark times them."""
 from __future__ import annotations
 
 import numpy as np
@@ -15,7 +17,7 @@ import torch
 import block_sparse_long_landmark_b200 as sa
 import oracle
 from block_sparse_long_landmark_b200 import inputs
-from _util import GAP, LSE_TOL, O_TOL, f64, round_mode, run_decode, run_prefill
+from _util import GAP, LSE_TOL, O_TOL, f64, round_mode, run_prefill
 
 pytestmark = pytest.mark.gpu
 
@@ -81,7 +83,12 @@ def test_long_prefill_256k_sampled():
 def _decode_sampled(wl, seqs):
     p = sa.params_for(wl)
     q, K, V = inputs.make_decode(wl, device="cuda")
-    _, (idx, sc, cnt), o, lse = run_decode(p, q, K, V)
+    # the configuration the benchmark times: one decode-step call
+    L = sa.landmarks(p, K)
+    ws = sa.workspace(p, ops=sa.DECODE_OPS)
+    (idx, sc, cnt), (o, lse) = sa.decode_step(p, q, L, K, V, ws)
+    torch.cuda.synchronize()
+    assert sa.check_status(ws) == 0
     gi, gs, gc = idx.cpu().numpy(), sc.cpu().numpy(), cnt.cpu().numpy()
     G = wl.Hq // wl.Hkv
     checked = exact = 0
