@@ -110,6 +110,25 @@ def test_varlen_entry_points_need_lengths():
     assert sa.sparse_attn_landmarks_update(_p(Hq=7), a, a, None, None, None) == sa.SA_ERR_ARG
 
 
+def test_decode_step_checks_arguments():
+    """The one-call decode step refuses what either of its two halves refuses,
+    and wants a workspace big enough for both of them; nothing is launched."""
+    p = _p(B=2, N=8192)
+    a = 256
+    big = 1 << 30
+    for kw, code in [(dict(Hq=7), sa.SA_ERR_ARG), (dict(d=96), sa.SA_ERR_UNSUPPORTED)]:
+        assert sa.sparse_attn_decode_step(_p(**kw), a, a, a, a, None, a, a, a, a, a, a, big, None) == code
+    for i in (0, 1, 2, 3, 5, 6, 7, 8, 9, 10):     # q L K V - idx score count o lse ws
+        ptrs = [a] * 11
+        ptrs[i] = None
+        assert sa.sparse_attn_decode_step(p, *ptrs[:4], None, *ptrs[5:], big, None) == sa.SA_ERR_ARG, i
+    assert sa.sparse_attn_decode_step(p, a + 8, a, a, a, None, a, a, a, a, a, a, big, None) == sa.SA_ERR_ARG
+    need = max(sa.sparse_attn_workspace_size(p, sa.SA_OP_SELECT_DECODE),
+               sa.sparse_attn_workspace_size(p, sa.SA_OP_DECODE))
+    assert sa.sparse_attn_decode_step(p, a, a, a, a, None, a, a, a, a, a, a, need - 256, None) == \
+        sa.SA_ERR_WORKSPACE
+
+
 def test_backward_entry_points_check_arguments():
     """Every call below fails its host-side checks before any launch."""
     p = _p()
