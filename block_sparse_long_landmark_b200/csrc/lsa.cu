@@ -411,14 +411,20 @@ __global__ void __launch_bounds__(kLsaThreads, 2) lsa_attend_kernel(LsaDecArgs a
     float *wst = reinterpret_cast<float *>(posv + ((pl.slice + 3) & ~3));      // [8 warps][HG][D + 2]
     int *misc = reinterpret_cast<int *>(wst + max((kLsaThreads / 32) * HG * (D + 2), 2 * pl.P * s.G + 2 * s.G));   // [4]
 
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // the list comes from the launch before this one
-    const int tot = a.cnt[2 * (size_t)bg + 1];
-    // this CTA's share of the kept positions, walked in rounds of pl.slice
-    const int t0 = (int)((long long)tot * pi / pl.P), t1 = (int)((long long)tot * (pi + 1) / pl.P);
     const int32_t *plist = a.pos + (size_t)bg * pl.pmax;
     const T *Kb = (const T *)a.K + (size_t)bg * s.N * D;
     const T *Vb = (const T *)a.V + (size_t)bg * s.N * D;
     const float sl2 = s.scale * kLog2e;
+    // Every list is [sink][the chosen clusters' keys][window], in that order,
+    // and the sink's and the window's rows are known before the list is: a CTA
+    // first attends to its share of those (part 0), while the launch before
+    // this one is still choosing the clusters, then to its share of the
+    // clusters' keys (part 1, list entries sink_n .. tot - nfix).
+    const int sink_n = min(s.sink, s.N), win0 = max(sink_n, s.N - s.window);
+    const int nfix = sink_n + (s.N - win0);
+    const int x0 = (int)((long long)nfix * pi / pl.P), x1 = (int)((long long)nfix * (pi + 1) / pl.P);
+    int c0 = 0, c1 = 0;
+    bool listed = false;
     for (int h0 = 0; h0 < s.G; h0 += HG) {
         const int nh = min(HG, s.G - h0);
         float qf[HG][EPV], acc[HG][EPV], m[HG], l[HG];
@@ -434,75 +440,87 @@ __global__ void __launch_bounds__(kLsaThreads, 2) lsa_attend_kernel(LsaDecArgs a
             m[h] = -CUDART_INF_F;
             l[h] = 0.f;
         }
-        for (int r0 = t0; r0 < t1; r0 += pl.slice) {
-            const int r1 = min(t1, r0 + pl.slice);
-            __syncthreads();                             // the previous round's positions are read
-            for (int i = tid; i < r1 - r0; i += kLsaThreads) {
-                posv[i] = plist[r0 + i];
-                SA_CHECK_START(a.status, posv[i], s.N);
+        for (int part = 0; part < 2; ++part) {
+            if (part == 1 && !listed) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");   // the list comes from the launch before this one
+                const int mid = max(0, min(a.cnt[2 * (size_t)bg + 1], pl.pmax) - nfix);
+                c0 = sink_n + (int)((long long)mid * pi / pl.P);
+                c1 = sink_n + (int)((long long)mid * (pi + 1) / pl.P);
+                listed = true;
             }
-            __syncthreads();
-            const int np = r1 - r0;
-            // rows of this lane group: vb + sub + u * RPW * 8 for the warp's bases vb
-            // (the trip count is the same for every lane: the row reductions
-            // shuffle over the whole warp); two rows per group in flight
-            constexpr int U = 4, NW = kLsaThreads / 32;
-            for (int vb = warp * RPW; vb < np; vb += U * RPW * NW) {
-                uint4 kr[U], vr[U];
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int v = min(vb + sub + u * RPW * NW, np - 1);
-                    const size_t row = (size_t)posv[v] * D + cv * EPV;
-                    kr[u] = *reinterpret_cast<const uint4 *>(Kb + row);
-                    vr[u] = *reinterpret_cast<const uint4 *>(Vb + row);
+            const int t0 = part == 0 ? x0 : c0, t1 = part == 0 ? x1 : c1;
+            // the part's positions, walked in rounds of pl.slice
+            for (int r0 = t0; r0 < t1; r0 += pl.slice) {
+                const int r1 = min(t1, r0 + pl.slice);
+                __syncthreads();                             // the previous round's positions are read
+                for (int i = tid; i < r1 - r0; i += kLsaThreads) {
+                    const int r = r0 + i;
+                    posv[i] = part == 1 ? plist[r] : r < sink_n ? r : win0 + (r - sink_n);
+                    SA_CHECK_START(a.status, posv[i], s.N);
                 }
-                // the U rows' scores for every head of the pass (summed over the lane group)
-                float z[U][HG];
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    float kf[EPV];
-                    load16(reinterpret_cast<const T *>(&kr[u]), kf);
-#pragma unroll
-                    for (int h = 0; h < HG; ++h) {
-                        float t = 0.f;
-#pragma unroll
-                        for (int e = 0; e < EPV; ++e) t = fmaf(qf[h][e], kf[e], t);
-                        for (int o = VPR / 2; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-                        // rows past the round (uniform over the lane group) and padded heads take no part
-                        z[u][h] = (vb + sub + u * RPW * NW < np && h < nh) ? t : -CUDART_INF_F;
-                    }
-                }
-                // one online-softmax step per head for the U rows: a single rescale
-#pragma unroll
-                for (int h = 0; h < HG; ++h) {
-                    float mn = m[h];
-#pragma unroll
-                    for (int u = 0; u < U; ++u) mn = fmaxf(mn, z[u][h]);
-                    if (mn == -CUDART_INF_F) {
-#pragma unroll
-                        for (int u = 0; u < U; ++u) z[u][h] = 0.f;
-                        continue;
-                    }
-                    const float corr = m[h] == -CUDART_INF_F ? 0.f : exp2f(m[h] - mn);
-                    float ps = 0.f;
+                __syncthreads();
+                const int np = r1 - r0;
+                // rows of this lane group: vb + sub + u * RPW * 8 for the warp's bases vb
+                // (the trip count is the same for every lane: the row reductions
+                // shuffle over the whole warp); two rows per group in flight
+                constexpr int U = 4, NW = kLsaThreads / 32;
+                for (int vb = warp * RPW; vb < np; vb += U * RPW * NW) {
+                    uint4 kr[U], vr[U];
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
-                        z[u][h] = exp2f(z[u][h] - mn);      // -inf rows give 0
-                        ps += z[u][h];
+                        const int v = min(vb + sub + u * RPW * NW, np - 1);
+                        const size_t row = (size_t)posv[v] * D + cv * EPV;
+                        kr[u] = *reinterpret_cast<const uint4 *>(Kb + row);
+                        vr[u] = *reinterpret_cast<const uint4 *>(Vb + row);
                     }
-                    l[h] = l[h] * corr + ps;
+                    // the U rows' scores for every head of the pass (summed over the lane group)
+                    float z[U][HG];
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e) acc[h][e] *= corr;
-                    m[h] = mn;
-                }
+                    for (int u = 0; u < U; ++u) {
+                        float kf[EPV];
+                        load16(reinterpret_cast<const T *>(&kr[u]), kf);
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    float vf[EPV];
-                    load16(reinterpret_cast<const T *>(&vr[u]), vf);
+                        for (int h = 0; h < HG; ++h) {
+                            float t = 0.f;
 #pragma unroll
-                    for (int h = 0; h < HG; ++h)
+                            for (int e = 0; e < EPV; ++e) t = fmaf(qf[h][e], kf[e], t);
+                            for (int o = VPR / 2; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+                            // rows past the round (uniform over the lane group) and padded heads take no part
+                            z[u][h] = (vb + sub + u * RPW * NW < np && h < nh) ? t : -CUDART_INF_F;
+                        }
+                    }
+                    // one online-softmax step per head for the U rows: a single rescale
 #pragma unroll
-                        for (int e = 0; e < EPV; ++e) acc[h][e] = fmaf(z[u][h], vf[e], acc[h][e]);
+                    for (int h = 0; h < HG; ++h) {
+                        float mn = m[h];
+#pragma unroll
+                        for (int u = 0; u < U; ++u) mn = fmaxf(mn, z[u][h]);
+                        if (mn == -CUDART_INF_F) {
+#pragma unroll
+                            for (int u = 0; u < U; ++u) z[u][h] = 0.f;
+                            continue;
+                        }
+                        const float corr = m[h] == -CUDART_INF_F ? 0.f : exp2f(m[h] - mn);
+                        float ps = 0.f;
+#pragma unroll
+                        for (int u = 0; u < U; ++u) {
+                            z[u][h] = exp2f(z[u][h] - mn);      // -inf rows give 0
+                            ps += z[u][h];
+                        }
+                        l[h] = l[h] * corr + ps;
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) acc[h][e] *= corr;
+                        m[h] = mn;
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        float vf[EPV];
+                        load16(reinterpret_cast<const T *>(&vr[u]), vf);
+#pragma unroll
+                        for (int h = 0; h < HG; ++h)
+#pragma unroll
+                            for (int e = 0; e < EPV; ++e) acc[h][e] = fmaf(z[u][h], vf[e], acc[h][e]);
+                    }
                 }
             }
         }
