@@ -26,10 +26,12 @@ Page names: [SAS] "Учёные научили трансформеры отби
 разреженное внимание для сверхдлинного контекста в языковых моделях"; [LSA] the
 Latent Sparse Attention post on rit.work.
 
-Parity status of the readings the pages leave open (tile-level shared lists
-per kv-head, gate only on selected blocks, s_local from the tile's own block,
-hierarchical weights over all kept blocks): parity unpinned against the pages;
-they are pinned only to the stated reading.
+Readings of what the pages leave open (tile-level shared lists per kv-head,
+the gate on selected blocks only, s_local from the tile's own block,
+hierarchical weights over all kept blocks) are implemented as stated.  Every
+function is pinned to the mathematics of its reading (closed forms, brute
+force on tiny inputs, library routines); the pages print no worked values that
+could decide between readings.
 """
 from __future__ import annotations
 
